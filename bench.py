@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the HiF4 W4A4 hot path on B200 — one JSON line on rank 0.
+
+Headline workload: the Wan2.2-14B-shaped FFN, per GPU 57600 tokens x 5120 ->
+13824 (tanh-GELU) -> 5120, both linears W4A4 HiF4 fake-quantized with a
+1 %-of-K protected-channel mask from the tail-percentile rule.  One step =
+for each linear: activation fake quantization (hif4_fake_quantize), weight
+decode (hif4_weight_decode), tcgen05 GEMM + epilogue (hif4_gemm_bf16) — the
+same kernels, in the same order, that hif4_linear_w4a4 launches.  value =
+FLOPs of both GEMMs (2 M N K each) over all ranks / max-over-ranks step time.
+
+The same JSON line carries the other rows of the path, each timed the same
+way: the quantizer sweep's largest size (quantize, dequantize; 2^30 BF16
+values) and the calibration workload (16 x 14400 tokens x 5120 channels),
+as GB/s of algorithmic bytes and a fraction of HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hif4|reference]
+
+Multi-GPU (torchrun, one process per GPU): tokens are sharded (each rank its
+own 57600-token batch, weights replicated), no data-path collective; weak
+scaling.  ``--impl reference`` times the CPU oracle (the only reference this
+method has) on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 HiF4 linear TFLOP/s & quantizer GB/s at Wan2.2 shapes, % of roofline"
+TOKENS, D_MODEL, D_FFN = 57600, 5120, 13824
+QUANT_N = 1 << 30
+CALIB_T, CALIB_C = 16 * 14400, 5120
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
+# hex digits) of the kernel source it was taken on; stale entries read as null.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=40)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["hif4", "reference"], default="hif4")
+    p.add_argument("--no-components", action="store_true", help="skip the quantizer / calibration lines")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-sample-rows", type=int, default=8)
+    p.add_argument("--tokens", type=int, default=TOKENS, help="tokens per GPU (default: Wan2.2 57600)")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK, source="fallback")
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "block_floating_point_hif4_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 100 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_ffn_sample(rows: int, seed: int = 3, threads: int | None = None, steps: int = 1, prep=None):
+    """Time the CPU oracle on `rows` tokens of the FFN workload (numpy-seeded
+    inputs of the same recipe).  Per step: activation fake quantization, the
+    full weight decode of W1 and W2, both FP64 products and the GELU.
+    Returns (flop per step, seconds per step list, threads)."""
+    import numpy as np
+
+    import oracle
+    from block_floating_point_hif4_b200 import workloads as wl
+    threads = threads or max(1, len(os.sched_getaffinity(0)))
+    if prep is None:
+        d = wl.ffn(M=max(rows, 2048), seed=seed)
+        x = d["x"]
+        p1 = oracle.percentile(x, threads=threads)
+        _, m1, _ = oracle.channel_mask(p1)
+        idx1 = np.nonzero(m1)[0].astype(np.int32)
+        h = wl.ffn_hidden(2048)
+        p2 = oracle.percentile(h, threads=threads)
+        _, m2, _ = oracle.channel_mask(p2)
+        idx2 = np.nonzero(m2)[0].astype(np.int32)
+        c1, mt1, _ = oracle.quantize(d["w1"], m1)
+        c2, mt2, _ = oracle.quantize(d["w2"], m2)
+        prep = dict(x=x[:rows].copy(), idx1=idx1, idx2=idx2, c1=c1, mt1=mt1, c2=c2, mt2=mt2,
+                    wm1=np.ascontiguousarray(d["w1"][:, idx1]), wm2=np.ascontiguousarray(d["w2"][:, idx2]))
+    P = prep
+    from block_floating_point_hif4_b200.workloads import f32_to_bf16_bits
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        w1 = _threaded_weight_hat(P["c1"], P["mt1"], D_FFN, D_MODEL, P["idx1"], P["wm1"], threads)
+        w2 = _threaded_weight_hat(P["c2"], P["mt2"], D_MODEL, D_FFN, P["idx2"], P["wm2"], threads)
+        xh = oracle.fake_quantize(P["x"], P["idx1"])
+        hid = oracle.linear(xh, w1, None, gelu=True, threads=threads)
+        hb = f32_to_bf16_bits(hid.astype(np.float32))
+        hh = oracle.fake_quantize(hb, P["idx2"])
+        oracle.linear(hh, w2, None, threads=threads)
+        times.append(time.perf_counter() - t0)
+    flop = 2 * 2.0 * rows * D_MODEL * D_FFN
+    return flop, times, threads, prep
+
+
+def _threaded_weight_hat(codes, meta, N, K, idx, wm, threads):
+    import numpy as np
+
+    import oracle
+    out = np.empty((N, K), np.float64)
+    bounds = np.linspace(0, N, threads + 1).astype(int)
+
+    def run(i):
+        a, b = bounds[i], bounds[i + 1]
+        if b > a:
+            out[a:b] = oracle.weight_hat(codes[a:b], meta[a:b], b - a, K, idx, wm[a:b])
+    ts = [threading.Thread(target=run, args=(i,)) for i in range(threads)]
+    [t.start() for t in ts]
+    [t.join() for t in ts]
+    return out
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = args.cpu_sample_rows
+    flop, times, threads, prep = oracle_ffn_sample(rows, steps=1)           # setup + first step
+    _, warm, _, _ = oracle_ffn_sample(rows, steps=max(0, args.warmup - 1), prep=prep)
+    _, timed, _, _ = oracle_ffn_sample(rows, steps=args.steps, prep=prep)
+    sec = sum(timed) / len(timed)
+    value = flop / sec / 1e12
+    sample = ("%d of %d tokens per step of the FFN workload (weight decode of W1, W2 in full each step), "
+              "FP64 oracle" % (rows, args.tokens))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(args):
+    return {"workload": "wan22_ffn_%dx%dx%d" % (args.tokens, D_MODEL, D_FFN), "tokens_per_gpu": args.tokens,
+            "d_model": D_MODEL, "d_ffn": D_FFN, "activation": "tanh-GELU",
+            "protected_channels": "1%% of K per linear (%d, %d) from the tail-percentile rule"
+                                  % (D_MODEL // 100, D_FFN // 100),
+            "l2": "inputs larger than L2 (X %.0f MB, H %.0f MB per GPU)" % (args.tokens * D_MODEL * 2 / 1e6,
+                                                                          args.tokens * D_FFN * 2 / 1e6),
+            "parallelism": "dp%d (tokens sharded, weights replicated, no collective)" % args.gpus}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    from block_floating_point_hif4_b200 import binding as H
+    from block_floating_point_hif4_b200 import workloads as wl
+    H.lib()
+    P = peaks()
+    M, D, F = args.tokens, D_MODEL, D_FFN
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- setup (untimed): inputs, calibration, weight quantization
+    x, _ = wl.device_rows(M, D, seed=3 + 1009 * rank, device=dev)
+    w1 = wl.device_weight(F, D, 0.015, seed=31, device=dev)
+    w2 = wl.device_weight(D, F, 0.015, seed=32, device=dev)
+    _, _, mask1, idx1 = H.calib_percentile_mask(x)
+    w1c, w1m = H.quantize(w1, mask1)
+    w1k = w1[:, idx1.long()].contiguous()
+    hbuf = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    ybuf = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(H.linear_w4a4_workspace(M, max(D, F), max(D, F)), dtype=torch.uint8, device=dev)
+    H.linear_w4a4(x, w1c, w1m, F, idx1, w1k, None, gelu=True, out=hbuf, workspace=ws)
+    _, _, mask2, idx2 = H.calib_percentile_mask(hbuf)
+    w2c, w2m = H.quantize(w2, mask2)
+    w2k = w2[:, idx2.long()].contiguous()
+    del w1, w2
+    xhat1 = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    xhat2 = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    what1 = torch.empty(F, D, dtype=torch.bfloat16, device=dev)
+    what2 = torch.empty(D, F, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+
+    stages = ["fake_quant_1", "weight_decode_1", "gemm_1", "fake_quant_2", "weight_decode_2", "gemm_2"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        H.fake_quantize(x, mask1, out=xhat1, status=status)
+        mark(1)
+        H.weight_decode(w1c, w1m, F, D, idx1, w1k, out=what1, status=status)
+        mark(2)
+        H.gemm_bf16(xhat1, what1, None, gelu=True, out=hbuf, status=status)
+        mark(3)
+        H.fake_quantize(hbuf, mask2, out=xhat2, status=status)
+        mark(4)
+        H.weight_decode(w2c, w2m, D, F, idx2, w2k, out=what2, status=status)
+        mark(5)
+        H.gemm_bf16(xhat2, what2, None, gelu=False, out=ybuf, status=status)
+        mark(6)
+
+    launches_per_step = 2 * (1 + 1 + 1 + 1)     # fake-quant, dequant, column scatter, GEMM per linear
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        barrier()
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_step = max_over_ranks(ms_total / args.steps)
+    per_stage = {s: [] for s in stages}
+    for k in range(args.steps):
+        for i, s in enumerate(stages):
+            per_stage[s].append(evs[k][i].elapsed_time(evs[k][i + 1]))
+    stage_ms = {s: statistics.mean(v) for s, v in per_stage.items()}
+    if H.get_status(status) not in (0, H.ERR_NONFINITE):
+        raise SystemExit("device status word reports an error: %d" % H.get_status(status))
+
+    flop_gemm = 2.0 * M * D * F                      # each of the two GEMMs
+    flop_step = 2 * flop_gemm
+    value = world * flop_step / (ms_step * 1e-3) / 1e12
+    gemm_ms = max_over_ranks((stage_ms["gemm_1"] + stage_ms["gemm_2"]) / 2)
+    achieved = flop_gemm / (gemm_ms * 1e-3) / 1e12
+    peak = P["bf16_tflops_sustained"]
+    gh = src_hash("hif4_linear.cu", "hif4_sm100.cuh")
+    traffic = NCU_TRAFFIC.get(("gemm", gh))
+    roofline = {"kernel": "k_gemm (hif4_gemm_bf16)", "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": "%s bf16 sustained (burst %.1f, frac %.3f)" % (P["source"], P["bf16_tflops"],
+                                                                            achieved / P["bf16_tflops"]),
+                "algorithmic_per_launch": "2*M*N*K = %.4g FLOP" % flop_gemm,
+                "avg_launch_ms": gemm_ms}
+
+    share = {s: v / sum(stage_ms.values()) for s, v in stage_ms.items()}
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(args),
+            "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
+            "stage_share": {s: round(v, 4) for s, v in share.items()}}
+
+    # ---- e2e: the public linear call with host buffers (pinned), copies timed
+    if not args.no_e2e:
+        xh = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=True)
+        xh.copy_(x)
+        yh = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=True)
+        xd = torch.empty_like(x)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            H.linear_w4a4(xd, w1c, w1m, F, idx1, w1k, None, gelu=True, out=hbuf, workspace=ws, status=status)
+            H.linear_w4a4(hbuf, w2c, w2m, D, idx2, w2k, None, gelu=False, out=ybuf, workspace=ws, status=status)
+            yh.copy_(ybuf, non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        line["e2e"] = {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": M * D * 2, "d2h_bytes_per_step": M * D * 2,
+                       "ms_per_step": e2e_ms, "api": "hif4_linear_w4a4 x2, pinned host X in, Y out"}
+        del xh, yh, xd
+
+    del xhat1, xhat2, what1, what2, hbuf, ybuf, ws, x
+    torch.cuda.empty_cache()
+
+    # ---- the other rows of the path: quantizer sweep and calibration
+    if not args.no_components:
+        comps = {}
+        n = QUANT_N
+        xq = wl.quant_sweep_torch(n, dev).view(-1, 1024)
+        codes = torch.empty(n // 1024, 512, dtype=torch.uint8, device=dev)
+        meta = torch.empty(n // 1024, 16, dtype=torch.int32, device=dev)
+        yq = torch.empty_like(xq)
+        comps["quantize"] = time_op(lambda: H.quantize(xq, codes=codes, meta=meta), args, stream, barrier,
+                                    max_over_ranks, world, n * 2.5625, P)
+        comps["dequantize"] = time_op(lambda: H.dequantize(codes, meta, 1024, out=yq), args, stream, barrier,
+                                      max_over_ranks, world, n * 2.5625, P)
+        comps["quantize"]["workload"] = comps["dequantize"]["workload"] = \
+            "quant_sweep 2^30 BF16 (rows of 5120, t3 x 0.05 x row lognormal), 2.5625 B/elem"
+        del xq, codes, meta, yq
+        torch.cuda.empty_cache()
+        acts = wl.calib_torch(CALIB_T, CALIB_C, dev)
+        cws = torch.empty(H.calib_workspace(CALIB_T, CALIB_C), dtype=torch.uint8, device=dev)
+        outs = (torch.empty(CALIB_C, dtype=torch.bfloat16, device=dev),
+                torch.empty(CALIB_C, dtype=torch.float32, device=dev),
+                torch.empty(CALIB_C, dtype=torch.uint8, device=dev),
+                torch.empty(CALIB_C // 100, dtype=torch.int32, device=dev))
+        comps["calib_percentile_mask"] = time_op(
+            lambda: H.calib_percentile_mask(acts, workspace=cws, out=outs), args, stream, barrier, max_over_ranks,
+            world, CALIB_T * CALIB_C * 2.0, P)
+        comps["calib_percentile_mask"]["workload"] = \
+            "calib 230400 x 5120 BF16, 2 B/elem read once (algorithmic); two radix passes read it twice"
+        del acts
+        line["components"] = comps
+
+    if rank == 0 and world == 1:
+        try:
+            flop, times, thr, _ = oracle_ffn_sample(args.cpu_sample_rows, steps=2)
+            sec = min(times)
+            line["cpu_baseline"] = {"value": flop / sec / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                    "sample": "%d of %d tokens of the FFN workload per step (full W1/W2 decode "
+                                              "each step), FP64 oracle, best of 2" % (args.cpu_sample_rows, M)}
+        except Exception as e:  # pragma: no cover
+            line["cpu_baseline"] = {"value": None, "unit": "TFLOP/s", "cores": None, "kind": "oracle",
+                                    "sample": "failed: %s" % e}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def time_op(fn, args, stream, barrier, max_over_ranks, world, bytes_per_call, P):
+    import torch
+    for _ in range(args.warmup):
+        fn()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    gbs = world * bytes_per_call / (ms * 1e-3) / 1e9
+    return {"value": gbs, "unit": "GB/s", "ms": ms, "bound": "hbm", "peak": P["hbm_gbs"],
+            "frac": gbs / world / P["hbm_gbs"], "peak_source": P["source"],
+            "l2": "inputs larger than L2"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,14 @@
+"""libhif4 — HiFloat4 (HiF4) W4A4 fake-quantized linear hot path on B200.
+
+The compute lives in ``libhif4.so`` (hand-written sm_100a CUDA kernels behind
+the C ABI in ``include/hif4.h``); :mod:`.binding` marshals torch tensors into
+it.  :mod:`.workloads` holds the seeded synthetic inputs.
+"""
+from .binding import (  # noqa: F401
+    Hif4Error, calib_percentile_mask, calib_workspace, dequantize, fake_quantize, gemm_bf16, get_status, lib,
+    linear_w4a4, linear_w4a4_workspace, quantize, reset_status, version, weight_decode,
+)
+
+__all__ = ["Hif4Error", "calib_percentile_mask", "calib_workspace", "dequantize", "fake_quantize",
+           "gemm_bf16", "get_status", "lib", "linear_w4a4", "linear_w4a4_workspace", "quantize", "reset_status",
+           "version", "weight_decode"]

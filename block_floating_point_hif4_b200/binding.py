@@ -1,0 +1,230 @@
+"""ctypes binding of libhif4.so — argument marshalling only.
+
+Every function here forwards to the C ABI declared in ``include/hif4.h`` with
+the same name (minus the ``hif4_`` prefix).  torch is used for device memory
+and the current CUDA stream; all HiF4 arithmetic runs in the library's CUDA
+kernels.  There is no CPU fallback: if ``libhif4.so`` is missing or fails to
+load, :func:`lib` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhif4.so")
+
+OK = 0
+ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_SHAPE, ERR_WORKSPACE = 1, 2, 3, 4
+ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED = 5, 6, 7, 8
+F32, BF16 = 0, 1
+FLAG_NONFINITE, FLAG_TIMEOUT, FLAG_BAD_INDEX = 1, 2, 4
+LINEAR_GELU_TANH = 1
+
+# (name, restype, argtypes) of every exported entry point
+_P, _I64, _U32, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_size_t
+SIGNATURES = {
+    "hif4_quantize": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "hif4_dequantize": (ctypes.c_int, [_P, _P, _I64, _I64, ctypes.c_int, _P, _I64, _P]),
+    "hif4_fake_quantize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _P]),
+    "hif4_linear_w4a4_workspace": (_SZ, [_I64, _I64, _I64]),
+    "hif4_linear_w4a4": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _I32, _P, _P, _P, _I64,
+                                        _U32, _P, _SZ, _P, _P]),
+    "hif4_weight_decode": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I32, _P, _P, _I64, _P, _P]),
+    "hif4_gemm_bf16": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P, _I64, _U32, _P, _P]),
+    "hif4_calib_workspace": (_SZ, [_I64, _I64]),
+    "hif4_calib_percentile_mask": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P, _P,
+                                                  _P, _P, _SZ, _P]),
+    "hif4_get_status": (ctypes.c_int, [_P, _P]),
+    "hif4_reset_status": (ctypes.c_int, [_P, _P]),
+    "hif4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "hif4_version": (ctypes.c_int, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Hif4Error(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        msg = lib().hif4_status_string(code).decode()
+        super().__init__("%s failed: status %d (%s)" % (fn, code, msg))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhif4.so (built in-tree by ``build.py``); raises if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError("libhif4.so is not built (run python -m block_floating_point_hif4_b200.build); "
+                                   "there is no CPU fallback")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != OK:
+        raise Hif4Error(fn, code)
+
+
+def _dev(t, name):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    return t
+
+
+# ------------------------------------------------------------------ calls
+
+def quantize(x: torch.Tensor, chan_mask: torch.Tensor | None = None, *, codes=None, meta=None,
+             status=None, stream=None):
+    """HiF4 codes (uint8 [rows, cols/2]) and meta (int32 bit patterns [rows, cols/64])."""
+    _dev(x, "x")
+    assert x.dim() == 2 and x.stride(1) == 1
+    dt = {torch.bfloat16: BF16, torch.float32: F32}[x.dtype]
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device)
+    if meta is None:
+        meta = torch.empty(rows, cols // 64, dtype=torch.int32, device=x.device)
+    _check("hif4_quantize", lib().hif4_quantize(_ptr(x), dt, rows, cols, x.stride(0), _ptr(chan_mask),
+                                                _ptr(codes), _ptr(meta), _ptr(status), _stream(stream)))
+    return codes, meta
+
+
+def dequantize(codes: torch.Tensor, meta: torch.Tensor, cols: int, dtype=torch.bfloat16, *, out=None,
+               stream=None):
+    _dev(codes, "codes")
+    rows = codes.shape[0]
+    if out is None:
+        out = torch.empty(rows, cols, dtype=dtype, device=codes.device)
+    dt = {torch.bfloat16: BF16, torch.float32: F32}[out.dtype]
+    _check("hif4_dequantize", lib().hif4_dequantize(_ptr(codes), _ptr(meta), rows, cols, dt, _ptr(out),
+                                                    out.stride(0), _stream(stream)))
+    return out
+
+
+def fake_quantize(x: torch.Tensor, chan_mask: torch.Tensor | None = None, *, out=None, status=None,
+                  stream=None):
+    _dev(x, "x")
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty(rows, cols, dtype=torch.bfloat16, device=x.device)
+    _check("hif4_fake_quantize", lib().hif4_fake_quantize(_ptr(x), rows, cols, x.stride(0), _ptr(chan_mask),
+                                                          _ptr(out), out.stride(0), _ptr(status),
+                                                          _stream(stream)))
+    return out
+
+
+def linear_w4a4_workspace(M: int, N: int, K: int) -> int:
+    return int(lib().hif4_linear_w4a4_workspace(M, N, K))
+
+
+def linear_w4a4(x: torch.Tensor, w_codes: torch.Tensor, w_meta: torch.Tensor, N: int,
+                mask_idx: torch.Tensor | None = None, w_masked: torch.Tensor | None = None,
+                bias: torch.Tensor | None = None, gelu: bool = False, *, out=None, workspace=None,
+                status=None, stream=None):
+    """y = fakequant(x) · deq(w)ᵀ + bias (BF16 out); protected columns in BF16."""
+    _dev(x, "x")
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    need = linear_w4a4_workspace(M, N, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    n_m = 0 if mask_idx is None else int(mask_idx.numel())
+    flags = LINEAR_GELU_TANH if gelu else 0
+    _check("hif4_linear_w4a4", lib().hif4_linear_w4a4(
+        _ptr(x), M, K, x.stride(0), _ptr(w_codes), _ptr(w_meta), N, _ptr(mask_idx) if n_m else None, n_m,
+        _ptr(w_masked) if n_m else None, _ptr(bias), _ptr(out), out.stride(0), flags, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+    return out
+
+
+def weight_decode(w_codes: torch.Tensor, w_meta: torch.Tensor, N: int, K: int,
+                  mask_idx: torch.Tensor | None = None, w_masked: torch.Tensor | None = None, *, out=None,
+                  status=None, stream=None):
+    """BF16 N x K decoded weight with the protected columns restored."""
+    _dev(w_codes, "w_codes")
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.bfloat16, device=w_codes.device)
+    n_m = 0 if mask_idx is None else int(mask_idx.numel())
+    _check("hif4_weight_decode", lib().hif4_weight_decode(
+        _ptr(w_codes), _ptr(w_meta), N, K, _ptr(mask_idx) if n_m else None, n_m, _ptr(w_masked) if n_m else None,
+        _ptr(out), out.stride(0), _ptr(status), _stream(stream)))
+    return out
+
+
+def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None, gelu: bool = False, *,
+              out=None, status=None, stream=None):
+    """y = a · bᵀ + bias on BF16 operands (tcgen05, FP32 accumulate, BF16 out)."""
+    _dev(a, "a")
+    assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16 and a.stride(1) == 1 and b.stride(1) == 1
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    _check("hif4_gemm_bf16", lib().hif4_gemm_bf16(
+        _ptr(a), M, K, a.stride(0), _ptr(b), N, b.stride(0), _ptr(bias), _ptr(out), out.stride(0),
+        LINEAR_GELU_TANH if gelu else 0, _ptr(status), _stream(stream)))
+    return out
+
+
+def calib_workspace(T: int, C: int) -> int:
+    return int(lib().hif4_calib_workspace(T, C))
+
+
+def calib_percentile_mask(acts: torch.Tensor, q=(999, 1000), frac=(1, 100), *, workspace=None, out=None,
+                          stream=None):
+    """-> (pct bf16 [C], ratio f32 [C], mask uint8 [C], mask_idx int32 [n_top])."""
+    _dev(acts, "acts")
+    assert acts.dtype == torch.bfloat16 and acts.dim() == 2 and acts.stride(1) == 1
+    T, C = acts.shape
+    n_top = (C * frac[0]) // frac[1]
+    dev = acts.device
+    if out is None:
+        out = (torch.empty(C, dtype=torch.bfloat16, device=dev), torch.empty(C, dtype=torch.float32, device=dev),
+               torch.empty(C, dtype=torch.uint8, device=dev), torch.empty(max(n_top, 1), dtype=torch.int32,
+                                                                            device=dev))
+    pct, ratio, mask, midx = out
+    need = calib_workspace(T, C)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check("hif4_calib_percentile_mask", lib().hif4_calib_percentile_mask(
+        _ptr(acts), T, C, acts.stride(0), q[0], q[1], frac[0], frac[1], _ptr(pct), _ptr(ratio), _ptr(mask),
+        _ptr(midx), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return pct, ratio, mask, midx[:n_top]
+
+
+def get_status(status: torch.Tensor, stream=None) -> int:
+    return int(lib().hif4_get_status(_ptr(status), _stream(stream)))
+
+
+def reset_status(status: torch.Tensor, stream=None) -> None:
+    _check("hif4_reset_status", lib().hif4_reset_status(_ptr(status), _stream(stream)))
+
+
+def version() -> int:
+    return int(lib().hif4_version())

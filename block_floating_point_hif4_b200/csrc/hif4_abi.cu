@@ -1,0 +1,95 @@
+// hif4_abi.cu — status handling and per-device caches of libhif4.
+#include <mutex>
+
+#include "hif4_internal.cuh"
+
+namespace hif4 {
+
+namespace {
+std::mutex g_mu;
+constexpr int kMaxDev = 64;
+int g_sms[kMaxDev] = {0};
+struct OccEntry {
+    const void *kernel;
+    int dev, threads;
+    size_t smem;
+    int blocks;
+};
+OccEntry g_occ[256];
+int g_nocc = 0;
+} // namespace
+
+int sm_count()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    int &v = g_sms[dev & (kMaxDev - 1)];
+    if (v == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        v = n;
+    }
+    return v;
+}
+
+int blocks_per_sm(const void *kernel, int threads, size_t dyn_smem)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (int i = 0; i < g_nocc; ++i)
+            if (g_occ[i].kernel == kernel && g_occ[i].dev == dev && g_occ[i].threads == threads &&
+                g_occ[i].smem == dyn_smem)
+                return g_occ[i].blocks;
+    }
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, dyn_smem) != cudaSuccess || b < 1)
+        b = 1;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_nocc < 256) g_occ[g_nocc++] = OccEntry{kernel, dev, threads, dyn_smem, b};
+    return b;
+}
+
+} // namespace hif4
+
+extern "C" hif4_status hif4_get_status(const uint32_t *status_word, hif4_stream_t stream)
+{
+    if (!status_word) return HIF4_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t w = 0;
+    if (cudaMemcpyAsync(&w, status_word, sizeof w, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return HIF4_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HIF4_ERR_CUDA;
+    if (w & HIF4_FLAG_TIMEOUT) return HIF4_ERR_TIMEOUT;
+    if (w & HIF4_FLAG_BAD_INDEX) return HIF4_ERR_INVALID_ARG;
+    if (w & HIF4_FLAG_NONFINITE) return HIF4_ERR_NONFINITE;
+    return HIF4_OK;
+}
+
+extern "C" hif4_status hif4_reset_status(uint32_t *status_word, hif4_stream_t stream)
+{
+    if (!status_word) return HIF4_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(status_word, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HIF4_ERR_CUDA;
+    return HIF4_OK;
+}
+
+extern "C" const char *hif4_status_string(hif4_status s)
+{
+    switch (s) {
+    case HIF4_OK: return "ok";
+    case HIF4_ERR_INVALID_ARG: return "invalid argument";
+    case HIF4_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case HIF4_ERR_SHAPE: return "shape error (cols/K must be a multiple of 64, ld >= cols)";
+    case HIF4_ERR_WORKSPACE: return "workspace missing or too small";
+    case HIF4_ERR_CUDA: return "CUDA runtime error";
+    case HIF4_ERR_NONFINITE: return "non-finite input mapped (NaN -> 0, Inf -> +-FLT_MAX)";
+    case HIF4_ERR_TIMEOUT: return "bounded device wait timed out";
+    case HIF4_ERR_UNSUPPORTED: return "unsupported device or size";
+    }
+    return "unknown status";
+}
+
+extern "C" int hif4_version(void) { return 100; }

@@ -1,0 +1,354 @@
+// hif4_calib.cu — tail-aware percentile calibration and channel mask.
+//
+// [Tail-Aware HiFloat4 summary on agents-report.net, "Why tail percentiles";
+// arXiv abstract: "activation-tail-aware percentile calibration module for
+// channel-mask construction".]  Rank rule and mask rule are the library's
+// readings: per channel, the |x| key at ascending rank
+// k = floor(q_num (T-1) / q_den); mask = top floor(C m_num / m_den) channels
+// by (percentile desc, channel asc); ratio = percentile / lower median over
+// channels.
+//
+// Exact order statistic by a two-pass radix select on the 15-bit BF16
+// magnitude key (bits & 0x7FFF, whose order is the |x| order):
+//   pass 1  per-channel histogram of key >> 7 (the exponent byte, 256 bins);
+//   pass 2  per-channel histogram of key & 127 restricted to the bin that
+//           holds rank k (128 bins);
+//   final   bin + low bits -> the key; one warp per channel;
+//   mask    one block: 32768-bin histogram of the C percentiles, block scans
+//           for the median and the top-n threshold, index-order scan for
+//           ties and for the sorted index list.
+// Histogram blocks own a 64-channel slab and a token range; a warp reads one
+// 128-byte row segment per load (lane = channel pair), so the slab's shared
+// histogram (bin-major, channel-minor) is updated without bank conflicts.
+#include <cuda_bf16.h>
+
+#include "hif4_internal.cuh"
+
+namespace hif4 {
+namespace {
+
+constexpr int kSlab = 64;          // channels per histogram block
+constexpr int kHistThreads = 256;  // 8 warps
+constexpr int kRowUnroll = 16;     // rows in flight per warp
+constexpr int kBins1 = 256;
+constexpr int kBins2 = 128;
+
+struct HistArgs {
+    const uint16_t *acts;
+    int64_t T;
+    int C;
+    int64_t lda;
+    int nslab;
+    int64_t rows_per_split;
+    uint32_t *hist1;   // [C][256]
+    uint32_t *hist2;   // [C][128]
+    uint32_t k;        // target ascending rank
+};
+
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Bin holding ascending rank k of a histogram of `nbins` counts, and the
+// number of elements in lower bins.  Called by a full warp.
+__device__ __forceinline__ void warp_select_bin(const uint32_t *h, int nbins, uint32_t k, uint32_t &bin,
+                                                uint32_t &below)
+{
+    const int lane = threadIdx.x & 31;
+    const int per = nbins / 32;
+    uint32_t c[8];
+    uint32_t sum = 0;
+    for (int i = 0; i < per; ++i) {
+        c[i] = h[lane * per + i];
+        sum += c[i];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const bool mine = excl <= k && k < incl;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, mine);
+    const int owner = ballot ? __ffs(ballot) - 1 : 31;
+    uint32_t b = 0, bl = 0;
+    if (lane == owner) {
+        uint32_t run = excl;
+        int i = 0;
+        for (; i < per - 1; ++i) {
+            if (k < run + c[i]) break;
+            run += c[i];
+        }
+        b = (uint32_t)(lane * per + i);
+        bl = run;
+    }
+    bin = __shfl_sync(0xffffffffu, b, owner);
+    below = __shfl_sync(0xffffffffu, bl, owner);
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kHistThreads) k_hist(HistArgs a)
+{
+    constexpr int NB = PASS == 1 ? kBins1 : kBins2;
+    extern __shared__ uint32_t h[];                    // [NB][kSlab]
+    __shared__ uint32_t target[kSlab];
+    const int slab = blockIdx.x % a.nslab;
+    const int split = blockIdx.x / a.nslab;
+    const int c0 = slab * kSlab;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i < NB * kSlab; i += kHistThreads) h[i] = 0;
+    if (PASS == 2) {
+        for (int j = warp; j < kSlab; j += kHistThreads / 32) {
+            uint32_t bin = 0xFFFFFFFFu, below = 0;
+            if (c0 + j < a.C) warp_select_bin(a.hist1 + (size_t)(c0 + j) * kBins1, kBins1, a.k, bin, below);
+            if (lane == 0) target[j] = bin;
+        }
+    }
+    __syncthreads();
+
+    const int ch0 = 2 * lane, ch1 = 2 * lane + 1;        // local channels of this lane
+    const bool v0 = c0 + ch0 < a.C, v1 = c0 + ch1 < a.C;
+    uint32_t tb0 = 0, tb1 = 0;
+    if (PASS == 2) {
+        tb0 = target[ch0];
+        tb1 = target[ch1];
+    }
+    // Conflict-free order: lanes 0-15 touch even channels first, 16-31 odd.
+    const bool swap = lane >= 16;
+    const int64_t t0 = (int64_t)split * a.rows_per_split;
+    int64_t t1 = t0 + a.rows_per_split;
+    if (t1 > a.T) t1 = a.T;
+    const uint16_t *col = a.acts + c0 + ch0;
+
+    for (int64_t t = t0 + warp; t < t1; t += (int64_t)(kHistThreads / 32) * kRowUnroll) {
+        uint32_t w[kRowUnroll];
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
+            w[u] = 0;
+            if (r < t1) {
+                const uint16_t *p = col + r * a.lda;
+                if (v1) w[u] = ldg_nc_u32(p);
+                else if (v0) w[u] = (uint32_t)*p;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) {
+            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
+            if (r >= t1) break;
+            const uint32_t k0 = w[u] & 0x7FFFu, k1 = (w[u] >> 16) & 0x7FFFu;
+            const uint32_t ka = swap ? k1 : k0, kb = swap ? k0 : k1;
+            const int ca = swap ? ch1 : ch0, cb = swap ? ch0 : ch1;
+            const bool va = swap ? v1 : v0, vb = swap ? v0 : v1;
+            if (PASS == 1) {
+                if (va) atomicAdd(&h[(ka >> 7) * kSlab + ca], 1u);
+                if (vb) atomicAdd(&h[(kb >> 7) * kSlab + cb], 1u);
+            } else {
+                const uint32_t ta = swap ? tb1 : tb0, tbb = swap ? tb0 : tb1;
+                if (va && (ka >> 7) == ta) atomicAdd(&h[(ka & 127u) * kSlab + ca], 1u);
+                if (vb && (kb >> 7) == tbb) atomicAdd(&h[(kb & 127u) * kSlab + cb], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    uint32_t *g = PASS == 1 ? a.hist1 : a.hist2;
+    for (int i = threadIdx.x; i < NB * kSlab; i += kHistThreads) {
+        const uint32_t v = h[i];
+        const int bin = i / kSlab, ch = i % kSlab;
+        if (v && c0 + ch < a.C) atomicAdd(&g[(size_t)(c0 + ch) * NB + bin], v);
+    }
+}
+
+// pct[c] = key at rank k: one warp per channel.
+__global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, uint32_t k, uint16_t *pct)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= C) return;
+    uint32_t b1, below1, b2, below2;
+    warp_select_bin(hist1 + (size_t)warp * kBins1, kBins1, k, b1, below1);
+    warp_select_bin(hist2 + (size_t)warp * kBins2, kBins2, k - below1, b2, below2);
+    if ((threadIdx.x & 31) == 0) pct[warp] = (uint16_t)((b1 << 7) | b2);
+}
+
+constexpr int kMaskThreads = 1024;
+constexpr int kKeys = 32768;
+
+// Block-wide exclusive scan of one value per thread (1024 threads).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratch, uint32_t &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    __syncthreads();
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = scratch[lane];
+        uint32_t si = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, si, o);
+            if (lane >= o) si += t;
+        }
+        scratch[32 + lane] = si - s;
+        if (lane == 31) scratch[64] = si;
+    }
+    __syncthreads();
+    total = scratch[64];
+    return scratch[32 + warp] + incl - v;
+}
+
+__global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int C, uint32_t n_top, float *ratio,
+                                                      uint8_t *mask, int32_t *mask_idx)
+{
+    extern __shared__ uint32_t hist[];                 // [kKeys]
+    __shared__ uint32_t scratch[72];
+    __shared__ uint32_t sel[4];                        // med key, tau key, count above tau
+    for (int i = threadIdx.x; i < kKeys; i += kMaskThreads) hist[i] = 0;
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += kMaskThreads) atomicAdd(&hist[pct[c] & 0x7FFFu], 1u);
+    __syncthreads();
+
+    // each thread owns 32 consecutive keys
+    constexpr int PER = kKeys / kMaskThreads;
+    uint32_t local = 0;
+    for (int i = 0; i < PER; ++i) local += hist[threadIdx.x * PER + i];
+    uint32_t total;
+    const uint32_t excl = block_excl_scan(local, scratch, total);
+    const uint32_t r_med = (uint32_t)(C - 1) / 2u;
+    const uint32_t r_tau = (uint32_t)C - n_top;        // ascending rank of the n_top-th largest
+    {
+        uint32_t run = excl;
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t cnt = hist[threadIdx.x * PER + i];
+            const uint32_t key = (uint32_t)(threadIdx.x * PER + i);
+            if (cnt && run <= r_med && r_med < run + cnt) sel[0] = key;
+            if (n_top && cnt && run <= r_tau && r_tau < run + cnt) {
+                sel[1] = key;
+                sel[2] = (uint32_t)C - (run + cnt);      // channels strictly above tau
+            }
+            run += cnt;
+        }
+    }
+    __syncthreads();
+    const uint32_t med_key = sel[0];
+    const uint32_t tau = n_top ? sel[1] : 0x10000u;
+    const uint32_t above = n_top ? sel[2] : 0u;
+    const uint32_t need_eq = n_top - above;            // ties at tau taken by lowest index
+    const float med = __uint_as_float(med_key << 16);
+
+    uint32_t eq_base = 0, m_base = 0;
+    for (int c0 = 0; c0 < C; c0 += kMaskThreads) {
+        const int c = c0 + threadIdx.x;
+        const bool in = c < C;
+        const uint32_t key = in ? (pct[c] & 0x7FFFu) : 0u;
+        const uint32_t eq = in && n_top && key == tau;
+        uint32_t tot_eq;
+        const uint32_t eq_rank = eq_base + block_excl_scan(eq, scratch, tot_eq);
+        const uint32_t m = in && n_top && (key > tau || (eq && eq_rank < need_eq));
+        uint32_t tot_m;
+        const uint32_t m_pos = m_base + block_excl_scan(m, scratch, tot_m);
+        if (in) {
+            mask[c] = (uint8_t)m;
+            float rt;
+            if (med_key == 0) rt = key ? __int_as_float(0x7F800000) : 0.0f;
+            else rt = __fdiv_rn(__uint_as_float(key << 16), med);
+            ratio[c] = rt;
+            if (m && mask_idx) mask_idx[m_pos] = c;
+        }
+        eq_base += tot_eq;
+        m_base += tot_m;
+    }
+}
+
+size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
+
+} // namespace
+} // namespace hif4
+
+using namespace hif4;
+
+extern "C" size_t hif4_calib_workspace(int64_t tokens, int64_t channels)
+{
+    (void)tokens;
+    if (channels <= 0) return 0;
+    return a256((size_t)channels * kBins1 * 4) + a256((size_t)channels * kBins2 * 4);
+}
+
+extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t channels,
+                                                  int64_t lda, uint32_t q_num, uint32_t q_den,
+                                                  uint32_t mask_num, uint32_t mask_den, void *pct,
+                                                  float *ratio, uint8_t *mask, int32_t *mask_idx_out,
+                                                  void *workspace, size_t ws_bytes, hif4_stream_t stream)
+{
+    if (tokens <= 0 || channels <= 0) return HIF4_ERR_INVALID_ARG;
+    if (!acts || !pct || !ratio || !mask) return HIF4_ERR_INVALID_ARG;
+    if (q_den == 0 || q_num > q_den || mask_den == 0 || mask_num > mask_den) return HIF4_ERR_INVALID_ARG;
+    if (lda < channels) return HIF4_ERR_SHAPE;
+    if (tokens > 0xFFFFFFFFll || channels > (1 << 24)) return HIF4_ERR_UNSUPPORTED;
+    if (!aligned16(acts) || (lda * 2) % 16 != 0) return HIF4_ERR_ALIGNMENT;
+    if (!aligned_to(pct, 2) || !aligned_to(ratio, 4) || (mask_idx_out && !aligned_to(mask_idx_out, 4)))
+        return HIF4_ERR_ALIGNMENT;
+    const size_t need = hif4_calib_workspace(tokens, channels);
+    if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
+    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *hist1 = static_cast<uint32_t *>(workspace);
+    uint32_t *hist2 = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                                   a256((size_t)channels * kBins1 * 4));
+    if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return HIF4_ERR_CUDA;
+
+    const uint64_t kk = ((uint64_t)q_num * (uint64_t)(tokens - 1)) / q_den;
+    HistArgs a{};
+    a.acts = static_cast<const uint16_t *>(acts);
+    a.T = tokens;
+    a.C = (int)channels;
+    a.lda = lda;
+    a.nslab = (int)((channels + kSlab - 1) / kSlab);
+    a.hist1 = hist1;
+    a.hist2 = hist2;
+    a.k = (uint32_t)kk;
+
+    const size_t smem1 = (size_t)kBins1 * kSlab * 4, smem2 = (size_t)kBins2 * kSlab * 4;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr[dev & 63]) {
+        if (cudaFuncSetAttribute(k_hist<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
+            cudaFuncSetAttribute(k_hist<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mask, cudaFuncAttributeMaxDynamicSharedMemorySize, kKeys * 4) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        attr[dev & 63] = true;
+    }
+    // Token splits: enough blocks for every SM to hold its resident maximum.
+    const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1>), kHistThreads, smem1);
+    const int64_t want = (int64_t)per_sm * sm_count();
+    int64_t splits = (want + a.nslab - 1) / a.nslab;
+    const int64_t min_rows = (int64_t)(kHistThreads / 32) * kRowUnroll;
+    if (splits * min_rows > tokens) splits = (tokens + min_rows - 1) / min_rows;
+    if (splits < 1) splits = 1;
+    a.rows_per_split = (tokens + splits - 1) / splits;
+    const int grid = (int)(a.nslab * splits);
+
+    k_hist<1><<<grid, kHistThreads, smem1, s>>>(a);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    k_hist<2><<<grid, kHistThreads, smem2, s>>>(a);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    k_finalize<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(hist1, hist2, (int)channels, a.k,
+                                                                   static_cast<uint16_t *>(pct));
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    const uint32_t n_top = (uint32_t)(((uint64_t)channels * mask_num) / mask_den);
+    k_mask<<<1, kMaskThreads, kKeys * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
+                                             mask_idx_out);
+    return launch_status();
+}

@@ -1,0 +1,499 @@
+// hif4_linear.cu — the W4A4 HiF4 fake-quantized linear layer on sm_100a.
+//
+//   y = xhat * what^T + bias        [Tail-Aware HiFloat4 arXiv abstract:
+//                                    W4A4 fake quantization of the main linears]
+// xhat: activations fake-quantized along K in 64-element units (protected
+//       channels kept in BF16), written once to the workspace;
+// what: HiF4 weights decoded to BF16 (protected columns restored from the
+//       caller's BF16 copy), written once to the workspace;
+// GEMM: persistent, warp-specialized tcgen05 kernel.  Every dequantized
+//       operand is exact in BF16 (at most 6 significant bits), so the BF16
+//       tensor-core product with FP32 accumulation is the fake-quant linear.
+//
+// GEMM structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: 128x64 A and 256x64 B BF16 tiles, 128-byte
+//               swizzle, 4-stage smem ring (48 KB per stage);
+//   warp 1      allocates 512 TMEM columns (two 128x256 FP32 accumulators)
+//               and issues tcgen05.mma (M=128, N=256, K=16) from one thread;
+//   warps 2-5   epilogue: tcgen05.ld of its 32-lane quarter, + bias,
+//               optional tanh-GELU, BF16 round-to-nearest-even, global store;
+//               it drains one accumulator while the next tile accumulates.
+// Every mbarrier wait is bounded; a wait that gives up sets the block's abort
+// flag, the others leave their loops, TMEM is freed and HIF4_FLAG_TIMEOUT is
+// raised in the status word.
+#include <cuda_bf16.h>
+
+#include "hif4_internal.cuh"
+#include "hif4_sm100.cuh"
+
+namespace hif4 {
+
+hif4_status fake_quantize_bf16(const void *x, int64_t rows, int64_t cols, int64_t ldx,
+                               const uint8_t *chan_mask, void *xhat, int64_t ldxh,
+                               uint32_t *status, cudaStream_t s);
+
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int THREADS = 192;
+constexpr int GROUP_M = 16;
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t TIMEOUT_NS = 4000000000ull;   // 4 s: far above any launch
+
+struct Args {
+    int M, N, K;
+    int num_m, num_n, num_k, num_tiles;
+    const uint16_t *bias;   // BF16 [N] or null
+    uint16_t *y;            // BF16 M x N, leading dimension ldy
+    int64_t ldy;
+    uint32_t flags;
+    uint32_t *status;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Args &g, int &mb, int &nb)
+{
+    const int per_group = GROUP_M * g.num_n;
+    const int gi = t / per_group;
+    const int first_m = gi * GROUP_M;
+    const int gm = min(g.num_m - first_m, GROUP_M);
+    const int r = t - gi * per_group;
+    mb = first_m + r % gm;
+    nb = r / gm;
+}
+
+__device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float gelu_tanh(float x)
+{
+    const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+    return 0.5f * x * (1.0f + tanh_approx(u));
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Args g)
+{
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * A_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars;
+    uint64_t *empty = bars + STAGES;
+    uint64_t *tfull = bars + 2 * STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_holder + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- producer
+            uint32_t stage = 0, phase = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
+                int mb, nb;
+                tile_coords(t, g, mb, nb);
+                for (int kb = 0; kb < g.num_k; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, g.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
+                    tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let our own copies land before the block leaves: wait (with
+                // a short limit, ignoring the abort flag) on the most recent
+                // phase of every stage we loaded.
+                for (uint32_t i = 0; i < STAGES && i < issued; ++i) {
+                    uint32_t s = (stage + STAGES - 1 - i) % STAGES;
+                    uint32_t ph = (s < stage) ? phase : (phase ^ 1u);
+                    mbar_wait_bounded(&full[s], ph, nullptr, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------- MMA issuer
+            const uint32_t idesc = idesc_bf16_f32(BM, BN);
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
+                if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, g.timeout_ns)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                for (int kb = 0; kb < g.num_k; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, g.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_addr(sA + stage * A_BYTES);
+                    const uint32_t b0 = smem_addr(sB + stage * B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16(d, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
+                                 (kb | k) != 0);
+                    mma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                acc ^= 1u;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // No MMA may still be running when TMEM is released.
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0, nullptr, 100000000ull);
+        }
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
+            int mb, nb;
+            tile_coords(t, g, mb, nb);
+            if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, g.timeout_ns)) break;
+            tc_fence_after();
+            const int row = mb * BM + q * 32 + lane;
+            uint16_t *yrow = g.y + (int64_t)row * g.ldy;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = nb * BN + c * 32;
+                if (n0 >= g.N) break;                          // warp-uniform
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
+                tmem_ld_wait();
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                if (g.bias) {
+                    if (n0 + 32 <= g.N) {
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(g.bias + n0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 b = __ldg(bp + i);
+                            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                v[8 * i + 2 * h] += __uint_as_float(bw[h] << 16);
+                                v[8 * i + 2 * h + 1] += __uint_as_float(bw[h] & 0xFFFF0000u);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < g.N) v[j] += __uint_as_float((uint32_t)g.bias[n0 + j] << 16);
+                    }
+                }
+                if (gelu) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+                }
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+                    packed[j] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                if (row < g.M) {
+                    if (n0 + 32 <= g.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (n0 + j < g.N) yrow[n0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            acc ^= 1u;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
+}
+
+// ----------------------------------------------------------- host helpers
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// BF16 rows x cols (K-major, leading dimension ld elements), boxes of
+// box_rows x 64 with 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld, int box_rows)
+{
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+} // namespace gemm
+
+namespace {
+
+// mask[k] = 1 for k in mask_idx, else 0; flags out-of-range or unsorted
+// indices in the status word (they are then ignored).
+__global__ void k_mask_prep(uint8_t *mask, int K, const int32_t *idx, int n, uint32_t *status)
+{
+    uint32_t bad = 0;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < K || i < n; i += gridDim.x * blockDim.x) {
+        if (i < n) {
+            const int v = idx[i];
+            if (v < 0 || v >= K || (i > 0 && idx[i - 1] >= v)) bad = 1;
+        }
+        if (i < K) {
+            int lo = 0, hi = n;                    // first index with idx >= i
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (idx[mid] < i) lo = mid + 1;
+                else hi = mid;
+            }
+            mask[i] = (lo < n && idx[lo] == i) ? 1 : 0;
+        }
+    }
+    if (bad) status_or(status, HIF4_FLAG_BAD_INDEX);
+}
+
+// what[n, idx[j]] = w_masked[n, j] (protected weight columns kept in BF16).
+__global__ void k_scatter_cols(uint16_t *what, int64_t K, const uint16_t *wm, const int32_t *idx, int n_m,
+                               int64_t N)
+{
+    const int64_t total = N * (int64_t)n_m;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = e / n_m;
+        const int j = (int)(e - n * n_m);
+        const int k = idx[j];
+        if (k >= 0 && k < K) what[n * K + k] = wm[e];
+    }
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+} // namespace
+} // namespace hif4
+
+using namespace hif4;
+
+namespace hif4 {
+namespace {
+
+hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N, int64_t ldb,
+                        const void *bias, void *y, int64_t ldy, uint32_t flags, uint32_t *status, cudaStream_t s)
+{
+    using namespace gemm;
+    CUtensorMap tmA, tmB;
+    if (!make_map(&tmA, a, M, K, lda, BM) || !make_map(&tmB, b, N, K, ldb, BN)) return HIF4_ERR_CUDA;
+    Args g{};
+    g.M = (int)M;
+    g.N = (int)N;
+    g.K = (int)K;
+    g.num_m = (int)((M + BM - 1) / BM);
+    g.num_n = (int)((N + BN - 1) / BN);
+    g.num_k = (int)(K / BK);
+    g.num_tiles = g.num_m * g.num_n;
+    g.bias = static_cast<const uint16_t *>(bias);
+    g.y = static_cast<uint16_t *>(y);
+    g.ldy = ldy;
+    g.flags = flags;
+    g.status = status;
+    g.timeout_ns = TIMEOUT_NS;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev & 63]) {
+        if (cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        attr_set[dev & 63] = true;
+    }
+    int grid = sm_count();
+    if (grid > g.num_tiles) grid = g.num_tiles;
+    k_gemm<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmB, g);
+    return launch_status();
+}
+
+hif4_status check_gemm_args(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N,
+                            int64_t ldb, const void *bias, const void *y, int64_t ldy, uint32_t flags)
+{
+    if (M < 0 || N < 0 || K < 0) return HIF4_ERR_INVALID_ARG;
+    if (K % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
+    if (M == 0 || N == 0) return HIF4_OK;
+    if (K == 0) return HIF4_ERR_SHAPE;
+    if (!a || !b || !y) return HIF4_ERR_INVALID_ARG;
+    if (flags & ~HIF4_LINEAR_GELU_TANH) return HIF4_ERR_INVALID_ARG;
+    if (lda < K || ldb < K || ldy < N) return HIF4_ERR_SHAPE;
+    if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return HIF4_ERR_UNSUPPORTED;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(y) || (lda * 2) % 16 || (ldb * 2) % 16 || (ldy * 2) % 16)
+        return HIF4_ERR_ALIGNMENT;
+    if (bias && !aligned16(bias)) return HIF4_ERR_ALIGNMENT;
+    return HIF4_OK;
+}
+
+} // namespace
+} // namespace hif4
+
+extern "C" hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N,
+                                      int64_t ldb, const void *bias, void *y, int64_t ldy, uint32_t flags,
+                                      uint32_t *status, hif4_stream_t stream)
+{
+    hif4_status st = check_gemm_args(a, M, K, lda, b, N, ldb, bias, y, ldy, flags);
+    if (st != HIF4_OK || M == 0 || N == 0) return st;
+    return launch_gemm(a, M, K, lda, b, N, ldb, bias, y, ldy, flags, status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" hif4_status hif4_weight_decode(const uint8_t *w_codes, const uint32_t *w_meta, int64_t N, int64_t K,
+                                          const int32_t *mask_idx, int32_t n_masked, const void *w_masked,
+                                          void *what, int64_t ldw, uint32_t *status, hif4_stream_t stream)
+{
+    (void)status;
+    if (N < 0 || K < 0 || n_masked < 0) return HIF4_ERR_INVALID_ARG;
+    if (K % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
+    if (N == 0 || K == 0) return HIF4_OK;
+    if (!w_codes || !w_meta || !what) return HIF4_ERR_INVALID_ARG;
+    if (n_masked > 0 && (!mask_idx || !w_masked)) return HIF4_ERR_INVALID_ARG;
+    if (n_masked > K) return HIF4_ERR_INVALID_ARG;
+    if (n_masked > 0 && (!aligned_to(mask_idx, 4) || !aligned_to(w_masked, 2))) return HIF4_ERR_ALIGNMENT;
+    hif4_status st = hif4_dequantize(w_codes, w_meta, N, K, HIF4_BF16, what, ldw, stream);
+    if (st != HIF4_OK || n_masked == 0) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t total = N * (int64_t)n_masked;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+    k_scatter_cols<<<blocks, 256, 0, s>>>(static_cast<uint16_t *>(what), ldw, static_cast<const uint16_t *>(w_masked),
+                                          mask_idx, n_masked, N);
+    return launch_status();
+}
+
+extern "C" size_t hif4_linear_w4a4_workspace(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return align256((size_t)M * K * 2) + align256((size_t)N * K * 2) + align256((size_t)K);
+}
+
+extern "C" hif4_status hif4_linear_w4a4(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                        const uint8_t *w_codes, const uint32_t *w_meta, int64_t N,
+                                        const int32_t *mask_idx, int32_t n_masked, const void *w_masked,
+                                        const void *bias, void *y, int64_t ldy, uint32_t flags,
+                                        void *workspace, size_t ws_bytes, uint32_t *status,
+                                        hif4_stream_t stream)
+{
+    if (n_masked < 0) return HIF4_ERR_INVALID_ARG;
+    hif4_status st = check_gemm_args(x, M, K, ldx, x, N, K, bias, y, ldy, flags);
+    if (st != HIF4_OK || M == 0 || N == 0) return st;
+    if (!w_codes || !w_meta) return HIF4_ERR_INVALID_ARG;
+    if (n_masked > 0 && (!mask_idx || !w_masked)) return HIF4_ERR_INVALID_ARG;
+    if (n_masked > K) return HIF4_ERR_INVALID_ARG;
+    if (!aligned_to(w_codes, 4) || !aligned_to(w_meta, 4)) return HIF4_ERR_ALIGNMENT;
+    if (n_masked > 0 && (!aligned_to(mask_idx, 4) || !aligned_to(w_masked, 2))) return HIF4_ERR_ALIGNMENT;
+    const size_t need = hif4_linear_w4a4_workspace(M, N, K);
+    if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
+    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *xhat = reinterpret_cast<uint16_t *>(ws);
+    uint16_t *what = reinterpret_cast<uint16_t *>(ws + align256((size_t)M * K * 2));
+    uint8_t *mask = ws + align256((size_t)M * K * 2) + align256((size_t)N * K * 2);
+
+    // 1. protected-channel mask (u8 per input channel) from the sorted indices
+    const uint8_t *chan_mask = nullptr;
+    if (n_masked > 0) {
+        const int64_t work = K > n_masked ? K : n_masked;
+        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask, (int)K, mask_idx, n_masked, status);
+        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+        chan_mask = mask;
+    }
+    // 2. activation fake quantization along K
+    st = fake_quantize_bf16(x, M, K, ldx, chan_mask, xhat, K, status, s);
+    if (st != HIF4_OK) return st;
+    // 3. weight decode to BF16, protected columns restored
+    st = hif4_weight_decode(w_codes, w_meta, N, K, mask_idx, n_masked, w_masked, what, K, status, stream);
+    if (st != HIF4_OK) return st;
+    // 4. tcgen05 GEMM + bias (+ GELU)
+    return launch_gemm(xhat, M, K, K, what, N, K, bias, y, ldy, flags, status, s);
+}

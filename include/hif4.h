@@ -1,0 +1,207 @@
+/*
+ * hif4.h — C ABI of libhif4: the data-parallel hot path of Tail-Aware
+ * HiFloat4 W4A4 post-training quantization on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [HiF4 format]  Huawei HiF4 calibration article (hwcomputing.csdn.net),
+ *                  section 1 "HiFloat4 (HiF4) format" (64-element unit, E6M2
+ *                  level-1 scale, 8 + 16 E1 micro-exponents, S1P2 elements).
+ *   [HiGPTQ]       same article, section 3.1 (units run along the input
+ *                  channels, i.e. along the reduction dimension K).
+ *   [TA abstract]  "Tail-Aware HiFloat4: W4A4 Post-Training Quantization for
+ *                  Wan2.2", arXiv 2605.26628 record, abstract (W4A4 fake
+ *                  quantization of the main linears, tail-aware percentile
+ *                  calibration for channel-mask construction).
+ *   [TA summary]   agents-report.net summary of that report, "Method
+ *                  overview" and "Why tail percentiles".
+ *
+ * Numerics (decode sign convention, encode rule, percentile rank and mask
+ * rule — the parts the pages leave open) are fixed in the repository's
+ * specification and restated in each call's comment below.
+ *
+ * Conventions for every call:
+ *   - Ownership: the caller allocates every buffer; the library allocates
+ *     nothing and keeps no state between calls except, per device, one
+ *     resolved driver entry point (tensor-map encoder) and cached occupancy.
+ *   - Pointers named x, y, codes, meta, acts, pct, ratio, mask, workspace,
+ *     status are DEVICE pointers unless stated otherwise.
+ *   - Execution: asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are checked on the host before any launch;
+ *     a failed check launches nothing and returns its error.  After each
+ *     launch the library checks cudaGetLastError and returns HIF4_ERR_CUDA.
+ *   - Layout: row-major; "ld" arguments are leading dimensions in ELEMENTS.
+ *     Units are 64 consecutive elements of a row, so cols (K) % 64 == 0.
+ *   - Alignment: x / y / acts base pointers and ld * element size must be
+ *     multiples of 16 bytes (HIF4_ERR_ALIGNMENT otherwise).
+ *   - Device-side errors are sticky bits in an optional caller-provided
+ *     device word `status` (HIF4_FLAG_*); read it with hif4_get_status.
+ */
+#ifndef HIF4_H
+#define HIF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *hif4_stream_t; /* == cudaStream_t */
+
+typedef enum {
+    HIF4_OK = 0,
+    HIF4_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad ratio */
+    HIF4_ERR_ALIGNMENT = 2,   /* pointer or leading dimension not 16-byte aligned */
+    HIF4_ERR_SHAPE = 3,       /* cols / K not a multiple of 64, ld < cols */
+    HIF4_ERR_WORKSPACE = 4,   /* workspace null or smaller than *_workspace() */
+    HIF4_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+    HIF4_ERR_NONFINITE = 6,   /* device flag: a NaN/Inf input was mapped */
+    HIF4_ERR_TIMEOUT = 7,     /* device flag: a bounded wait gave up */
+    HIF4_ERR_UNSUPPORTED = 8  /* no sm_100 device, or size beyond a limit */
+} hif4_status;
+
+typedef enum { HIF4_F32 = 0, HIF4_BF16 = 1 } hif4_dtype;
+
+/* Bits of the device status word. */
+#define HIF4_FLAG_NONFINITE 0x1u /* NaN -> 0, +-Inf -> +-FLT_MAX was applied */
+#define HIF4_FLAG_TIMEOUT 0x2u   /* a pipeline wait hit its iteration limit */
+#define HIF4_FLAG_BAD_INDEX 0x4u /* a mask index was out of range or unsorted */
+
+/* Flags of hif4_linear_w4a4. */
+#define HIF4_LINEAR_GELU_TANH 0x1u /* y = bf16(gelu_tanh(acc + bias)) */
+
+/*
+ * hif4_quantize — HiF4 "direct conversion" (round to nearest) of a
+ * rows x cols matrix along its rows [HiF4 format; HiGPTQ].
+ *
+ * For each 64-element unit (masked columns counted as 0):
+ *   c  = largest E6M2 code with 6.5 * v(c) < max|x|  (0 if none),
+ *        v(c) = 2^(E-31) (1 + f/4), c = E<<2 | f;
+ *   t_k = 0 / 1 / 2 as max|x| of 4-group k is <= 1.75 S / <= 3.5 S / more;
+ *   e2[j] = [max(t_2j, t_2j+1) == 2],  e3[k] = max(0, t_k - e2[k/2]);
+ *   m_i = RNE(|x_i| / (S 2^(e2+e3) / 4)), ties to even, min 7; sign dropped at 0.
+ *   NaN -> 0 and +-Inf -> +-FLT_MAX (sets HIF4_FLAG_NONFINITE).
+ *
+ * x         rows x cols, F32 or BF16, leading dimension ldx (elements).
+ * chan_mask NULL or `cols` bytes (device); nonzero = protected column: it is
+ *           excluded from the scale choice and gets code 0.
+ * codes     out, rows x cols/2 bytes, dense; element 2b in the low nibble of
+ *           byte b, code = sign << 3 | m.
+ * meta      out, rows x cols/64 uint32, dense; c | e2 << 8 | e3 << 16.
+ * status    NULL or a device word that receives HIF4_FLAG_* bits (OR-ed).
+ * Errors: INVALID_ARG (null x/codes/meta with rows > 0, rows < 0, dtype),
+ *         SHAPE (cols % 64, ldx < cols), ALIGNMENT (x, ldx; codes/meta 4 B).
+ */
+hif4_status hif4_quantize(const void *x, hif4_dtype dtype, int64_t rows, int64_t cols,
+                          int64_t ldx, const uint8_t *chan_mask, uint8_t *codes,
+                          uint32_t *meta, uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_dequantize — y = (-1)^s (m/4) 2^(e2+e3) v(c) [HiF4 format; the
+ * decode formula is an image on that page — this sign convention, an E1 bit
+ * of 1 doubling the value, is the library's reading].  Exact in BF16/F32.
+ * codes/meta as produced by hif4_quantize (dense); y rows x cols with ldy.
+ * Code 8 (sign with m = 0) decodes to -0.
+ */
+hif4_status hif4_dequantize(const uint8_t *codes, const uint32_t *meta, int64_t rows,
+                            int64_t cols, hif4_dtype out_dtype, void *y, int64_t ldy,
+                            hif4_stream_t stream);
+
+/*
+ * hif4_fake_quantize — activation fake quantization of the W4A4 linear
+ * [TA abstract]: xhat = deq(q(x with masked -> 0)) and xhat = x on masked
+ * columns.  x, xhat: BF16 rows x cols (ldx, ldxh).  chan_mask as in
+ * hif4_quantize.  Bit-identical to hif4_quantize followed by hif4_dequantize
+ * with the masked columns copied.
+ */
+hif4_status hif4_fake_quantize(const void *x, int64_t rows, int64_t cols, int64_t ldx,
+                               const uint8_t *chan_mask, void *xhat, int64_t ldxh,
+                               uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_linear_w4a4 — the fake-quantized W4A4 linear layer [TA abstract]:
+ *   y = xhat * what^T + bias   (FP32 accumulation, BF16 output),
+ * xhat = hif4_fake_quantize(x) with the columns in mask_idx kept in BF16;
+ * what = deq(w_codes, w_meta) with column mask_idx[j] replaced by
+ * w_masked[:, j].  The dequantized operands are exact in BF16, so the
+ * product runs on the tcgen05 BF16 tensor cores.
+ *
+ * x        BF16 M x K, ldx.            w_codes/w_meta  HiF4 N x K (dense),
+ *          quantized with hif4_quantize using the same protected columns.
+ * mask_idx NULL or n_masked sorted distinct column indices (device int32).
+ * w_masked NULL or BF16 N x n_masked, dense (row n = W[n, mask_idx[:]]).
+ * bias     NULL or BF16 [N].           y  BF16 M x N, ldy.
+ * flags    0 or HIF4_LINEAR_GELU_TANH (tanh-form GELU applied to acc + bias).
+ * workspace >= hif4_linear_w4a4_workspace(M, N, K) bytes, 256-byte aligned.
+ * Errors: SHAPE (K % 64, M/N/K <= 0), ALIGNMENT, WORKSPACE, INVALID_ARG.
+ * Bad mask indices are reported through status (HIF4_FLAG_BAD_INDEX).
+ */
+size_t hif4_linear_w4a4_workspace(int64_t M, int64_t N, int64_t K);
+hif4_status hif4_linear_w4a4(const void *x, int64_t M, int64_t K, int64_t ldx,
+                             const uint8_t *w_codes, const uint32_t *w_meta, int64_t N,
+                             const int32_t *mask_idx, int32_t n_masked, const void *w_masked,
+                             const void *bias, void *y, int64_t ldy, uint32_t flags,
+                             void *workspace, size_t ws_bytes, uint32_t *status,
+                             hif4_stream_t stream);
+
+/*
+ * hif4_weight_decode — the weight half of the fake-quantized linear:
+ * what = deq(w_codes, w_meta) as BF16 (N x K, leading dimension ldw) with
+ * column mask_idx[j] replaced by w_masked[:, j] (BF16 N x n_masked, dense).
+ * Stage 3 of hif4_linear_w4a4; callers with static weights may run it once.
+ * Errors as hif4_linear_w4a4.
+ */
+hif4_status hif4_weight_decode(const uint8_t *w_codes, const uint32_t *w_meta, int64_t N, int64_t K,
+                               const int32_t *mask_idx, int32_t n_masked, const void *w_masked,
+                               void *what, int64_t ldw, uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_gemm_bf16 — the product stage of hif4_linear_w4a4 on operands that are
+ * already BF16: y = a * b^T + bias (FP32 accumulation in tensor memory,
+ * BF16 round-to-nearest-even output), optional tanh-GELU (flags as for the
+ * linear).  a: M x K (lda), b: N x K (ldb), both K-major; K % 64 == 0.
+ * Persistent tcgen05 kernel, 128 x 256 output tiles, TMA-fed.
+ */
+hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N,
+                           int64_t ldb, const void *bias, void *y, int64_t ldy, uint32_t flags,
+                           uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_calib_percentile_mask — tail-aware percentile calibration and the
+ * channel mask [TA summary "Why tail percentiles"; TA abstract].
+ *   pct[c]   = the |x| value (as non-negative BF16) at 0-based ascending rank
+ *              k = floor(q_num (T-1) / q_den) among the T tokens of channel c,
+ *              keys compared as 15-bit BF16 magnitudes (+-0 equal);
+ *   med      = lower median over channels of pct (rank floor((C-1)/2));
+ *   ratio[c] = fp32(pct[c]) / fp32(med)  (+Inf / 0 when med == 0);
+ *   mask[c]  = 1 for the floor(C mask_num / mask_den) channels with the
+ *              largest pct, ties to the lower channel index.
+ * acts  BF16 T x C (lda).  pct BF16 [C], ratio F32 [C], mask u8 [C] (device).
+ * mask_idx_out  NULL or int32 [floor(C mask_num / mask_den)]: the masked
+ *               channels in ascending order (ready for hif4_linear_w4a4).
+ * workspace >= hif4_calib_workspace(T, C) bytes.
+ */
+size_t hif4_calib_workspace(int64_t tokens, int64_t channels);
+hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t channels,
+                                       int64_t lda, uint32_t q_num, uint32_t q_den,
+                                       uint32_t mask_num, uint32_t mask_den, void *pct,
+                                       float *ratio, uint8_t *mask, int32_t *mask_idx_out,
+                                       void *workspace, size_t ws_bytes,
+                                       hif4_stream_t stream);
+
+/* Synchronizes `stream`, reads the device status word and maps its bits:
+ * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX -> HIF4_ERR_INVALID_ARG,
+ * NONFINITE -> HIF4_ERR_NONFINITE, none -> HIF4_OK.  The word is not cleared. */
+hif4_status hif4_get_status(const uint32_t *status_word, hif4_stream_t stream);
+/* Clears the device status word (asynchronously, on `stream`). */
+hif4_status hif4_reset_status(uint32_t *status_word, hif4_stream_t stream);
+
+const char *hif4_status_string(hif4_status s);
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int hif4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HIF4_H */

@@ -1,0 +1,96 @@
+"""GPU parity: hif4_calib_percentile_mask against the CPU oracle, bit for bit
+(percentiles, ratios, mask, sorted mask indices).
+
+Method: Tail-Aware HiFloat4 summary (agents-report.net), "Why tail
+percentiles"; arXiv abstract (percentile calibration for channel masks).
+Rank and mask rules are the library's readings.
+"""
+import threading
+
+import numpy as np
+import pytest
+
+import oracle
+from block_floating_point_hif4_b200 import workloads as wl
+from tests._util import THREADS, to_dev_bf16, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def H():
+    import block_floating_point_hif4_b200 as h
+    from block_floating_point_hif4_b200 import build
+    build.build()
+    return h
+
+
+def run_gpu(H, acts_bits, q=(999, 1000), frac=(1, 100)):
+    pct, ratio, mask, midx = H.calib_percentile_mask(to_dev_bf16(acts_bits), q, frac)
+    return (to_host_bits(pct), ratio.cpu().numpy(), mask.cpu().numpy(), midx.cpu().numpy())
+
+
+def oracle_all(acts_bits, q=(999, 1000), frac=(1, 100)):
+    p = oracle.percentile(acts_bits, q[0], q[1], threads=THREADS)
+    r, m, n = oracle.channel_mask(p, frac[0], frac[1])
+    return p, r, m, np.nonzero(m)[0].astype(np.int32)
+
+
+def assert_same(g, o):
+    assert np.array_equal(g[0], o[0]), "percentile mismatch at %s" % np.argwhere(g[0] != o[0])[:5].ravel()
+    assert np.array_equal(g[1].view(np.uint32), o[1].view(np.uint32))
+    assert np.array_equal(g[2], o[2])
+    assert np.array_equal(g[3], o[3])
+
+
+@pytest.mark.parametrize("T,C", [(1, 1), (2, 3), (17, 64), (1000, 65), (3001, 130), (14400, 320)])
+def test_small_shapes(H, T, C):
+    acts, _ = wl.calib(T=T, C=C, seed=4 + T + C)
+    assert_same(run_gpu(H, acts), oracle_all(acts))
+
+
+def test_other_ratios_and_ties(H):
+    rng = np.random.default_rng(9)
+    acts = rng.integers(0, 6, (500, 200)).astype(np.uint16) * 0x80 + 0x3F00     # heavy ties
+    acts[rng.random(acts.shape) < 0.5] |= 0x8000                                # signs do not matter
+    for q, frac in [((1, 2), (1, 10)), ((0, 1), (3, 7)), ((1, 1), (0, 100)), ((999, 1000), (1, 1))]:
+        assert_same(run_gpu(H, acts, q, frac), oracle_all(acts, q, frac))
+
+
+def test_zero_median(H):
+    acts = np.zeros((50, 100), np.uint16)
+    acts[:, 97:] = 0x4000
+    assert_same(run_gpu(H, acts, (999, 1000), (2, 100)), oracle_all(acts, (999, 1000), (2, 100)))
+
+
+def test_medium_full_compare(H):
+    """One prompt's worth of tokens (14400) x 5120 channels, every channel."""
+    acts, _ = wl.calib(T=14400, C=5120, seed=4)
+    assert_same(run_gpu(H, acts), oracle_all(acts))
+
+
+@pytest.mark.slow
+def test_full_size_workload(H):
+    """16 prompts x 14400 tokens x 5120 channels (2.36 GB), the benchmark's
+    launch configuration: 256 sampled channels bit-exact against the oracle;
+    mask and ratios checked against the properties that define them."""
+    import torch
+    T, C = wl.CALIB_TOKENS, wl.WAN_DIM
+    acts, spikes = wl.calib(T=T, C=C, seed=4)
+    g = run_gpu(H, acts)
+    sample = np.sort(np.random.default_rng(44).choice(C, 256, replace=False))
+    sub = np.ascontiguousarray(acts[:, sample])
+    p_ref = oracle.percentile(sub, threads=THREADS)
+    assert np.array_equal(g[0][sample], p_ref)
+    pct = g[0].astype(np.int64)
+    n_top = C // 100
+    order = np.lexsort((np.arange(C), -pct))
+    want = np.zeros(C, np.uint8)
+    want[order[:n_top]] = 1
+    assert np.array_equal(g[2], want)
+    assert np.array_equal(g[3], np.nonzero(want)[0])
+    med = np.sort(pct)[(C - 1) // 2]
+    fp = wl.bf16_bits_to_f32(g[0].astype(np.uint16))
+    assert np.array_equal(g[1], fp / wl.bf16_bits_to_f32(np.array([med], np.uint16))[0])
+    del acts
+    torch.cuda.empty_cache()
