@@ -251,20 +251,16 @@ def main():
     M, D, F = args.tokens, D_MODEL, D_FFN
     stream = torch.cuda.current_stream()
 
+    from block_floating_point_hif4_b200 import sharding
+
     def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
+        sharding.barrier(dev)
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return sharding.max_over_ranks(v, dev)
 
     # ---- setup (untimed): inputs, calibration, weight quantization
-    x, _ = wl.device_rows(M, D, seed=3 + 1009 * rank, device=dev)
+    x, _ = wl.device_rows(M, D, seed=sharding.rank_seed(3, rank), device=dev)
     w1 = wl.device_weight(F, D, 0.015, seed=31, device=dev)
     w2 = wl.device_weight(D, F, 0.015, seed=32, device=dev)
     _, _, mask1, idx1 = H.calib_percentile_mask(x)
@@ -333,7 +329,7 @@ def main():
 
     flop_gemm = 2.0 * M * D * F                      # each of the two GEMMs
     flop_step = 2 * flop_gemm
-    value = world * flop_step / (ms_step * 1e-3) / 1e12
+    value = sharding.aggregate_throughput(flop_step, world, ms_step * 1e-3) / 1e12
     gemm_ms = max_over_ranks((stage_ms["gemm_1"] + stage_ms["gemm_2"]) / 2)
     achieved = flop_gemm / (gemm_ms * 1e-3) / 1e12
     peak = P["bf16_tflops_sustained"]

@@ -23,6 +23,7 @@ ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED = 5, 6, 7, 8
 F32, BF16 = 0, 1
 FLAG_NONFINITE, FLAG_TIMEOUT, FLAG_BAD_INDEX = 1, 2, 4
 LINEAR_GELU_TANH = 1
+LINEAR_OUT_F32 = 2
 
 # (name, restype, argtypes) of every exported entry point
 _P, _I64, _U32, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_size_t
@@ -155,7 +156,7 @@ def linear_w4a4(x: torch.Tensor, w_codes: torch.Tensor, w_meta: torch.Tensor, N:
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     n_m = 0 if mask_idx is None else int(mask_idx.numel())
-    flags = LINEAR_GELU_TANH if gelu else 0
+    flags = (LINEAR_GELU_TANH if gelu else 0) | (LINEAR_OUT_F32 if out.dtype == torch.float32 else 0)
     _check("hif4_linear_w4a4", lib().hif4_linear_w4a4(
         _ptr(x), M, K, x.stride(0), _ptr(w_codes), _ptr(w_meta), N, _ptr(mask_idx) if n_m else None, n_m,
         _ptr(w_masked) if n_m else None, _ptr(bias), _ptr(out), out.stride(0), flags, _ptr(workspace),
@@ -186,9 +187,10 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None
     N = b.shape[0]
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    flags = (LINEAR_GELU_TANH if gelu else 0) | (LINEAR_OUT_F32 if out.dtype == torch.float32 else 0)
     _check("hif4_gemm_bf16", lib().hif4_gemm_bf16(
         _ptr(a), M, K, a.stride(0), _ptr(b), N, b.stride(0), _ptr(bias), _ptr(out), out.stride(0),
-        LINEAR_GELU_TANH if gelu else 0, _ptr(status), _stream(stream)))
+        flags, _ptr(status), _stream(stream)))
     return out
 
 

@@ -90,7 +90,9 @@ __device__ __forceinline__ void warp_select_bin(const uint32_t *h, int nbins, ui
     below = __shfl_sync(0xffffffffu, bl, owner);
 }
 
-template <int PASS>
+// PAIR: 4-byte loads of a channel pair (needs a 4-byte aligned base and an
+// even leading dimension); otherwise two 2-byte loads.
+template <int PASS, bool PAIR>
 __global__ void __launch_bounds__(kHistThreads) k_hist(HistArgs a)
 {
     constexpr int NB = PASS == 1 ? kBins1 : kBins2;
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(kHistThreads) k_hist(HistArgs a)
             w[u] = 0;
             if (r < t1) {
                 const uint16_t *p = col + r * a.lda;
-                if (v1) w[u] = ldg_nc_u32(p);
-                else if (v0) w[u] = (uint32_t)*p;
+                if (PAIR && v1) w[u] = ldg_nc_u32(p);
+                else w[u] = (v0 ? (uint32_t)__ldg(p) : 0u) | (v1 ? (uint32_t)__ldg(p + 1) << 16 : 0u);
             }
         }
 #pragma unroll
@@ -295,7 +297,8 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     if (q_den == 0 || q_num > q_den || mask_den == 0 || mask_num > mask_den) return HIF4_ERR_INVALID_ARG;
     if (lda < channels) return HIF4_ERR_SHAPE;
     if (tokens > 0xFFFFFFFFll || channels > (1 << 24)) return HIF4_ERR_UNSUPPORTED;
-    if (!aligned16(acts) || (lda * 2) % 16 != 0) return HIF4_ERR_ALIGNMENT;
+    if (!aligned_to(acts, 2)) return HIF4_ERR_ALIGNMENT;
+    const bool pair = aligned_to(acts, 4) && (lda % 2 == 0);
     if (!aligned_to(pct, 2) || !aligned_to(ratio, 4) || (mask_idx_out && !aligned_to(mask_idx_out, 4)))
         return HIF4_ERR_ALIGNMENT;
     const size_t need = hif4_calib_workspace(tokens, channels);
@@ -324,14 +327,16 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr[dev & 63]) {
-        if (cudaFuncSetAttribute(k_hist<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
-            cudaFuncSetAttribute(k_hist<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
+        if (cudaFuncSetAttribute(k_hist<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
+            cudaFuncSetAttribute(k_hist<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
+            cudaFuncSetAttribute(k_hist<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
+            cudaFuncSetAttribute(k_hist<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
             cudaFuncSetAttribute(k_mask, cudaFuncAttributeMaxDynamicSharedMemorySize, kKeys * 4) != cudaSuccess)
             return HIF4_ERR_CUDA;
         attr[dev & 63] = true;
     }
     // Token splits: enough blocks for every SM to hold its resident maximum.
-    const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1>), kHistThreads, smem1);
+    const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1, true>), kHistThreads, smem1);
     const int64_t want = (int64_t)per_sm * sm_count();
     int64_t splits = (want + a.nslab - 1) / a.nslab;
     const int64_t min_rows = (int64_t)(kHistThreads / 32) * kRowUnroll;
@@ -340,9 +345,11 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.rows_per_split = (tokens + splits - 1) / splits;
     const int grid = (int)(a.nslab * splits);
 
-    k_hist<1><<<grid, kHistThreads, smem1, s>>>(a);
+    if (pair) k_hist<1, true><<<grid, kHistThreads, smem1, s>>>(a);
+    else k_hist<1, false><<<grid, kHistThreads, smem1, s>>>(a);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    k_hist<2><<<grid, kHistThreads, smem2, s>>>(a);
+    if (pair) k_hist<2, true><<<grid, kHistThreads, smem2, s>>>(a);
+    else k_hist<2, false><<<grid, kHistThreads, smem2, s>>>(a);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     k_finalize<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(hist1, hist2, (int)channels, a.k,
                                                                    static_cast<uint16_t *>(pct));

@@ -51,7 +51,7 @@ struct Args {
     int M, N, K;
     int num_m, num_n, num_k, num_tiles;
     const uint16_t *bias;   // BF16 [N] or null
-    uint16_t *y;            // BF16 M x N, leading dimension ldy
+    void *y;                // BF16 (or F32 with HIF4_LINEAR_OUT_F32) M x N, leading dimension ldy
     int64_t ldy;
     uint32_t flags;
     uint32_t *status;
@@ -203,6 +203,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         // -------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
+        const bool out_f32 = (g.flags & HIF4_LINEAR_OUT_F32) != 0;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
             int mb, nb;
@@ -210,7 +211,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, g.timeout_ns)) break;
             tc_fence_after();
             const int row = mb * BM + q * 32 + lane;
-            uint16_t *yrow = g.y + (int64_t)row * g.ldy;
+            uint16_t *yrow = static_cast<uint16_t *>(g.y) + (int64_t)row * g.ldy;
+            float *yrow32 = static_cast<float *>(g.y) + (int64_t)row * g.ldy;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 const int n0 = nb * BN + c * 32;
@@ -243,6 +245,21 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                 if (gelu) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+                }
+                if (out_f32) {
+                    if (row < g.M) {
+                        if (n0 + 32 <= g.N) {
+                            float4 *dst = reinterpret_cast<float4 *>(yrow32 + n0);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (n0 + j < g.N) yrow32[n0 + j] = v[j];
+                        }
+                    }
+                    continue;
                 }
                 uint32_t packed[16];
 #pragma unroll
@@ -378,7 +395,7 @@ hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const 
     g.num_k = (int)(K / BK);
     g.num_tiles = g.num_m * g.num_n;
     g.bias = static_cast<const uint16_t *>(bias);
-    g.y = static_cast<uint16_t *>(y);
+    g.y = y;
     g.ldy = ldy;
     g.flags = flags;
     g.status = status;
@@ -405,10 +422,11 @@ hif4_status check_gemm_args(const void *a, int64_t M, int64_t K, int64_t lda, co
     if (M == 0 || N == 0) return HIF4_OK;
     if (K == 0) return HIF4_ERR_SHAPE;
     if (!a || !b || !y) return HIF4_ERR_INVALID_ARG;
-    if (flags & ~HIF4_LINEAR_GELU_TANH) return HIF4_ERR_INVALID_ARG;
+    if (flags & ~(HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_OUT_F32)) return HIF4_ERR_INVALID_ARG;
     if (lda < K || ldb < K || ldy < N) return HIF4_ERR_SHAPE;
     if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return HIF4_ERR_UNSUPPORTED;
-    if (!aligned16(a) || !aligned16(b) || !aligned16(y) || (lda * 2) % 16 || (ldb * 2) % 16 || (ldy * 2) % 16)
+    const int64_t ysz = (flags & HIF4_LINEAR_OUT_F32) ? 4 : 2;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(y) || (lda * 2) % 16 || (ldb * 2) % 16 || (ldy * ysz) % 16)
         return HIF4_ERR_ALIGNMENT;
     if (bias && !aligned16(bias)) return HIF4_ERR_ALIGNMENT;
     return HIF4_OK;

@@ -67,8 +67,9 @@ typedef enum { HIF4_F32 = 0, HIF4_BF16 = 1 } hif4_dtype;
 #define HIF4_FLAG_TIMEOUT 0x2u   /* a pipeline wait hit its iteration limit */
 #define HIF4_FLAG_BAD_INDEX 0x4u /* a mask index was out of range or unsorted */
 
-/* Flags of hif4_linear_w4a4. */
-#define HIF4_LINEAR_GELU_TANH 0x1u /* y = bf16(gelu_tanh(acc + bias)) */
+/* Flags of hif4_linear_w4a4 / hif4_gemm_bf16. */
+#define HIF4_LINEAR_GELU_TANH 0x1u /* y = gelu_tanh(acc + bias) */
+#define HIF4_LINEAR_OUT_F32 0x2u   /* y is FP32 (the accumulator, unrounded) instead of BF16 */
 
 /*
  * hif4_quantize — HiF4 "direct conversion" (round to nearest) of a
@@ -130,8 +131,10 @@ hif4_status hif4_fake_quantize(const void *x, int64_t rows, int64_t cols, int64_
  *          quantized with hif4_quantize using the same protected columns.
  * mask_idx NULL or n_masked sorted distinct column indices (device int32).
  * w_masked NULL or BF16 N x n_masked, dense (row n = W[n, mask_idx[:]]).
- * bias     NULL or BF16 [N].           y  BF16 M x N, ldy.
- * flags    0 or HIF4_LINEAR_GELU_TANH (tanh-form GELU applied to acc + bias).
+ * bias     NULL or BF16 [N].           y  BF16 (FP32 with OUT_F32) M x N, ldy.
+ * flags    HIF4_LINEAR_GELU_TANH: tanh-form GELU applied to acc + bias;
+ *          HIF4_LINEAR_OUT_F32: store the FP32 result instead of its BF16
+ *          round-to-nearest-even (the BF16 output is exactly that rounding).
  * workspace >= hif4_linear_w4a4_workspace(M, N, K) bytes, 256-byte aligned.
  * Errors: SHAPE (K % 64, M/N/K <= 0), ALIGNMENT, WORKSPACE, INVALID_ARG.
  * Bad mask indices are reported through status (HIF4_FLAG_BAD_INDEX).
@@ -176,7 +179,8 @@ hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64_t lda, con
  *   ratio[c] = fp32(pct[c]) / fp32(med)  (+Inf / 0 when med == 0);
  *   mask[c]  = 1 for the floor(C mask_num / mask_den) channels with the
  *              largest pct, ties to the lower channel index.
- * acts  BF16 T x C (lda).  pct BF16 [C], ratio F32 [C], mask u8 [C] (device).
+ * acts  BF16 T x C (lda; 2-byte alignment suffices).  pct BF16 [C], ratio
+ *       F32 [C], mask u8 [C] (device).
  * mask_idx_out  NULL or int32 [floor(C mask_num / mask_den)]: the masked
  *               channels in ascending order (ready for hif4_linear_w4a4).
  * workspace >= hif4_calib_workspace(T, C) bytes.

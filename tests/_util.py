@@ -26,10 +26,11 @@ def meta_u32(t) -> np.ndarray:
     return t.cpu().numpy().view(np.uint32)
 
 
-def assert_linear_close(y_gpu_bits: np.ndarray, y_ref: np.ndarray, rel_fro=5e-3, row_rel=2e-2):
-    """Tolerance of the fake-quantized linear: relative Frobenius error <= 5e-3
-    and every element within 2e-2 x the RMS of its row (FP64 reference)."""
-    y = bf16_bits_to_f64(y_gpu_bits)
+def assert_linear_close(y_gpu: np.ndarray, y_ref: np.ndarray, rel_fro=5e-3, row_rel=2e-2):
+    """Tolerance of the fake-quantized linear on its FP32 result: relative
+    Frobenius error <= 5e-3 and every element within 2e-2 x the RMS of its
+    row (FP64 reference).  Accepts FP32/FP64 values or BF16 bit patterns."""
+    y = bf16_bits_to_f64(y_gpu) if y_gpu.dtype == np.uint16 else np.asarray(y_gpu, np.float64)
     assert y.shape == y_ref.shape
     assert np.all(np.isfinite(y))
     err = y - y_ref

@@ -1,9 +1,12 @@
 """GPU parity: hif4_linear_w4a4 (tcgen05 GEMM on the fake-quantized operands)
 against the FP64 oracle linear on the same seeded inputs.
 
-Tolerance (FP32 accumulation, BF16 output): relative Frobenius error <= 5e-3
-and |dY| <= 2e-2 x the row's RMS, every row for small shapes, a seeded
-1024-row sample (last row included) for the Wan2.2-shaped workloads.
+Tolerance, on the FP32 result (HIF4_LINEAR_OUT_F32): relative Frobenius
+error <= 5e-3 and |dY| <= 2e-2 x the row's RMS, every row for small shapes, a
+seeded 1024-row sample (last row included) for the Wan2.2-shaped workloads.
+The BF16 output is checked to be exactly the round-to-nearest-even of that
+FP32 result (BF16 rounding alone can reach 2e-2 x RMS on elements larger
+than ~10 x RMS, so the bound is not applied to the rounded output).
 Method: Tail-Aware HiFloat4 arXiv abstract (W4A4 HiF4 fake quantization of
 the main linears, protected channels kept in high precision).
 """
@@ -42,11 +45,16 @@ def run_case(H, x_bits, w_bits, mask_idx=None, bias_bits=None, gelu=False, rows=
     wmask = None if chan_mask is None else to_dev_bf16(np.ascontiguousarray(w_bits[:, mask_idx]))
     bias = None if bias_bits is None else to_dev_bf16(bias_bits)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    y = H.linear_w4a4(to_dev_bf16(x_bits), wc, wm, N, midx, wmask, bias, gelu=gelu, status=status)
+    xd = to_dev_bf16(x_bits)
+    y = H.linear_w4a4(xd, wc, wm, N, midx, wmask, bias, gelu=gelu, status=status)
+    y32 = H.linear_w4a4(xd, wc, wm, N, midx, wmask, bias, gelu=gelu, status=status,
+                        out=torch.empty(M, N, dtype=torch.float32, device="cuda"))
     torch.cuda.synchronize()
     assert H.get_status(status) == 0
+    # the BF16 output is exactly the round-to-nearest-even of the FP32 result
+    assert torch.equal(y, y32.to(torch.bfloat16))
     rows = np.arange(M) if rows is None else rows
-    y_rows = to_host_bits(y[torch.from_numpy(rows).cuda()])
+    y_rows = y32[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
     # oracle
     ref_c, ref_m, _ = oracle.quantize(w_bits, chan_mask)
     assert np.array_equal(ref_c, wc.cpu().numpy()) and np.array_equal(ref_m, meta_u32(wm))
@@ -73,10 +81,10 @@ def test_tiny_workload(H):
     wc, wm = H.quantize(torch.from_numpy(W).cuda())
     ref_wc, ref_wm, _ = oracle.quantize(W)
     assert np.array_equal(wc.cpu().numpy(), ref_wc) and np.array_equal(meta_u32(wm), ref_wm)
-    y = H.linear_w4a4(to_dev_bf16(xhat_bits), wc, wm, 512)
+    y = H.linear_w4a4(to_dev_bf16(xhat_bits), wc, wm, 512, out=torch.empty(128, 512, device="cuda"))
     what = oracle.dequantize(ref_wc, ref_wm, 512)
     y_ref = oracle.linear(ref_x, what, None, threads=THREADS)
-    assert_linear_close(to_host_bits(y), y_ref)
+    assert_linear_close(y.cpu().numpy().astype(np.float64), y_ref)
     del w_bits
 
 
