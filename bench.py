@@ -55,6 +55,7 @@ def parse():
     p.add_argument("--impl", choices=["hif4", "reference"], default="hif4")
     p.add_argument("--no-components", action="store_true", help="skip the quantizer / calibration lines")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-rows", type=int, default=8)
     p.add_argument("--tokens", type=int, default=TOKENS, help="tokens per GPU (default: Wan2.2 57600)")
     return p.parse_args()
@@ -412,7 +413,7 @@ def main():
         del acts
         line["components"] = comps
 
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
             flop, times, thr, _ = oracle_ffn_sample(args.cpu_sample_rows, steps=2)
             sec = min(times)

@@ -1,0 +1,74 @@
+"""Run one libhif4 operation a few times on seeded device inputs — the
+command to put under a profiler (ncu) or to time one kernel in isolation.
+
+    python -m block_floating_point_hif4_b200.profile OP [--log2n N] [--tokens T] [--reps R]
+
+OP: quantize | dequantize | fake_quantize | gemm | calib | linear.
+Sizes default to small cases that still exceed the 126 MB L2 (a few hundred
+MB on the device).  Prints the mean CUDA-event time per call.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "gemm", "calib", "linear"])
+    p.add_argument("--log2n", type=int, default=28, help="elements for quantize/dequantize/fake_quantize")
+    p.add_argument("--tokens", type=int, default=57600)
+    p.add_argument("--channels", type=int, default=5120)
+    p.add_argument("--n", type=int, default=5120, help="output features for gemm/linear")
+    p.add_argument("--reps", type=int, default=3)
+    a = p.parse_args(argv)
+
+    import torch
+
+    from . import binding as H
+    from . import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H.lib()
+    if a.op in ("quantize", "dequantize", "fake_quantize"):
+        n = 1 << a.log2n
+        x = wl.quant_sweep_torch(n, dev).view(-1, 1024)
+        codes, meta = H.quantize(x)
+        y = torch.empty_like(x)
+        fn = {"quantize": lambda: H.quantize(x, codes=codes, meta=meta),
+              "dequantize": lambda: H.dequantize(codes, meta, 1024, out=y),
+              "fake_quantize": lambda: H.fake_quantize(x, out=y)}[a.op]
+        nbytes = n * (4.0 if a.op == "fake_quantize" else 2.5625)
+    elif a.op == "calib":
+        x = wl.calib_torch(a.tokens, a.channels, dev)
+        ws = torch.empty(H.calib_workspace(a.tokens, a.channels), dtype=torch.uint8, device=dev)
+        fn = lambda: H.calib_percentile_mask(x, workspace=ws)  # noqa: E731
+        nbytes = 2.0 * a.tokens * a.channels
+    else:
+        x, _ = wl.device_rows(a.tokens, a.channels, seed=3, device=dev)
+        w = wl.device_weight(a.n, a.channels, 0.015, seed=31, device=dev)
+        y = torch.empty(a.tokens, a.n, dtype=torch.bfloat16, device=dev)
+        if a.op == "gemm":
+            fn = lambda: H.gemm_bf16(x, w, out=y)  # noqa: E731
+        else:
+            wc, wm = H.quantize(w)
+            ws = torch.empty(H.linear_w4a4_workspace(a.tokens, a.n, a.channels), dtype=torch.uint8, device=dev)
+            fn = lambda: H.linear_w4a4(x, wc, wm, a.n, out=y, workspace=ws)  # noqa: E731
+        nbytes = 2.0 * a.tokens * a.n * a.channels          # FLOPs for the GEMM-shaped ops
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.reps
+    unit = "TFLOP/s" if a.op in ("gemm", "linear") else "GB/s"
+    rate = nbytes / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print("%s: %.4f ms per call, %.1f %s" % (a.op, ms, rate, unit))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
