@@ -39,6 +39,9 @@ SIGNATURES = {
     "hif4_calib_workspace": (_SZ, [_I64, _I64]),
     "hif4_calib_percentile_mask": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P, _P,
                                                   _P, _P, _SZ, _P]),
+    "hif4_calib_noalloc_scratch_bytes": (_SZ, []),
+    "hif4_calib_percentile_mask_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P,
+                                                          _P, _P, _P]),
     "hif4_get_status": (ctypes.c_int, [_P, _P]),
     "hif4_reset_status": (ctypes.c_int, [_P, _P]),
     "hif4_status_string": (ctypes.c_char_p, [ctypes.c_int]),

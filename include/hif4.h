@@ -193,6 +193,37 @@ hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t
                                        void *workspace, size_t ws_bytes,
                                        hif4_stream_t stream);
 
+/*
+ * hif4_calib_percentile_mask_noalloc — the same computation as
+ * hif4_calib_percentile_mask, for callers that cannot allocate device memory
+ * (a runtime that gives all device memory to its own pool at start-up, a
+ * plugin host that forbids allocation inside its enqueue callback).  The
+ * source pages have no counterpart of this call; it exists only for such
+ * callers.
+ *
+ * Its scratch is one fixed array of hif4_calib_noalloc_scratch_bytes()
+ * bytes (16 MiB) in device memory, which every GPU that loads the library
+ * holds until the process exits.  The call allocates nothing: it forwards to
+ * hif4_calib_percentile_mask with that array as the workspace, which clears
+ * what must start at zero on every call.
+ *   - Sizes whose hif4_calib_workspace(tokens, channels) exceeds the array
+ *     are rejected with HIF4_ERR_WORKSPACE before any launch (with the
+ *     current histogram layout: channels <= 10922).
+ *   - The first call on a device looks up the array's device address once
+ *     (that device must be current); make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents: calls whose execution overlaps on the GPU (different streams
+ *     without ordering) race and give wrong results.  Order them.
+ * Arguments and outputs are those of hif4_calib_percentile_mask.
+ */
+size_t hif4_calib_noalloc_scratch_bytes(void);
+hif4_status hif4_calib_percentile_mask_noalloc(const void *acts, int64_t tokens, int64_t channels,
+                                               int64_t lda, uint32_t q_num, uint32_t q_den,
+                                               uint32_t mask_num, uint32_t mask_den, void *pct,
+                                               float *ratio, uint8_t *mask, int32_t *mask_idx_out,
+                                               hif4_stream_t stream);
+
 /* Synchronizes `stream`, reads the device status word and maps its bits:
  * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX -> HIF4_ERR_INVALID_ARG,
  * NONFINITE -> HIF4_ERR_NONFINITE, none -> HIF4_OK.  The word is not cleared. */
