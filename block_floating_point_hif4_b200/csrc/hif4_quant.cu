@@ -243,6 +243,318 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a)
     if (bad) status_or(a.status, HIF4_FLAG_NONFINITE);
 }
 
+// ------------------------------------------------- BF16 input, fast kernel
+//
+// One lane owns 16 consecutive elements of a unit (one 256-bit load; two
+// level-2 groups, four level-3 groups); 4 lanes share a unit, a warp covers 8
+// units (1 KB of BF16).
+//   * Maxima are taken on 16-bit magnitude keys (bits & 0x7FFF, whose order is
+//     the |x| order) with max.u16x2; a unit key >= 0x7F80 means a NaN/Inf.
+//   * The scale code comes from the bits of the unit maximum a: within a's
+//     binade the four thresholds 6.5 v(c) sit at mantissa offsets
+//     2^17 {1, 14, 27, 40}, so c = 4 (e - 99) + #{thresholds below the mantissa}.
+//   * 1.75 S and 3.5 S are exact BF16 values, so the group exponents are
+//     integer comparisons of keys.
+//   * |x| / step = |x| (H + L) with H + L a two-term expansion of
+//     16 / (4 + f) (times a power of two): for BF16 inputs the FP32 result of
+//     fma(|x|, H, |x| L) is exact at every rounding tie and at least 1/448 away
+//     from a tie otherwise, so round-to-nearest-even by the 1.5 * 2^23 magic
+//     addition is exact.  Products run as packed f32x2 operations.
+//   * Units with a non-finite input or a scale clamped at the top code (255)
+//     take the generic FP32 path (sanitize, exact half-way comparisons).
+
+typedef unsigned long long u64;
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ u64 pk(float lo, float hi)
+{
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk(u64 v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 fmul2(u64 a, u64 b)
+{
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 ffma2(u64 a, u64 b, u64 c)
+{
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ u64 fadd2(u64 a, u64 b)
+{
+    u64 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Scale code from the FP32 bits of the unit maximum (exact; see above).
+__device__ __forceinline__ uint32_t scale_code_from_bits(uint32_t bits)
+{
+    const int32_t ea = (int32_t)(bits >> 23);
+    const int32_t qm = ((int32_t)(bits & 0x7FFFFFu) - 1) >> 17;       // -1 .. 63
+    int32_t f = ((qm + 12) * 79) >> 10;                                 // floor((qm + 12) / 13)
+    f = f > 4 ? 4 : f;
+    int32_t c = ((ea - 99) << 2) + f;
+    c = c < 0 ? 0 : c;
+    return (uint32_t)(c > 255 ? 255 : c);
+}
+
+// 4 / (4 + f) as an unevaluated sum hi + lo of two FP32 values.
+__device__ __forceinline__ void recip_pair(uint32_t f, float &hi, float &lo)
+{
+    const uint32_t h = f == 0 ? 0x3F800000u : f == 1 ? 0x3F4CCCCDu : f == 2 ? 0x3F2AAAABu : 0x3F124925u;
+    const uint32_t l = f == 0 ? 0u : f == 1 ? 0xB24CCCCDu : f == 2 ? 0xB2AAAAABu : 0xB2DB6DB7u;
+    hi = bits_f(h);
+    lo = bits_f(l);
+}
+
+__device__ __forceinline__ void ld256(const void *p, uint32_t (&w)[8])
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void st256(void *p, const uint32_t (&w)[8])
+{
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
+// Generic FP32 path for one lane's 16 elements (all 4 lanes of the unit call
+// it together; `mask` = the lanes taking this path).
+template <int MODE>
+__device__ __forceinline__ void slow_lane16(const uint32_t (&w)[8], const uint32_t (&mw)[8], uint32_t q4,
+                                         uint32_t mask, uint32_t &bad, uint32_t (&out)[8], uint32_t &meta)
+{
+    float v[16];
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = sanitize(bf16_lo(w[i] & ~mw[i]), bad);
+        v[2 * i + 1] = sanitize(bf16_hi(w[i] & ~mw[i]), bad);
+    }
+    float a4[4];
+    for (int k = 0; k < 4; ++k) {
+        a4[k] = 0.0f;
+        for (int i = 0; i < 4; ++i) a4[k] = fmaxf(a4[k], fabsf(v[4 * k + i]));
+    }
+    float a = fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]));
+    a = fmaxf(a, __shfl_xor_sync(mask, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(mask, a, 2));
+    const uint32_t c = select_scale_code(a);
+    const float S = e6m2_value(c);
+    const float T1 = 1.75f * S, T2 = 3.5f * S;
+    const float rS = __frcp_rn(S);
+    uint32_t part = 0;
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t e2 = fmaxf(a4[2 * j], a4[2 * j + 1]) > T2;
+        part |= e2 << (8 + 2 * q4 + j);
+        for (int h = 0; h < 2; ++h) {
+            const int k = 2 * j + h;
+            const uint32_t e3 = e2 ? (a4[k] > T2) : (a4[k] > T1);
+            part |= e3 << (16 + 4 * q4 + k);
+            const int E = (int)(e2 + e3);
+            const float step = ldexp_small(S, E - 2), inv = ldexp_small(rS, 2 - E);
+            for (int i = 4 * k; i < 4 * k + 4; ++i) {
+                const uint32_t m = round_exact(fabsf(v[i]), inv, step);
+                const uint32_t sgn = (m != 0u) ? (f_bits(v[i]) >> 31) : 0u;
+                if (MODE == 0) {
+                    if ((i & 7) == 0) out[i >> 3] = 0;
+                    out[i >> 3] |= (m | (sgn << 3)) << (4 * (i & 7));
+                } else {
+                    v[i] = bits_f(f_bits((float)m * step) | (sgn << 31));
+                }
+            }
+        }
+    }
+    if (MODE == 0) {
+        part |= __shfl_xor_sync(mask, part, 1);
+        part |= __shfl_xor_sync(mask, part, 2);
+        meta = part | c;
+    } else {
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t y = pack_bf16_exact(v[2 * i], v[2 * i + 1]);
+            out[i] = (y & ~mw[i]) | (w[i] & mw[i]);
+        }
+    }
+}
+
+constexpr int kUnroll16 = 2;
+
+template <bool MASK, bool CONTIG, int MODE>
+__global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
+{
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t q4 = lane & 3u;
+    const uint32_t nocts = (a.total_units + 7u) >> 3;                 // 8 units per warp step
+    const uint32_t gwarp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
+    const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
+    const u64 NMAGIC2 = pk(-12582912.0f, -12582912.0f);
+    uint32_t bad = 0;
+
+    for (uint32_t o0 = gwarp; o0 < nocts; o0 += nwarps * kUnroll16) {
+        uint32_t raw[kUnroll16][8], mraw[kUnroll16][4], unit[kUnroll16], row[kUnroll16], cu[kUnroll16];
+#pragma unroll
+        for (int u = 0; u < kUnroll16; ++u) {
+            const uint32_t o = o0 + (uint32_t)u * nwarps;
+            unit[u] = o * 8u + (lane >> 2);
+            const bool active = o < nocts && unit[u] < a.total_units;
+            row[u] = (!CONTIG || MASK) ? a.upr_div.div(unit[u]) : 0u;
+            cu[u] = unit[u] - row[u] * a.upr;
+            const int64_t e = CONTIG ? (int64_t)unit[u] * HIF4_UNIT + q4 * 16
+                                     : (int64_t)row[u] * a.ldx + (int64_t)cu[u] * HIF4_UNIT + q4 * 16;
+            if (active) {
+                ld256(static_cast<const uint16_t *>(a.x) + e, raw[u]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) raw[u][i] = 0;
+            }
+            if (MASK) {
+                if (active) {
+                    const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu[u] * HIF4_UNIT + q4 * 16));
+                    mraw[u][0] = m4.x; mraw[u][1] = m4.y; mraw[u][2] = m4.z; mraw[u][3] = m4.w;
+                } else {
+                    mraw[u][0] = mraw[u][1] = mraw[u][2] = mraw[u][3] = 0;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll16; ++u) {
+            const uint32_t o = o0 + (uint32_t)u * nwarps;
+            if (o >= nocts) break;                                      // warp-uniform
+            const bool active = unit[u] < a.total_units;
+            const uint32_t (&w)[8] = raw[u];
+            // protected columns: 16-bit lane masks (all ones where the mask byte is nonzero)
+            uint32_t mw[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mw[i] = 0;
+            if (MASK) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t x = mraw[u][i];
+                    const uint32_t nz = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x);   // bit 7 set <=> byte != 0
+                    mw[2 * i] = __byte_perm(nz, 0, 0x9988);                        // bytes 0,0,1,1 (sign-replicated)
+                    mw[2 * i + 1] = __byte_perm(nz, 0, 0xBBAA);                    // bytes 2,2,3,3
+                }
+            }
+            uint32_t mk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
+            const uint32_t G0 = max_u16x2(mk[0], mk[1]), G1 = max_u16x2(mk[2], mk[3]);
+            const uint32_t G2 = max_u16x2(mk[4], mk[5]), G3 = max_u16x2(mk[6], mk[7]);
+            const uint32_t A01 = max_u16x2(__byte_perm(G0, G1, 0x5410), __byte_perm(G0, G1, 0x7632));
+            const uint32_t A23 = max_u16x2(__byte_perm(G2, G3, 0x5410), __byte_perm(G2, G3, 0x7632));
+            const uint32_t A8 = max_u16x2(__byte_perm(A01, A23, 0x5410), __byte_perm(A01, A23, 0x7632));
+            uint32_t ak = max(A8 & 0xFFFFu, A8 >> 16);
+            ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 1));
+            ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 2));
+            const uint32_t c = scale_code_from_bits(ak << 16);
+            uint32_t out[8];
+            uint32_t meta = 0;
+            const bool slow = ak >= 0x7F80u || c == 255u;                 // unit-uniform
+            if (slow) {
+                slow_lane16<MODE>(w, mw, q4, __activemask(), bad, out, meta);
+            } else {
+                const float S = e6m2_value(c);
+                const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
+                const uint32_t a8_0 = A8 & 0xFFFFu, a8_1 = A8 >> 16;
+                const uint32_t a4[4] = {A01 & 0xFFFFu, A01 >> 16, A23 & 0xFFFFu, A23 >> 16};
+                const uint32_t e2_0 = a8_0 > T2, e2_1 = a8_1 > T2;
+                const uint32_t th0 = e2_0 ? T2 : T1, th1 = e2_1 ? T2 : T1;
+                const uint32_t e3[4] = {a4[0] > th0, a4[1] > th0, a4[2] > th1, a4[3] > th1};
+                float ih, il;
+                recip_pair(c & 3u, ih, il);
+                const uint32_t E6 = c >> 2;
+                u64 HH[4], LL[4], ST[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t E = (k < 2 ? e2_0 : e2_1) + e3[k];
+                    const float pw = bits_f((160u - E6 - E) << 23);         // 2^(33 - E6 - E)
+                    HH[k] = pk(ih * pw, ih * pw);
+                    LL[k] = pk(il * pw, il * pw);
+                    if (MODE == 1) {
+                        const float st = ldexp_small(S, (int)E - 2);
+                        ST[k] = pk(st, st);
+                    }
+                }
+                if (MODE == 0) {
+                    uint32_t tb[16];
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const u64 ax = pk(bits_f(mk[p] << 16), bits_f(mk[p] & 0xFFFF0000u));
+                        const u64 r = ffma2(ax, HH[p >> 1], fmul2(ax, LL[p >> 1]));
+                        const u64 t = fadd2(r, MAGIC2);                    // low byte = RNE(r) <= 8
+                        float tl, th;
+                        upk(t, tl, th);
+                        tb[2 * p] = f_bits(tl);
+                        tb[2 * p + 1] = f_bits(th);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t *t8 = tb + 8 * h;
+                        const uint32_t *w4 = w + 4 * h;
+                        const uint32_t Ae = __byte_perm(__byte_perm(t8[0], t8[2], 0x0040), __byte_perm(t8[4], t8[6], 0x0040), 0x5410);
+                        const uint32_t Bo = __byte_perm(__byte_perm(t8[1], t8[3], 0x0040), __byte_perm(t8[5], t8[7], 0x0040), 0x5410);
+                        uint32_t C = Ae | (Bo << 4);
+                        C -= (C >> 3) & 0x11111111u;                        // m = 8 -> 7 (saturation)
+                        const uint32_t SE = __byte_perm(__byte_perm(w4[0], w4[1], 0x00D9), __byte_perm(w4[2], w4[3], 0x00D9), 0x5410);
+                        const uint32_t SO = __byte_perm(__byte_perm(w4[0], w4[1], 0x00FB), __byte_perm(w4[2], w4[3], 0x00FB), 0x5410);
+                        const uint32_t sg = ((SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u)) & 0x88888888u;
+                        const uint32_t nz = ((C | (C >> 1) | (C >> 2)) & 0x11111111u) << 3;
+                        out[h] = C | (sg & nz);
+                    }
+                    uint32_t part = (e2_0 << (8 + 2 * q4)) | (e2_1 << (9 + 2 * q4)) |
+                                    ((e3[0] | e3[1] << 1 | e3[2] << 2 | e3[3] << 3) << (16 + 4 * q4));
+                    part |= __shfl_xor_sync(0xffffffffu, part, 1);
+                    part |= __shfl_xor_sync(0xffffffffu, part, 2);
+                    meta = part | c;
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint32_t wz = w[p] & ~mw[p];
+                        const u64 x = pk(bits_f(wz << 16), bits_f(wz & 0xFFFF0000u));
+                        const u64 r = ffma2(x, HH[p >> 1], fmul2(x, LL[p >> 1]));
+                        const u64 mf = fadd2(fadd2(r, MAGIC2), NMAGIC2);   // signed RNE(r), +0 when 0
+                        float ml, mh;
+                        upk(mf, ml, mh);
+                        ml = fminf(fmaxf(ml, -7.0f), 7.0f);
+                        mh = fminf(fmaxf(mh, -7.0f), 7.0f);
+                        float yl, yh;
+                        upk(fmul2(pk(ml, mh), ST[p >> 1]), yl, yh);
+                        const uint32_t y = pack_bf16_exact(yl, yh);
+                        out[p] = MASK ? ((y & ~mw[p]) | (w[p] & mw[p])) : y;
+                    }
+                }
+            }
+            if (!active) continue;
+            if (MODE == 0) {
+                asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(a.codes + (size_t)unit[u] * 32 + q4 * 8),
+                             "r"(out[0]), "r"(out[1])
+                             : "memory");
+                if (q4 == 0) a.meta[unit[u]] = meta;
+            } else {
+                const int64_t e = CONTIG ? (int64_t)unit[u] * HIF4_UNIT + q4 * 16
+                                         : (int64_t)row[u] * a.ldo + (int64_t)cu[u] * HIF4_UNIT + q4 * 16;
+                st256(static_cast<uint16_t *>(a.out) + e, out);
+            }
+        }
+    }
+    if (bad) status_or(a.status, HIF4_FLAG_NONFINITE);
+}
+
 // ------------------------------------------------------------- dequantize
 
 struct DequantArgs {
@@ -332,9 +644,31 @@ int grid_for(K kernel, uint32_t total_units)
     return (int)(g < 1 ? 1 : g);
 }
 
-template <bool BF16, bool MASK, int MODE>
-hif4_status launch_quant(const QuantArgs &qa, bool contig, cudaStream_t s)
+template <typename K>
+int grid_for16(K kernel, uint32_t total_units)
 {
+    const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(kernel), kThreads, 0);
+    const uint64_t octs = (total_units + 7ull) / 8ull;
+    const uint64_t warps_needed = (octs + kUnroll16 - 1) / kUnroll16;
+    const uint64_t blocks_needed = (warps_needed + kThreads / 32 - 1) / (kThreads / 32);
+    uint64_t g = (uint64_t)per_sm * (uint64_t)sm_count();
+    if (blocks_needed < g) g = blocks_needed;
+    return (int)(g < 1 ? 1 : g);
+}
+
+template <bool BF16, bool MASK, int MODE>
+hif4_status launch_quant(const QuantArgs &qa, bool contig, bool fast, cudaStream_t s)
+{
+    if (BF16 && fast) {
+        if (contig) {
+            auto k = k_quant_bf16<MASK, true, MODE>;
+            k<<<grid_for16(k, qa.total_units), kThreads, 0, s>>>(qa);
+        } else {
+            auto k = k_quant_bf16<MASK, false, MODE>;
+            k<<<grid_for16(k, qa.total_units), kThreads, 0, s>>>(qa);
+        }
+        return launch_status();
+    }
     if (contig) {
         auto k = k_quant<BF16, MASK, true, MODE>;
         k<<<grid_for(k, qa.total_units), kThreads, 0, s>>>(qa);
@@ -373,8 +707,11 @@ hif4_status fake_quantize_bf16(const void *x, int64_t rows, int64_t cols, int64_
     qa.total_units = (uint32_t)(rows * (cols / HIF4_UNIT));
     qa.status = status;
     const bool contig = (ldx == cols) && (ldxh == cols);
-    return chan_mask ? launch_quant<true, true, 1>(qa, contig, s)
-                     : launch_quant<true, false, 1>(qa, contig, s);
+    // 256-bit accesses need 32-byte aligned rows; otherwise the 16-byte kernel
+    const bool fast = aligned_to(x, 32) && aligned_to(xhat, 32) && (ldx * 2) % 32 == 0 && (ldxh * 2) % 32 == 0 &&
+                      (!chan_mask || aligned_to(chan_mask, 16));
+    return chan_mask ? launch_quant<true, true, 1>(qa, contig, fast, s)
+                     : launch_quant<true, false, 1>(qa, contig, fast, s);
 }
 
 } // namespace hif4
@@ -407,9 +744,14 @@ extern "C" hif4_status hif4_quantize(const void *x, hif4_dtype dtype, int64_t ro
     qa.status = status;
     const bool contig = ldx == cols;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // 256-bit loads need 32-byte aligned rows; otherwise the 16-byte kernel
+    const bool fast = aligned_to(x, 32) && (ldx * 2) % 32 == 0 && aligned_to(codes, 8) &&
+                      (!chan_mask || aligned_to(chan_mask, 16));
     if (dtype == HIF4_BF16)
-        return chan_mask ? launch_quant<true, true, 0>(qa, contig, s) : launch_quant<true, false, 0>(qa, contig, s);
-    return chan_mask ? launch_quant<false, true, 0>(qa, contig, s) : launch_quant<false, false, 0>(qa, contig, s);
+        return chan_mask ? launch_quant<true, true, 0>(qa, contig, fast, s)
+                         : launch_quant<true, false, 0>(qa, contig, fast, s);
+    return chan_mask ? launch_quant<false, true, 0>(qa, contig, false, s)
+                     : launch_quant<false, false, 0>(qa, contig, false, s);
 }
 
 extern "C" hif4_status hif4_dequantize(const uint8_t *codes, const uint32_t *meta, int64_t rows,

@@ -82,6 +82,24 @@ def test_ragged_shapes(H, rows, cols):
     check_roundtrip(H, wl.f32_to_bf16_bits(x), "bf16")
 
 
+def test_unaligned_view_uses_16_byte_path(H):
+    """A row view starting 16 bytes past a 32-byte boundary (still 16-byte
+    aligned) must give the same result through the 16-byte kernel."""
+    torch = _torch()
+    rng = np.random.default_rng(15)
+    x = wl.f32_to_bf16_bits(rng.standard_normal((9, 192)).astype(np.float32))
+    big = torch.zeros(9, 192 + 8, dtype=torch.bfloat16, device="cuda")
+    big[:, 8:] = to_dev_bf16(x)
+    view = big[:, 8:]
+    assert view.data_ptr() % 32 == 16
+    c, m = H.quantize(view)
+    ref_c, ref_m, _ = oracle.quantize(x)
+    assert np.array_equal(c.cpu().numpy(), ref_c) and np.array_equal(meta_u32(m), ref_m)
+    y = H.fake_quantize(view)
+    ref = oracle.fake_quantize(x)
+    assert np.array_equal(to_host_bits(y), wl.f32_to_bf16_bits(ref.astype(np.float32)))
+
+
 def test_strided_rows_and_mask(H):
     rng = np.random.default_rng(5)
     x = rng.standard_normal((37, 256)).astype(np.float32)
