@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include "hif4_internal.cuh"
+#include "hif4_sm100.cuh"
 
 namespace hif4 {
 
@@ -271,6 +272,14 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
     asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
+// PTX prmt (byte permute); a selector nibble with bit 3 set replicates the
+// sign bit of the selected byte into the whole byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
 __device__ __forceinline__ u64 pk(float lo, float hi)
 {
     u64 r;
@@ -391,6 +400,115 @@ __device__ __forceinline__ void slow_lane16(const uint32_t (&w)[8], const uint32
     }
 }
 
+template <bool MASK, int MODE>
+__device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t (&mraw)[4], uint32_t q4,
+                                         uint32_t &bad, uint32_t (&out)[8], uint32_t &meta)
+{
+    const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
+    const u64 NMAGIC2 = pk(-12582912.0f, -12582912.0f);
+    // protected columns: 16-bit lane masks (all ones where the mask byte is nonzero)
+    uint32_t mw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mw[i] = 0;
+    if (MASK) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t x = mraw[i];
+            const uint32_t nz = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x);   // bit 7 set <=> byte != 0
+            mw[2 * i] = prmt(nz, 0, 0x9988);                        // bytes 0,0,1,1 (sign-replicated)
+            mw[2 * i + 1] = prmt(nz, 0, 0xBBAA);                    // bytes 2,2,3,3
+        }
+    }
+    uint32_t mk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
+    const uint32_t G0 = max_u16x2(mk[0], mk[1]), G1 = max_u16x2(mk[2], mk[3]);
+    const uint32_t G2 = max_u16x2(mk[4], mk[5]), G3 = max_u16x2(mk[6], mk[7]);
+    const uint32_t A01 = max_u16x2(prmt(G0, G1, 0x5410), prmt(G0, G1, 0x7632));
+    const uint32_t A23 = max_u16x2(prmt(G2, G3, 0x5410), prmt(G2, G3, 0x7632));
+    const uint32_t A8 = max_u16x2(prmt(A01, A23, 0x5410), prmt(A01, A23, 0x7632));
+    uint32_t ak = max(A8 & 0xFFFFu, A8 >> 16);
+    ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 1));
+    ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 2));
+    const uint32_t c = scale_code_from_bits(ak << 16);
+    meta = 0;
+    const bool slow = ak >= 0x7F80u || c == 255u;                 // unit-uniform
+    if (slow) {
+        slow_lane16<MODE>(w, mw, q4, __activemask(), bad, out, meta);
+    } else {
+        const float S = e6m2_value(c);
+        const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
+        const uint32_t a8_0 = A8 & 0xFFFFu, a8_1 = A8 >> 16;
+        const uint32_t a4[4] = {A01 & 0xFFFFu, A01 >> 16, A23 & 0xFFFFu, A23 >> 16};
+        const uint32_t e2_0 = a8_0 > T2, e2_1 = a8_1 > T2;
+        const uint32_t th0 = e2_0 ? T2 : T1, th1 = e2_1 ? T2 : T1;
+        const uint32_t e3[4] = {a4[0] > th0, a4[1] > th0, a4[2] > th1, a4[3] > th1};
+        float ih, il;
+        recip_pair(c & 3u, ih, il);
+        const uint32_t E6 = c >> 2;
+        u64 HH[4], LL[4], ST[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t E = (k < 2 ? e2_0 : e2_1) + e3[k];
+            const float pw = bits_f((160u - E6 - E) << 23);         // 2^(33 - E6 - E)
+            HH[k] = pk(ih * pw, ih * pw);
+            LL[k] = pk(il * pw, il * pw);
+            if (MODE == 1) {
+                const float st = ldexp_small(S, (int)E - 2);
+                ST[k] = pk(st, st);
+            }
+        }
+        if (MODE == 0) {
+            uint32_t tb[16];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const u64 ax = pk(bits_f(mk[p] << 16), bits_f(mk[p] & 0xFFFF0000u));
+                const u64 r = ffma2(ax, HH[p >> 1], fmul2(ax, LL[p >> 1]));
+                const u64 t = fadd2(r, MAGIC2);                    // low byte = RNE(r) <= 8
+                float tl, th;
+                upk(t, tl, th);
+                tb[2 * p] = f_bits(tl);
+                tb[2 * p + 1] = f_bits(th);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t *t8 = tb + 8 * h;
+                const uint32_t *w4 = w + 4 * h;
+                const uint32_t Ae = prmt(prmt(t8[0], t8[2], 0x0040), prmt(t8[4], t8[6], 0x0040), 0x5410);
+                const uint32_t Bo = prmt(prmt(t8[1], t8[3], 0x0040), prmt(t8[5], t8[7], 0x0040), 0x5410);
+                uint32_t C = Ae | (Bo << 4);
+                C -= (C >> 3) & 0x11111111u;                        // m = 8 -> 7 (saturation)
+                const uint32_t SE = prmt(prmt(w4[0], w4[1], 0x00D9), prmt(w4[2], w4[3], 0x00D9), 0x5410);
+                const uint32_t SO = prmt(prmt(w4[0], w4[1], 0x00FB), prmt(w4[2], w4[3], 0x00FB), 0x5410);
+                const uint32_t sg = ((SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u)) & 0x88888888u;
+                const uint32_t nz = ((C | (C >> 1) | (C >> 2)) & 0x11111111u) << 3;
+                out[h] = C | (sg & nz);
+            }
+            uint32_t part = (e2_0 << (8 + 2 * q4)) | (e2_1 << (9 + 2 * q4)) |
+                            ((e3[0] | e3[1] << 1 | e3[2] << 2 | e3[3] << 3) << (16 + 4 * q4));
+            part |= __shfl_xor_sync(0xffffffffu, part, 1);
+            part |= __shfl_xor_sync(0xffffffffu, part, 2);
+            meta = part | c;
+        } else {
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const uint32_t wz = w[p] & ~mw[p];
+                const u64 x = pk(bits_f(wz << 16), bits_f(wz & 0xFFFF0000u));
+                const u64 r = ffma2(x, HH[p >> 1], fmul2(x, LL[p >> 1]));
+                const u64 mf = fadd2(fadd2(r, MAGIC2), NMAGIC2);   // signed RNE(r), +0 when 0
+                float ml, mh;
+                upk(mf, ml, mh);
+                ml = fminf(fmaxf(ml, -7.0f), 7.0f);
+                mh = fminf(fmaxf(mh, -7.0f), 7.0f);
+                float yl, yh;
+                upk(fmul2(pk(ml, mh), ST[p >> 1]), yl, yh);
+                const uint32_t y = pack_bf16_exact(yl, yh);
+                out[p] = MASK ? ((y & ~mw[p]) | (w[p] & mw[p])) : y;
+            }
+        }
+    }
+}
+
 constexpr int kUnroll16 = 2;
 
 template <bool MASK, bool CONTIG, int MODE>
@@ -401,12 +519,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
     const uint32_t nocts = (a.total_units + 7u) >> 3;                 // 8 units per warp step
     const uint32_t gwarp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
-    const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
-    const u64 NMAGIC2 = pk(-12582912.0f, -12582912.0f);
     uint32_t bad = 0;
 
     for (uint32_t o0 = gwarp; o0 < nocts; o0 += nwarps * kUnroll16) {
-        uint32_t raw[kUnroll16][8], mraw[kUnroll16][4], unit[kUnroll16], row[kUnroll16], cu[kUnroll16];
+        uint32_t raw[kUnroll16][8], mraw[kUnroll16][4] = {}, unit[kUnroll16], row[kUnroll16], cu[kUnroll16];
 #pragma unroll
         for (int u = 0; u < kUnroll16; ++u) {
             const uint32_t o = o0 + (uint32_t)u * nwarps;
@@ -437,108 +553,8 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
             if (o >= nocts) break;                                      // warp-uniform
             const bool active = unit[u] < a.total_units;
             const uint32_t (&w)[8] = raw[u];
-            // protected columns: 16-bit lane masks (all ones where the mask byte is nonzero)
-            uint32_t mw[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mw[i] = 0;
-            if (MASK) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t x = mraw[u][i];
-                    const uint32_t nz = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x);   // bit 7 set <=> byte != 0
-                    mw[2 * i] = __byte_perm(nz, 0, 0x9988);                        // bytes 0,0,1,1 (sign-replicated)
-                    mw[2 * i + 1] = __byte_perm(nz, 0, 0xBBAA);                    // bytes 2,2,3,3
-                }
-            }
-            uint32_t mk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
-            const uint32_t G0 = max_u16x2(mk[0], mk[1]), G1 = max_u16x2(mk[2], mk[3]);
-            const uint32_t G2 = max_u16x2(mk[4], mk[5]), G3 = max_u16x2(mk[6], mk[7]);
-            const uint32_t A01 = max_u16x2(__byte_perm(G0, G1, 0x5410), __byte_perm(G0, G1, 0x7632));
-            const uint32_t A23 = max_u16x2(__byte_perm(G2, G3, 0x5410), __byte_perm(G2, G3, 0x7632));
-            const uint32_t A8 = max_u16x2(__byte_perm(A01, A23, 0x5410), __byte_perm(A01, A23, 0x7632));
-            uint32_t ak = max(A8 & 0xFFFFu, A8 >> 16);
-            ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 1));
-            ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 2));
-            const uint32_t c = scale_code_from_bits(ak << 16);
-            uint32_t out[8];
-            uint32_t meta = 0;
-            const bool slow = ak >= 0x7F80u || c == 255u;                 // unit-uniform
-            if (slow) {
-                slow_lane16<MODE>(w, mw, q4, __activemask(), bad, out, meta);
-            } else {
-                const float S = e6m2_value(c);
-                const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
-                const uint32_t a8_0 = A8 & 0xFFFFu, a8_1 = A8 >> 16;
-                const uint32_t a4[4] = {A01 & 0xFFFFu, A01 >> 16, A23 & 0xFFFFu, A23 >> 16};
-                const uint32_t e2_0 = a8_0 > T2, e2_1 = a8_1 > T2;
-                const uint32_t th0 = e2_0 ? T2 : T1, th1 = e2_1 ? T2 : T1;
-                const uint32_t e3[4] = {a4[0] > th0, a4[1] > th0, a4[2] > th1, a4[3] > th1};
-                float ih, il;
-                recip_pair(c & 3u, ih, il);
-                const uint32_t E6 = c >> 2;
-                u64 HH[4], LL[4], ST[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t E = (k < 2 ? e2_0 : e2_1) + e3[k];
-                    const float pw = bits_f((160u - E6 - E) << 23);         // 2^(33 - E6 - E)
-                    HH[k] = pk(ih * pw, ih * pw);
-                    LL[k] = pk(il * pw, il * pw);
-                    if (MODE == 1) {
-                        const float st = ldexp_small(S, (int)E - 2);
-                        ST[k] = pk(st, st);
-                    }
-                }
-                if (MODE == 0) {
-                    uint32_t tb[16];
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const u64 ax = pk(bits_f(mk[p] << 16), bits_f(mk[p] & 0xFFFF0000u));
-                        const u64 r = ffma2(ax, HH[p >> 1], fmul2(ax, LL[p >> 1]));
-                        const u64 t = fadd2(r, MAGIC2);                    // low byte = RNE(r) <= 8
-                        float tl, th;
-                        upk(t, tl, th);
-                        tb[2 * p] = f_bits(tl);
-                        tb[2 * p + 1] = f_bits(th);
-                    }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t *t8 = tb + 8 * h;
-                        const uint32_t *w4 = w + 4 * h;
-                        const uint32_t Ae = __byte_perm(__byte_perm(t8[0], t8[2], 0x0040), __byte_perm(t8[4], t8[6], 0x0040), 0x5410);
-                        const uint32_t Bo = __byte_perm(__byte_perm(t8[1], t8[3], 0x0040), __byte_perm(t8[5], t8[7], 0x0040), 0x5410);
-                        uint32_t C = Ae | (Bo << 4);
-                        C -= (C >> 3) & 0x11111111u;                        // m = 8 -> 7 (saturation)
-                        const uint32_t SE = __byte_perm(__byte_perm(w4[0], w4[1], 0x00D9), __byte_perm(w4[2], w4[3], 0x00D9), 0x5410);
-                        const uint32_t SO = __byte_perm(__byte_perm(w4[0], w4[1], 0x00FB), __byte_perm(w4[2], w4[3], 0x00FB), 0x5410);
-                        const uint32_t sg = ((SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u)) & 0x88888888u;
-                        const uint32_t nz = ((C | (C >> 1) | (C >> 2)) & 0x11111111u) << 3;
-                        out[h] = C | (sg & nz);
-                    }
-                    uint32_t part = (e2_0 << (8 + 2 * q4)) | (e2_1 << (9 + 2 * q4)) |
-                                    ((e3[0] | e3[1] << 1 | e3[2] << 2 | e3[3] << 3) << (16 + 4 * q4));
-                    part |= __shfl_xor_sync(0xffffffffu, part, 1);
-                    part |= __shfl_xor_sync(0xffffffffu, part, 2);
-                    meta = part | c;
-                } else {
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const uint32_t wz = w[p] & ~mw[p];
-                        const u64 x = pk(bits_f(wz << 16), bits_f(wz & 0xFFFF0000u));
-                        const u64 r = ffma2(x, HH[p >> 1], fmul2(x, LL[p >> 1]));
-                        const u64 mf = fadd2(fadd2(r, MAGIC2), NMAGIC2);   // signed RNE(r), +0 when 0
-                        float ml, mh;
-                        upk(mf, ml, mh);
-                        ml = fminf(fmaxf(ml, -7.0f), 7.0f);
-                        mh = fminf(fmaxf(mh, -7.0f), 7.0f);
-                        float yl, yh;
-                        upk(fmul2(pk(ml, mh), ST[p >> 1]), yl, yh);
-                        const uint32_t y = pack_bf16_exact(yl, yh);
-                        out[p] = MASK ? ((y & ~mw[p]) | (w[p] & mw[p])) : y;
-                    }
-                }
-            }
+            uint32_t out[8], meta;
+            encode16<MASK, MODE>(w, mraw[u], q4, bad, out, meta);
             if (!active) continue;
             if (MODE == 0) {
                 asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(a.codes + (size_t)unit[u] * 32 + q4 * 8),
@@ -553,6 +569,94 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
         }
     }
     if (bad) status_or(a.status, HIF4_FLAG_NONFINITE);
+}
+
+// ------------------------------------------- BF16 input, TMA-staged kernel
+//
+// Contiguous rows only.  A block streams chunks of 64 units (8 KB of BF16)
+// through a 6-stage shared-memory ring filled by cp.async.bulk copies that
+// complete on per-stage mbarriers, so each SM keeps ~100-150 KB of reads in
+// flight without holding them in registers.  Chunks are dealt to blocks
+// round-robin; thread t of the block encodes elements [16 (t % 4), +16) of
+// unit (chunk * 64 + t / 4) with encode16 above.
+
+constexpr int kStages = 6;
+constexpr int kChunkUnits = kThreads / 4;                 // 64 units
+constexpr uint32_t kChunkBytes = kChunkUnits * HIF4_UNIT * 2;   // 8 KB
+constexpr size_t kTmaSmem = (size_t)kStages * kChunkBytes + 128;
+constexpr uint64_t kWaitNs = 2000000000ull;               // 2 s: far above any chunk
+
+template <bool MASK, int MODE>
+__global__ void __launch_bounds__(kThreads, 3) k_quant_tma(QuantArgs a)
+{
+    using namespace sm100;
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + (size_t)kStages * kChunkBytes);
+    __shared__ uint32_t abort_flag;
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, q4 = lane & 3u;
+    const uint32_t nchunks = (a.total_units + kChunkUnits - 1) / kChunkUnits;
+    const uint32_t my_n = nchunks > blockIdx.x ? (nchunks - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
+    const uint16_t *x = static_cast<const uint16_t *>(a.x);
+
+    if (tid == 0) {
+        for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto issue = [&](uint32_t i) {
+        const uint32_t chunk = blockIdx.x + i * gridDim.x;
+        const uint32_t u0 = chunk * kChunkUnits;
+        const uint32_t nu = min((uint32_t)kChunkUnits, a.total_units - u0);
+        const uint32_t st = i % kStages;
+        mbar_arrive_expect_tx(&full[st], nu * HIF4_UNIT * 2);
+        bulk_load(sm + (size_t)st * kChunkBytes, x + (size_t)u0 * HIF4_UNIT, nu * HIF4_UNIT * 2, &full[st]);
+    };
+    if (tid == 0)
+        for (uint32_t i = 0; i < my_n && i < (uint32_t)kStages; ++i) issue(i);
+
+    uint32_t bad = 0, i = 0;
+    for (; i < my_n; ++i) {
+        const uint32_t st = i % kStages;
+        const bool ok = mbar_wait_bounded(&full[st], (i / kStages) & 1u, &abort_flag, kWaitNs);
+        const uint32_t unit = (blockIdx.x + i * gridDim.x) * kChunkUnits + (tid >> 2);
+        const bool active = unit < a.total_units;
+        uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (ok && active) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + (size_t)st * kChunkBytes + tid * 32u);
+            const uint4 lo = src[0], hi = src[1];
+            w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+            w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+        }
+        // stage st consumed by every thread; leave together if any wait gave up
+        if (__syncthreads_or(!ok)) break;
+        if (tid == 0 && i + kStages < my_n) issue(i + kStages);
+        uint32_t mraw[4] = {0, 0, 0, 0};
+        uint32_t cu = 0;
+        if (MASK && active) {
+            cu = unit - a.upr_div.div(unit) * a.upr;
+            const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + q4 * 16));
+            mraw[0] = m4.x; mraw[1] = m4.y; mraw[2] = m4.z; mraw[3] = m4.w;
+        }
+        uint32_t out[8], meta;
+        encode16<MASK, MODE>(w, mraw, q4, bad, out, meta);
+        if (!active) continue;
+        if (MODE == 0) {
+            asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(a.codes + (size_t)unit * 32 + q4 * 8), "r"(out[0]),
+                         "r"(out[1])
+                         : "memory");
+            if (q4 == 0) a.meta[unit] = meta;
+        } else {
+            st256(static_cast<uint16_t *>(a.out) + (size_t)unit * HIF4_UNIT + q4 * 16, out);
+        }
+    }
+    if (bad) status_or(a.status, HIF4_FLAG_NONFINITE);
+    if (tid == 0 && i < my_n) {
+        // gave up: let the copies this block still has in flight land first
+        for (uint32_t j = i; j < my_n && j < i + kStages; ++j)
+            mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1u, nullptr, 100000000ull);
+        status_or(a.status, HIF4_FLAG_TIMEOUT);
+    }
 }
 
 // ------------------------------------------------------------- dequantize
@@ -656,9 +760,29 @@ int grid_for16(K kernel, uint32_t total_units)
     return (int)(g < 1 ? 1 : g);
 }
 
+template <bool MASK, int MODE>
+hif4_status launch_quant_tma(const QuantArgs &qa, cudaStream_t s)
+{
+    auto k = k_quant_tma<MASK, MODE>;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr[dev & 63]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTmaSmem) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        attr[dev & 63] = true;
+    }
+    const uint32_t nchunks = (qa.total_units + kChunkUnits - 1) / kChunkUnits;
+    int grid = blocks_per_sm(reinterpret_cast<const void *>(k), kThreads, kTmaSmem) * sm_count();
+    if ((uint32_t)grid > nchunks) grid = (int)nchunks;
+    k<<<grid, kThreads, kTmaSmem, s>>>(qa);
+    return launch_status();
+}
+
 template <bool BF16, bool MASK, int MODE>
 hif4_status launch_quant(const QuantArgs &qa, bool contig, bool fast, cudaStream_t s)
 {
+    if (BF16 && fast && contig) return launch_quant_tma<MASK, MODE>(qa, s);
     if (BF16 && fast) {
         if (contig) {
             auto k = k_quant_bf16<MASK, true, MODE>;
