@@ -280,6 +280,14 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
 }
+// a * b + c on the integer multiply-add path (keeps byte/nibble packing off
+// the ALU pipe).
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
 __device__ __forceinline__ u64 pk(float lo, float hi)
 {
     u64 r;
@@ -462,7 +470,7 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
             uint32_t tb[16];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const u64 ax = pk(bits_f(mk[p] << 16), bits_f(mk[p] & 0xFFFF0000u));
+                const u64 ax = pk(bits_f(imad(mk[p], 65536u, 0u)), bits_f(mk[p] & 0xFFFF0000u));
                 const u64 r = ffma2(ax, HH[p >> 1], fmul2(ax, LL[p >> 1]));
                 const u64 t = fadd2(r, MAGIC2);                    // low byte = RNE(r) <= 8
                 float tl, th;
@@ -474,15 +482,16 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
             for (int h = 0; h < 2; ++h) {
                 const uint32_t *t8 = tb + 8 * h;
                 const uint32_t *w4 = w + 4 * h;
-                const uint32_t Ae = prmt(prmt(t8[0], t8[2], 0x0040), prmt(t8[4], t8[6], 0x0040), 0x5410);
-                const uint32_t Bo = prmt(prmt(t8[1], t8[3], 0x0040), prmt(t8[5], t8[7], 0x0040), 0x5410);
-                uint32_t C = Ae | (Bo << 4);
-                C -= (C >> 3) & 0x11111111u;                        // m = 8 -> 7 (saturation)
+                // nibble i = t_i - 0x4B400000 = m_i (0..8): a digit sum, no carries
+                uint32_t C = imad(t8[0], 1u, 0u - 0x4B400000u * 0x11111111u);
+#pragma unroll
+                for (int i = 1; i < 8; ++i) C = imad(t8[i], 1u << (4 * i), C);
+                const uint32_t nz = (C + 0x77777777u) & 0x88888888u;   // bit 3 of nibble <=> m >= 1
+                C -= (C >> 3) & 0x11111111u;                           // m = 8 -> 7 (saturation)
                 const uint32_t SE = prmt(prmt(w4[0], w4[1], 0x00D9), prmt(w4[2], w4[3], 0x00D9), 0x5410);
                 const uint32_t SO = prmt(prmt(w4[0], w4[1], 0x00FB), prmt(w4[2], w4[3], 0x00FB), 0x5410);
-                const uint32_t sg = ((SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u)) & 0x88888888u;
-                const uint32_t nz = ((C | (C >> 1) | (C >> 2)) & 0x11111111u) << 3;
-                out[h] = C | (sg & nz);
+                const uint32_t sg = (SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u);
+                out[h] = C | (sg & nz);                                // sign only where m != 0
             }
             uint32_t part = (e2_0 << (8 + 2 * q4)) | (e2_1 << (9 + 2 * q4)) |
                             ((e3[0] | e3[1] << 1 | e3[2] << 2 | e3[3] << 3) << (16 + 4 * q4));
