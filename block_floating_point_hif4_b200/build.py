@@ -21,11 +21,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
-BUILD = os.path.join(HERE, "_build")
-LIB = os.path.join(HERE, "libhif4.so")
+BUILD = os.environ.get("HIF4_BUILD_DIR", os.path.join(HERE, "_build"))
+LIB = os.environ.get("HIF4_LIB_OUT", os.path.join(HERE, "libhif4.so"))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "-I" + INCLUDE,
-         "--expt-relaxed-constexpr", "-Xptxas", "-v"]
+         "--expt-relaxed-constexpr", "-Xptxas", "-v"] + os.environ.get("HIF4_NVCC_EXTRA", "").split()
 
 
 def nvcc() -> str:

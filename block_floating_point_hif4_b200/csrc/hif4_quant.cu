@@ -483,9 +483,10 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
                 const uint32_t *t8 = tb + 8 * h;
                 const uint32_t *w4 = w + 4 * h;
                 // nibble i = t_i - 0x4B400000 = m_i (0..8): a digit sum, no carries
-                uint32_t C = imad(t8[0], 1u, 0u - 0x4B400000u * 0x11111111u);
-#pragma unroll
-                for (int i = 1; i < 8; ++i) C = imad(t8[i], 1u << (4 * i), C);
+                const uint32_t c01 = imad(t8[1], 16u, t8[0]), c23 = imad(t8[3], 16u, t8[2]);
+                const uint32_t c45 = imad(t8[5], 16u, t8[4]), c67 = imad(t8[7], 16u, t8[6]);
+                const uint32_t c03 = imad(c23, 256u, c01), c47 = imad(c67, 256u, c45);
+                uint32_t C = imad(c47, 65536u, c03 - 0x4B400000u * 0x11111111u);
                 const uint32_t nz = (C + 0x77777777u) & 0x88888888u;   // bit 3 of nibble <=> m >= 1
                 C -= (C >> 3) & 0x11111111u;                           // m = 8 -> 7 (saturation)
                 const uint32_t SE = prmt(prmt(w4[0], w4[1], 0x00D9), prmt(w4[2], w4[3], 0x00D9), 0x5410);
@@ -589,14 +590,20 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
 // round-robin; thread t of the block encodes elements [16 (t % 4), +16) of
 // unit (chunk * 64 + t / 4) with encode16 above.
 
-constexpr int kStages = 6;
+#ifndef HIF4_QT_STAGES
+#define HIF4_QT_STAGES 6
+#endif
+#ifndef HIF4_QT_MINB
+#define HIF4_QT_MINB 3
+#endif
+constexpr int kStages = HIF4_QT_STAGES;
 constexpr int kChunkUnits = kThreads / 4;                 // 64 units
 constexpr uint32_t kChunkBytes = kChunkUnits * HIF4_UNIT * 2;   // 8 KB
 constexpr size_t kTmaSmem = (size_t)kStages * kChunkBytes + 128;
 constexpr uint64_t kWaitNs = 2000000000ull;               // 2 s: far above any chunk
 
 template <bool MASK, int MODE>
-__global__ void __launch_bounds__(kThreads, 3) k_quant_tma(QuantArgs a)
+__global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs a)
 {
     using namespace sm100;
     extern __shared__ __align__(128) uint8_t sm[];
