@@ -8,6 +8,7 @@
 // so every rounding decision below is taken by exact FP32 comparison.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -33,6 +34,11 @@ int sm_count();
 // Resident blocks per SM for `kernel` at this block size (cached per kernel
 // and device).
 int blocks_per_sm(const void *kernel, int threads, size_t dyn_smem);
+// 2-D BF16 tensor map (inner x outer elements, rows row_stride_bytes apart)
+// with box_inner x box_outer boxes, optionally 128-byte swizzled; the driver's
+// encoder is resolved once through the runtime.  False if unavailable.
+bool make_tensor_map_bf16_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
 // Exact unsigned 32-bit division by a fixed divisor d >= 1 via a multiply:
 // q = (umulhi(n, m) + n) >> s with s = ceil(log2 d),

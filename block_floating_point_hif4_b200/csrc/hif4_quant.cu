@@ -675,6 +675,262 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
     }
 }
 
+// ------------------------------- BF16 quantize, 32 elements per lane, TMA 2-D
+//
+// Halves the per-unit work of encode16 per element: two lanes share a unit,
+// each encodes 32 elements (four level-2 groups).  A block stages chunks of
+// 128 units (16 KB) with 2-D TMA tile loads whose 128-byte swizzle makes the
+// per-lane 64-byte shared-memory reads bank-conflict free: 16-byte piece p of
+// unit row r sits at piece p ^ (r % 8).  The per-group scaling 4/(S 2^E) is
+// derived from the E = 0 value by subtracting E from the FP32 exponent field.
+
+#ifndef HIF4_Q32_STAGES
+#define HIF4_Q32_STAGES 4
+#endif
+#ifndef HIF4_Q32_MINB
+#define HIF4_Q32_MINB 2
+#endif
+constexpr int kQ32Stages = HIF4_Q32_STAGES;
+constexpr int kQ32Units = kThreads / 2;                       // 128 units per chunk
+constexpr uint32_t kQ32Bytes = kQ32Units * HIF4_UNIT * 2;     // 16 KB
+constexpr size_t kQ32Smem = (size_t)kQ32Stages * kQ32Bytes + 1024 + 128;
+
+// Generic FP32 path for a lane holding NW words (2 NW elements) of a unit
+// split over 64 / (2 NW) lanes; `part` = this lane's index within the unit.
+template <int NW>
+__device__ __forceinline__ void slow_codes(const uint32_t (&w)[NW], const uint32_t (&mw)[NW], uint32_t part_idx,
+                                           uint32_t mask, uint32_t &bad, uint32_t (&out)[NW / 4], uint32_t &meta)
+{
+    constexpr int NE = 2 * NW, NG = NE / 4;
+    float v[NE];
+    for (int i = 0; i < NW; ++i) {
+        v[2 * i] = sanitize(bf16_lo(w[i] & ~mw[i]), bad);
+        v[2 * i + 1] = sanitize(bf16_hi(w[i] & ~mw[i]), bad);
+    }
+    float a4[NG];
+    float a = 0.0f;
+    for (int k = 0; k < NG; ++k) {
+        a4[k] = 0.0f;
+        for (int i = 0; i < 4; ++i) a4[k] = fmaxf(a4[k], fabsf(v[4 * k + i]));
+        a = fmaxf(a, a4[k]);
+    }
+    for (int o = 1; o < 64 / NE; o <<= 1) a = fmaxf(a, __shfl_xor_sync(mask, a, o));
+    const uint32_t c = select_scale_code(a);
+    const float S = e6m2_value(c);
+    const float T1 = 1.75f * S, T2 = 3.5f * S;
+    const float rS = __frcp_rn(S);
+    uint32_t part = 0;
+    for (int i = 0; i < NW / 4; ++i) out[i] = 0;
+    for (int j = 0; j < NG / 2; ++j) {
+        const uint32_t e2 = fmaxf(a4[2 * j], a4[2 * j + 1]) > T2;
+        part |= e2 << (8 + (NG / 2) * part_idx + j);
+        for (int h = 0; h < 2; ++h) {
+            const int k = 2 * j + h;
+            const uint32_t e3 = e2 ? (a4[k] > T2) : (a4[k] > T1);
+            part |= e3 << (16 + NG * part_idx + k);
+            const int E = (int)(e2 + e3);
+            const float step = ldexp_small(S, E - 2), inv = ldexp_small(rS, 2 - E);
+            for (int i = 4 * k; i < 4 * k + 4; ++i) {
+                const uint32_t m = round_exact(fabsf(v[i]), inv, step);
+                const uint32_t sgn = (m != 0u) ? (f_bits(v[i]) >> 31) : 0u;
+                out[i >> 3] |= (m | (sgn << 3)) << (4 * (i & 7));
+            }
+        }
+    }
+    for (int o = 1; o < 64 / NE; o <<= 1) part |= __shfl_xor_sync(mask, part, o);
+    meta = part | c;
+}
+
+// Codes of 8 elements from their rounded values t (low bits m <= 8) and the
+// 4 BF16 words holding them (for the signs).
+__device__ __forceinline__ uint32_t pack8(const uint32_t *t8, const uint32_t *w4)
+{
+    const uint32_t c01 = imad(t8[1], 16u, t8[0]), c23 = imad(t8[3], 16u, t8[2]);
+    const uint32_t c45 = imad(t8[5], 16u, t8[4]), c67 = imad(t8[7], 16u, t8[6]);
+    const uint32_t c03 = imad(c23, 256u, c01), c47 = imad(c67, 256u, c45);
+    uint32_t C = imad(c47, 65536u, c03 - 0x4B400000u * 0x11111111u);    // nibble i = m_i
+    const uint32_t nz = (C + 0x77777777u) & 0x88888888u;                // bit 3 <=> m >= 1
+    C -= (C >> 3) & 0x11111111u;                                        // m = 8 -> 7
+    const uint32_t SE = prmt(prmt(w4[0], w4[1], 0x00D9), prmt(w4[2], w4[3], 0x00D9), 0x5410);
+    const uint32_t SO = prmt(prmt(w4[0], w4[1], 0x00FB), prmt(w4[2], w4[3], 0x00FB), 0x5410);
+    return C | (((SE & 0x0F0F0F0Fu) | (SO & 0xF0F0F0F0u)) & nz);
+}
+
+template <bool MASK>
+__device__ __forceinline__ void encode32(const uint32_t (&w)[16], const uint32_t (&mraw)[8], uint32_t p2,
+                                         uint32_t &bad, uint32_t (&out)[4], uint32_t &meta)
+{
+    const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
+    uint32_t mw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mw[i] = 0;
+    if (MASK) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t x = mraw[i];
+            const uint32_t nz = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x);
+            mw[2 * i] = prmt(nz, 0, 0x9988);
+            mw[2 * i + 1] = prmt(nz, 0, 0xBBAA);
+        }
+    }
+    uint32_t mk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
+    uint32_t A[4];                                           // [a4_2j, a4_2j+1]
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t G0 = max_u16x2(mk[4 * j], mk[4 * j + 1]), G1 = max_u16x2(mk[4 * j + 2], mk[4 * j + 3]);
+        A[j] = max_u16x2(prmt(G0, G1, 0x5410), prmt(G0, G1, 0x7632));
+    }
+    const uint32_t A8a = max_u16x2(prmt(A[0], A[1], 0x5410), prmt(A[0], A[1], 0x7632));   // [a8_0, a8_1]
+    const uint32_t A8b = max_u16x2(prmt(A[2], A[3], 0x5410), prmt(A[2], A[3], 0x7632));   // [a8_2, a8_3]
+    const uint32_t m2 = max_u16x2(A8a, A8b);
+    uint32_t ak = max(m2 & 0xFFFFu, m2 >> 16);
+    ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 1));
+    const uint32_t c = scale_code_from_bits(ak << 16);
+    if (ak >= 0x7F80u || c == 255u) {                        // unit-uniform
+        slow_codes<16>(w, mw, p2, __activemask(), bad, out, meta);
+        return;
+    }
+    const float S = e6m2_value(c);
+    const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
+    const uint32_t a8[4] = {A8a & 0xFFFFu, A8a >> 16, A8b & 0xFFFFu, A8b >> 16};
+    uint32_t e2[4], E[8], e2bits = 0, e3bits = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        e2[j] = a8[j] > T2;
+        const uint32_t th = e2[j] ? T2 : T1;
+        const uint32_t e3a = (A[j] & 0xFFFFu) > th, e3b = (A[j] >> 16) > th;
+        E[2 * j] = e2[j] + e3a;
+        E[2 * j + 1] = e2[j] + e3b;
+        e2bits |= e2[j] << j;
+        e3bits |= (e3a << (2 * j)) | (e3b << (2 * j + 1));
+    }
+    float ih, il;
+    recip_pair(c & 3u, ih, il);
+    if ((c & 3u) == 0) il = bits_f(0x21800000u);             // 2^-60: keeps the exponent arithmetic valid
+    const float pw0 = bits_f((160u - (c >> 2)) << 23);       // 2^(33 - E6)
+    const uint32_t H0 = f_bits(ih * pw0), L0 = f_bits(il * pw0);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        uint32_t tb[16];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int k = 4 * hh + (p >> 1);
+            const float H = bits_f(imad(E[k], 0xFF800000u, H0));   // exponent - E
+            const float L = bits_f(imad(E[k], 0xFF800000u, L0));
+            const uint32_t m = mk[8 * hh + p];
+            const u64 ax = pk(bits_f(imad(m, 65536u, 0u)), bits_f(m & 0xFFFF0000u));
+            const u64 r = ffma2(ax, pk(H, H), fmul2(ax, pk(L, L)));
+            float tl, th;
+            upk(fadd2(r, MAGIC2), tl, th);
+            tb[2 * p] = f_bits(tl);
+            tb[2 * p + 1] = f_bits(th);
+        }
+        out[2 * hh] = pack8(tb, w + 8 * hh);
+        out[2 * hh + 1] = pack8(tb + 8, w + 8 * hh + 4);
+    }
+    uint32_t part = (e2bits << (8 + 4 * p2)) | (e3bits << (16 + 8 * p2));
+    part |= __shfl_xor_sync(0xffffffffu, part, 1);
+    meta = part | c;
+}
+
+template <bool MASK>
+__global__ void __launch_bounds__(kThreads, HIF4_Q32_MINB) k_quant32(const __grid_constant__ CUtensorMap tm, QuantArgs a)
+{
+    using namespace sm100;
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + (size_t)kQ32Stages * kQ32Bytes);
+    __shared__ uint32_t abort_flag;
+    const uint32_t tid = threadIdx.x, p2 = tid & 1u, r = tid >> 1;
+    const uint32_t nchunks = (a.total_units + kQ32Units - 1) / kQ32Units;
+    const uint32_t my_n = nchunks > blockIdx.x ? (nchunks - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
+
+    if (tid == 0) {
+        for (int st = 0; st < kQ32Stages; ++st) mbar_init(&full[st], 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tm);
+    }
+    __syncthreads();
+    auto issue = [&](uint32_t i) {
+        const uint32_t st = i % kQ32Stages;
+        mbar_arrive_expect_tx(&full[st], kQ32Bytes);
+        tma_load_2d(sm + (size_t)st * kQ32Bytes, &tm, 0, (int32_t)((blockIdx.x + i * gridDim.x) * kQ32Units),
+                    &full[st]);
+    };
+    if (tid == 0)
+        for (uint32_t i = 0; i < my_n && i < (uint32_t)kQ32Stages; ++i) issue(i);
+
+    uint32_t bad = 0, i = 0;
+    for (; i < my_n; ++i) {
+        const uint32_t st = i % kQ32Stages;
+        const bool ok = mbar_wait_bounded(&full[st], (i / kQ32Stages) & 1u, &abort_flag, kWaitNs);
+        const uint32_t unit = (blockIdx.x + i * gridDim.x) * kQ32Units + r;
+        const bool active = unit < a.total_units;
+        uint32_t w[16];
+        if (ok) {
+            const uint8_t *row = sm + (size_t)st * kQ32Bytes + r * 128u;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + (((4u * p2 + kk) ^ (r & 7u)) << 4));
+                w[4 * kk] = v.x; w[4 * kk + 1] = v.y; w[4 * kk + 2] = v.z; w[4 * kk + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) w[k] = 0;
+        }
+        if (__syncthreads_or(!ok)) break;                    // stage consumed; leave together on a time-out
+        if (tid == 0 && i + kQ32Stages < my_n) issue(i + kQ32Stages);
+        uint32_t mraw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (MASK && active) {
+            const uint32_t cu = unit - a.upr_div.div(unit) * a.upr;
+            const uint4 *mp = reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + p2 * 32);
+            const uint4 m0 = __ldg(mp), m1 = __ldg(mp + 1);
+            mraw[0] = m0.x; mraw[1] = m0.y; mraw[2] = m0.z; mraw[3] = m0.w;
+            mraw[4] = m1.x; mraw[5] = m1.y; mraw[6] = m1.z; mraw[7] = m1.w;
+        }
+        uint32_t out[4], meta;
+        encode32<MASK>(w, mraw, p2, bad, out, meta);
+        if (!active) continue;
+        asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(a.codes + (size_t)unit * 32 + p2 * 16),
+                     "r"(out[0]), "r"(out[1]), "r"(out[2]), "r"(out[3])
+                     : "memory");
+        if (p2 == 0) a.meta[unit] = meta;
+    }
+    if (bad) status_or(a.status, HIF4_FLAG_NONFINITE);
+    if (tid == 0 && i < my_n) {
+        for (uint32_t j = i; j < my_n && j < i + kQ32Stages; ++j)
+            mbar_wait_bounded(&full[j % kQ32Stages], (j / kQ32Stages) & 1u, nullptr, 100000000ull);
+        status_or(a.status, HIF4_FLAG_TIMEOUT);
+    }
+}
+
+template <bool MASK>
+hif4_status launch_quant32(const QuantArgs &qa, cudaStream_t s, bool &done)
+{
+    done = false;
+    CUtensorMap tm;
+    if (!make_tensor_map_bf16_2d(&tm, qa.x, HIF4_UNIT, qa.total_units, HIF4_UNIT * 2, HIF4_UNIT, kQ32Units, true))
+        return HIF4_OK;                                      // no encoder: caller uses another kernel
+    auto k = k_quant32<MASK>;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr[dev & 63]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQ32Smem) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        attr[dev & 63] = true;
+    }
+    const uint32_t nchunks = (qa.total_units + kQ32Units - 1) / kQ32Units;
+    int grid = blocks_per_sm(reinterpret_cast<const void *>(k), kThreads, kQ32Smem) * sm_count();
+    if ((uint32_t)grid > nchunks) grid = (int)nchunks;
+    k<<<grid, kThreads, kQ32Smem, s>>>(tm, qa);
+    done = true;
+    return launch_status();
+}
+
 // ------------------------------------------------------------- dequantize
 
 struct DequantArgs {
@@ -798,6 +1054,11 @@ hif4_status launch_quant_tma(const QuantArgs &qa, cudaStream_t s)
 template <bool BF16, bool MASK, int MODE>
 hif4_status launch_quant(const QuantArgs &qa, bool contig, bool fast, cudaStream_t s)
 {
+    if (BF16 && MODE == 0 && fast && contig) {
+        bool done = false;
+        const hif4_status st = launch_quant32<MASK>(qa, s, done);
+        if (done || st != HIF4_OK) return st;
+    }
     if (BF16 && fast && contig) return launch_quant_tma<MASK, MODE>(qa, s);
     if (BF16 && fast) {
         if (contig) {
