@@ -685,10 +685,10 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
 // derived from the E = 0 value by subtracting E from the FP32 exponent field.
 
 #ifndef HIF4_Q32_STAGES
-#define HIF4_Q32_STAGES 4
+#define HIF4_Q32_STAGES 3
 #endif
 #ifndef HIF4_Q32_MINB
-#define HIF4_Q32_MINB 2
+#define HIF4_Q32_MINB 4
 #endif
 constexpr int kQ32Stages = HIF4_Q32_STAGES;
 constexpr int kQ32Units = kThreads / 2;                       // 128 units per chunk
