@@ -43,6 +43,7 @@ struct HistArgs {
     uint32_t *hist1;   // [C][256]
     uint32_t *hist2;   // [C][128]
     uint32_t k;        // target ascending rank
+    const uint32_t *needed;   // null, or per 64-channel slab: nonzero = process
 };
 
 __device__ __forceinline__ uint32_t ldg_nc_u32(const void *p)
@@ -55,7 +56,7 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void *p)
 // Bin holding ascending rank k of a histogram of `nbins` counts, and the
 // number of elements in lower bins.  Called by a full warp.
 __device__ __forceinline__ void warp_select_bin(const uint32_t *h, int nbins, uint32_t k, uint32_t &bin,
-                                                uint32_t &below)
+                                                uint32_t &below, uint32_t *total = nullptr)
 {
     const int lane = threadIdx.x & 31;
     const int per = nbins / 32;
@@ -88,6 +89,7 @@ __device__ __forceinline__ void warp_select_bin(const uint32_t *h, int nbins, ui
     }
     bin = __shfl_sync(0xffffffffu, b, owner);
     below = __shfl_sync(0xffffffffu, bl, owner);
+    if (total) *total = __shfl_sync(0xffffffffu, incl, 31);
 }
 
 // PAIR: 4-byte loads of a channel pair (needs a 4-byte aligned base and an
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(kHistThreads) k_hist(HistArgs a)
     const int split = blockIdx.x / a.nslab;
     const int c0 = slab * kSlab;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (a.needed && !a.needed[slab]) return;                 // block-uniform
 
     for (int i = threadIdx.x; i < NB * kSlab; i += kHistThreads) h[i] = 0;
     if (PASS == 2) {
@@ -167,14 +170,174 @@ __global__ void __launch_bounds__(kHistThreads) k_hist(HistArgs a)
 }
 
 // pct[c] = key at rank k: one warp per channel.
-__global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, uint32_t k, uint16_t *pct)
+__global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, uint32_t k, uint16_t *pct,
+                           const uint8_t *failed)
 {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (warp >= C) return;
+    if (failed && !failed[warp]) return;
     uint32_t b1, below1, b2, below2;
     warp_select_bin(hist1 + (size_t)warp * kBins1, kBins1, k, b1, below1);
     warp_select_bin(hist2 + (size_t)warp * kBins2, kBins2, k - below1, b2, below2);
     if ((threadIdx.x & 31) == 0) pct[warp] = (uint16_t)((b1 << 7) | b2);
+}
+
+// ------------------------------------------------------- windowed single pass
+//
+// A row sample (about 4096 rows) gives each channel a window of 256 keys — two
+// binades — starting at the binade that holds its sampled tail quantile at
+// ten times the target tail mass (the 99th percentile for q = 0.999).  One
+// pass over all tokens then counts the keys at or above the window start
+// (`ge`) and histograms the keys inside the window; the target rank k is in
+// the window iff T - ge <= k < T - ge + (window count), and then the window
+// histogram gives the exact key.  Channels where it is not fall back to the
+// exact two-pass radix select (launched always; blocks of slabs without a
+// failed channel exit at once), so the result never depends on the sample.
+//
+// Hot loop: a lane owns 4 channels (one 8-byte load per row); with the keys
+// packed in 16-bit halves, (x | 0x80008000) - (lo pair) sets bit 15 of a half
+// exactly when key >= lo (lo <= 0x8000, so no borrow crosses halves), so the
+// common case — every key below the window — costs four instructions per
+// 4-byte word.  The window histogram lives in shared memory as 16-bit counts
+// (a block covers at most 65535 rows).
+
+constexpr int kWinSlab = 128;       // channels per block
+constexpr int kWinBins = 256;
+constexpr int kWinUnroll = 16;
+
+struct WinArgs {
+    const uint16_t *acts;
+    int64_t T;
+    int C;
+    int64_t lda;
+    int nslab;
+    int64_t rows_per_split;
+    const uint32_t *hs;     // sample histogram [C][256] of key >> 7
+    uint32_t r_lo;          // sample rank whose binade starts the window
+    uint32_t *ge;           // [C] keys >= window start
+    uint32_t *whist;        // [C][256]
+    uint32_t *lo;           // [C] window start key
+};
+
+template <bool V8>
+__global__ void __launch_bounds__(kHistThreads) k_window(WinArgs a)
+{
+    extern __shared__ uint32_t h[];                    // [256 bins][64 words], u16 count per channel
+    __shared__ uint32_t lo_s[kWinSlab];
+    __shared__ uint32_t ge_s[kWinSlab];
+    const int slab = blockIdx.x % a.nslab;
+    const int split = blockIdx.x / a.nslab;
+    const int c0 = slab * kWinSlab;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i < kWinBins * kWinSlab / 2; i += kHistThreads) h[i] = 0;
+    for (int j = warp; j < kWinSlab; j += kHistThreads / 32) {
+        uint32_t lo = 0x8000u;                         // channel past C: never counted
+        if (c0 + j < a.C) {
+            uint32_t bin, below;
+            warp_select_bin(a.hs + (size_t)(c0 + j) * 256, 256, a.r_lo, bin, below);
+            lo = bin << 7;
+            if (split == 0 && lane == 0) a.lo[c0 + j] = lo;
+        }
+        if (lane == 0) {
+            lo_s[j] = lo;
+            ge_s[j] = 0;
+        }
+    }
+    __syncthreads();
+
+    const int ch = 4 * lane;
+    const uint32_t LO01 = lo_s[ch] | (lo_s[ch + 1] << 16), LO23 = lo_s[ch + 2] | (lo_s[ch + 3] << 16);
+    const bool all4 = c0 + ch + 3 < a.C;
+    uint32_t ge[4] = {0, 0, 0, 0};
+    const int64_t t0 = (int64_t)split * a.rows_per_split;
+    int64_t t1 = t0 + a.rows_per_split;
+    if (t1 > a.T) t1 = a.T;
+    const uint16_t *col = a.acts + c0 + ch;
+
+    for (int64_t t = t0 + warp; t < t1; t += (int64_t)(kHistThreads / 32) * kWinUnroll) {
+        uint32_t w01[kWinUnroll], w23[kWinUnroll];
+#pragma unroll
+        for (int u = 0; u < kWinUnroll; ++u) {
+            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
+            w01[u] = w23[u] = 0;
+            if (r < t1) {
+                const uint16_t *p = col + r * a.lda;
+                if (V8 && all4) {
+                    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                                 : "=r"(w01[u]), "=r"(w23[u]) : "l"(p));
+                } else {
+                    uint32_t e[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (c0 + ch + j < a.C) e[j] = __ldg(p + j);
+                    w01[u] = e[0] | (e[1] << 16);
+                    w23[u] = e[2] | (e[3] << 16);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kWinUnroll; ++u) {
+            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
+            if (r >= t1) break;
+            const uint32_t D01 = (w01[u] | 0x80008000u) - LO01;
+            const uint32_t D23 = (w23[u] | 0x80008000u) - LO23;
+            if ((D01 | D23) & 0x80008000u) {           // some key at or above its window start
+                const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (d[j] & 0x8000u) {
+                        ++ge[j];
+                        const uint32_t off = d[j] - 0x8000u;          // key - lo
+                        if (off < (uint32_t)kWinBins)
+                            atomicAdd(&h[off * (kWinSlab / 2) + 2 * lane + (j >> 1)], 1u << (16 * (j & 1)));
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        if (ge[j]) atomicAdd(&ge_s[ch + j], ge[j]);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kWinBins * kWinSlab / 2; i += kHistThreads) {
+        const uint32_t v = h[i];
+        if (!v) continue;
+        const int bin = i / (kWinSlab / 2), c = c0 + 2 * (i % (kWinSlab / 2));
+        if ((v & 0xFFFFu) && c < a.C) atomicAdd(&a.whist[(size_t)c * kWinBins + bin], v & 0xFFFFu);
+        if ((v >> 16) && c + 1 < a.C) atomicAdd(&a.whist[(size_t)(c + 1) * kWinBins + bin], v >> 16);
+    }
+    for (int j = threadIdx.x; j < kWinSlab; j += kHistThreads)
+        if (ge_s[j] && c0 + j < a.C) atomicAdd(&a.ge[c0 + j], ge_s[j]);
+}
+
+// Key at rank k from the window counts (one warp per channel); a channel
+// whose rank is outside its window is marked for the exact fallback, and its
+// window row is cleared for reuse as the fallback's first histogram.
+__global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint32_t *lo, int C, uint64_t T, uint32_t k,
+                               uint16_t *pct, uint8_t *failed, uint32_t *needed)
+{
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (c >= C) return;
+    uint32_t *row = whist + (size_t)c * kWinBins;
+    const uint64_t below = T - ge[c];
+    bool ok = false;
+    if ((uint64_t)k >= below) {
+        uint32_t bin, cum, total;
+        warp_select_bin(row, kWinBins, (uint32_t)((uint64_t)k - below), bin, cum, &total);
+        if ((uint64_t)k - below < total) {
+            ok = true;
+            if (lane == 0) pct[c] = (uint16_t)(lo[c] + bin);
+        }
+    }
+    if (!ok) {
+        for (int i = lane; i < kWinBins; i += 32) row[i] = 0;
+        if (lane == 0) {
+            failed[c] = 1;
+            atomicOr(&needed[c / kSlab], 1u);
+        }
+    }
 }
 
 constexpr int kMaskThreads = 1024;
@@ -274,6 +437,36 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
 
+struct CalibLayout {
+    size_t hs, whist, hist2, ge, lo, failed, needed, total;
+};
+
+CalibLayout calib_layout(int64_t C)
+{
+    CalibLayout L{};
+    const size_t nslab = (size_t)((C + kSlab - 1) / kSlab);
+    L.hs = 0;
+    L.whist = L.hs + a256((size_t)C * 256 * 4);
+    L.hist2 = L.whist + a256((size_t)C * 256 * 4);
+    L.ge = L.hist2 + a256((size_t)C * kBins2 * 4);
+    L.lo = L.ge + a256((size_t)C * 4);
+    L.failed = L.lo + a256((size_t)C * 4);
+    L.needed = L.failed + a256((size_t)C);
+    L.total = L.needed + a256(nslab * 4);
+    return L;
+}
+
+// Token splits so that every SM can hold its resident maximum of blocks.
+int64_t splits_for(int64_t rows, int64_t nslab, int per_sm, int64_t min_rows, int64_t max_rows)
+{
+    const int64_t want = (int64_t)per_sm * sm_count();
+    int64_t splits = (want + nslab - 1) / nslab;
+    if (splits * min_rows > rows) splits = (rows + min_rows - 1) / min_rows;
+    if (splits < 1) splits = 1;
+    while ((rows + splits - 1) / splits > max_rows) ++splits;
+    return splits;
+}
+
 } // namespace
 } // namespace hif4
 
@@ -283,7 +476,7 @@ extern "C" size_t hif4_calib_workspace(int64_t tokens, int64_t channels)
 {
     (void)tokens;
     if (channels <= 0) return 0;
-    return a256((size_t)channels * kBins1 * 4) + a256((size_t)channels * kBins2 * 4);
+    return calib_layout(channels).total;
 }
 
 extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t channels,
@@ -299,30 +492,27 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     if (tokens > 0xFFFFFFFFll || channels > (1 << 24)) return HIF4_ERR_UNSUPPORTED;
     if (!aligned_to(acts, 2)) return HIF4_ERR_ALIGNMENT;
     const bool pair = aligned_to(acts, 4) && (lda % 2 == 0);
+    const bool v8 = aligned_to(acts, 8) && (lda % 4 == 0);
     if (!aligned_to(pct, 2) || !aligned_to(ratio, 4) || (mask_idx_out && !aligned_to(mask_idx_out, 4)))
         return HIF4_ERR_ALIGNMENT;
-    const size_t need = hif4_calib_workspace(tokens, channels);
-    if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
+    const CalibLayout L = calib_layout(channels);
+    if (!workspace || ws_bytes < L.total) return HIF4_ERR_WORKSPACE;
     if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint32_t *hist1 = static_cast<uint32_t *>(workspace);
-    uint32_t *hist2 = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
-                                                   a256((size_t)channels * kBins1 * 4));
-    if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return HIF4_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *hs = reinterpret_cast<uint32_t *>(ws + L.hs);
+    uint32_t *whist = reinterpret_cast<uint32_t *>(ws + L.whist);
+    uint32_t *hist2 = reinterpret_cast<uint32_t *>(ws + L.hist2);
+    uint32_t *ge = reinterpret_cast<uint32_t *>(ws + L.ge);
+    uint32_t *lo = reinterpret_cast<uint32_t *>(ws + L.lo);
+    uint8_t *failed = ws + L.failed;
+    uint32_t *needed = reinterpret_cast<uint32_t *>(ws + L.needed);
+    if (cudaMemsetAsync(workspace, 0, L.total, s) != cudaSuccess) return HIF4_ERR_CUDA;
 
     const uint64_t kk = ((uint64_t)q_num * (uint64_t)(tokens - 1)) / q_den;
-    HistArgs a{};
-    a.acts = static_cast<const uint16_t *>(acts);
-    a.T = tokens;
-    a.C = (int)channels;
-    a.lda = lda;
-    a.nslab = (int)((channels + kSlab - 1) / kSlab);
-    a.hist1 = hist1;
-    a.hist2 = hist2;
-    a.k = (uint32_t)kk;
-
     const size_t smem1 = (size_t)kBins1 * kSlab * 4, smem2 = (size_t)kBins2 * kSlab * 4;
+    const size_t smemw = (size_t)kWinBins * kWinSlab / 2 * 4;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -331,29 +521,87 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
             cudaFuncSetAttribute(k_hist<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
             cudaFuncSetAttribute(k_hist<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) != cudaSuccess ||
             cudaFuncSetAttribute(k_hist<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess ||
+            cudaFuncSetAttribute(k_window<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemw) != cudaSuccess ||
+            cudaFuncSetAttribute(k_window<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smemw) != cudaSuccess ||
             cudaFuncSetAttribute(k_mask, cudaFuncAttributeMaxDynamicSharedMemorySize, kKeys * 4) != cudaSuccess)
             return HIF4_ERR_CUDA;
         attr[dev & 63] = true;
     }
-    // Token splits: enough blocks for every SM to hold its resident maximum.
-    const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1, true>), kHistThreads, smem1);
-    const int64_t want = (int64_t)per_sm * sm_count();
-    int64_t splits = (want + a.nslab - 1) / a.nslab;
+    const int nslab64 = (int)((channels + kSlab - 1) / kSlab);
+    const int per_sm1 = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1, true>), kHistThreads, smem1);
     const int64_t min_rows = (int64_t)(kHistThreads / 32) * kRowUnroll;
-    if (splits * min_rows > tokens) splits = (tokens + min_rows - 1) / min_rows;
-    if (splits < 1) splits = 1;
-    a.rows_per_split = (tokens + splits - 1) / splits;
-    const int grid = (int)(a.nslab * splits);
 
+    // 1. sample histogram: every R-th row (about 4096 rows)
+    const int64_t R = tokens / 4096 > 1 ? tokens / 4096 : 1;
+    const int64_t Ts = (tokens + R - 1) / R;
+    HistArgs sa{};
+    sa.acts = static_cast<const uint16_t *>(acts);
+    sa.T = Ts;
+    sa.C = (int)channels;
+    sa.lda = lda * R;
+    sa.nslab = nslab64;
+    sa.hist1 = hs;
+    sa.hist2 = hist2;
+    sa.k = 0;
+    sa.needed = nullptr;
+    int64_t sp = splits_for(Ts, nslab64, per_sm1, min_rows, INT64_MAX);
+    sa.rows_per_split = (Ts + sp - 1) / sp;
+    if (pair) k_hist<1, true><<<(int)(nslab64 * sp), kHistThreads, smem1, s>>>(sa);
+    else k_hist<1, false><<<(int)(nslab64 * sp), kHistThreads, smem1, s>>>(sa);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+
+    // 2. windowed pass over every token
+    WinArgs wa{};
+    wa.acts = static_cast<const uint16_t *>(acts);
+    wa.T = tokens;
+    wa.C = (int)channels;
+    wa.lda = lda;
+    wa.nslab = (int)((channels + kWinSlab - 1) / kWinSlab);
+    wa.hs = hs;
+    {
+        // ascending sample rank: ten times the target's tail mass below the top
+        const uint64_t tail = ((uint64_t)(tokens - kk) * 10ull * (uint64_t)Ts + (uint64_t)tokens - 1) / (uint64_t)tokens;
+        wa.r_lo = (uint32_t)((uint64_t)Ts > tail + 1 ? (uint64_t)Ts - 1 - tail : 0);
+    }
+    wa.ge = ge;
+    wa.whist = whist;
+    wa.lo = lo;
+    const int per_smw = blocks_per_sm(reinterpret_cast<const void *>(k_window<true>), kHistThreads, smemw);
+    const int64_t spw = splits_for(tokens, wa.nslab, per_smw, (int64_t)(kHistThreads / 32) * kWinUnroll, 65535);
+    wa.rows_per_split = (tokens + spw - 1) / spw;
+    if (v8) k_window<true><<<(int)(wa.nslab * spw), kHistThreads, smemw, s>>>(wa);
+    else k_window<false><<<(int)(wa.nslab * spw), kHistThreads, smemw, s>>>(wa);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    k_window_final<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(whist, ge, lo, (int)channels, (uint64_t)tokens,
+                                                                       (uint32_t)kk, static_cast<uint16_t *>(pct),
+                                                                       failed, needed);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+
+    // 3. exact two-pass radix select for the channels outside their window
+    HistArgs a{};
+    a.acts = static_cast<const uint16_t *>(acts);
+    a.T = tokens;
+    a.C = (int)channels;
+    a.lda = lda;
+    a.nslab = nslab64;
+    a.hist1 = whist;
+    a.hist2 = hist2;
+    a.k = (uint32_t)kk;
+    a.needed = needed;
+    const int64_t splits = splits_for(tokens, nslab64, per_sm1, min_rows, INT64_MAX);
+    a.rows_per_split = (tokens + splits - 1) / splits;
+    const int grid = (int)(nslab64 * splits);
     if (pair) k_hist<1, true><<<grid, kHistThreads, smem1, s>>>(a);
     else k_hist<1, false><<<grid, kHistThreads, smem1, s>>>(a);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     if (pair) k_hist<2, true><<<grid, kHistThreads, smem2, s>>>(a);
     else k_hist<2, false><<<grid, kHistThreads, smem2, s>>>(a);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    k_finalize<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(hist1, hist2, (int)channels, a.k,
-                                                                   static_cast<uint16_t *>(pct));
+    k_finalize<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(whist, hist2, (int)channels, a.k,
+                                                                   static_cast<uint16_t *>(pct), failed);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+
+    // 4. median over channels, ratios, top-n mask
     const uint32_t n_top = (uint32_t)(((uint64_t)channels * mask_num) / mask_den);
     k_mask<<<1, kMaskThreads, kKeys * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
                                              mask_idx_out);

@@ -49,6 +49,22 @@ def test_small_shapes(H, T, C):
     assert_same(run_gpu(H, acts), oracle_all(acts))
 
 
+@pytest.mark.parametrize("kind", ["t3", "cauchy", "wide"])
+def test_heavy_tails_exercise_exact_fallback(H, kind):
+    """Tails far heavier than Gaussian put the target rank outside the sampled
+    window for many channels, so the exact two-pass select must take over."""
+    rng = np.random.default_rng({"t3": 21, "cauchy": 22, "wide": 23}[kind])
+    T, C = 9000, 200
+    if kind == "t3":
+        x = rng.standard_t(3, (T, C))
+    elif kind == "cauchy":
+        x = rng.standard_cauchy((T, C))
+    else:
+        x = rng.standard_normal((T, C)) * np.exp(rng.uniform(-30, 30, (T, 1)))
+    acts = wl.f32_to_bf16_bits(x.astype(np.float32))
+    assert_same(run_gpu(H, acts), oracle_all(acts))
+
+
 def test_other_ratios_and_ties(H):
     rng = np.random.default_rng(9)
     acts = rng.integers(0, 6, (500, 200)).astype(np.uint16) * 0x80 + 0x3F00     # heavy ties
