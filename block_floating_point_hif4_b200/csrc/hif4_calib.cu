@@ -184,9 +184,10 @@ __global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, 
 
 // ------------------------------------------------------- windowed single pass
 //
-// A row sample (about 4096 rows) gives each channel a window of 256 keys — two
-// binades — starting at the binade that holds its sampled tail quantile at
-// ten times the target tail mass (the 99th percentile for q = 0.999).  One
+// A row sample (about 2048 rows) gives each channel a window of 256 keys (at
+// least a factor 2 in value) starting at the sample's exact order statistic
+// at ten times the target tail mass (its 99th percentile for q = 0.999),
+// found by the same two-pass radix select run on the sampled rows.  One
 // pass over all tokens then counts the keys at or above the window start
 // (`ge`) and histograms the keys inside the window; the target rank k is in
 // the window iff T - ge <= k < T - ge + (window count), and then the window
@@ -212,11 +213,9 @@ struct WinArgs {
     int64_t lda;
     int nslab;
     int64_t rows_per_split;
-    const uint32_t *hs;     // sample histogram [C][256] of key >> 7
-    uint32_t r_lo;          // sample rank whose binade starts the window
+    const uint16_t *lo;     // [C] window start key (a sample order statistic)
     uint32_t *ge;           // [C] keys >= window start
     uint32_t *whist;        // [C][256]
-    uint32_t *lo;           // [C] window start key
 };
 
 template <bool V8>
@@ -231,18 +230,9 @@ __global__ void __launch_bounds__(kHistThreads) k_window(WinArgs a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     for (int i = threadIdx.x; i < kWinBins * kWinSlab / 2; i += kHistThreads) h[i] = 0;
-    for (int j = warp; j < kWinSlab; j += kHistThreads / 32) {
-        uint32_t lo = 0x8000u;                         // channel past C: never counted
-        if (c0 + j < a.C) {
-            uint32_t bin, below;
-            warp_select_bin(a.hs + (size_t)(c0 + j) * 256, 256, a.r_lo, bin, below);
-            lo = bin << 7;
-            if (split == 0 && lane == 0) a.lo[c0 + j] = lo;
-        }
-        if (lane == 0) {
-            lo_s[j] = lo;
-            ge_s[j] = 0;
-        }
+    for (int j = threadIdx.x; j < kWinSlab; j += kHistThreads) {
+        lo_s[j] = c0 + j < a.C ? (uint32_t)a.lo[c0 + j] : 0x8000u;   // past C: never counted
+        ge_s[j] = 0;
     }
     __syncthreads();
 
@@ -314,7 +304,7 @@ __global__ void __launch_bounds__(kHistThreads) k_window(WinArgs a)
 // Key at rank k from the window counts (one warp per channel); a channel
 // whose rank is outside its window is marked for the exact fallback, and its
 // window row is cleared for reuse as the fallback's first histogram.
-__global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint32_t *lo, int C, uint64_t T, uint32_t k,
+__global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint16_t *lo, int C, uint64_t T, uint32_t k,
                                uint16_t *pct, uint8_t *failed, uint32_t *needed)
 {
     const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -328,7 +318,7 @@ __global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint32
         warp_select_bin(row, kWinBins, (uint32_t)((uint64_t)k - below), bin, cum, &total);
         if ((uint64_t)k - below < total) {
             ok = true;
-            if (lane == 0) pct[c] = (uint16_t)(lo[c] + bin);
+            if (lane == 0) pct[c] = (uint16_t)((uint32_t)lo[c] + bin);
         }
     }
     if (!ok) {
@@ -438,7 +428,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct CalibLayout {
-    size_t hs, whist, hist2, ge, lo, failed, needed, total;
+    size_t hs, hs2, whist, hist2, ge, lo, failed, needed, total;
 };
 
 CalibLayout calib_layout(int64_t C)
@@ -446,11 +436,12 @@ CalibLayout calib_layout(int64_t C)
     CalibLayout L{};
     const size_t nslab = (size_t)((C + kSlab - 1) / kSlab);
     L.hs = 0;
-    L.whist = L.hs + a256((size_t)C * 256 * 4);
+    L.hs2 = L.hs + a256((size_t)C * kBins1 * 4);
+    L.whist = L.hs2 + a256((size_t)C * kBins2 * 4);
     L.hist2 = L.whist + a256((size_t)C * 256 * 4);
     L.ge = L.hist2 + a256((size_t)C * kBins2 * 4);
     L.lo = L.ge + a256((size_t)C * 4);
-    L.failed = L.lo + a256((size_t)C * 4);
+    L.failed = L.lo + a256((size_t)C * 2);
     L.needed = L.failed + a256((size_t)C);
     L.total = L.needed + a256(nslab * 4);
     return L;
@@ -502,10 +493,11 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *hs = reinterpret_cast<uint32_t *>(ws + L.hs);
+    uint32_t *hs2 = reinterpret_cast<uint32_t *>(ws + L.hs2);
     uint32_t *whist = reinterpret_cast<uint32_t *>(ws + L.whist);
     uint32_t *hist2 = reinterpret_cast<uint32_t *>(ws + L.hist2);
     uint32_t *ge = reinterpret_cast<uint32_t *>(ws + L.ge);
-    uint32_t *lo = reinterpret_cast<uint32_t *>(ws + L.lo);
+    uint16_t *lo = reinterpret_cast<uint16_t *>(ws + L.lo);
     uint8_t *failed = ws + L.failed;
     uint32_t *needed = reinterpret_cast<uint32_t *>(ws + L.needed);
     if (cudaMemsetAsync(workspace, 0, L.total, s) != cudaSuccess) return HIF4_ERR_CUDA;
@@ -531,9 +523,12 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     const int per_sm1 = blocks_per_sm(reinterpret_cast<const void *>(k_hist<1, true>), kHistThreads, smem1);
     const int64_t min_rows = (int64_t)(kHistThreads / 32) * kRowUnroll;
 
-    // 1. sample histogram: every R-th row (about 4096 rows)
-    const int64_t R = tokens / 4096 > 1 ? tokens / 4096 : 1;
+    // 1. window starts: exact order statistic of a row sample (every R-th row,
+    //    about 2048 rows) at ten times the target tail mass below the top
+    const int64_t R = tokens / 2048 > 1 ? tokens / 2048 : 1;
     const int64_t Ts = (tokens + R - 1) / R;
+    const uint64_t tail = ((uint64_t)(tokens - kk) * 10ull * (uint64_t)Ts + (uint64_t)tokens - 1) / (uint64_t)tokens;
+    const uint32_t r_lo = (uint32_t)((uint64_t)Ts > tail + 1 ? (uint64_t)Ts - 1 - tail : 0);
     HistArgs sa{};
     sa.acts = static_cast<const uint16_t *>(acts);
     sa.T = Ts;
@@ -541,13 +536,18 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     sa.lda = lda * R;
     sa.nslab = nslab64;
     sa.hist1 = hs;
-    sa.hist2 = hist2;
-    sa.k = 0;
+    sa.hist2 = hs2;
+    sa.k = r_lo;
     sa.needed = nullptr;
-    int64_t sp = splits_for(Ts, nslab64, per_sm1, min_rows, INT64_MAX);
+    const int64_t sp = splits_for(Ts, nslab64, per_sm1, min_rows, INT64_MAX);
     sa.rows_per_split = (Ts + sp - 1) / sp;
     if (pair) k_hist<1, true><<<(int)(nslab64 * sp), kHistThreads, smem1, s>>>(sa);
     else k_hist<1, false><<<(int)(nslab64 * sp), kHistThreads, smem1, s>>>(sa);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (pair) k_hist<2, true><<<(int)(nslab64 * sp), kHistThreads, smem2, s>>>(sa);
+    else k_hist<2, false><<<(int)(nslab64 * sp), kHistThreads, smem2, s>>>(sa);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    k_finalize<<<(int)((channels * 32 + 255) / 256), 256, 0, s>>>(hs, hs2, (int)channels, r_lo, lo, nullptr);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
 
     // 2. windowed pass over every token
@@ -557,15 +557,9 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     wa.C = (int)channels;
     wa.lda = lda;
     wa.nslab = (int)((channels + kWinSlab - 1) / kWinSlab);
-    wa.hs = hs;
-    {
-        // ascending sample rank: ten times the target's tail mass below the top
-        const uint64_t tail = ((uint64_t)(tokens - kk) * 10ull * (uint64_t)Ts + (uint64_t)tokens - 1) / (uint64_t)tokens;
-        wa.r_lo = (uint32_t)((uint64_t)Ts > tail + 1 ? (uint64_t)Ts - 1 - tail : 0);
-    }
+    wa.lo = lo;
     wa.ge = ge;
     wa.whist = whist;
-    wa.lo = lo;
     const int per_smw = blocks_per_sm(reinterpret_cast<const void *>(k_window<true>), kHistThreads, smemw);
     const int64_t spw = splits_for(tokens, wa.nslab, per_smw, (int64_t)(kHistThreads / 32) * kWinUnroll, 65535);
     wa.rows_per_split = (tokens + spw - 1) / spw;
