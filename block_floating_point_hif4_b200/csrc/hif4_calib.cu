@@ -240,51 +240,58 @@ __global__ void __launch_bounds__(kHistThreads) k_window(WinArgs a)
     const uint32_t LO01 = lo_s[ch] | (lo_s[ch + 1] << 16), LO23 = lo_s[ch + 2] | (lo_s[ch + 3] << 16);
     const bool all4 = c0 + ch + 3 < a.C;
     uint32_t ge[4] = {0, 0, 0, 0};
+    uint32_t *hrow = h + 2 * lane;                     // word of channels (ch, ch+1); +1: (ch+2, ch+3)
     const int64_t t0 = (int64_t)split * a.rows_per_split;
     int64_t t1 = t0 + a.rows_per_split;
     if (t1 > a.T) t1 = a.T;
-    const uint16_t *col = a.acts + c0 + ch;
+    constexpr int RS = kHistThreads / 32;              // rows between a warp's consecutive rows
 
-    for (int64_t t = t0 + warp; t < t1; t += (int64_t)(kHistThreads / 32) * kWinUnroll) {
+    // one row: counts keys at or above the window start, histograms the keys inside it
+    auto row = [&](uint32_t w01, uint32_t w23) {
+        const uint32_t D01 = (w01 | 0x80008000u) - LO01;
+        const uint32_t D23 = (w23 | 0x80008000u) - LO23;
+        if ((D01 | D23) & 0x80008000u) {
+            const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t off = d[j] - 0x8000u;  // key - lo (wraps when key < lo)
+                ge[j] += off < 0x8000u;
+                if (off < (uint32_t)kWinBins) atomicAdd(hrow + off * (kWinSlab / 2) + (j >> 1), 1u << (16 * (j & 1)));
+            }
+        }
+    };
+    auto load = [&](const uint16_t *p, uint32_t &w01, uint32_t &w23) {
+        if (V8 && all4) {
+            asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(w01), "=r"(w23) : "l"(p));
+        } else {
+            uint32_t e[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (c0 + ch + q < a.C) e[q] = __ldg(p + q);
+            w01 = e[0] | (e[1] << 16);
+            w23 = e[2] | (e[3] << 16);
+        }
+    };
+
+    const int64_t step = (int64_t)RS * a.lda;           // elements between a warp's rows
+    int64_t t = t0 + warp;
+    const uint16_t *p = a.acts + (size_t)t * a.lda + c0 + ch;
+    // full iterations: kWinUnroll rows in flight, no bounds checks
+    for (; t + (int64_t)(kWinUnroll - 1) * RS < t1; t += (int64_t)kWinUnroll * RS) {
         uint32_t w01[kWinUnroll], w23[kWinUnroll];
 #pragma unroll
         for (int u = 0; u < kWinUnroll; ++u) {
-            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
-            w01[u] = w23[u] = 0;
-            if (r < t1) {
-                const uint16_t *p = col + r * a.lda;
-                if (V8 && all4) {
-                    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-                                 : "=r"(w01[u]), "=r"(w23[u]) : "l"(p));
-                } else {
-                    uint32_t e[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        if (c0 + ch + j < a.C) e[j] = __ldg(p + j);
-                    w01[u] = e[0] | (e[1] << 16);
-                    w23[u] = e[2] | (e[3] << 16);
-                }
-            }
+            load(p, w01[u], w23[u]);
+            p += step;
         }
 #pragma unroll
-        for (int u = 0; u < kWinUnroll; ++u) {
-            const int64_t r = t + (int64_t)u * (kHistThreads / 32);
-            if (r >= t1) break;
-            const uint32_t D01 = (w01[u] | 0x80008000u) - LO01;
-            const uint32_t D23 = (w23[u] | 0x80008000u) - LO23;
-            if ((D01 | D23) & 0x80008000u) {           // some key at or above its window start
-                const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (d[j] & 0x8000u) {
-                        ++ge[j];
-                        const uint32_t off = d[j] - 0x8000u;          // key - lo
-                        if (off < (uint32_t)kWinBins)
-                            atomicAdd(&h[off * (kWinSlab / 2) + 2 * lane + (j >> 1)], 1u << (16 * (j & 1)));
-                    }
-                }
-            }
-        }
+        for (int u = 0; u < kWinUnroll; ++u) row(w01[u], w23[u]);
+    }
+    for (; t < t1; t += RS) {                           // tail
+        uint32_t w01, w23;
+        load(p, w01, w23);
+        p += step;
+        row(w01, w23);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
