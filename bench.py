@@ -82,19 +82,29 @@ def src_hash(*names):
 # --------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 100 ms while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 50 ms; started before the warm-up (the tool
+    takes a moment to start) and filtered to the timed region by timestamp."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, uuid):
         self.uuid = uuid
         self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        import datetime
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        import datetime
+        self.t1 = datetime.datetime.now()
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -113,6 +123,7 @@ class ClockSampler:
         return False
 
     def summary(self):
+        import datetime
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in self.lines:
@@ -120,6 +131,9 @@ class ClockSampler:
             if len(f) < 9:
                 continue
             try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                if self.t0 and self.t1 and not (self.t0 <= ts <= self.t1):
+                    continue
                 sm.append(float(f[1]))
                 mx = float(f[2])
             except ValueError:
@@ -304,20 +318,21 @@ def main():
 
     launches_per_step = 2 * (1 + 1 + 1 + 1)     # fake-quant, dequant, column scatter, GEMM per linear
 
-    for _ in range(args.warmup):
-        step()
-    barrier()
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
+        for _ in range(args.warmup):
+            step()
         barrier()
+        clk.mark_start()
         t_start.record(stream)
         for k in range(args.steps):
             step(evs[k])
         t_end.record(stream)
         barrier()
+        clk.mark_end()
     ms_total = t_start.elapsed_time(t_end)
     ms_step = max_over_ranks(ms_total / args.steps)
     per_stage = {s: [] for s in stages}
