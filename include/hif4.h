@@ -208,7 +208,7 @@ hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t
  * what must start at zero on every call.
  *   - Sizes whose hif4_calib_workspace(tokens, channels) exceeds the array
  *     are rejected with HIF4_ERR_WORKSPACE before any launch (with the
- *     current histogram layout: channels <= 10922).
+ *     current histogram layout: channels <= 5448).
  *   - The first call on a device looks up the array's device address once
  *     (that device must be current); make that first call before any stream
  *     capture begins.
