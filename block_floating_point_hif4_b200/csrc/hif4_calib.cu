@@ -56,6 +56,7 @@ struct PassArgs {
     uint32_t *hist1;         // [C][256]
     uint32_t *hist2;         // [C][128]
     uint32_t k;              // target ascending rank (pass 2)
+    const uint16_t *tbin;    // pass 2: [C] bin of hist1 that holds rank k
     const uint32_t *needed;  // null, or per slab: nonzero = process
     const uint16_t *lo;      // window pass: [C] window start key
     uint32_t *ge;            // window pass: [C]
@@ -138,11 +139,8 @@ __global__ void __launch_bounds__(kThreads) k_pass(PassArgs a)
 
     for (int i = threadIdx.x; i < NB * kSlab / 2; i += kThreads) h[i] = 0;
     if (MODE == 2) {
-        for (int j = warp; j < kSlab; j += kRS) {
-            uint32_t bin = 0x1000u, below;             // past C: matches no key
-            if (c0 + j < a.C) warp_select_bin(a.hist1 + (size_t)(c0 + j) * kBins1, kBins1, a.k, bin, below);
-            if (lane == 0) par[j] = bin;
-        }
+        for (int j = threadIdx.x; j < kSlab; j += kThreads)
+            par[j] = c0 + j < a.C ? (uint32_t)a.tbin[c0 + j] : 0u;   // counts past C are dropped
     }
     if (MODE == 3) {
         for (int j = threadIdx.x; j < kSlab; j += kThreads) {
@@ -240,6 +238,17 @@ __global__ void __launch_bounds__(kThreads) k_pass(PassArgs a)
     if (MODE == 3)
         for (int j = threadIdx.x; j < kSlab; j += kThreads)
             if (ge_s[j] && c0 + j < a.C) atomicAdd(&a.ge[c0 + j], ge_s[j]);
+}
+
+// Bin of the first radix histogram that holds rank k (one warp per channel).
+__global__ void k_select1(const uint32_t *hist1, int C, uint32_t k, uint16_t *tbin, const uint8_t *failed)
+{
+    const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (c >= C) return;
+    if (failed && !failed[c]) return;
+    uint32_t b, below;
+    warp_select_bin(hist1 + (size_t)c * kBins1, kBins1, k, b, below);
+    if ((threadIdx.x & 31) == 0) tbin[c] = (uint16_t)b;
 }
 
 // Key at rank k from the two radix histograms (one warp per channel); with
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct CalibLayout {
-    size_t hs, hs2, whist, hist2, ge, lo, failed, needed, total;
+    size_t hs, hs2, whist, hist2, ge, lo, tbin, failed, needed, total;
 };
 
 CalibLayout calib_layout(int64_t C)
@@ -396,7 +405,8 @@ CalibLayout calib_layout(int64_t C)
     L.hist2 = L.whist + a256((size_t)C * kWinBins * 4);
     L.ge = L.hist2 + a256((size_t)C * kBins2 * 4);
     L.lo = L.ge + a256((size_t)C * 4);
-    L.failed = L.lo + a256((size_t)C * 2);
+    L.tbin = L.lo + a256((size_t)C * 2);
+    L.failed = L.tbin + a256((size_t)C * 2);
     L.needed = L.failed + a256((size_t)C);
     L.total = L.needed + a256(nslab * 4);
     return L;
@@ -479,6 +489,7 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     uint32_t *hist2 = reinterpret_cast<uint32_t *>(ws + L.hist2);
     uint32_t *ge = reinterpret_cast<uint32_t *>(ws + L.ge);
     uint16_t *lo = reinterpret_cast<uint16_t *>(ws + L.lo);
+    uint16_t *tbin = reinterpret_cast<uint16_t *>(ws + L.tbin);
     uint8_t *failed = ws + L.failed;
     uint32_t *needed = reinterpret_cast<uint32_t *>(ws + L.needed);
     if (cudaMemsetAsync(workspace, 0, L.total, s) != cudaSuccess) return HIF4_ERR_CUDA;
@@ -504,7 +515,10 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     sa.hist1 = hs;
     sa.hist2 = hs2;
     sa.k = r_lo;
+    sa.tbin = tbin;
     if ((st = launch_pass<1>(sa, v8s, s)) != HIF4_OK) return st;
+    k_select1<<<fgrid, 256, 0, s>>>(hs, (int)channels, r_lo, tbin, nullptr);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     if ((st = launch_pass<2>(sa, v8s, s)) != HIF4_OK) return st;
     k_finalize<<<fgrid, 256, 0, s>>>(hs, hs2, (int)channels, r_lo, lo, nullptr);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
@@ -529,8 +543,11 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.hist1 = whist;
     a.hist2 = hist2;
     a.k = (uint32_t)kk;
+    a.tbin = tbin;
     a.needed = needed;
     if ((st = launch_pass<1>(a, v8, s)) != HIF4_OK) return st;
+    k_select1<<<fgrid, 256, 0, s>>>(whist, (int)channels, (uint32_t)kk, tbin, failed);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     if ((st = launch_pass<2>(a, v8, s)) != HIF4_OK) return st;
     k_finalize<<<fgrid, 256, 0, s>>>(whist, hist2, (int)channels, (uint32_t)kk, static_cast<uint16_t *>(pct), failed);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
