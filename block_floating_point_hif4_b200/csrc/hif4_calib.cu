@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include "hif4_internal.cuh"
+#include "hif4_sm100.cuh"
 
 namespace hif4 {
 namespace {
@@ -61,6 +62,7 @@ struct PassArgs {
     const uint16_t *lo;      // window pass: [C] window start key
     uint32_t *ge;            // window pass: [C]
     uint32_t *whist;         // window pass: [C][256]
+    uint32_t *timed_out;     // set to 1 when a TMA transfer never lands
 };
 
 // Bin holding ascending rank k of a histogram of `nbins` (multiple of 32)
@@ -251,6 +253,174 @@ __global__ void k_select1(const uint32_t *hist1, int C, uint32_t k, uint16_t *tb
     if ((threadIdx.x & 31) == 0) tbin[c] = (uint16_t)b;
 }
 
+// TMA-staged variant of k_pass.  A 2-D tensor map over the (strided) rows
+// lands 64-row x 128-channel tiles (16 KB) in a 3-stage shared ring
+// (cp.async.bulk.tensor with mbarrier completion), so loads stay in flight
+// while the warps count.  A warp reads its rows' 4-channel words with 8-byte
+// shared loads (256 contiguous bytes per warp: no bank conflicts).
+//
+// Work split: the grid is persistent (every block resident at once) and
+// block b takes units [b share, (b+1) share) of the slab-major space
+// u = slab * T + row, so all blocks carry equal rows and no wave tail is
+// left.  A share crosses at most a few slab boundaries; each slab segment
+// zeroes and flushes the shared counters (share <= 65535 rows keeps the
+// 16-bit counters exact).  Rows past a segment inside a tile are skipped by
+// count; channels past C land in counters that are never flushed.
+constexpr int kTmaRows = 64;
+constexpr int kTmaStages = 3;
+constexpr uint32_t kTileBytes = kTmaRows * kSlab * 2;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+template <int MODE>
+__device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *hrow, uint32_t swap, uint32_t P01,
+                                          uint32_t P23, uint32_t (&ge)[4])
+{
+    if (MODE == 1) {
+        const uint32_t wa = swap ? w23 : w01, wb = swap ? w01 : w23;
+        const uint32_t ha = swap, hb = swap ^ 1u;
+        atomicAdd(hrow + ((wa >> 7) & 0xFFu) * (kSlab / 2) + ha, 1u);
+        atomicAdd(hrow + ((wa >> 23) & 0xFFu) * (kSlab / 2) + ha, 0x10000u);
+        atomicAdd(hrow + ((wb >> 7) & 0xFFu) * (kSlab / 2) + hb, 1u);
+        atomicAdd(hrow + ((wb >> 23) & 0xFFu) * (kSlab / 2) + hb, 0x10000u);
+    } else if (MODE == 2) {
+        const uint32_t x01 = (w01 & 0x7F807F80u) ^ P01, x23 = (w23 & 0x7F807F80u) ^ P23;
+        if (!(x01 & 0xFFFFu)) atomicAdd(hrow + (w01 & 127u) * (kSlab / 2), 1u);
+        if (!(x01 >> 16)) atomicAdd(hrow + ((w01 >> 16) & 127u) * (kSlab / 2), 0x10000u);
+        if (!(x23 & 0xFFFFu)) atomicAdd(hrow + (w23 & 127u) * (kSlab / 2) + 1, 1u);
+        if (!(x23 >> 16)) atomicAdd(hrow + ((w23 >> 16) & 127u) * (kSlab / 2) + 1, 0x10000u);
+    } else {
+        // bit 15 of each half of D is set iff that key >= lo; the half then
+        // holds 0x8000 + (key - lo)
+        const uint32_t D01 = (w01 | 0x80008000u) - P01;
+        const uint32_t D23 = (w23 | 0x80008000u) - P23;
+        if ((D01 | D23) & 0x80008000u) {
+            const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t off = d[j] - 0x8000u;
+                ge[j] += off < 0x8000u;
+                if (off < (uint32_t)kWinBins) atomicAdd(hrow + off * (kSlab / 2) + (j >> 1), 1u << (16 * (j & 1)));
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads) k_pass_tma(const __grid_constant__ CUtensorMap tm, PassArgs a)
+{
+    using namespace sm100;
+    constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
+    extern __shared__ __align__(128) uint8_t smraw[];
+    uint8_t *tiles = smraw;                                             // kTmaStages x 16 KB
+    uint32_t *h = reinterpret_cast<uint32_t *>(smraw + kTmaStages * kTileBytes);   // [NB][kSlab / 2]
+    __shared__ uint64_t full[kTmaStages];
+    __shared__ uint16_t par[kSlab];                                     // 16-bit: keeps two blocks per SM
+    __shared__ uint32_t ge_s[kSlab];
+    __shared__ uint32_t abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ch = 4 * lane;
+    const uint32_t swap = lane >= 16 ? 1u : 0u;
+    uint32_t *hrow = h + 2 * lane;
+
+    const int64_t total = (int64_t)a.nslab * a.T;
+    int64_t cur = (int64_t)blockIdx.x * a.rows_per_split;
+    const int64_t end = cur + a.rows_per_split < total ? cur + a.rows_per_split : total;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kTmaStages; ++st) mbar_init(&full[st], 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tm);
+    }
+    uint32_t g = 0;                                    // tiles consumed: ring slot and phase
+    while (cur < end) {                                // block-uniform
+        const int slab = (int)(cur / a.T);
+        const int64_t t0 = cur - (int64_t)slab * a.T;
+        const int64_t t1 = t0 + (end - cur) < a.T ? t0 + (end - cur) : a.T;
+        cur += t1 - t0;
+        if (a.needed && !a.needed[slab]) continue;
+        const int c0 = slab * kSlab;
+        __syncthreads();                               // previous segment flushed
+        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kThreads) h[i] = 0;
+        if (MODE == 2)
+            for (int j = threadIdx.x; j < kSlab; j += kThreads) par[j] = c0 + j < a.C ? a.tbin[c0 + j] : (uint16_t)0;
+        if (MODE == 3)
+            for (int j = threadIdx.x; j < kSlab; j += kThreads) {
+                par[j] = c0 + j < a.C ? a.lo[c0 + j] : (uint16_t)0x8000u;
+                ge_s[j] = 0;
+            }
+        __syncthreads();
+        const int nchunks = (int)((t1 - t0 + kTmaRows - 1) / kTmaRows);
+        auto issue = [&](int ci) {
+            const uint32_t st = (g + (uint32_t)ci) % kTmaStages;
+            mbar_arrive_expect_tx(&full[st], kTileBytes);
+            tma_load_2d(tiles + st * kTileBytes, &tm, c0, (int32_t)(t0 + (int64_t)ci * kTmaRows), &full[st]);
+        };
+        if (threadIdx.x == 0)
+            for (int ci = 0; ci < nchunks && ci < kTmaStages; ++ci) issue(ci);
+        uint32_t P01 = 0, P23 = 0;
+        if (MODE == 2) {
+            P01 = ((uint32_t)par[ch] << 7) | ((uint32_t)par[ch + 1] << 23);
+            P23 = ((uint32_t)par[ch + 2] << 7) | ((uint32_t)par[ch + 3] << 23);
+        }
+        if (MODE == 3) {
+            P01 = (uint32_t)par[ch] | ((uint32_t)par[ch + 1] << 16);
+            P23 = (uint32_t)par[ch + 2] | ((uint32_t)par[ch + 3] << 16);
+        }
+        uint32_t ge[4] = {0, 0, 0, 0};
+        int ci = 0;
+        for (; ci < nchunks; ++ci) {
+            const uint32_t gi = g + (uint32_t)ci;
+            const uint32_t st = gi % kTmaStages;
+            const bool ok = mbar_wait_bounded(&full[st], (gi / kTmaStages) & 1u, &abort_flag, kWaitNs);
+            const int64_t left = t1 - (t0 + (int64_t)ci * kTmaRows);
+            const uint8_t *tile = tiles + st * kTileBytes + ch * 2;
+            if (ok && left >= kTmaRows) {
+#pragma unroll
+                for (int i = 0; i < kTmaRows / kRS; ++i) {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(tile + (warp + i * kRS) * (kSlab * 2));
+                    count_row<MODE>(v.x, v.y, hrow, swap, P01, P23, ge);
+                }
+            } else if (ok) {
+                for (int r = warp; r < (int)left; r += kRS) {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(tile + r * (kSlab * 2));
+                    count_row<MODE>(v.x, v.y, hrow, swap, P01, P23, ge);
+                }
+            }
+            if (__syncthreads_or(!ok)) break;          // slot consumed; on a time-out all leave together
+            if (threadIdx.x == 0 && ci + kTmaStages < nchunks) issue(ci + kTmaStages);
+        }
+        if (ci < nchunks) {                            // time-out: let issued copies land, flag, stop
+            if (threadIdx.x == 0) {
+                for (int cj = ci; cj < nchunks && cj < ci + kTmaStages; ++cj) {
+                    const uint32_t gj = g + (uint32_t)cj;
+                    mbar_wait_bounded(&full[gj % kTmaStages], (gj / kTmaStages) & 1u, nullptr, 100000000ull);
+                }
+                atomicOr(a.timed_out, 1u);
+            }
+            return;
+        }
+        g += (uint32_t)nchunks;
+        if (MODE == 3) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (ge[j]) atomicAdd(&ge_s[ch + j], ge[j]);
+        }
+        __syncthreads();
+        uint32_t *gh = MODE == 1 ? a.hist1 : MODE == 2 ? a.hist2 : a.whist;
+        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kThreads) {
+            const uint32_t v = h[i];
+            if (!v) continue;
+            const int bin = i / (kSlab / 2), wi = i % (kSlab / 2);
+            const int c = c0 + 4 * (wi >> 1) + 2 * (wi & 1);
+            if ((v & 0xFFFFu) && c < a.C) atomicAdd(&gh[(size_t)c * NB + bin], v & 0xFFFFu);
+            if ((v >> 16) && c + 1 < a.C) atomicAdd(&gh[(size_t)(c + 1) * NB + bin], v >> 16);
+        }
+        if (MODE == 3)
+            for (int j = threadIdx.x; j < kSlab; j += kThreads)
+                if (ge_s[j] && c0 + j < a.C) atomicAdd(&a.ge[c0 + j], ge_s[j]);
+    }
+}
+
 // Key at rank k from the two radix histograms (one warp per channel); with
 // `failed`, only the channels it marks.
 __global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, uint32_t k, uint16_t *out,
@@ -326,10 +496,21 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratc
     return scratch[32 + warp] + incl - v;
 }
 
+// A time-out in an earlier pass (timed_out != 0) poisons the outputs instead:
+// every ratio NaN, the mask all zero, every mask index -1.
 __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int C, uint32_t n_top, float *ratio,
-                                                      uint8_t *mask, int32_t *mask_idx)
+                                                      uint8_t *mask, int32_t *mask_idx, const uint32_t *timed_out)
 {
     extern __shared__ uint32_t hist[];                 // [kKeys]
+    if (*timed_out) {                                  // block-uniform
+        for (int c = threadIdx.x; c < C; c += kMaskThreads) {
+            ratio[c] = __int_as_float(0x7FC00000);
+            mask[c] = 0;
+        }
+        if (mask_idx)
+            for (uint32_t i = threadIdx.x; i < n_top; i += kMaskThreads) mask_idx[i] = -1;
+        return;
+    }
     __shared__ uint32_t scratch[72];
     __shared__ uint32_t sel[4];                        // med key, tau key, count above tau
     for (int i = threadIdx.x; i < kKeys; i += kMaskThreads) hist[i] = 0;
@@ -392,7 +573,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
 size_t a256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct CalibLayout {
-    size_t hs, hs2, whist, hist2, ge, lo, tbin, failed, needed, total;
+    size_t hs, hs2, whist, hist2, ge, lo, tbin, failed, needed, timed_out, total;
 };
 
 CalibLayout calib_layout(int64_t C)
@@ -408,7 +589,8 @@ CalibLayout calib_layout(int64_t C)
     L.tbin = L.lo + a256((size_t)C * 2);
     L.failed = L.tbin + a256((size_t)C * 2);
     L.needed = L.failed + a256((size_t)C);
-    L.total = L.needed + a256(nslab * 4);
+    L.timed_out = L.needed + a256(nslab * 4);
+    L.total = L.timed_out + 256;
     return L;
 }
 
@@ -426,8 +608,47 @@ int64_t splits_for(int64_t rows, int nslab, int per_sm)
 }
 
 template <int MODE>
-hif4_status launch_pass(const PassArgs &a0, bool v8, cudaStream_t s)
+hif4_status launch_pass_tma(const PassArgs &a0, cudaStream_t s, bool &done)
 {
+    constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
+    const size_t smem = (size_t)kTmaStages * kTileBytes + (size_t)NB * kSlab / 2 * 4;
+    done = false;
+    if (a0.T > INT32_MAX - kTmaRows) return HIF4_OK;   // TMA row coordinates are int32
+    CUtensorMap tm;
+    if (!make_tensor_map_bf16_2d(&tm, a0.acts, (uint64_t)a0.C, (uint64_t)a0.T, (uint64_t)a0.lda * 2, kSlab, kTmaRows,
+                                 false))
+        return HIF4_OK;
+    auto k = k_pass_tma<MODE>;
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr[dev & 63]) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        attr[dev & 63] = true;
+    }
+    PassArgs a = a0;
+    // equal shares of the slab-major (slab, row) space, one block per
+    // resident slot, 4..65535 tiles' worth of rows each
+    const int64_t slots = (int64_t)blocks_per_sm(reinterpret_cast<const void *>(k), kThreads, smem) * sm_count();
+    const int64_t total = (int64_t)a.nslab * a.T;
+    int64_t share = (total + slots - 1) / slots;
+    if (share < 4 * kTmaRows) share = 4 * kTmaRows;
+    if (share > kMaxRowsPerBlock) share = kMaxRowsPerBlock;
+    a.rows_per_split = share;
+    k<<<(int)((total + share - 1) / share), kThreads, smem, s>>>(tm, a);
+    done = true;
+    return launch_status();
+}
+
+template <int MODE>
+hif4_status launch_pass(const PassArgs &a0, bool v8, bool tma, cudaStream_t s)
+{
+    if (tma) {
+        bool done = false;
+        const hif4_status st = launch_pass_tma<MODE>(a0, s, done);
+        if (done || st != HIF4_OK) return st;
+    }
     constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
     const size_t smem = (size_t)NB * kSlab / 2 * 4;
     auto kt = k_pass<MODE, true>;
@@ -492,6 +713,7 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     uint16_t *tbin = reinterpret_cast<uint16_t *>(ws + L.tbin);
     uint8_t *failed = ws + L.failed;
     uint32_t *needed = reinterpret_cast<uint32_t *>(ws + L.needed);
+    uint32_t *timed_out = reinterpret_cast<uint32_t *>(ws + L.timed_out);
     if (cudaMemsetAsync(workspace, 0, L.total, s) != cudaSuccess) return HIF4_ERR_CUDA;
 
     const uint64_t kk = ((uint64_t)q_num * (uint64_t)(tokens - 1)) / q_den;
@@ -516,15 +738,19 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     sa.hist2 = hs2;
     sa.k = r_lo;
     sa.tbin = tbin;
-    if ((st = launch_pass<1>(sa, v8s, s)) != HIF4_OK) return st;
+    sa.timed_out = timed_out;
+    // TMA needs a 16-byte aligned base and row stride (the box is 256 bytes wide)
+    const bool tmas = aligned16(acts) && ((lda * R * 2) % 16 == 0);
+    if ((st = launch_pass<1>(sa, v8s, tmas, s)) != HIF4_OK) return st;
     k_select1<<<fgrid, 256, 0, s>>>(hs, (int)channels, r_lo, tbin, nullptr);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    if ((st = launch_pass<2>(sa, v8s, s)) != HIF4_OK) return st;
+    if ((st = launch_pass<2>(sa, v8s, tmas, s)) != HIF4_OK) return st;
     k_finalize<<<fgrid, 256, 0, s>>>(hs, hs2, (int)channels, r_lo, lo, nullptr);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
 
     // 2-3. windowed pass over every token, then the key where rank k falls
     const bool v8 = aligned_to(acts, 8) && (lda % 4 == 0);
+    const bool tma = aligned16(acts) && ((lda * 2) % 16 == 0);
     PassArgs a{};
     a.acts = static_cast<const uint16_t *>(acts);
     a.T = tokens;
@@ -534,7 +760,8 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.lo = lo;
     a.ge = ge;
     a.whist = whist;
-    if ((st = launch_pass<3>(a, v8, s)) != HIF4_OK) return st;
+    a.timed_out = timed_out;
+    if ((st = launch_pass<3>(a, v8, tma, s)) != HIF4_OK) return st;
     k_window_final<<<fgrid, 256, 0, s>>>(whist, ge, lo, (int)channels, (uint64_t)tokens, (uint32_t)kk,
                                          static_cast<uint16_t *>(pct), failed, needed);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
@@ -545,10 +772,10 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.k = (uint32_t)kk;
     a.tbin = tbin;
     a.needed = needed;
-    if ((st = launch_pass<1>(a, v8, s)) != HIF4_OK) return st;
+    if ((st = launch_pass<1>(a, v8, tma, s)) != HIF4_OK) return st;
     k_select1<<<fgrid, 256, 0, s>>>(whist, (int)channels, (uint32_t)kk, tbin, failed);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    if ((st = launch_pass<2>(a, v8, s)) != HIF4_OK) return st;
+    if ((st = launch_pass<2>(a, v8, tma, s)) != HIF4_OK) return st;
     k_finalize<<<fgrid, 256, 0, s>>>(whist, hist2, (int)channels, (uint32_t)kk, static_cast<uint16_t *>(pct), failed);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
 
@@ -563,6 +790,6 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     }
     const uint32_t n_top = (uint32_t)(((uint64_t)channels * mask_num) / mask_den);
     k_mask<<<1, kMaskThreads, kKeys * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
-                                             mask_idx_out);
+                                             mask_idx_out, timed_out);
     return launch_status();
 }
