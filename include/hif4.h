@@ -184,6 +184,9 @@ hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64_t lda, con
  * mask_idx_out  NULL or int32 [floor(C mask_num / mask_den)]: the masked
  *               channels in ascending order (ready for hif4_linear_w4a4).
  * workspace >= hif4_calib_workspace(T, C) bytes.
+ * Every wait on a tile copy inside the passes is bounded (2 s); if one runs
+ * out, the passes stop and the outputs are poisoned instead of computed:
+ * every ratio NaN, mask all zero, every mask_idx_out entry -1.
  */
 size_t hif4_calib_workspace(int64_t tokens, int64_t channels);
 hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t channels,
@@ -208,7 +211,7 @@ hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t
  * what must start at zero on every call.
  *   - Sizes whose hif4_calib_workspace(tokens, channels) exceeds the array
  *     are rejected with HIF4_ERR_WORKSPACE before any launch (with the
- *     current histogram layout: channels <= 5448).
+ *     current histogram layout: channels <= 5445).
  *   - The first call on a device looks up the array's device address once
  *     (that device must be current); make that first call before any stream
  *     capture begins.
