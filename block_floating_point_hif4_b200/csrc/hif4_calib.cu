@@ -253,24 +253,39 @@ __global__ void k_select1(const uint32_t *hist1, int C, uint32_t k, uint16_t *tb
     if ((threadIdx.x & 31) == 0) tbin[c] = (uint16_t)b;
 }
 
-// TMA-staged variant of k_pass.  A 2-D tensor map over the (strided) rows
-// lands 64-row x 128-channel tiles (16 KB) in a 3-stage shared ring
-// (cp.async.bulk.tensor with mbarrier completion), so loads stay in flight
-// while the warps count.  A warp reads its rows' 4-channel words with 8-byte
-// shared loads (256 contiguous bytes per warp: no bank conflicts).
+// TMA-staged variant of k_pass, warp-specialized, one block per SM.  A 2-D
+// tensor map over the (strided) rows lands 128-row x 128-channel tiles
+// (32 KB) in a 5-stage shared ring beside the 64 KB counter array.  One
+// producer warp issues the copies (cp.async.bulk.tensor, completion on a
+// "full" mbarrier per slot) and refills a slot once all sixteen consumer
+// warps have released it (an "empty" mbarrier per slot), so consumers never
+// wait on one another inside a segment and up to 160 KB per SM stay in
+// flight.  A consumer warp takes rows warp, warp + 16, ... (8 per tile): it
+// loads them all first (8-byte shared loads, 256 contiguous bytes per warp).
+// Pass 1 counts every key.  Passes 2 and 3 count few keys (those in the
+// target bin, those at or above the window start), so each lane first
+// marks its rows holding a candidate (a cheap superset test), then the warp
+// visits marked rows one per lane per round: the count is paid per marked
+// row instead of per divergent row.
 //
-// Work split: the grid is persistent (every block resident at once) and
-// block b takes units [b share, (b+1) share) of the slab-major space
-// u = slab * T + row, so all blocks carry equal rows and no wave tail is
-// left.  A share crosses at most a few slab boundaries; each slab segment
-// zeroes and flushes the shared counters (share <= 65535 rows keeps the
-// 16-bit counters exact).  Rows past a segment inside a tile are skipped by
-// count; channels past C land in counters that are never flushed.
-constexpr int kTmaRows = 64;
-constexpr int kTmaStages = 3;
-constexpr uint32_t kTileBytes = kTmaRows * kSlab * 2;
+// Work split: one block per SM; block b takes units [b share, (b+1) share)
+// of the slab-major space u = slab * T + row, so all blocks carry equal
+// rows and no wave tail is left.  A share crosses at most a few slab
+// boundaries; each slab segment zeroes and flushes the shared counters
+// (share <= 65535 rows keeps the 16-bit counters exact).  Rows past a
+// segment inside a tile are skipped; channels past C land in counters that
+// are never flushed.
+constexpr int kTmaRows = 128;
+constexpr int kTmaStages = 5;
+constexpr int kConsumers = 16;                       // consumer warps
+constexpr int kTmaThreads = (kConsumers + 1) * 32;   // + one producer warp
+constexpr int kRowsPerWarp = kTmaRows / kConsumers;  // 8
+constexpr uint32_t kRowBytes = kSlab * 2;
+constexpr uint32_t kTileBytes = kTmaRows * kRowBytes;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
+// One row's four keys of this lane (words w01 = channels ch, ch+1 and
+// w23 = ch+2, ch+3) into the shared counters.
 template <int MODE>
 __device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *hrow, uint32_t swap, uint32_t P01,
                                           uint32_t P23, uint32_t (&ge)[4])
@@ -289,32 +304,43 @@ __device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *
         if (!(x23 & 0xFFFFu)) atomicAdd(hrow + (w23 & 127u) * (kSlab / 2) + 1, 1u);
         if (!(x23 >> 16)) atomicAdd(hrow + ((w23 >> 16) & 127u) * (kSlab / 2) + 1, 0x10000u);
     } else {
-        // bit 15 of each half of D is set iff that key >= lo; the half then
-        // holds 0x8000 + (key - lo)
-        const uint32_t D01 = (w01 | 0x80008000u) - P01;
-        const uint32_t D23 = (w23 | 0x80008000u) - P23;
-        if ((D01 | D23) & 0x80008000u) {
-            const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
+        // D = (w | 0x80008000) - P: bit 15 of each half is set iff that key
+        // >= lo, the half then holding 0x8000 + (key - lo)
+        const uint32_t D01 = (w01 | 0x80008000u) - P01, D23 = (w23 | 0x80008000u) - P23;
+        const uint32_t d[4] = {D01 & 0xFFFFu, D01 >> 16, D23 & 0xFFFFu, D23 >> 16};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t off = d[j] - 0x8000u;
-                ge[j] += off < 0x8000u;
-                if (off < (uint32_t)kWinBins) atomicAdd(hrow + off * (kSlab / 2) + (j >> 1), 1u << (16 * (j & 1)));
-            }
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t off = d[j] - 0x8000u;
+            ge[j] += off < 0x8000u;
+            if (off < (uint32_t)kWinBins) atomicAdd(hrow + off * (kSlab / 2) + (j >> 1), 1u << (16 * (j & 1)));
         }
     }
 }
 
+// Superset test for a row that count_row<MODE> (2 or 3) may count: true
+// whenever it counts something.
 template <int MODE>
-__global__ void __launch_bounds__(kThreads) k_pass_tma(const __grid_constant__ CUtensorMap tm, PassArgs a)
+__device__ __forceinline__ bool row_candidate(uint32_t w01, uint32_t w23, uint32_t P01, uint32_t P23)
+{
+    if (MODE == 2) {
+        // a 16-bit half of x is zero (bit 15 of every half of x is clear)
+        const uint32_t x01 = (w01 & 0x7F807F80u) ^ P01, x23 = (w23 & 0x7F807F80u) ^ P23;
+        return (((x01 - 0x00010001u) | (x23 - 0x00010001u)) & 0x80008000u) != 0u;
+    } else {
+        return ((((w01 | 0x80008000u) - P01) | ((w23 | 0x80008000u) - P23)) & 0x80008000u) != 0u;
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_constant__ CUtensorMap tm, PassArgs a)
 {
     using namespace sm100;
     constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
     extern __shared__ __align__(128) uint8_t smraw[];
-    uint8_t *tiles = smraw;                                             // kTmaStages x 16 KB
+    uint8_t *tiles = smraw;                                             // kTmaStages x 32 KB
     uint32_t *h = reinterpret_cast<uint32_t *>(smraw + kTmaStages * kTileBytes);   // [NB][kSlab / 2]
-    __shared__ uint64_t full[kTmaStages];
-    __shared__ uint16_t par[kSlab];                                     // 16-bit: keeps two blocks per SM
+    __shared__ uint64_t full[kTmaStages], empty[kTmaStages];
+    __shared__ uint16_t par[kSlab];
     __shared__ uint32_t ge_s[kSlab];
     __shared__ uint32_t abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -326,7 +352,10 @@ __global__ void __launch_bounds__(kThreads) k_pass_tma(const __grid_constant__ C
     int64_t cur = (int64_t)blockIdx.x * a.rows_per_split;
     const int64_t end = cur + a.rows_per_split < total ? cur + a.rows_per_split : total;
     if (threadIdx.x == 0) {
-        for (int st = 0; st < kTmaStages; ++st) mbar_init(&full[st], 1);
+        for (int st = 0; st < kTmaStages; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], kConsumers);
+        }
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm);
@@ -340,58 +369,91 @@ __global__ void __launch_bounds__(kThreads) k_pass_tma(const __grid_constant__ C
         if (a.needed && !a.needed[slab]) continue;
         const int c0 = slab * kSlab;
         __syncthreads();                               // previous segment flushed
-        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kThreads) h[i] = 0;
+        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kTmaThreads) h[i] = 0;
         if (MODE == 2)
-            for (int j = threadIdx.x; j < kSlab; j += kThreads) par[j] = c0 + j < a.C ? a.tbin[c0 + j] : (uint16_t)0;
+            for (int j = threadIdx.x; j < kSlab; j += kTmaThreads)
+                par[j] = c0 + j < a.C ? a.tbin[c0 + j] : (uint16_t)0;
         if (MODE == 3)
-            for (int j = threadIdx.x; j < kSlab; j += kThreads) {
+            for (int j = threadIdx.x; j < kSlab; j += kTmaThreads) {
                 par[j] = c0 + j < a.C ? a.lo[c0 + j] : (uint16_t)0x8000u;
                 ge_s[j] = 0;
             }
         __syncthreads();
         const int nchunks = (int)((t1 - t0 + kTmaRows - 1) / kTmaRows);
-        auto issue = [&](int ci) {
-            const uint32_t st = (g + (uint32_t)ci) % kTmaStages;
-            mbar_arrive_expect_tx(&full[st], kTileBytes);
-            tma_load_2d(tiles + st * kTileBytes, &tm, c0, (int32_t)(t0 + (int64_t)ci * kTmaRows), &full[st]);
-        };
-        if (threadIdx.x == 0)
-            for (int ci = 0; ci < nchunks && ci < kTmaStages; ++ci) issue(ci);
-        uint32_t P01 = 0, P23 = 0;
-        if (MODE == 2) {
-            P01 = ((uint32_t)par[ch] << 7) | ((uint32_t)par[ch + 1] << 23);
-            P23 = ((uint32_t)par[ch + 2] << 7) | ((uint32_t)par[ch + 3] << 23);
-        }
-        if (MODE == 3) {
-            P01 = (uint32_t)par[ch] | ((uint32_t)par[ch + 1] << 16);
-            P23 = (uint32_t)par[ch + 2] | ((uint32_t)par[ch + 3] << 16);
-        }
-        uint32_t ge[4] = {0, 0, 0, 0};
-        int ci = 0;
-        for (; ci < nchunks; ++ci) {
-            const uint32_t gi = g + (uint32_t)ci;
-            const uint32_t st = gi % kTmaStages;
-            const bool ok = mbar_wait_bounded(&full[st], (gi / kTmaStages) & 1u, &abort_flag, kWaitNs);
-            const int64_t left = t1 - (t0 + (int64_t)ci * kTmaRows);
-            const uint8_t *tile = tiles + st * kTileBytes + ch * 2;
-            if (ok && left >= kTmaRows) {
-#pragma unroll
-                for (int i = 0; i < kTmaRows / kRS; ++i) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(tile + (warp + i * kRS) * (kSlab * 2));
-                    count_row<MODE>(v.x, v.y, hrow, swap, P01, P23, ge);
-                }
-            } else if (ok) {
-                for (int r = warp; r < (int)left; r += kRS) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(tile + r * (kSlab * 2));
-                    count_row<MODE>(v.x, v.y, hrow, swap, P01, P23, ge);
+        bool ok = true;
+        int issued = 0;
+        if (warp == kConsumers) {
+            // producer: one lane issues every tile of the segment in order
+            if (lane == 0) {
+                for (; issued < nchunks; ++issued) {
+                    const uint32_t gi = g + (uint32_t)issued, st = gi % kTmaStages;
+                    if (gi >= (uint32_t)kTmaStages &&
+                        !mbar_wait_bounded(&empty[st], (gi / kTmaStages - 1u) & 1u, &abort_flag, kWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[st], kTileBytes);
+                    tma_load_2d(tiles + st * kTileBytes, &tm, c0, (int32_t)(t0 + (int64_t)issued * kTmaRows),
+                                &full[st]);
                 }
             }
-            if (__syncthreads_or(!ok)) break;          // slot consumed; on a time-out all leave together
-            if (threadIdx.x == 0 && ci + kTmaStages < nchunks) issue(ci + kTmaStages);
+        } else {
+            uint32_t P01 = 0, P23 = 0;
+            if (MODE == 2) {
+                P01 = ((uint32_t)par[ch] << 7) | ((uint32_t)par[ch + 1] << 23);
+                P23 = ((uint32_t)par[ch + 2] << 7) | ((uint32_t)par[ch + 3] << 23);
+            }
+            if (MODE == 3) {
+                P01 = (uint32_t)par[ch] | ((uint32_t)par[ch + 1] << 16);
+                P23 = (uint32_t)par[ch + 2] | ((uint32_t)par[ch + 3] << 16);
+            }
+            uint32_t ge[4] = {0, 0, 0, 0};
+            for (int ci = 0; ci < nchunks; ++ci) {
+                const uint32_t gi = g + (uint32_t)ci, st = gi % kTmaStages;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(&full[st], (gi / kTmaStages) & 1u, &abort_flag, kWaitNs));
+                if (!ok) break;
+                // rows warp + 16 i of this tile that lie inside the segment
+                const int64_t left = t1 - (t0 + (int64_t)ci * kTmaRows);
+                const int rows_here = left >= kTmaRows ? kTmaRows : (int)left;
+                const int nmine = rows_here > warp ? (rows_here - warp + kConsumers - 1) / kConsumers : 0;
+                const uint32_t valid = (1u << nmine) - 1u;
+                const uint8_t *tile = tiles + st * kTileBytes + ch * 2 + warp * kRowBytes;
+                uint2 v[kRowsPerWarp];
+#pragma unroll
+                for (int i = 0; i < kRowsPerWarp; ++i)
+                    v[i] = *reinterpret_cast<const uint2 *>(tile + i * (kConsumers * kRowBytes));
+                if (MODE == 1) {
+#pragma unroll
+                    for (int i = 0; i < kRowsPerWarp; ++i)
+                        if (valid >> i & 1u) count_row<1>(v[i].x, v[i].y, hrow, swap, P01, P23, ge);
+                } else {
+                    uint32_t marked = 0;
+#pragma unroll
+                    for (int i = 0; i < kRowsPerWarp; ++i)
+                        marked |= (uint32_t)row_candidate<MODE>(v[i].x, v[i].y, P01, P23) << i;
+                    marked &= valid;
+                    while (__any_sync(0xffffffffu, marked != 0u)) {
+                        if (marked) {
+                            const int i = __ffs(marked) - 1;
+                            marked &= marked - 1u;
+                            const uint2 w = *reinterpret_cast<const uint2 *>(tile + i * (kConsumers * kRowBytes));
+                            count_row<MODE>(w.x, w.y, hrow, swap, P01, P23, ge);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+            if (MODE == 3) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (ge[j]) atomicAdd(&ge_s[ch + j], ge[j]);
+            }
         }
-        if (ci < nchunks) {                            // time-out: let issued copies land, flag, stop
-            if (threadIdx.x == 0) {
-                for (int cj = ci; cj < nchunks && cj < ci + kTmaStages; ++cj) {
+        if (__syncthreads_or(!ok)) {                   // time-out: let issued copies land, flag, stop
+            if (warp == kConsumers && lane == 0) {
+                for (int cj = issued - kTmaStages < 0 ? 0 : issued - kTmaStages; cj < issued; ++cj) {
                     const uint32_t gj = g + (uint32_t)cj;
                     mbar_wait_bounded(&full[gj % kTmaStages], (gj / kTmaStages) & 1u, nullptr, 100000000ull);
                 }
@@ -400,23 +462,17 @@ __global__ void __launch_bounds__(kThreads) k_pass_tma(const __grid_constant__ C
             return;
         }
         g += (uint32_t)nchunks;
-        if (MODE == 3) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (ge[j]) atomicAdd(&ge_s[ch + j], ge[j]);
-        }
-        __syncthreads();
         uint32_t *gh = MODE == 1 ? a.hist1 : MODE == 2 ? a.hist2 : a.whist;
-        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kThreads) {
-            const uint32_t v = h[i];
-            if (!v) continue;
+        for (int i = threadIdx.x; i < NB * kSlab / 2; i += kTmaThreads) {
+            const uint32_t hv = h[i];
+            if (!hv) continue;
             const int bin = i / (kSlab / 2), wi = i % (kSlab / 2);
             const int c = c0 + 4 * (wi >> 1) + 2 * (wi & 1);
-            if ((v & 0xFFFFu) && c < a.C) atomicAdd(&gh[(size_t)c * NB + bin], v & 0xFFFFu);
-            if ((v >> 16) && c + 1 < a.C) atomicAdd(&gh[(size_t)(c + 1) * NB + bin], v >> 16);
+            if ((hv & 0xFFFFu) && c < a.C) atomicAdd(&gh[(size_t)c * NB + bin], hv & 0xFFFFu);
+            if ((hv >> 16) && c + 1 < a.C) atomicAdd(&gh[(size_t)(c + 1) * NB + bin], hv >> 16);
         }
         if (MODE == 3)
-            for (int j = threadIdx.x; j < kSlab; j += kThreads)
+            for (int j = threadIdx.x; j < kSlab; j += kTmaThreads)
                 if (ge_s[j] && c0 + j < a.C) atomicAdd(&a.ge[c0 + j], ge_s[j]);
     }
 }
@@ -630,13 +686,13 @@ hif4_status launch_pass_tma(const PassArgs &a0, cudaStream_t s, bool &done)
     PassArgs a = a0;
     // equal shares of the slab-major (slab, row) space, one block per
     // resident slot, 4..65535 tiles' worth of rows each
-    const int64_t slots = (int64_t)blocks_per_sm(reinterpret_cast<const void *>(k), kThreads, smem) * sm_count();
+    const int64_t slots = (int64_t)blocks_per_sm(reinterpret_cast<const void *>(k), kTmaThreads, smem) * sm_count();
     const int64_t total = (int64_t)a.nslab * a.T;
     int64_t share = (total + slots - 1) / slots;
     if (share < 4 * kTmaRows) share = 4 * kTmaRows;
     if (share > kMaxRowsPerBlock) share = kMaxRowsPerBlock;
     a.rows_per_split = share;
-    k<<<(int)((total + share - 1) / share), kThreads, smem, s>>>(tm, a);
+    k<<<(int)((total + share - 1) / share), kTmaThreads, smem, s>>>(tm, a);
     done = true;
     return launch_status();
 }
