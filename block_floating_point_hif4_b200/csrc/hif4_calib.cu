@@ -522,6 +522,10 @@ __global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint16
 
 constexpr int kMaskThreads = 1024;
 constexpr int kKeys = 32768;
+// Key histogram slot with one pad word per 32 keys: thread t's 32 consecutive
+// keys then sit in 32 different banks across a warp.
+constexpr int kKeySlots = kKeys + kKeys / 32;
+__device__ __forceinline__ int key_slot(uint32_t key) { return (int)(key + (key >> 5)); }
 
 // Block-wide exclusive scan of one value per thread (1024 threads).
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratch, uint32_t &total)
@@ -557,7 +561,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratc
 __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int C, uint32_t n_top, float *ratio,
                                                       uint8_t *mask, int32_t *mask_idx, const uint32_t *timed_out)
 {
-    extern __shared__ uint32_t hist[];                 // [kKeys]
+    extern __shared__ uint32_t hist[];                 // [kKeySlots]
     if (*timed_out) {                                  // block-uniform
         for (int c = threadIdx.x; c < C; c += kMaskThreads) {
             ratio[c] = __int_as_float(0x7FC00000);
@@ -569,15 +573,15 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
     }
     __shared__ uint32_t scratch[72];
     __shared__ uint32_t sel[4];                        // med key, tau key, count above tau
-    for (int i = threadIdx.x; i < kKeys; i += kMaskThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < kKeySlots; i += kMaskThreads) hist[i] = 0;
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += kMaskThreads) atomicAdd(&hist[pct[c] & 0x7FFFu], 1u);
+    for (int c = threadIdx.x; c < C; c += kMaskThreads) atomicAdd(&hist[key_slot(pct[c] & 0x7FFFu)], 1u);
     __syncthreads();
 
     // each thread owns 32 consecutive keys
     constexpr int PER = kKeys / kMaskThreads;
     uint32_t local = 0;
-    for (int i = 0; i < PER; ++i) local += hist[threadIdx.x * PER + i];
+    for (int i = 0; i < PER; ++i) local += hist[threadIdx.x * (PER + 1) + i];
     uint32_t total;
     const uint32_t excl = block_excl_scan(local, scratch, total);
     const uint32_t r_med = (uint32_t)(C - 1) / 2u;
@@ -585,7 +589,7 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
     {
         uint32_t run = excl;
         for (int i = 0; i < PER; ++i) {
-            const uint32_t cnt = hist[threadIdx.x * PER + i];
+            const uint32_t cnt = hist[threadIdx.x * (PER + 1) + i];
             const uint32_t key = (uint32_t)(threadIdx.x * PER + i);
             if (cnt && run <= r_med && r_med < run + cnt) sel[0] = key;
             if (n_top && cnt && run <= r_tau && r_tau < run + cnt) {
@@ -840,12 +844,12 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     int dev = 0;
     cudaGetDevice(&dev);
     if (!mattr[dev & 63]) {
-        if (cudaFuncSetAttribute(k_mask, cudaFuncAttributeMaxDynamicSharedMemorySize, kKeys * 4) != cudaSuccess)
+        if (cudaFuncSetAttribute(k_mask, cudaFuncAttributeMaxDynamicSharedMemorySize, kKeySlots * 4) != cudaSuccess)
             return HIF4_ERR_CUDA;
         mattr[dev & 63] = true;
     }
     const uint32_t n_top = (uint32_t)(((uint64_t)channels * mask_num) / mask_den);
-    k_mask<<<1, kMaskThreads, kKeys * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
+    k_mask<<<1, kMaskThreads, kKeySlots * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
                                              mask_idx_out, timed_out);
     return launch_status();
 }
