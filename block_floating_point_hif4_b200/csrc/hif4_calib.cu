@@ -11,7 +11,7 @@
 //
 // Pipeline (all on the device, one stream):
 //   1. sample  — the exact order statistic, per channel, of a row sample
-//                (about 8192 rows) at four times the target's tail mass
+//                (about 4096 rows) at four times the target's tail mass
 //                below the top, by a two-pass radix select (pass 1: key >> 7,
 //                the exponent byte; pass 2: key & 127 inside the bin that
 //                holds the rank);
@@ -262,11 +262,12 @@ __global__ void k_select1(const uint32_t *hist1, int C, uint32_t k, uint16_t *tb
 // wait on one another inside a segment and up to 160 KB per SM stay in
 // flight.  A consumer warp takes rows warp, warp + 16, ... (8 per tile): it
 // loads them all first (8-byte shared loads, 256 contiguous bytes per warp).
-// Pass 1 counts every key.  Passes 2 and 3 count few keys (those in the
-// target bin, those at or above the window start), so each lane first
-// marks its rows holding a candidate (a cheap superset test), then the warp
-// visits marked rows one per lane per round: the count is paid per marked
-// row instead of per divergent row.
+// Passes 1 and 2 count every row with straight-line predicated atomics (the
+// bin that holds the target often holds several percent of the keys).  The
+// window pass counts few keys (those at or above the window start), so each
+// lane first marks its rows holding one (a cheap superset test), then the
+// warp visits marked rows one per lane per round: the count is paid per
+// marked row instead of per divergent row.
 //
 // Work split: one block per SM; block b takes units [b share, (b+1) share)
 // of the slab-major space u = slab * T + row, so all blocks carry equal
@@ -284,25 +285,35 @@ constexpr uint32_t kRowBytes = kSlab * 2;
 constexpr uint32_t kTileBytes = kTmaRows * kRowBytes;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
+// Shared counter layout of the TMA passes: [bin][64 words], word
+// 2 l + col of lane l holding two 16-bit counts.  Lanes below 16 keep
+// channels 4l, 4l+1 in col 0 and 4l+2, 4l+3 in col 1; lanes from 16 on keep
+// them the other way round, so that lanes l and l + 16 (same bank pair) hit
+// different banks in every counting instruction.
+__device__ __forceinline__ int slot_channel(int wi)
+{
+    const int l = wi >> 1;
+    return 4 * l + 2 * ((wi & 1) ^ (l >= 16 ? 1 : 0));
+}
+
 // One row's four keys of this lane (words w01 = channels ch, ch+1 and
-// w23 = ch+2, ch+3) into the shared counters.
+// w23 = ch+2, ch+3) into the shared counters (h01 / h23: this lane's
+// columns for the two words).
 template <int MODE>
-__device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *hrow, uint32_t swap, uint32_t P01,
+__device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *h01, uint32_t *h23, uint32_t P01,
                                           uint32_t P23, uint32_t (&ge)[4])
 {
     if (MODE == 1) {
-        const uint32_t wa = swap ? w23 : w01, wb = swap ? w01 : w23;
-        const uint32_t ha = swap, hb = swap ^ 1u;
-        atomicAdd(hrow + ((wa >> 7) & 0xFFu) * (kSlab / 2) + ha, 1u);
-        atomicAdd(hrow + ((wa >> 23) & 0xFFu) * (kSlab / 2) + ha, 0x10000u);
-        atomicAdd(hrow + ((wb >> 7) & 0xFFu) * (kSlab / 2) + hb, 1u);
-        atomicAdd(hrow + ((wb >> 23) & 0xFFu) * (kSlab / 2) + hb, 0x10000u);
+        atomicAdd(h01 + ((w01 >> 7) & 0xFFu) * (kSlab / 2), 1u);
+        atomicAdd(h01 + ((w01 >> 23) & 0xFFu) * (kSlab / 2), 0x10000u);
+        atomicAdd(h23 + ((w23 >> 7) & 0xFFu) * (kSlab / 2), 1u);
+        atomicAdd(h23 + ((w23 >> 23) & 0xFFu) * (kSlab / 2), 0x10000u);
     } else if (MODE == 2) {
         const uint32_t x01 = (w01 & 0x7F807F80u) ^ P01, x23 = (w23 & 0x7F807F80u) ^ P23;
-        if (!(x01 & 0xFFFFu)) atomicAdd(hrow + (w01 & 127u) * (kSlab / 2), 1u);
-        if (!(x01 >> 16)) atomicAdd(hrow + ((w01 >> 16) & 127u) * (kSlab / 2), 0x10000u);
-        if (!(x23 & 0xFFFFu)) atomicAdd(hrow + (w23 & 127u) * (kSlab / 2) + 1, 1u);
-        if (!(x23 >> 16)) atomicAdd(hrow + ((w23 >> 16) & 127u) * (kSlab / 2) + 1, 0x10000u);
+        if (!(x01 & 0xFFFFu)) atomicAdd(h01 + (w01 & 127u) * (kSlab / 2), 1u);
+        if (!(x01 >> 16)) atomicAdd(h01 + ((w01 >> 16) & 127u) * (kSlab / 2), 0x10000u);
+        if (!(x23 & 0xFFFFu)) atomicAdd(h23 + (w23 & 127u) * (kSlab / 2), 1u);
+        if (!(x23 >> 16)) atomicAdd(h23 + ((w23 >> 16) & 127u) * (kSlab / 2), 0x10000u);
     } else {
         // D = (w | 0x80008000) - P: bit 15 of each half is set iff that key
         // >= lo, the half then holding 0x8000 + (key - lo)
@@ -312,23 +323,17 @@ __device__ __forceinline__ void count_row(uint32_t w01, uint32_t w23, uint32_t *
         for (int j = 0; j < 4; ++j) {
             const uint32_t off = d[j] - 0x8000u;
             ge[j] += off < 0x8000u;
-            if (off < (uint32_t)kWinBins) atomicAdd(hrow + off * (kSlab / 2) + (j >> 1), 1u << (16 * (j & 1)));
+            if (off < (uint32_t)kWinBins)
+                atomicAdd((j < 2 ? h01 : h23) + off * (kSlab / 2), 1u << (16 * (j & 1)));
         }
     }
 }
 
-// Superset test for a row that count_row<MODE> (2 or 3) may count: true
-// whenever it counts something.
-template <int MODE>
+// Superset test for a row that the window count may count: true whenever
+// some key of the row is at or above its channel's window start.
 __device__ __forceinline__ bool row_candidate(uint32_t w01, uint32_t w23, uint32_t P01, uint32_t P23)
 {
-    if (MODE == 2) {
-        // a 16-bit half of x is zero (bit 15 of every half of x is clear)
-        const uint32_t x01 = (w01 & 0x7F807F80u) ^ P01, x23 = (w23 & 0x7F807F80u) ^ P23;
-        return (((x01 - 0x00010001u) | (x23 - 0x00010001u)) & 0x80008000u) != 0u;
-    } else {
-        return ((((w01 | 0x80008000u) - P01) | ((w23 | 0x80008000u) - P23)) & 0x80008000u) != 0u;
-    }
+    return ((((w01 | 0x80008000u) - P01) | ((w23 | 0x80008000u) - P23)) & 0x80008000u) != 0u;
 }
 
 template <int MODE>
@@ -345,8 +350,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
     __shared__ uint32_t abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ch = 4 * lane;
-    const uint32_t swap = lane >= 16 ? 1u : 0u;
-    uint32_t *hrow = h + 2 * lane;
+    uint32_t *h01 = h + 2 * lane + (lane >= 16 ? 1 : 0);
+    uint32_t *h23 = h + 2 * lane + (lane >= 16 ? 0 : 1);
 
     const int64_t total = (int64_t)a.nslab * a.T;
     int64_t cur = (int64_t)blockIdx.x * a.rows_per_split;
@@ -423,22 +428,22 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
 #pragma unroll
                 for (int i = 0; i < kRowsPerWarp; ++i)
                     v[i] = *reinterpret_cast<const uint2 *>(tile + i * (kConsumers * kRowBytes));
-                if (MODE == 1) {
+                if (MODE != 3) {
 #pragma unroll
                     for (int i = 0; i < kRowsPerWarp; ++i)
-                        if (valid >> i & 1u) count_row<1>(v[i].x, v[i].y, hrow, swap, P01, P23, ge);
+                        if (valid >> i & 1u) count_row<MODE>(v[i].x, v[i].y, h01, h23, P01, P23, ge);
                 } else {
                     uint32_t marked = 0;
 #pragma unroll
                     for (int i = 0; i < kRowsPerWarp; ++i)
-                        marked |= (uint32_t)row_candidate<MODE>(v[i].x, v[i].y, P01, P23) << i;
+                        marked |= (uint32_t)row_candidate(v[i].x, v[i].y, P01, P23) << i;
                     marked &= valid;
                     while (__any_sync(0xffffffffu, marked != 0u)) {
                         if (marked) {
                             const int i = __ffs(marked) - 1;
                             marked &= marked - 1u;
                             const uint2 w = *reinterpret_cast<const uint2 *>(tile + i * (kConsumers * kRowBytes));
-                            count_row<MODE>(w.x, w.y, hrow, swap, P01, P23, ge);
+                            count_row<MODE>(w.x, w.y, h01, h23, P01, P23, ge);
                         }
                     }
                 }
@@ -466,8 +471,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
         for (int i = threadIdx.x; i < NB * kSlab / 2; i += kTmaThreads) {
             const uint32_t hv = h[i];
             if (!hv) continue;
-            const int bin = i / (kSlab / 2), wi = i % (kSlab / 2);
-            const int c = c0 + 4 * (wi >> 1) + 2 * (wi & 1);
+            const int bin = i / (kSlab / 2);
+            const int c = c0 + slot_channel(i % (kSlab / 2));
             if ((hv & 0xFFFFu) && c < a.C) atomicAdd(&gh[(size_t)c * NB + bin], hv & 0xFFFFu);
             if ((hv >> 16) && c + 1 < a.C) atomicAdd(&gh[(size_t)(c + 1) * NB + bin], hv >> 16);
         }
@@ -781,9 +786,9 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     const int fgrid = (int)((channels * 32 + 255) / 256);
     hif4_status st;
 
-    // 1. window start: exact order statistic of every R-th row (about 8192
+    // 1. window start: exact order statistic of every R-th row (about 4096
     //    rows) at four times the target's tail mass below the top
-    const int64_t R = tokens / 8192 > 1 ? tokens / 8192 : 1;
+    const int64_t R = tokens / 4096 > 1 ? tokens / 4096 : 1;
     const int64_t Ts = (tokens + R - 1) / R;
     const uint64_t tail = ((uint64_t)(tokens - kk) * 4ull * (uint64_t)Ts + (uint64_t)tokens - 1) / (uint64_t)tokens;
     const uint32_t r_lo = (uint32_t)((uint64_t)Ts > tail + 1 ? (uint64_t)Ts - 1 - tail : 0);
