@@ -26,10 +26,12 @@
 //                depends on the sample;
 //   5. mask    — one block: median, ratios, top-n by (key desc, index asc).
 //
-// Streaming passes share one shape: a block owns a 128-channel slab and a
-// token range of at most 65535 rows (16-bit shared counters); a lane owns 4
-// channels and reads them with one 8-byte load per row; full iterations keep
-// 16 rows in flight with no bounds checks.
+// Streaming passes count keys of a 128-channel slab into 16-bit shared
+// counters (a lane owns 4 channels).  When the rows start on 16-byte
+// boundaries they run as k_pass_tma: TMA-staged tiles, a producer warp, one
+// block per SM over equal shares of the slab-major row space.  Otherwise
+// (2- or 8-byte aligned rows) they run as k_pass: plain loads, a block per
+// (slab, token range of at most 65535 rows), 16 rows in flight per warp.
 #include <cuda_bf16.h>
 
 #include "hif4_internal.cuh"
