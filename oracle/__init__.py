@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.orc_weight_hat.argtypes = [P, P, i64, i64, P, ctypes.c_int, P, P]
             L.orc_gelu_tanh.restype = ctypes.c_double
             L.orc_gelu_tanh.argtypes = [ctypes.c_double]
+            L.orc_round_bf16.restype = ctypes.c_uint16
+            L.orc_round_bf16.argtypes = [ctypes.c_double]
+            L.orc_round_bf16_array.restype = None
+            L.orc_round_bf16_array.argtypes = [P, i64, P]
             L.orc_linear.restype = None
             L.orc_linear.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, P]
             L.orc_percentile.restype = ctypes.c_int
@@ -175,6 +179,14 @@ def weight_hat(codes, meta, N, K, mask_idx=None, w_masked_bf16=None) -> np.ndarr
 
 def gelu_tanh(x: float) -> float:
     return lib().orc_gelu_tanh(float(x))
+
+
+def round_bf16(x) -> np.ndarray:
+    """double array -> BF16 bit patterns (uint16), one round-to-nearest-even step."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.zeros(x.shape, np.uint16)
+    lib().orc_round_bf16_array(_p(x), x.size, _p(out))
+    return out
 
 
 def linear(xhat: np.ndarray, what: np.ndarray, bias=None, gelu: bool = False,

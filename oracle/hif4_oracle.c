@@ -289,6 +289,37 @@ double orc_gelu_tanh(double x)
     return 0.5 * x * (1.0 + tanh(k * (x + 0.044715 * x * x * x)));
 }
 
+/* double -> BF16 bit pattern in one rounding: to nearest, ties to even (no
+ * intermediate FP32 rounding) [reading: the FFN's hidden activation is held
+ * in BF16 between the two linears].  BF16 keeps 8 significant bits, so the
+ * quantum is 2^(e-8) for |x| = m 2^e (m in [0.5, 1)), and 2^-133 below the
+ * normal range.  Magnitudes at or above the midpoint past the largest finite
+ * BF16 value go to Inf; NaN gives the quiet NaN with the input's sign. */
+uint16_t orc_round_bf16(double x)
+{
+    if (isnan(x)) return signbit(x) ? 0xFFC0u : 0x7FC0u;
+    const uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return sign | 0x7F80u;
+    int e;
+    frexp(a, &e);
+    int qe = e - 8;
+    if (qe < -133) qe = -133;
+    const double q = ldexp(1.0, qe);
+    const double r = nearbyint(a / q) * q;          /* a / q exact; default mode = ties to even */
+    if (r > ldexp(255.0, 120)) return sign | 0x7F80u;
+    const float f = (float)r;                        /* exact: r is a BF16 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return sign | (uint16_t)(u >> 16);
+}
+
+void orc_round_bf16_array(const double *x, long n, uint16_t *out)
+{
+    for (long i = 0; i < n; ++i) out[i] = orc_round_bf16(x[i]);
+}
+
 /* Fake-quantized linear layer [TA abstract]:  y = xhat * what^T + bias,
  * summed in double;  with gelu != 0 the GELU above is applied to each output.
  *   xhat M x K, what N x K, bias N or NULL, y M x N (all dense, row-major). */
