@@ -24,6 +24,7 @@ F32, BF16 = 0, 1
 FLAG_NONFINITE, FLAG_TIMEOUT, FLAG_BAD_INDEX = 1, 2, 4
 LINEAR_GELU_TANH = 1
 LINEAR_OUT_F32 = 2
+LINEAR_FAKE_QUANT_OUT = 4
 
 # (name, restype, argtypes) of every exported entry point
 _P, _I64, _U32, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_size_t
@@ -36,6 +37,10 @@ SIGNATURES = {
                                         _U32, _P, _SZ, _P, _P]),
     "hif4_weight_decode": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I32, _P, _P, _I64, _P, _P]),
     "hif4_gemm_bf16": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P, _I64, _U32, _P, _P]),
+    "hif4_gemm_bf16_fq": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P, _P, _I64, _U32, _P, _P]),
+    "hif4_ffn_w4a4_workspace": (_SZ, [_I64, _I64, _I64]),
+    "hif4_ffn_w4a4": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
+                                     _P, _P, _I64, _U32, _P, _SZ, _P, _P]),
     "hif4_calib_workspace": (_SZ, [_I64, _I64]),
     "hif4_calib_percentile_mask": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P, _P,
                                                   _P, _P, _SZ, _P]),
@@ -194,6 +199,54 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None
     _check("hif4_gemm_bf16", lib().hif4_gemm_bf16(
         _ptr(a), M, K, a.stride(0), _ptr(b), N, b.stride(0), _ptr(bias), _ptr(out), out.stride(0),
         flags, _ptr(status), _stream(stream)))
+    return out
+
+
+def gemm_bf16_fq(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None, gelu: bool = False,
+                 out_chan_mask: torch.Tensor | None = None, *, out=None, status=None, stream=None):
+    """hfq = fakequant(bf16(a · bᵀ + bias), optionally GELU'd) along N in the
+    GEMM epilogue; out_chan_mask (u8 [N], nonzero = protected) columns kept."""
+    _dev(a, "a")
+    assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16 and a.stride(1) == 1 and b.stride(1) == 1
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    flags = LINEAR_GELU_TANH if gelu else 0
+    _check("hif4_gemm_bf16_fq", lib().hif4_gemm_bf16_fq(
+        _ptr(a), M, K, a.stride(0), _ptr(b), N, b.stride(0), _ptr(bias), _ptr(out_chan_mask), _ptr(out),
+        out.stride(0), flags, _ptr(status), _stream(stream)))
+    return out
+
+
+def ffn_w4a4_workspace(M: int, D: int, F: int) -> int:
+    return int(lib().hif4_ffn_w4a4_workspace(M, D, F))
+
+
+def ffn_w4a4(x: torch.Tensor, w1_codes: torch.Tensor, w1_meta: torch.Tensor, F: int,
+             w2_codes: torch.Tensor, w2_meta: torch.Tensor,
+             mask1_idx: torch.Tensor | None = None, w1_masked: torch.Tensor | None = None,
+             b1: torch.Tensor | None = None, mask2_idx: torch.Tensor | None = None,
+             w2_masked: torch.Tensor | None = None, b2: torch.Tensor | None = None, *, out=None,
+             workspace=None, status=None, stream=None):
+    """y = fq(gelu(fq(x) · ŵ1ᵀ + b1)) · ŵ2ᵀ + b2, the W4A4 HiF4 FFN block (BF16 or FP32 out)."""
+    _dev(x, "x")
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, D = x.shape
+    if out is None:
+        out = torch.empty(M, D, dtype=torch.bfloat16, device=x.device)
+    need = ffn_w4a4_workspace(M, D, F)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    n1 = 0 if mask1_idx is None else int(mask1_idx.numel())
+    n2 = 0 if mask2_idx is None else int(mask2_idx.numel())
+    flags = LINEAR_OUT_F32 if out.dtype == torch.float32 else 0
+    _check("hif4_ffn_w4a4", lib().hif4_ffn_w4a4(
+        _ptr(x), M, D, x.stride(0), _ptr(w1_codes), _ptr(w1_meta), F, _ptr(mask1_idx) if n1 else None, n1,
+        _ptr(w1_masked) if n1 else None, _ptr(b1), _ptr(w2_codes), _ptr(w2_meta),
+        _ptr(mask2_idx) if n2 else None, n2, _ptr(w2_masked) if n2 else None, _ptr(b2), _ptr(out),
+        out.stride(0), flags, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
     return out
 
 

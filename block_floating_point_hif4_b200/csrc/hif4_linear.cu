@@ -16,13 +16,16 @@
 //   warp 1      allocates 512 TMEM columns (two 128x256 FP32 accumulators)
 //               and issues tcgen05.mma (M=128, N=256, K=16) from one thread;
 //   warps 2-5   epilogue: tcgen05.ld of its 32-lane quarter, + bias,
-//               optional tanh-GELU, BF16 round-to-nearest-even, global store;
-//               it drains one accumulator while the next tile accumulates.
+//               optional tanh-GELU, BF16 round-to-nearest-even, optional
+//               HiF4 fake quantization of the row's 64-column units, global
+//               store; it drains one accumulator while the next tile
+//               accumulates.
 // Every mbarrier wait is bounded; a wait that gives up sets the block's abort
 // flag, the others leave their loops, TMEM is freed and HIF4_FLAG_TIMEOUT is
 // raised in the status word.
 #include <cuda_bf16.h>
 
+#include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
 #include "hif4_sm100.cuh"
 
@@ -54,6 +57,7 @@ struct Args {
     void *y;                // BF16 (or F32 with HIF4_LINEAR_OUT_F32) M x N, leading dimension ldy
     int64_t ldy;
     uint32_t flags;
+    const uint8_t *out_mask;  // HIF4_LINEAR_FAKE_QUANT_OUT: u8 [N] protected output columns, or null
     uint32_t *status;
     uint64_t timeout_ns;
 };
@@ -69,17 +73,49 @@ __device__ __forceinline__ void tile_coords(int t, const Args &g, int &mb, int &
     nb = r / gm;
 }
 
-__device__ __forceinline__ float tanh_approx(float x)
-{
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
+// tanh-form GELU, 0.5 x (1 + tanh(u)) with u = sqrt(2/pi) (x + 0.044715 x^3),
+// evaluated as the identical x / (1 + exp(-2u)): expf and a correctly
+// rounded division keep it within a few FP32 ulps, so the BF16 rounding of
+// the result (and any re-quantization of it) rarely differs from the exact
+// function.  Large |x|: exp overflows to +Inf for x -> -inf (result -0) and
+// underflows to 0 for x -> +inf (result x).
 __device__ __forceinline__ float gelu_tanh(float x)
 {
     const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
-    return 0.5f * x * (1.0f + tanh_approx(u));
+    return __fdiv_rn(x, 1.0f + expf(-2.0f * u));
+}
+
+// 32 accumulator columns of one row -> + bias (BF16, 16-byte aligned, or
+// null) -> optional tanh-GELU -> 16 packed BF16 pairs (round to nearest
+// even; column 2j in the low half of w[j]).
+__device__ __forceinline__ void epi_pack32(const uint32_t (&r)[32], const uint16_t *bias, bool gelu,
+                                           uint32_t *w)
+{
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    if (bias) {
+        const uint4 *bp = reinterpret_cast<const uint4 *>(bias);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 b = __ldg(bp + i);
+            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                v[8 * i + 2 * h] += __uint_as_float(bw[h] << 16);
+                v[8 * i + 2 * h + 1] += __uint_as_float(bw[h] & 0xFFFF0000u);
+            }
+        }
+    }
+    if (gelu) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t *>(&h2);
+    }
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -204,6 +240,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
         const bool out_f32 = (g.flags & HIF4_LINEAR_OUT_F32) != 0;
+        const bool fq_out = (g.flags & HIF4_LINEAR_FAKE_QUANT_OUT) != 0;
+        uint32_t nonfinite = 0;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
             int mb, nb;
@@ -213,8 +251,56 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             const int row = mb * BM + q * 32 + lane;
             uint16_t *yrow = static_cast<uint16_t *>(g.y) + (int64_t)row * g.ldy;
             float *yrow32 = static_cast<float *>(g.y) + (int64_t)row * g.ldy;
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            // HiF4 fake-quant of the output along N: a thread holds whole
+            // 64-column units of its row (N % 64 == 0), so every unit
+            // decision is thread-local.
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int u = 0; fq_out && u < BN / 64; ++u) {
+                const int n0 = nb * BN + u * 64;
+                if (n0 >= g.N) break;                          // warp-uniform
+                uint32_t w[32];
+                {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tacc + u * 64, r);
+                    tmem_ld_wait();
+                    epi_pack32(r, g.bias ? g.bias + n0 : nullptr, gelu, w);
+                    tmem_ld_32x32b_x32(tacc + u * 64 + 32, r);
+                    tmem_ld_wait();
+                    epi_pack32(r, g.bias ? g.bias + n0 + 32 : nullptr, gelu, w + 16);
+                }
+                uint32_t out[32];
+                uint32_t mraw[16];
+                uint32_t any = 0;
+                if (g.out_mask) {
+                    const uint4 *mp = reinterpret_cast<const uint4 *>(g.out_mask + n0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 m = __ldg(mp + i);
+                        mraw[4 * i] = m.x;
+                        mraw[4 * i + 1] = m.y;
+                        mraw[4 * i + 2] = m.z;
+                        mraw[4 * i + 3] = m.w;
+                        any |= m.x | m.y | m.z | m.w;
+                    }
+                }
+                if (any) {                                     // warp-uniform: same columns
+                    uint32_t mw[32];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) enc::mask_words16(mraw + 4 * i, mw + 8 * i);
+                    enc::fq_unit64<true>(w, mw, out, nonfinite);
+                } else {
+                    enc::fq_unit64<false>(w, w, out, nonfinite);
+                }
+                if (row < g.M) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+                }
+            }
+#pragma unroll 1
+            for (int c = 0; !fq_out && c < BN / 32; ++c) {
                 const int n0 = nb * BN + c * 32;
                 if (n0 >= g.N) break;                          // warp-uniform
                 uint32_t r[32];
@@ -286,6 +372,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             acc ^= 1u;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (nonfinite) status_or(g.status, HIF4_FLAG_NONFINITE);
     }
 
     tc_fence_before();
@@ -356,7 +443,8 @@ namespace hif4 {
 namespace {
 
 hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N, int64_t ldb,
-                        const void *bias, void *y, int64_t ldy, uint32_t flags, uint32_t *status, cudaStream_t s)
+                        const void *bias, const uint8_t *out_mask, void *y, int64_t ldy, uint32_t flags,
+                        uint32_t *status, cudaStream_t s)
 {
     using namespace gemm;
     CUtensorMap tmA, tmB;
@@ -373,6 +461,7 @@ hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const 
     g.y = y;
     g.ldy = ldy;
     g.flags = flags;
+    g.out_mask = out_mask;
     g.status = status;
     g.timeout_ns = TIMEOUT_NS;
     static bool attr_set[64] = {false};
@@ -397,7 +486,12 @@ hif4_status check_gemm_args(const void *a, int64_t M, int64_t K, int64_t lda, co
     if (M == 0 || N == 0) return HIF4_OK;
     if (K == 0) return HIF4_ERR_SHAPE;
     if (!a || !b || !y) return HIF4_ERR_INVALID_ARG;
-    if (flags & ~(HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_OUT_F32)) return HIF4_ERR_INVALID_ARG;
+    if (flags & ~(HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_OUT_F32 | HIF4_LINEAR_FAKE_QUANT_OUT))
+        return HIF4_ERR_INVALID_ARG;
+    if (flags & HIF4_LINEAR_FAKE_QUANT_OUT) {
+        if (flags & HIF4_LINEAR_OUT_F32) return HIF4_ERR_INVALID_ARG;   // fake quant writes BF16
+        if (N % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
+    }
     if (lda < K || ldb < K || ldy < N) return HIF4_ERR_SHAPE;
     if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2) return HIF4_ERR_UNSUPPORTED;
     const int64_t ysz = (flags & HIF4_LINEAR_OUT_F32) ? 4 : 2;
@@ -416,7 +510,21 @@ extern "C" hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64
 {
     hif4_status st = check_gemm_args(a, M, K, lda, b, N, ldb, bias, y, ldy, flags);
     if (st != HIF4_OK || M == 0 || N == 0) return st;
-    return launch_gemm(a, M, K, lda, b, N, ldb, bias, y, ldy, flags, status, reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemm(a, M, K, lda, b, N, ldb, bias, nullptr, y, ldy, flags, status,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" hif4_status hif4_gemm_bf16_fq(const void *a, int64_t M, int64_t K, int64_t lda, const void *b,
+                                         int64_t N, int64_t ldb, const void *bias, const uint8_t *out_chan_mask,
+                                         void *y, int64_t ldy, uint32_t flags, uint32_t *status,
+                                         hif4_stream_t stream)
+{
+    flags |= HIF4_LINEAR_FAKE_QUANT_OUT;
+    hif4_status st = check_gemm_args(a, M, K, lda, b, N, ldb, bias, y, ldy, flags);
+    if (st != HIF4_OK || M == 0 || N == 0) return st;
+    if (out_chan_mask && !aligned16(out_chan_mask)) return HIF4_ERR_ALIGNMENT;
+    return launch_gemm(a, M, K, lda, b, N, ldb, bias, out_chan_mask, y, ldy, flags, status,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" hif4_status hif4_weight_decode(const uint8_t *w_codes, const uint32_t *w_meta, int64_t N, int64_t K,
@@ -456,6 +564,7 @@ extern "C" hif4_status hif4_linear_w4a4(const void *x, int64_t M, int64_t K, int
                                         hif4_stream_t stream)
 {
     if (n_masked < 0) return HIF4_ERR_INVALID_ARG;
+    if (flags & HIF4_LINEAR_FAKE_QUANT_OUT) return HIF4_ERR_INVALID_ARG;   // needs an output mask: hif4_ffn_w4a4
     hif4_status st = check_gemm_args(x, M, K, ldx, x, N, K, bias, y, ldy, flags);
     if (st != HIF4_OK || M == 0 || N == 0) return st;
     if (!w_codes || !w_meta) return HIF4_ERR_INVALID_ARG;
@@ -488,5 +597,97 @@ extern "C" hif4_status hif4_linear_w4a4(const void *x, int64_t M, int64_t K, int
     st = hif4_weight_decode(w_codes, w_meta, N, K, mask_idx, n_masked, w_masked, what, K, status, stream);
     if (st != HIF4_OK) return st;
     // 4. tcgen05 GEMM + bias (+ GELU)
-    return launch_gemm(xhat, M, K, K, what, N, K, bias, y, ldy, flags, status, s);
+    return launch_gemm(xhat, M, K, K, what, N, K, bias, nullptr, y, ldy, flags, status, s);
+}
+
+// ----------------------------------------------------------------- FFN block
+//
+//   H    = gelu_tanh(xhat1 * what1^T + b1)   rounded to BF16,
+//   Hhat = HiF4 fake quantization of H along F (mask2 columns kept),
+//   y    = Hhat * what2^T + b2,
+// with xhat1 the fake quantization of x along D (mask1 columns kept) and
+// what1 / what2 the decoded weights (protected columns restored).  The
+// second activation's fake quantization runs inside the first GEMM's
+// epilogue, so H never goes through HBM unquantized.
+// Workspace: xhat1 M x D | what1 F x D | Hhat M x F | what2 D x F (BF16) |
+// mask1 D | mask2 F (u8), each 256-byte aligned.
+
+extern "C" size_t hif4_ffn_w4a4_workspace(int64_t M, int64_t D, int64_t F)
+{
+    if (M <= 0 || D <= 0 || F <= 0) return 0;
+    return align256((size_t)M * D * 2) + align256((size_t)F * D * 2) + align256((size_t)M * F * 2) +
+           align256((size_t)D * F * 2) + align256((size_t)D) + align256((size_t)F);
+}
+
+extern "C" hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_t ldx,
+                                     const uint8_t *w1_codes, const uint32_t *w1_meta, int64_t F,
+                                     const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked,
+                                     const void *b1, const uint8_t *w2_codes, const uint32_t *w2_meta,
+                                     const int32_t *mask2_idx, int32_t n_mask2, const void *w2_masked,
+                                     const void *b2, void *y, int64_t ldy, uint32_t flags, void *workspace,
+                                     size_t ws_bytes, uint32_t *status, hif4_stream_t stream)
+{
+    if (n_mask1 < 0 || n_mask2 < 0) return HIF4_ERR_INVALID_ARG;
+    if (flags & ~HIF4_LINEAR_OUT_F32) return HIF4_ERR_INVALID_ARG;
+    if (M < 0 || D < 0 || F < 0) return HIF4_ERR_INVALID_ARG;
+    if (D % HIF4_UNIT != 0 || F % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
+    if (M == 0) return HIF4_OK;
+    if (D == 0 || F == 0) return HIF4_ERR_SHAPE;
+    // first GEMM (x -> Hhat) and second GEMM (Hhat -> y) shapes and pointers
+    hif4_status st = check_gemm_args(x, M, D, ldx, x, F, D, b1, x, F,
+                                     HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT);
+    if (st != HIF4_OK) return st;
+    st = check_gemm_args(x, M, F, F, x, D, F, b2, y, ldy, flags);
+    if (st != HIF4_OK) return st;
+    if (!w1_codes || !w1_meta || !w2_codes || !w2_meta) return HIF4_ERR_INVALID_ARG;
+    if (n_mask1 > D || n_mask2 > F) return HIF4_ERR_INVALID_ARG;
+    if ((n_mask1 > 0 && (!mask1_idx || !w1_masked)) || (n_mask2 > 0 && (!mask2_idx || !w2_masked)))
+        return HIF4_ERR_INVALID_ARG;
+    if (!aligned_to(w1_codes, 4) || !aligned_to(w1_meta, 4) || !aligned_to(w2_codes, 4) || !aligned_to(w2_meta, 4))
+        return HIF4_ERR_ALIGNMENT;
+    if ((n_mask1 > 0 && (!aligned_to(mask1_idx, 4) || !aligned_to(w1_masked, 2))) ||
+        (n_mask2 > 0 && (!aligned_to(mask2_idx, 4) || !aligned_to(w2_masked, 2))))
+        return HIF4_ERR_ALIGNMENT;
+    const size_t need = hif4_ffn_w4a4_workspace(M, D, F);
+    if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
+    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *p = static_cast<uint8_t *>(workspace);
+    uint16_t *xhat1 = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)M * D * 2);
+    uint16_t *what1 = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)F * D * 2);
+    uint16_t *hhat = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)M * F * 2);
+    uint16_t *what2 = reinterpret_cast<uint16_t *>(p);
+    p += align256((size_t)D * F * 2);
+    uint8_t *mask1 = p;
+    p += align256((size_t)D);
+    uint8_t *mask2 = p;
+
+    // 1. protected-channel masks from the sorted index lists
+    if (n_mask1 > 0) {
+        const int64_t work = D > n_mask1 ? D : n_mask1;
+        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask1, (int)D, mask1_idx, n_mask1, status);
+        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    }
+    if (n_mask2 > 0) {
+        const int64_t work = F > n_mask2 ? F : n_mask2;
+        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask2, (int)F, mask2_idx, n_mask2, status);
+        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    }
+    // 2. first activation fake quantization along D
+    st = fake_quantize_bf16(x, M, D, ldx, n_mask1 > 0 ? mask1 : nullptr, xhat1, D, status, s);
+    if (st != HIF4_OK) return st;
+    // 3. W1 decode; first GEMM with bias, GELU and the fake quantization of H
+    st = hif4_weight_decode(w1_codes, w1_meta, F, D, mask1_idx, n_mask1, w1_masked, what1, D, status, stream);
+    if (st != HIF4_OK) return st;
+    st = launch_gemm(xhat1, M, D, D, what1, F, D, b1, n_mask2 > 0 ? mask2 : nullptr, hhat, F,
+                     HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, s);
+    if (st != HIF4_OK) return st;
+    // 4. W2 decode; second GEMM with bias
+    st = hif4_weight_decode(w2_codes, w2_meta, D, F, mask2_idx, n_mask2, w2_masked, what2, F, status, stream);
+    if (st != HIF4_OK) return st;
+    return launch_gemm(hhat, M, F, F, what2, D, F, b2, nullptr, y, ldy, flags, status, s);
 }

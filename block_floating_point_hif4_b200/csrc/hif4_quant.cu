@@ -18,12 +18,15 @@
 // comparisons against the half-way points (k + 1/2) S 2^E / 4 (exact in FP32).
 #include <cuda_bf16.h>
 
+#include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
 #include "hif4_sm100.cuh"
 
 namespace hif4 {
 
 namespace {
+
+using namespace enc;
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
@@ -41,17 +44,6 @@ struct QuantArgs {
     uint32_t total_units;
     uint32_t *status;
 };
-
-// Exact RNE of |x| / step onto 0..7 (slow path).
-__device__ __forceinline__ uint32_t round_exact(float ax, float inv, float step)
-{
-    float k = floorf(fminf(ax * inv, 7.0f));
-    float mid = fmaf(k, step, 0.5f * step);       // (k + 1/2) step, exact
-    uint32_t ki = (uint32_t)k;
-    uint32_t up = (ax > mid) || (ax == mid && (ki & 1u));
-    uint32_t m = ki + up;
-    return m > 7u ? 7u : m;
-}
 
 // Loads the 8 elements of lane vector `e` (element offset) as FP32.
 template <bool BF16>
@@ -264,80 +256,6 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a)
 //   * Units with a non-finite input or a scale clamped at the top code (255)
 //     take the generic FP32 path (sanitize, exact half-way comparisons).
 
-typedef unsigned long long u64;
-
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-// PTX prmt (byte permute); a selector nibble with bit 3 set replicates the
-// sign bit of the selected byte into the whole byte.
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
-{
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-// a * b + c on the integer multiply-add path (keeps byte/nibble packing off
-// the ALU pipe).
-__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c)
-{
-    uint32_t d;
-    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-__device__ __forceinline__ u64 pk(float lo, float hi)
-{
-    u64 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void upk(u64 v, float &lo, float &hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ u64 fmul2(u64 a, u64 b)
-{
-    u64 d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ u64 ffma2(u64 a, u64 b, u64 c)
-{
-    u64 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ u64 fadd2(u64 a, u64 b)
-{
-    u64 d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// Scale code from the FP32 bits of the unit maximum (exact; see above).
-__device__ __forceinline__ uint32_t scale_code_from_bits(uint32_t bits)
-{
-    const int32_t ea = (int32_t)(bits >> 23);
-    const int32_t qm = ((int32_t)(bits & 0x7FFFFFu) - 1) >> 17;       // -1 .. 63
-    int32_t f = ((qm + 12) * 79) >> 10;                                 // floor((qm + 12) / 13)
-    f = f > 4 ? 4 : f;
-    int32_t c = ((ea - 99) << 2) + f;
-    c = c < 0 ? 0 : c;
-    return (uint32_t)(c > 255 ? 255 : c);
-}
-
-// 4 / (4 + f) as an unevaluated sum hi + lo of two FP32 values.
-__device__ __forceinline__ void recip_pair(uint32_t f, float &hi, float &lo)
-{
-    const uint32_t h = f == 0 ? 0x3F800000u : f == 1 ? 0x3F4CCCCDu : f == 2 ? 0x3F2AAAABu : 0x3F124925u;
-    const uint32_t l = f == 0 ? 0u : f == 1 ? 0xB24CCCCDu : f == 2 ? 0xB2AAAAABu : 0xB2DB6DB7u;
-    hi = bits_f(h);
-    lo = bits_f(l);
-}
-
 __device__ __forceinline__ void ld256(const void *p, uint32_t (&w)[8])
 {
     asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -413,28 +331,16 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
                                          uint32_t &bad, uint32_t (&out)[8], uint32_t &meta)
 {
     const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
-    const u64 NMAGIC2 = pk(-12582912.0f, -12582912.0f);
     // protected columns: 16-bit lane masks (all ones where the mask byte is nonzero)
     uint32_t mw[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mw[i] = 0;
-    if (MASK) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t x = mraw[i];
-            const uint32_t nz = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x);   // bit 7 set <=> byte != 0
-            mw[2 * i] = prmt(nz, 0, 0x9988);                        // bytes 0,0,1,1 (sign-replicated)
-            mw[2 * i + 1] = prmt(nz, 0, 0xBBAA);                    // bytes 2,2,3,3
-        }
-    }
+    if (MASK) mask_words16(mraw, mw);
     uint32_t mk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
-    const uint32_t G0 = max_u16x2(mk[0], mk[1]), G1 = max_u16x2(mk[2], mk[3]);
-    const uint32_t G2 = max_u16x2(mk[4], mk[5]), G3 = max_u16x2(mk[6], mk[7]);
-    const uint32_t A01 = max_u16x2(prmt(G0, G1, 0x5410), prmt(G0, G1, 0x7632));
-    const uint32_t A23 = max_u16x2(prmt(G2, G3, 0x5410), prmt(G2, G3, 0x7632));
-    const uint32_t A8 = max_u16x2(prmt(A01, A23, 0x5410), prmt(A01, A23, 0x7632));
+    uint32_t A01, A23, A8;
+    quarter_max(mk, A01, A23, A8);
     uint32_t ak = max(A8 & 0xFFFFu, A8 >> 16);
     ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 1));
     ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, 2));
@@ -445,33 +351,16 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
         slow_lane16<MODE>(w, mw, q4, __activemask(), bad, out, meta);
     } else {
         const float S = e6m2_value(c);
-        const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
-        const uint32_t a8_0 = A8 & 0xFFFFu, a8_1 = A8 >> 16;
-        const uint32_t a4[4] = {A01 & 0xFFFFu, A01 >> 16, A23 & 0xFFFFu, A23 >> 16};
-        const uint32_t e2_0 = a8_0 > T2, e2_1 = a8_1 > T2;
-        const uint32_t th0 = e2_0 ? T2 : T1, th1 = e2_1 ? T2 : T1;
-        const uint32_t e3[4] = {a4[0] > th0, a4[1] > th0, a4[2] > th1, a4[3] > th1};
-        float ih, il;
-        recip_pair(c & 3u, ih, il);
-        const uint32_t E6 = c >> 2;
-        u64 HH[4], LL[4], ST[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t E = (k < 2 ? e2_0 : e2_1) + e3[k];
-            const float pw = bits_f((160u - E6 - E) << 23);         // 2^(33 - E6 - E)
-            HH[k] = pk(ih * pw, ih * pw);
-            LL[k] = pk(il * pw, il * pw);
-            if (MODE == 1) {
-                const float st = ldexp_small(S, (int)E - 2);
-                ST[k] = pk(st, st);
-            }
-        }
+        Quarter pq;
+        plan_quarter(A01, A23, A8, c, S, pq);
+        const uint32_t e2_0 = pq.e2_0, e2_1 = pq.e2_1;
+        const uint32_t *e3 = pq.e3;
         if (MODE == 0) {
             uint32_t tb[16];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
                 const u64 ax = pk(bits_f(imad(mk[p], 65536u, 0u)), bits_f(mk[p] & 0xFFFF0000u));
-                const u64 r = ffma2(ax, HH[p >> 1], fmul2(ax, LL[p >> 1]));
+                const u64 r = ffma2(ax, pq.HH[p >> 1], fmul2(ax, pq.LL[p >> 1]));
                 const u64 t = fadd2(r, MAGIC2);                    // low byte = RNE(r) <= 8
                 float tl, th;
                 upk(t, tl, th);
@@ -500,21 +389,7 @@ __device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t 
             part |= __shfl_xor_sync(0xffffffffu, part, 2);
             meta = part | c;
         } else {
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint32_t wz = w[p] & ~mw[p];
-                const u64 x = pk(bits_f(wz << 16), bits_f(wz & 0xFFFF0000u));
-                const u64 r = ffma2(x, HH[p >> 1], fmul2(x, LL[p >> 1]));
-                const u64 mf = fadd2(fadd2(r, MAGIC2), NMAGIC2);   // signed RNE(r), +0 when 0
-                float ml, mh;
-                upk(mf, ml, mh);
-                ml = fminf(fmaxf(ml, -7.0f), 7.0f);
-                mh = fminf(fmaxf(mh, -7.0f), 7.0f);
-                float yl, yh;
-                upk(fmul2(pk(ml, mh), ST[p >> 1]), yl, yh);
-                const uint32_t y = pack_bf16_exact(yl, yh);
-                out[p] = MASK ? ((y & ~mw[p]) | (w[p] & mw[p])) : y;
-            }
+            fq_quarter<MASK>(w, mw, pq, S, out);
         }
     }
 }

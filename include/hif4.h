@@ -70,6 +70,10 @@ typedef enum { HIF4_F32 = 0, HIF4_BF16 = 1 } hif4_dtype;
 /* Flags of hif4_linear_w4a4 / hif4_gemm_bf16. */
 #define HIF4_LINEAR_GELU_TANH 0x1u /* y = gelu_tanh(acc + bias) */
 #define HIF4_LINEAR_OUT_F32 0x2u   /* y is FP32 (the accumulator, unrounded) instead of BF16 */
+/* y (BF16) is replaced by its HiF4 fake quantization along N in 64-column
+ * units: deq(q(y with protected columns -> 0)), protected columns kept
+ * (hif4_gemm_bf16_fq; hif4_ffn_w4a4 uses it for the hidden activation). */
+#define HIF4_LINEAR_FAKE_QUANT_OUT 0x4u
 
 /*
  * hif4_quantize — HiF4 "direct conversion" (round to nearest) of a
@@ -168,6 +172,53 @@ hif4_status hif4_weight_decode(const uint8_t *w_codes, const uint32_t *w_meta, i
 hif4_status hif4_gemm_bf16(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N,
                            int64_t ldb, const void *bias, void *y, int64_t ldy, uint32_t flags,
                            uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_gemm_bf16_fq — hif4_gemm_bf16 whose BF16 output is fake-quantized in
+ * the epilogue [TA abstract: W4A4 HiF4 fake quantization of the activations
+ * that enter the main linears; fusion of the second FFN activation]:
+ *   h    = bf16_rne(acc + bias), or of gelu_tanh(acc + bias) with GELU,
+ *   y    = deq(q(h with the out_chan_mask columns -> 0)) along N in 64-column
+ *          units, the out_chan_mask columns keeping h.
+ * Identical, bit for bit, to hif4_gemm_bf16 followed by hif4_fake_quantize
+ * with that mask.  HIF4_LINEAR_FAKE_QUANT_OUT is implied; OUT_F32 is refused.
+ * out_chan_mask  NULL (no protected column) or u8 [N], nonzero = protected,
+ *                16-byte aligned.
+ * Errors: SHAPE (N % 64 != 0, others as hif4_gemm_bf16), ALIGNMENT,
+ * INVALID_ARG.  Non-finite h values raise HIF4_FLAG_NONFINITE (mapped as the
+ * quantizer maps them).
+ */
+hif4_status hif4_gemm_bf16_fq(const void *a, int64_t M, int64_t K, int64_t lda, const void *b, int64_t N,
+                              int64_t ldb, const void *bias, const uint8_t *out_chan_mask, void *y,
+                              int64_t ldy, uint32_t flags, uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_ffn_w4a4 — the W4A4 HiF4 feed-forward block of a DiT layer [TA
+ * abstract: fake-quantized main linears, protected channels in BF16; the
+ * tanh-form GELU between them is the library's reading]:
+ *   xhat1 = fake_quantize(x, mask1)                       M x D
+ *   Hhat  = fake_quantize(bf16(gelu_tanh(xhat1 what1^T + b1)), mask2)   M x F
+ *   y     = Hhat what2^T + b2                             M x D
+ * what1 = deq(w1) with columns mask1 restored from w1_masked (F x n_mask1);
+ * what2 = deq(w2) with columns mask2 restored from w2_masked (D x n_mask2).
+ * Hhat is produced inside the first GEMM's epilogue (hif4_gemm_bf16_fq).
+ * x      BF16 M x D, ldx.   w1_codes/w1_meta HiF4 F x D, quantized with
+ *        hif4_quantize and mask1; w2_codes/w2_meta HiF4 D x F with mask2.
+ * mask1_idx / mask2_idx  NULL or sorted distinct column indices (device
+ *        int32) of D / F.   b1 BF16 [F] or NULL; b2 BF16 [D] or NULL.
+ * y      BF16 M x D (FP32 with HIF4_LINEAR_OUT_F32, the only flag), ldy.
+ * workspace >= hif4_ffn_w4a4_workspace(M, D, F) bytes, 256-byte aligned.
+ * Errors: SHAPE (D or F not a multiple of 64), ALIGNMENT, WORKSPACE,
+ * INVALID_ARG; bad mask indices through status (HIF4_FLAG_BAD_INDEX).
+ */
+size_t hif4_ffn_w4a4_workspace(int64_t M, int64_t D, int64_t F);
+hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_t ldx,
+                          const uint8_t *w1_codes, const uint32_t *w1_meta, int64_t F,
+                          const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked,
+                          const void *b1, const uint8_t *w2_codes, const uint32_t *w2_meta,
+                          const int32_t *mask2_idx, int32_t n_mask2, const void *w2_masked,
+                          const void *b2, void *y, int64_t ldy, uint32_t flags, void *workspace,
+                          size_t ws_bytes, uint32_t *status, hif4_stream_t stream);
 
 /*
  * hif4_calib_percentile_mask — tail-aware percentile calibration and the

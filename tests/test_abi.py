@@ -51,6 +51,9 @@ def test_workspace_sizes(L):
     assert ws >= 2 * (M * K + N * K) + K
     assert L.hif4_linear_w4a4_workspace(0, 1, 64) == 0
     assert L.hif4_calib_workspace(230400, 5120) >= 5120 * 384 * 4
+    D, F = 5120, 13824
+    assert L.hif4_ffn_w4a4_workspace(M, D, F) >= 2 * (M * D + F * D + M * F + D * F) + D + F
+    assert L.hif4_ffn_w4a4_workspace(M, 0, F) == 0
 
 
 def test_argument_errors_return_before_any_launch(L):
@@ -88,4 +91,21 @@ def test_argument_errors_return_before_any_launch(L):
                                         1 << 30, None) == 1
     assert L.hif4_calib_percentile_mask(fake, 10, 8, 8, 999, 1000, 1, 100, fake, fake, fake, None, fake, 8,
                                         None) == 4
+    # fused fake-quant GEMM: N % 64, FP32 output refused, misaligned mask
+    assert L.hif4_gemm_bf16_fq(fake, 4, 64, 64, fake, 100, 64, None, None, fake, 100, 0, None, None) == 3
+    assert L.hif4_gemm_bf16_fq(fake, 4, 64, 64, fake, 64, 64, None, None, fake, 64, 2, None, None) == 1
+    assert L.hif4_gemm_bf16_fq(fake, 4, 64, 64, fake, 64, 64, None, P(0x1001), fake, 64, 0, None, None) == 2
+    # the plain linear refuses the fused-output flag (it has no output mask)
+    assert L.hif4_linear_w4a4(fake, 4, 64, 64, fake, fake, 64, None, 0, None, None, fake, 64, 4, fake,
+                              1 << 30, None, None) == 1
+    # FFN block: F % 64, unknown flag, workspace too small, mask2 count without indices
+    ffn = L.hif4_ffn_w4a4
+    assert ffn(fake, 4, 64, 64, fake, fake, 100, None, 0, None, None, fake, fake, None, 0, None, None, fake, 64,
+               0, fake, 1 << 30, None, None) == 3
+    assert ffn(fake, 4, 64, 64, fake, fake, 128, None, 0, None, None, fake, fake, None, 0, None, None, fake, 64,
+               1, fake, 1 << 30, None, None) == 1
+    assert ffn(fake, 4, 64, 64, fake, fake, 128, None, 0, None, None, fake, fake, None, 0, None, None, fake, 64,
+               0, fake, 64, None, None) == 4
+    assert ffn(fake, 4, 64, 64, fake, fake, 128, None, 0, None, None, fake, fake, None, 2, None, None, fake, 64,
+               0, fake, 1 << 30, None, None) == 1
     assert L.hif4_get_status(None, None) == 1
