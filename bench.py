@@ -4,10 +4,12 @@
 Headline workload: the Wan2.2-14B-shaped FFN, per GPU 57600 tokens x 5120 ->
 13824 (tanh-GELU) -> 5120, both linears W4A4 HiF4 fake-quantized with a
 1 %-of-K protected-channel mask from the tail-percentile rule.  One step =
-for each linear: activation fake quantization (hif4_fake_quantize), weight
-decode (hif4_weight_decode), tcgen05 GEMM + epilogue (hif4_gemm_bf16) — the
-same kernels, in the same order, that hif4_linear_w4a4 launches.  value =
-FLOPs of both GEMMs (2 M N K each) over all ranks / max-over-ranks step time.
+fake quantization of X (hif4_fake_quantize), W1 decode (hif4_weight_decode),
+the first tcgen05 GEMM with bias, GELU and the fake quantization of the
+hidden activation in its epilogue (hif4_gemm_bf16_fq), W2 decode, the second
+GEMM (hif4_gemm_bf16) — the kernels, in the order, that hif4_ffn_w4a4
+launches.  value = FLOPs of both GEMMs (2 M N K each) over all ranks /
+max-over-ranks step time.
 
 The same JSON line carries the other rows of the path, each timed the same
 way: the quantizer sweep's largest size (quantize, dequantize; 2^30 BF16
@@ -151,7 +153,8 @@ class ClockSampler:
 def oracle_ffn_sample(rows: int, seed: int = 3, threads: int | None = None, steps: int = 1, prep=None):
     """Time the CPU oracle on `rows` tokens of the FFN workload (numpy-seeded
     inputs of the same recipe).  Per step: activation fake quantization, the
-    full weight decode of W1 and W2, both FP64 products and the GELU.
+    full weight decode of W1 and W2, both FP64 products, the GELU, the BF16
+    rounding and fake quantization of the hidden activation.
     Returns (flop per step, seconds per step list, threads)."""
     import numpy as np
 
@@ -173,7 +176,6 @@ def oracle_ffn_sample(rows: int, seed: int = 3, threads: int | None = None, step
         prep = dict(x=x[:rows].copy(), idx1=idx1, idx2=idx2, c1=c1, mt1=mt1, c2=c2, mt2=mt2,
                     wm1=np.ascontiguousarray(d["w1"][:, idx1]), wm2=np.ascontiguousarray(d["w2"][:, idx2]))
     P = prep
-    from block_floating_point_hif4_b200.workloads import f32_to_bf16_bits
     times = []
     for _ in range(steps):
         t0 = time.perf_counter()
@@ -181,8 +183,7 @@ def oracle_ffn_sample(rows: int, seed: int = 3, threads: int | None = None, step
         w2 = _threaded_weight_hat(P["c2"], P["mt2"], D_MODEL, D_FFN, P["idx2"], P["wm2"], threads)
         xh = oracle.fake_quantize(P["x"], P["idx1"])
         hid = oracle.linear(xh, w1, None, gelu=True, threads=threads)
-        hb = f32_to_bf16_bits(hid.astype(np.float32))
-        hh = oracle.fake_quantize(hb, P["idx2"])
+        hh = oracle.fake_quantize(oracle.round_bf16(hid), P["idx2"])
         oracle.linear(hh, w2, None, threads=threads)
         times.append(time.perf_counter() - t0)
     flop = 2 * 2.0 * rows * D_MODEL * D_FFN
@@ -286,6 +287,7 @@ def main():
     ws = torch.empty(H.linear_w4a4_workspace(M, max(D, F), max(D, F)), dtype=torch.uint8, device=dev)
     H.linear_w4a4(x, w1c, w1m, F, idx1, w1k, None, gelu=True, out=hbuf, workspace=ws)
     _, _, mask2, idx2 = H.calib_percentile_mask(hbuf)
+    del hbuf, ws
     w2c, w2m = H.quantize(w2, mask2)
     w2k = w2[:, idx2.long()].contiguous()
     del w1, w2
@@ -296,7 +298,7 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
-    stages = ["fake_quant_1", "weight_decode_1", "gemm_1", "fake_quant_2", "weight_decode_2", "gemm_2"]
+    stages = ["fake_quant_1", "weight_decode_1", "gemm_1_gelu_fq", "weight_decode_2", "gemm_2"]
 
     def step(evs=None):
         def mark(i):
@@ -307,19 +309,18 @@ def main():
         mark(1)
         H.weight_decode(w1c, w1m, F, D, idx1, w1k, out=what1, status=status)
         mark(2)
-        H.gemm_bf16(xhat1, what1, None, gelu=True, out=hbuf, status=status)
+        H.gemm_bf16_fq(xhat1, what1, None, gelu=True, out_chan_mask=mask2, out=xhat2, status=status)
         mark(3)
-        H.fake_quantize(hbuf, mask2, out=xhat2, status=status)
-        mark(4)
         H.weight_decode(w2c, w2m, D, F, idx2, w2k, out=what2, status=status)
-        mark(5)
+        mark(4)
         H.gemm_bf16(xhat2, what2, None, gelu=False, out=ybuf, status=status)
-        mark(6)
+        mark(5)
 
-    launches_per_step = 2 * (1 + 1 + 1 + 1)     # fake-quant, dequant, column scatter, GEMM per linear
+    # fake-quant, 2 x (dequant + column scatter), 2 x GEMM
+    launches_per_step = 1 + 2 * 2 + 2
 
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
@@ -346,12 +347,12 @@ def main():
     flop_gemm = 2.0 * M * D * F                      # each of the two GEMMs
     flop_step = 2 * flop_gemm
     value = sharding.aggregate_throughput(flop_step, world, ms_step * 1e-3) / 1e12
-    gemm_ms = max_over_ranks((stage_ms["gemm_1"] + stage_ms["gemm_2"]) / 2)
+    gemm_ms = max_over_ranks((stage_ms["gemm_1_gelu_fq"] + stage_ms["gemm_2"]) / 2)
     achieved = flop_gemm / (gemm_ms * 1e-3) / 1e12
     peak = P["bf16_tflops_sustained"]
     gh = src_hash("hif4_linear.cu", "hif4_sm100.cuh")
     traffic = NCU_TRAFFIC.get(("gemm", gh))
-    roofline = {"kernel": "k_gemm (hif4_gemm_bf16)", "bound": "tensor", "achieved": achieved, "peak": peak,
+    roofline = {"kernel": "k_gemm (hif4_gemm_bf16_fq, hif4_gemm_bf16)", "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_source": "%s bf16 sustained (burst %.1f, frac %.3f)" % (P["source"], P["bf16_tflops"],
                                                                             achieved / P["bf16_tflops"]),
@@ -374,10 +375,12 @@ def main():
         yh = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=True)
         xd = torch.empty_like(x)
 
+        ws = torch.empty(H.ffn_w4a4_workspace(M, D, F), dtype=torch.uint8, device=dev)
+
         def e2e_step():
             xd.copy_(xh, non_blocking=True)
-            H.linear_w4a4(xd, w1c, w1m, F, idx1, w1k, None, gelu=True, out=hbuf, workspace=ws, status=status)
-            H.linear_w4a4(hbuf, w2c, w2m, D, idx2, w2k, None, gelu=False, out=ybuf, workspace=ws, status=status)
+            H.ffn_w4a4(xd, w1c, w1m, F, w2c, w2m, idx1, w1k, None, idx2, w2k, None, out=ybuf, workspace=ws,
+                       status=status)
             yh.copy_(ybuf, non_blocking=True)
         for _ in range(args.warmup):
             e2e_step()
@@ -392,10 +395,10 @@ def main():
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
         line["e2e"] = {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": M * D * 2, "d2h_bytes_per_step": M * D * 2,
-                       "ms_per_step": e2e_ms, "api": "hif4_linear_w4a4 x2, pinned host X in, Y out"}
-        del xh, yh, xd
+                       "ms_per_step": e2e_ms, "api": "hif4_ffn_w4a4, pinned host X in, Y out"}
+        del xh, yh, xd, ws
 
-    del xhat1, xhat2, what1, what2, hbuf, ybuf, ws, x
+    del xhat1, xhat2, what1, what2, ybuf, x
     torch.cuda.empty_cache()
 
     # ---- the other rows of the path: quantizer sweep and calibration
