@@ -3,7 +3,10 @@ command to put under a profiler (ncu) or to time one kernel in isolation.
 
     python -m block_floating_point_hif4_b200.profile OP [--log2n N] [--tokens T] [--reps R]
 
-OP: quantize | dequantize | fake_quantize | gemm | calib | linear.
+OP: quantize | dequantize | fake_quantize | gemm | gemm_gelu | gemm_fq | calib |
+linear | ffn.  gemm_fq is the FFN's first GEMM: bias-free, tanh-GELU and the
+HiF4 fake quantization of its output (1 % protected columns) in the epilogue;
+ffn is the whole W4A4 FFN block (hif4_ffn_w4a4, --n = hidden width).
 Sizes default to small cases that still exceed the 126 MB L2 (a few hundred
 MB on the device).  Prints the mean CUDA-event time per call.
 """
@@ -15,7 +18,8 @@ import sys
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "gemm", "calib", "linear"])
+    p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "gemm", "gemm_gelu", "gemm_fq",
+                                  "calib", "linear", "ffn"])
     p.add_argument("--log2n", type=int, default=28, help="elements for quantize/dequantize/fake_quantize")
     p.add_argument("--tokens", type=int, default=57600)
     p.add_argument("--channels", type=int, default=5120)
@@ -50,11 +54,25 @@ def main(argv=None):
         y = torch.empty(a.tokens, a.n, dtype=torch.bfloat16, device=dev)
         if a.op == "gemm":
             fn = lambda: H.gemm_bf16(x, w, out=y)  # noqa: E731
+        elif a.op == "gemm_gelu":
+            fn = lambda: H.gemm_bf16(x, w, gelu=True, out=y)  # noqa: E731
+        elif a.op == "gemm_fq":
+            g = torch.Generator(device=dev)
+            g.manual_seed(5)
+            cm = (torch.rand(a.n, device=dev, generator=g) < 0.01).to(torch.uint8)
+            fn = lambda: H.gemm_bf16_fq(x, w, gelu=True, out_chan_mask=cm, out=y)  # noqa: E731
+        elif a.op == "ffn":
+            w2 = wl.device_weight(a.channels, a.n, 0.015, seed=32, device=dev)
+            w1c, w1m = H.quantize(w)
+            w2c, w2m = H.quantize(w2)
+            y = torch.empty(a.tokens, a.channels, dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(H.ffn_w4a4_workspace(a.tokens, a.channels, a.n), dtype=torch.uint8, device=dev)
+            fn = lambda: H.ffn_w4a4(x, w1c, w1m, a.n, w2c, w2m, out=y, workspace=ws)  # noqa: E731
         else:
             wc, wm = H.quantize(w)
             ws = torch.empty(H.linear_w4a4_workspace(a.tokens, a.n, a.channels), dtype=torch.uint8, device=dev)
             fn = lambda: H.linear_w4a4(x, wc, wm, a.n, out=y, workspace=ws)  # noqa: E731
-        nbytes = 2.0 * a.tokens * a.n * a.channels          # FLOPs for the GEMM-shaped ops
+        nbytes = 2.0 * a.tokens * a.n * a.channels * (2 if a.op == "ffn" else 1)   # FLOPs
     fn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -64,7 +82,7 @@ def main(argv=None):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.reps
-    unit = "TFLOP/s" if a.op in ("gemm", "linear") else "GB/s"
+    unit = "TFLOP/s" if a.op in ("gemm", "gemm_gelu", "gemm_fq", "linear", "ffn") else "GB/s"
     rate = nbytes / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print("%s: %.4f ms per call, %.1f %s" % (a.op, ms, rate, unit))
     return 0
