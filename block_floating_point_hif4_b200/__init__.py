@@ -5,11 +5,13 @@ the C ABI in ``include/hif4.h``); :mod:`.binding` marshals torch tensors into
 it.  :mod:`.workloads` holds the seeded synthetic inputs.
 """
 from .binding import (  # noqa: F401
-    Hif4Error, calib_percentile_mask, calib_workspace, dequantize, fake_quantize, ffn_w4a4, ffn_w4a4_workspace,
+    Hif4Error, calib_percentile_mask, calib_workspace, dequantize, fake_quantize, ffn_w4a4, ffn_w4a4_host,
+    ffn_w4a4_host_workspace, ffn_w4a4_workspace,
     gemm_bf16, gemm_bf16_fq, get_status, lib, linear_w4a4, linear_w4a4_workspace, quantize, reset_status,
     version, weight_decode,
 )
 
 __all__ = ["Hif4Error", "calib_percentile_mask", "calib_workspace", "dequantize", "fake_quantize", "ffn_w4a4",
-           "ffn_w4a4_workspace", "gemm_bf16", "gemm_bf16_fq", "get_status", "lib", "linear_w4a4",
-           "linear_w4a4_workspace", "quantize", "reset_status", "version", "weight_decode"]
+           "ffn_w4a4_host", "ffn_w4a4_host_workspace", "ffn_w4a4_workspace", "gemm_bf16", "gemm_bf16_fq",
+           "get_status", "lib", "linear_w4a4", "linear_w4a4_workspace", "quantize", "reset_status", "version",
+           "weight_decode"]

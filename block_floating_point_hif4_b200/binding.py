@@ -39,6 +39,9 @@ SIGNATURES = {
     "hif4_gemm_bf16": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P, _I64, _U32, _P, _P]),
     "hif4_gemm_bf16_fq": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P, _P, _I64, _U32, _P, _P]),
     "hif4_ffn_w4a4_workspace": (_SZ, [_I64, _I64, _I64]),
+    "hif4_ffn_w4a4_host_workspace": (_SZ, [_I64, _I64, _I64, _I64, _U32]),
+    "hif4_ffn_w4a4_host": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _I32, _P, _P, _P, _P, _P, _I32,
+                                          _P, _P, _P, _I64, _I64, _U32, _P, _SZ, _P, _P]),
     "hif4_ffn_w4a4": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I64, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
                                      _P, _P, _I64, _U32, _P, _SZ, _P, _P]),
     "hif4_calib_workspace": (_SZ, [_I64, _I64]),
@@ -247,6 +250,39 @@ def ffn_w4a4(x: torch.Tensor, w1_codes: torch.Tensor, w1_meta: torch.Tensor, F: 
         _ptr(mask2_idx) if n2 else None, n2, _ptr(w2_masked) if n2 else None, _ptr(b2), _ptr(out),
         out.stride(0), flags, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
+    return out
+
+
+def ffn_w4a4_host_workspace(M: int, D: int, F: int, chunk_rows: int = 0, out_f32: bool = False) -> int:
+    return int(lib().hif4_ffn_w4a4_host_workspace(M, D, F, chunk_rows, LINEAR_OUT_F32 if out_f32 else 0))
+
+
+def ffn_w4a4_host(x_host: torch.Tensor, w1_codes: torch.Tensor, w1_meta: torch.Tensor, F: int,
+                  w2_codes: torch.Tensor, w2_meta: torch.Tensor,
+                  mask1_idx: torch.Tensor | None = None, w1_masked: torch.Tensor | None = None,
+                  b1: torch.Tensor | None = None, mask2_idx: torch.Tensor | None = None,
+                  w2_masked: torch.Tensor | None = None, b2: torch.Tensor | None = None, *, out=None,
+                  chunk_rows: int = 0, workspace=None, status=None, stream=None):
+    """The FFN block on HOST (ideally pinned) x; y returned in a host tensor.
+    Copies overlap compute chunk by chunk.  Asynchronous on `stream`."""
+    assert x_host.device.type == "cpu" and x_host.dtype == torch.bfloat16 and x_host.stride(1) == 1
+    M, D = x_host.shape
+    if out is None:
+        out = torch.empty(M, D, dtype=torch.bfloat16, pin_memory=x_host.is_pinned())
+    assert out.device.type == "cpu" and out.stride(1) == 1
+    f32 = out.dtype == torch.float32
+    dev = w1_codes.device
+    if workspace is None:
+        need = ffn_w4a4_host_workspace(M, D, F, chunk_rows, f32)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    n1 = 0 if mask1_idx is None else int(mask1_idx.numel())
+    n2 = 0 if mask2_idx is None else int(mask2_idx.numel())
+    _check("hif4_ffn_w4a4_host", lib().hif4_ffn_w4a4_host(
+        ctypes.c_void_p(x_host.data_ptr()), M, D, x_host.stride(0), _ptr(w1_codes), _ptr(w1_meta), F,
+        _ptr(mask1_idx) if n1 else None, n1, _ptr(w1_masked) if n1 else None, _ptr(b1), _ptr(w2_codes),
+        _ptr(w2_meta), _ptr(mask2_idx) if n2 else None, n2, _ptr(w2_masked) if n2 else None, _ptr(b2),
+        ctypes.c_void_p(out.data_ptr()), out.stride(0), chunk_rows, LINEAR_OUT_F32 if f32 else 0,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
     return out
 
 

@@ -613,6 +613,76 @@ extern "C" hif4_status hif4_linear_w4a4(const void *x, int64_t M, int64_t K, int
 // Workspace: xhat1 M x D | what1 F x D | Hhat M x F | what2 D x F (BF16) |
 // mask1 D | mask2 F (u8), each 256-byte aligned.
 
+namespace hif4 {
+namespace {
+
+// The FFN on `rows` device rows once the masks are built and the weights
+// decoded: fake quantization of x along D into xhat1 (rows x D), the first
+// GEMM with bias, GELU and the fake quantization of H into hhat (rows x F),
+// the second GEMM with bias into y.
+hif4_status ffn_rows(const void *x, int64_t rows, int64_t D, int64_t ldx, const uint16_t *what1,
+                     const uint16_t *what2, int64_t F, const uint8_t *mask1, const uint8_t *mask2, const void *b1,
+                     const void *b2, uint16_t *xhat1, uint16_t *hhat, void *y, int64_t ldy, uint32_t flags,
+                     uint32_t *status, cudaStream_t s)
+{
+    hif4_status st = fake_quantize_bf16(x, rows, D, ldx, mask1, xhat1, D, status, s);
+    if (st != HIF4_OK) return st;
+    st = launch_gemm(xhat1, rows, D, D, what1, F, D, b1, mask2, hhat, F,
+                     HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, s);
+    if (st != HIF4_OK) return st;
+    return launch_gemm(hhat, rows, F, F, what2, D, F, b2, nullptr, y, ldy, flags, status, s);
+}
+
+// Host-side checks shared by both FFN entry points (device x / y pointers
+// are checked by the caller where they exist).
+hif4_status check_ffn_weights(int64_t D, int64_t F, const uint8_t *w1_codes, const uint32_t *w1_meta,
+                              const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked, const void *b1,
+                              const uint8_t *w2_codes, const uint32_t *w2_meta, const int32_t *mask2_idx,
+                              int32_t n_mask2, const void *w2_masked, const void *b2)
+{
+    if (n_mask1 < 0 || n_mask2 < 0 || D < 0 || F < 0) return HIF4_ERR_INVALID_ARG;
+    if (D % HIF4_UNIT != 0 || F % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
+    if (D == 0 || F == 0) return HIF4_ERR_SHAPE;
+    if (D > INT32_MAX / 2 || F > INT32_MAX / 2) return HIF4_ERR_UNSUPPORTED;
+    if (!w1_codes || !w1_meta || !w2_codes || !w2_meta) return HIF4_ERR_INVALID_ARG;
+    if (n_mask1 > D || n_mask2 > F) return HIF4_ERR_INVALID_ARG;
+    if ((n_mask1 > 0 && (!mask1_idx || !w1_masked)) || (n_mask2 > 0 && (!mask2_idx || !w2_masked)))
+        return HIF4_ERR_INVALID_ARG;
+    if (!aligned_to(w1_codes, 4) || !aligned_to(w1_meta, 4) || !aligned_to(w2_codes, 4) || !aligned_to(w2_meta, 4))
+        return HIF4_ERR_ALIGNMENT;
+    if ((n_mask1 > 0 && (!aligned_to(mask1_idx, 4) || !aligned_to(w1_masked, 2))) ||
+        (n_mask2 > 0 && (!aligned_to(mask2_idx, 4) || !aligned_to(w2_masked, 2))))
+        return HIF4_ERR_ALIGNMENT;
+    if ((b1 && !aligned16(b1)) || (b2 && !aligned16(b2))) return HIF4_ERR_ALIGNMENT;
+    return HIF4_OK;
+}
+
+// Masks from the sorted index lists and both weight decodes (once per call).
+hif4_status ffn_prepare(int64_t D, int64_t F, const uint8_t *w1_codes, const uint32_t *w1_meta,
+                        const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked, const uint8_t *w2_codes,
+                        const uint32_t *w2_meta, const int32_t *mask2_idx, int32_t n_mask2, const void *w2_masked,
+                        uint16_t *what1, uint16_t *what2, uint8_t *mask1, uint8_t *mask2, uint32_t *status,
+                        cudaStream_t s)
+{
+    if (n_mask1 > 0) {
+        const int64_t work = D > n_mask1 ? D : n_mask1;
+        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask1, (int)D, mask1_idx, n_mask1, status);
+        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    }
+    if (n_mask2 > 0) {
+        const int64_t work = F > n_mask2 ? F : n_mask2;
+        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask2, (int)F, mask2_idx, n_mask2, status);
+        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    }
+    hif4_stream_t hs = reinterpret_cast<hif4_stream_t>(s);
+    hif4_status st = hif4_weight_decode(w1_codes, w1_meta, F, D, mask1_idx, n_mask1, w1_masked, what1, D, status, hs);
+    if (st != HIF4_OK) return st;
+    return hif4_weight_decode(w2_codes, w2_meta, D, F, mask2_idx, n_mask2, w2_masked, what2, F, status, hs);
+}
+
+} // namespace
+} // namespace hif4
+
 extern "C" size_t hif4_ffn_w4a4_workspace(int64_t M, int64_t D, int64_t F)
 {
     if (M <= 0 || D <= 0 || F <= 0) return 0;
@@ -628,27 +698,16 @@ extern "C" hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_
                                      const void *b2, void *y, int64_t ldy, uint32_t flags, void *workspace,
                                      size_t ws_bytes, uint32_t *status, hif4_stream_t stream)
 {
-    if (n_mask1 < 0 || n_mask2 < 0) return HIF4_ERR_INVALID_ARG;
     if (flags & ~HIF4_LINEAR_OUT_F32) return HIF4_ERR_INVALID_ARG;
-    if (M < 0 || D < 0 || F < 0) return HIF4_ERR_INVALID_ARG;
-    if (D % HIF4_UNIT != 0 || F % HIF4_UNIT != 0) return HIF4_ERR_SHAPE;
-    if (M == 0) return HIF4_OK;
-    if (D == 0 || F == 0) return HIF4_ERR_SHAPE;
+    if (M < 0) return HIF4_ERR_INVALID_ARG;
+    hif4_status st = check_ffn_weights(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, b1, w2_codes,
+                                       w2_meta, mask2_idx, n_mask2, w2_masked, b2);
+    if (st != HIF4_OK || M == 0) return st;
     // first GEMM (x -> Hhat) and second GEMM (Hhat -> y) shapes and pointers
-    hif4_status st = check_gemm_args(x, M, D, ldx, x, F, D, b1, x, F,
-                                     HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT);
+    st = check_gemm_args(x, M, D, ldx, x, F, D, b1, x, F, HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT);
     if (st != HIF4_OK) return st;
     st = check_gemm_args(x, M, F, F, x, D, F, b2, y, ldy, flags);
     if (st != HIF4_OK) return st;
-    if (!w1_codes || !w1_meta || !w2_codes || !w2_meta) return HIF4_ERR_INVALID_ARG;
-    if (n_mask1 > D || n_mask2 > F) return HIF4_ERR_INVALID_ARG;
-    if ((n_mask1 > 0 && (!mask1_idx || !w1_masked)) || (n_mask2 > 0 && (!mask2_idx || !w2_masked)))
-        return HIF4_ERR_INVALID_ARG;
-    if (!aligned_to(w1_codes, 4) || !aligned_to(w1_meta, 4) || !aligned_to(w2_codes, 4) || !aligned_to(w2_meta, 4))
-        return HIF4_ERR_ALIGNMENT;
-    if ((n_mask1 > 0 && (!aligned_to(mask1_idx, 4) || !aligned_to(w1_masked, 2))) ||
-        (n_mask2 > 0 && (!aligned_to(mask2_idx, 4) || !aligned_to(w2_masked, 2))))
-        return HIF4_ERR_ALIGNMENT;
     const size_t need = hif4_ffn_w4a4_workspace(M, D, F);
     if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
     if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
@@ -667,28 +726,177 @@ extern "C" hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_
     p += align256((size_t)D);
     uint8_t *mask2 = p;
 
-    // 1. protected-channel masks from the sorted index lists
-    if (n_mask1 > 0) {
-        const int64_t work = D > n_mask1 ? D : n_mask1;
-        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask1, (int)D, mask1_idx, n_mask1, status);
-        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    st = ffn_prepare(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, w2_codes, w2_meta, mask2_idx,
+                     n_mask2, w2_masked, what1, what2, mask1, mask2, status, s);
+    if (st != HIF4_OK) return st;
+    return ffn_rows(x, M, D, ldx, what1, what2, F, n_mask1 > 0 ? mask1 : nullptr, n_mask2 > 0 ? mask2 : nullptr,
+                    b1, b2, xhat1, hhat, y, ldy, flags, status, s);
+}
+
+// ---------------------------------------------- FFN block on host activations
+//
+// The tokens stream through the GPU in chunks of C rows.  Two copy streams
+// run beside the caller's stream: chunk i+1 is copied in while chunk i
+// computes and chunk i-1 is copied out, with double-buffered device staging
+// (xs[2], ys[2]) ordered by events:
+//   h2d:     wait x_free[s]  -> copy x rows into xs[s]  -> record x_ready[s]
+//   compute: wait x_ready[s] -> fake-quant xs[s]        -> record x_free[s]
+//            GEMM 1 (+ fake quant of H)  -> wait y_free[s] -> GEMM 2 into ys[s]
+//            -> record y_ready[s]
+//   d2h:     wait y_ready[s] -> copy ys[s] out          -> record y_free[s]
+// with s = i % 2.  The weights are decoded once per call.  The streams and
+// events are created per call and released once their work completes.
+// Workspace: what1 F x D | what2 D x F | mask1 D | mask2 F | xhat1 C x D |
+// hhat C x F | xs 2 x C x D | ys 2 x C x D (x 2 for FP32 output).
+
+namespace hif4 {
+namespace {
+
+size_t ffn_host_layout(int64_t C, int64_t D, int64_t F, uint32_t flags, size_t *off)
+{
+    const size_t ysz = (flags & HIF4_LINEAR_OUT_F32) ? 4 : 2;
+    size_t o = 0;
+    const size_t sizes[8] = {(size_t)F * D * 2, (size_t)D * F * 2, (size_t)D, (size_t)F,
+                             (size_t)C * D * 2, (size_t)C * F * 2, 2 * align256((size_t)C * D * 2),
+                             2 * align256((size_t)C * D * ysz)};
+    for (int i = 0; i < 8; ++i) {
+        if (off) off[i] = o;
+        o += align256(sizes[i]);
     }
-    if (n_mask2 > 0) {
-        const int64_t work = F > n_mask2 ? F : n_mask2;
-        k_mask_prep<<<(int)((work + 255) / 256), 256, 0, s>>>(mask2, (int)F, mask2_idx, n_mask2, status);
-        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    return o;
+}
+
+int64_t ffn_host_chunk(int64_t M, int64_t chunk_rows)
+{
+    if (chunk_rows > 0) return chunk_rows < M ? chunk_rows : M;
+    const int64_t n = (M + 8191) / 8192;                      // chunks of at most 8192 rows
+    int64_t c = (M + n - 1) / n;
+    c = (c + 127) / 128 * 128;                                // whole 128-row GEMM tiles
+    return c < M ? c : M;
+}
+
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t x_ready[2] = {}, x_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
+    bool make()
+    {
+        if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
+        if (cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
+        cudaEvent_t *all[10] = {&start, &done, &x_ready[0], &x_ready[1], &x_free[0],
+                                &x_free[1], &y_ready[0], &y_ready[1], &y_free[0], &y_free[1]};
+        for (cudaEvent_t *e : all)
+            if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+        return true;
     }
-    // 2. first activation fake quantization along D
-    st = fake_quantize_bf16(x, M, D, ldx, n_mask1 > 0 ? mask1 : nullptr, xhat1, D, status, s);
+    ~HostPipe()
+    {
+        // Destroying a stream or an event with work pending is allowed: its
+        // resources are released once that work completes.
+        cudaEvent_t all[10] = {start, done, x_ready[0], x_ready[1], x_free[0],
+                               x_free[1], y_ready[0], y_ready[1], y_free[0], y_free[1]};
+        for (cudaEvent_t e : all)
+            if (e) cudaEventDestroy(e);
+        if (h2d) cudaStreamDestroy(h2d);
+        if (d2h) cudaStreamDestroy(d2h);
+    }
+};
+
+} // namespace
+} // namespace hif4
+
+extern "C" size_t hif4_ffn_w4a4_host_workspace(int64_t M, int64_t D, int64_t F, int64_t chunk_rows, uint32_t flags)
+{
+    if (M <= 0 || D <= 0 || F <= 0) return 0;
+    return ffn_host_layout(ffn_host_chunk(M, chunk_rows), D, F, flags, nullptr);
+}
+
+extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t D, int64_t ldx,
+                                          const uint8_t *w1_codes, const uint32_t *w1_meta, int64_t F,
+                                          const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked,
+                                          const void *b1, const uint8_t *w2_codes, const uint32_t *w2_meta,
+                                          const int32_t *mask2_idx, int32_t n_mask2, const void *w2_masked,
+                                          const void *b2, void *y_host, int64_t ldy, int64_t chunk_rows,
+                                          uint32_t flags, void *workspace, size_t ws_bytes, uint32_t *status,
+                                          hif4_stream_t stream)
+{
+    if (flags & ~HIF4_LINEAR_OUT_F32) return HIF4_ERR_INVALID_ARG;
+    if (M < 0 || chunk_rows < 0) return HIF4_ERR_INVALID_ARG;
+    hif4_status st = check_ffn_weights(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, b1, w2_codes,
+                                       w2_meta, mask2_idx, n_mask2, w2_masked, b2);
+    if (st != HIF4_OK || M == 0) return st;
+    if (!x_host || !y_host) return HIF4_ERR_INVALID_ARG;
+    if (ldx < D || ldy < D) return HIF4_ERR_SHAPE;
+    if (M > INT32_MAX / 2) return HIF4_ERR_UNSUPPORTED;
+    const size_t ysz = (flags & HIF4_LINEAR_OUT_F32) ? 4 : 2;
+    const int64_t C = ffn_host_chunk(M, chunk_rows);
+    size_t off[8];
+    const size_t need = ffn_host_layout(C, D, F, flags, off);
+    if (!workspace || ws_bytes < need) return HIF4_ERR_WORKSPACE;
+    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *what1 = reinterpret_cast<uint16_t *>(ws + off[0]);
+    uint16_t *what2 = reinterpret_cast<uint16_t *>(ws + off[1]);
+    uint8_t *mask1 = ws + off[2];
+    uint8_t *mask2 = ws + off[3];
+    uint16_t *xhat1 = reinterpret_cast<uint16_t *>(ws + off[4]);
+    uint16_t *hhat = reinterpret_cast<uint16_t *>(ws + off[5]);
+    uint8_t *xs[2] = {ws + off[6], ws + off[6] + align256((size_t)C * D * 2)};
+    uint8_t *ys[2] = {ws + off[7], ws + off[7] + align256((size_t)C * D * ysz)};
+
+    HostPipe P;
+    if (!P.make()) return HIF4_ERR_CUDA;
+    // the copy streams start after everything already queued on the caller's stream
+    if (cudaEventRecord(P.start, s) != cudaSuccess || cudaStreamWaitEvent(P.h2d, P.start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(P.d2h, P.start, 0) != cudaSuccess)
+        return HIF4_ERR_CUDA;
+    st = ffn_prepare(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, w2_codes, w2_meta, mask2_idx,
+                     n_mask2, w2_masked, what1, what2, mask1, mask2, status, s);
     if (st != HIF4_OK) return st;
-    // 3. W1 decode; first GEMM with bias, GELU and the fake quantization of H
-    st = hif4_weight_decode(w1_codes, w1_meta, F, D, mask1_idx, n_mask1, w1_masked, what1, D, status, stream);
-    if (st != HIF4_OK) return st;
-    st = launch_gemm(xhat1, M, D, D, what1, F, D, b1, n_mask2 > 0 ? mask2 : nullptr, hhat, F,
-                     HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, s);
-    if (st != HIF4_OK) return st;
-    // 4. W2 decode; second GEMM with bias
-    st = hif4_weight_decode(w2_codes, w2_meta, D, F, mask2_idx, n_mask2, w2_masked, what2, F, status, stream);
-    if (st != HIF4_OK) return st;
-    return launch_gemm(hhat, M, F, F, what2, D, F, b2, nullptr, y, ldy, flags, status, s);
+
+    // On any failure below, the caller's stream still waits for the copies
+    // already queued, so no buffer is released under a running copy.
+    auto join = [&](hif4_status result) {
+        if (cudaEventRecord(P.done, P.h2d) == cudaSuccess) cudaStreamWaitEvent(s, P.done, 0);
+        if (cudaEventRecord(P.done, P.d2h) == cudaSuccess) cudaStreamWaitEvent(s, P.done, 0);
+        return result;
+    };
+    const uint8_t *xh = static_cast<const uint8_t *>(x_host);
+    uint8_t *yh = static_cast<uint8_t *>(y_host);
+    const int64_t nchunks = (M + C - 1) / C;
+    for (int64_t i = 0; i < nchunks; ++i) {
+        const int sl = (int)(i & 1);
+        const int64_t r0 = i * C;
+        const int64_t rows = M - r0 < C ? M - r0 : C;
+        // copy in (waits for the compute that last read this staging slot)
+        if (i >= 2 && cudaStreamWaitEvent(P.h2d, P.x_free[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        if (cudaMemcpy2DAsync(xs[sl], (size_t)D * 2, xh + (size_t)r0 * ldx * 2, (size_t)ldx * 2, (size_t)D * 2,
+                              (size_t)rows, cudaMemcpyHostToDevice, P.h2d) != cudaSuccess ||
+            cudaEventRecord(P.x_ready[sl], P.h2d) != cudaSuccess)
+            return join(HIF4_ERR_CUDA);
+        // compute
+        if (cudaStreamWaitEvent(s, P.x_ready[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = fake_quantize_bf16(xs[sl], rows, D, D, n_mask1 > 0 ? mask1 : nullptr, xhat1, D, status, s);
+        if (st != HIF4_OK) return join(st);
+        if (cudaEventRecord(P.x_free[sl], s) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = launch_gemm(xhat1, rows, D, D, what1, F, D, b1, n_mask2 > 0 ? mask2 : nullptr, hhat, F,
+                         HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, s);
+        if (st != HIF4_OK) return join(st);
+        if (i >= 2 && cudaStreamWaitEvent(s, P.y_free[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = launch_gemm(hhat, rows, F, F, what2, D, F, b2, nullptr, ys[sl], D, flags, status, s);
+        if (st != HIF4_OK) return join(st);
+        if (cudaEventRecord(P.y_ready[sl], s) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        // copy out
+        if (cudaStreamWaitEvent(P.d2h, P.y_ready[sl], 0) != cudaSuccess ||
+            cudaMemcpy2DAsync(yh + (size_t)r0 * ldy * ysz, (size_t)ldy * ysz, ys[sl], (size_t)D * ysz,
+                              (size_t)D * ysz, (size_t)rows, cudaMemcpyDeviceToHost, P.d2h) != cudaSuccess ||
+            cudaEventRecord(P.y_free[sl], P.d2h) != cudaSuccess)
+            return join(HIF4_ERR_CUDA);
+    }
+    // the caller's stream completes only after the last row has landed on the host
+    if (cudaEventRecord(P.done, P.d2h) != cudaSuccess || cudaStreamWaitEvent(s, P.done, 0) != cudaSuccess)
+        return join(HIF4_ERR_CUDA);
+    return HIF4_OK;
 }

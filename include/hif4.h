@@ -221,6 +221,31 @@ hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_t ldx,
                           size_t ws_bytes, uint32_t *status, hif4_stream_t stream);
 
 /*
+ * hif4_ffn_w4a4_host — hif4_ffn_w4a4 on HOST activations: x_host (BF16
+ * M x D, ldx) and y_host (BF16, or FP32 with HIF4_LINEAR_OUT_F32, M x D,
+ * ldy) are host buffers.  The rows stream through the GPU in chunks of
+ * chunk_rows (0 = automatic: at most 8192, whole 128-row tiles), the copy of
+ * chunk i+1 to the device and of chunk i-1 back to the host overlapping the
+ * compute of chunk i (two internal copy streams, double-buffered staging in
+ * the workspace).  The results equal hif4_ffn_w4a4 on the same rows.
+ * Page-locked host buffers (cudaHostAlloc / cudaHostRegister) are needed for
+ * the overlap; pageable ones give the same results with serialized copies.
+ * Asynchronous on `stream`: when `stream` completes, y_host holds the
+ * result; x_host and y_host must stay valid until then.
+ * workspace >= hif4_ffn_w4a4_host_workspace(M, D, F, chunk_rows, flags)
+ * bytes, 256-byte aligned.  Other arguments and errors as hif4_ffn_w4a4.
+ */
+size_t hif4_ffn_w4a4_host_workspace(int64_t M, int64_t D, int64_t F, int64_t chunk_rows, uint32_t flags);
+hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t D, int64_t ldx,
+                               const uint8_t *w1_codes, const uint32_t *w1_meta, int64_t F,
+                               const int32_t *mask1_idx, int32_t n_mask1, const void *w1_masked,
+                               const void *b1, const uint8_t *w2_codes, const uint32_t *w2_meta,
+                               const int32_t *mask2_idx, int32_t n_mask2, const void *w2_masked,
+                               const void *b2, void *y_host, int64_t ldy, int64_t chunk_rows,
+                               uint32_t flags, void *workspace, size_t ws_bytes, uint32_t *status,
+                               hif4_stream_t stream);
+
+/*
  * hif4_calib_percentile_mask — tail-aware percentile calibration and the
  * channel mask [TA summary "Why tail percentiles"; TA abstract].
  *   pct[c]   = the |x| value (as non-negative BF16) at 0-based ascending rank

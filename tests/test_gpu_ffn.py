@@ -187,3 +187,42 @@ def test_ffn_full_size(H):
     idx2 = np.nonzero(m2)[0].astype(np.int32)
     run_ffn(H, d["x"], d["w1"], d["w2"], idx1, idx2, None, None, rows=rows)
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("M,chunk", [(1000, 256), (777, 0), (300, 1000)])
+def test_ffn_host_pipeline_equals_device_call(H, M, chunk):
+    """hif4_ffn_w4a4_host (pinned host x / y, chunked, copies overlapping
+    compute) gives exactly the rows hif4_ffn_w4a4 gives on device buffers:
+    per-row work and per-element accumulation order do not depend on the
+    chunking.  Strided host rows, a ragged last chunk and FP32 output."""
+    import torch
+    D, F = 256, 512
+    rng = np.random.default_rng(M + chunk)
+    x_bits = _bf16(rng, (M, D))
+    w1, w2 = _bf16(rng, (F, D), 1.0 / 16), _bf16(rng, (D, F), 1.0 / 22)
+    b1, b2 = to_dev_bf16(_bf16(rng, (F,), 0.1)), to_dev_bf16(_bf16(rng, (D,), 0.1))
+    idx1 = np.array([3, 77], np.int32)
+    idx2 = np.sort(rng.choice(F, 6, replace=False)).astype(np.int32)
+    w1c, w1m = _quantize_w(H, w1, idx1)
+    w2c, w2m = _quantize_w(H, w2, idx2)
+    i1 = torch.from_numpy(idx1).cuda()
+    i2 = torch.from_numpy(idx2).cuda()
+    w1k = to_dev_bf16(np.ascontiguousarray(w1[:, idx1]))
+    w2k = to_dev_bf16(np.ascontiguousarray(w2[:, idx2]))
+    args = (w1c, w1m, F, w2c, w2m, i1, w1k, b1, i2, w2k, b2)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y_dev = H.ffn_w4a4(to_dev_bf16(x_bits), *args, status=status)
+    y_dev32 = H.ffn_w4a4(to_dev_bf16(x_bits), *args, status=status,
+                         out=torch.empty(M, D, dtype=torch.float32, device="cuda"))
+    # host rows with a leading dimension larger than D
+    xh = torch.zeros(M, D + 64, dtype=torch.bfloat16, pin_memory=True)
+    xh[:, :D] = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16)
+    yh = torch.full((M, D + 32), float("nan"), dtype=torch.bfloat16, pin_memory=True)
+    H.ffn_w4a4_host(xh[:, :D], *args, out=yh[:, :D], chunk_rows=chunk, status=status)
+    yh32 = H.ffn_w4a4_host(xh[:, :D], *args, out=torch.empty(M, D, dtype=torch.float32, pin_memory=True),
+                           chunk_rows=chunk, status=status)
+    torch.cuda.synchronize()
+    assert H.get_status(status) == 0
+    assert torch.equal(yh[:, :D].view(torch.int16), y_dev.cpu().view(torch.int16))
+    assert torch.isnan(yh[:, D:]).all()                       # the padding past D is untouched
+    assert torch.equal(yh32.view(torch.int32), y_dev32.cpu().view(torch.int32))
