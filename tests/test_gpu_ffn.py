@@ -189,12 +189,14 @@ def test_ffn_full_size(H):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("M,chunk", [(1000, 256), (777, 0), (300, 1000)])
+@pytest.mark.parametrize("M,chunk", [(1000, 256), (777, 0), (300, 1000), (40000, 0)])
 def test_ffn_host_pipeline_equals_device_call(H, M, chunk):
     """hif4_ffn_w4a4_host (pinned host x / y, chunked, copies overlapping
     compute) gives exactly the rows hif4_ffn_w4a4 gives on device buffers:
     per-row work and per-element accumulation order do not depend on the
-    chunking.  Strided host rows, a ragged last chunk and FP32 output."""
+    chunking.  Strided host rows, a ragged last chunk, the automatic ramped
+    schedule (40000 rows: 1024, 2048, 4096, 4 middle chunks, 4096, 2048,
+    1024) and FP32 output."""
     import torch
     D, F = 256, 512
     rng = np.random.default_rng(M + chunk)
