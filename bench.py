@@ -392,11 +392,33 @@ def main():
         e1.record(stream)
         barrier()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        # the copies alone (same bytes, both directions at once, no compute):
+        # the end-to-end bound when they take longer than the compute
+        yd = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+        xd = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+            with torch.cuda.stream(s_in):
+                xd.copy_(xh, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                yh.copy_(yd, non_blocking=True)
+            stream.wait_stream(s_in)
+            stream.wait_stream(s_out)
+        c1.record(stream)
+        barrier()
+        copy_ms = max_over_ranks(c0.elapsed_time(c1) / args.steps)
         line["e2e"] = {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                        "h2d_bytes_per_step": M * D * 2, "d2h_bytes_per_step": M * D * 2,
                        "ms_per_step": e2e_ms,
+                       "copies_alone_ms_per_step": copy_ms,
+                       "bound": "host copies" if copy_ms > ms_step else "compute",
                        "api": "hif4_ffn_w4a4_host: pinned host X in, Y out, copies overlapped with compute"}
-        del xh, yh, ws
+        del xh, yh, ws, xd, yd
 
     del xhat1, xhat2, what1, what2, ybuf, x
     torch.cuda.empty_cache()
