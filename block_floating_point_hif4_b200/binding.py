@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libhif4.so")
 
 OK = 0
 ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_SHAPE, ERR_WORKSPACE = 1, 2, 3, 4
-ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED = 5, 6, 7, 8
+ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_FORMAT = 5, 6, 7, 8, 9
 F32, BF16 = 0, 1
 FLAG_NONFINITE, FLAG_TIMEOUT, FLAG_BAD_INDEX = 1, 2, 4
 LINEAR_GELU_TANH = 1
@@ -50,6 +50,10 @@ SIGNATURES = {
     "hif4_calib_noalloc_scratch_bytes": (_SZ, []),
     "hif4_calib_percentile_mask_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P,
                                                           _P, _P, _P]),
+    "hif4_ptq_state_bytes": (_SZ, [_I64, _I64, _I32]),
+    "hif4_ptq_state_pack": (ctypes.c_int, [_I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ]),
+    "hif4_ptq_state_info": (ctypes.c_int, [_P, _SZ, _P, _P, _P]),
+    "hif4_ptq_state_unpack": (ctypes.c_int, [_P, _SZ, _P, _P, _P, _P]),
     "hif4_get_status": (ctypes.c_int, [_P, _P]),
     "hif4_reset_status": (ctypes.c_int, [_P, _P]),
     "hif4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -310,6 +314,47 @@ def calib_percentile_mask(acts: torch.Tensor, q=(999, 1000), frac=(1, 100), *, w
         _ptr(acts), T, C, acts.stride(0), q[0], q[1], frac[0], frac[1], _ptr(pct), _ptr(ratio), _ptr(mask),
         _ptr(midx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return pct, ratio, mask, midx[:n_top]
+
+
+def ptq_state_pack(codes: torch.Tensor, meta: torch.Tensor, mask_idx: torch.Tensor | None = None,
+                   w_masked: torch.Tensor | None = None) -> bytes:
+    """Compact PTQ state record of one layer (see hif4.h) from its HiF4 codes
+    [N, K/2] u8, meta [N, K/64] i32, protected indices [n] i32 and their BF16
+    weight columns [N, n]; tensors on any device (copied to host memory)."""
+    c = codes.detach().to("cpu").contiguous()
+    m = meta.detach().to("cpu").contiguous()
+    N, K = c.shape[0], c.shape[1] * 2
+    n = 0 if mask_idx is None else int(mask_idx.numel())
+    idx = None if n == 0 else mask_idx.detach().to("cpu", torch.int32).contiguous()
+    wm = None if n == 0 else w_masked.detach().to("cpu").contiguous()
+    size = int(lib().hif4_ptq_state_bytes(N, K, n))
+    if size == 0:
+        raise Hif4Error("hif4_ptq_state_bytes", ERR_INVALID_ARG)
+    out = ctypes.create_string_buffer(size)
+    _check("hif4_ptq_state_pack", lib().hif4_ptq_state_pack(
+        N, K, _ptr(c), _ptr(m), _ptr(idx), n, _ptr(wm), ctypes.cast(out, ctypes.c_void_p), size))
+    return out.raw
+
+
+def ptq_state_unpack(record: bytes, device=None):
+    """-> (codes u8 [N, K/2], meta i32 [N, K/64], mask_idx i32 [n] or None,
+    w_masked bf16 [N, n] or None), on `device` (default: host)."""
+    buf = ctypes.create_string_buffer(bytes(record), len(record))
+    N, K, n = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+    _check("hif4_ptq_state_info", lib().hif4_ptq_state_info(
+        ctypes.cast(buf, ctypes.c_void_p), len(record), ctypes.byref(N), ctypes.byref(K), ctypes.byref(n)))
+    N, K, n = N.value, K.value, n.value
+    codes = torch.empty(N, K // 2, dtype=torch.uint8)
+    meta = torch.empty(N, K // 64, dtype=torch.int32)
+    idx = torch.empty(n, dtype=torch.int32) if n else None
+    wm = torch.empty(N, n, dtype=torch.bfloat16) if n else None
+    _check("hif4_ptq_state_unpack", lib().hif4_ptq_state_unpack(
+        ctypes.cast(buf, ctypes.c_void_p), len(record), _ptr(codes), _ptr(meta), _ptr(idx), _ptr(wm)))
+    if device is not None:
+        codes, meta = codes.to(device), meta.to(device)
+        idx = None if idx is None else idx.to(device)
+        wm = None if wm is None else wm.to(device)
+    return codes, meta, idx, wm
 
 
 def get_status(status: torch.Tensor, stream=None) -> int:

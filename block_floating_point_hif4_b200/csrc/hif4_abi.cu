@@ -121,6 +121,7 @@ extern "C" const char *hif4_status_string(hif4_status s)
     case HIF4_ERR_NONFINITE: return "non-finite input mapped (NaN -> 0, Inf -> +-FLT_MAX)";
     case HIF4_ERR_TIMEOUT: return "bounded device wait timed out";
     case HIF4_ERR_UNSUPPORTED: return "unsupported device or size";
+    case HIF4_ERR_FORMAT: return "serialized state malformed, truncated or corrupted";
     }
     return "unknown status";
 }

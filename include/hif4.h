@@ -57,7 +57,8 @@ typedef enum {
     HIF4_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
     HIF4_ERR_NONFINITE = 6,   /* device flag: a NaN/Inf input was mapped */
     HIF4_ERR_TIMEOUT = 7,     /* device flag: a bounded wait gave up */
-    HIF4_ERR_UNSUPPORTED = 8  /* no sm_100 device, or size beyond a limit */
+    HIF4_ERR_UNSUPPORTED = 8, /* no sm_100 device, or size beyond a limit */
+    HIF4_ERR_FORMAT = 9       /* serialized state malformed, truncated or corrupted */
 } hif4_status;
 
 typedef enum { HIF4_F32 = 0, HIF4_BF16 = 1 } hif4_dtype;
@@ -302,6 +303,38 @@ hif4_status hif4_calib_percentile_mask_noalloc(const void *acts, int64_t tokens,
                                                uint32_t mask_num, uint32_t mask_den, void *pct,
                                                float *ratio, uint8_t *mask, int32_t *mask_idx_out,
                                                hif4_stream_t stream);
+
+/*
+ * Compact PTQ state of one linear layer [TA summary, "Method overview":
+ * compact deltas that restore the quantized behaviour are stored instead of
+ * the full BF16 weights]: its HiF4 codes and metadata (as hif4_quantize
+ * writes them, N x K), the protected-column indices and those columns' BF16
+ * weights (as hif4_linear_w4a4 takes them) in one self-describing record.
+ * Version 1 layout (little-endian; sections at 64-byte offsets):
+ *   0 "HIF4PTQS" | 8 u32 version 1 | 12 u32 64 | 16 i64 N | 24 i64 K |
+ *   32 i32 n_masked | 36 u32 0 | 40 u64 total bytes | 48 16 zero bytes |
+ *   64 mask_idx i32[n_masked] | codes u8[N][K/2] | meta u32[N][K/64] |
+ *   w_masked u16[N][n_masked] | u32 CRC-32 (IEEE, reflected 0xEDB88320) of
+ *   every byte before it.
+ * All pointers are HOST pointers; no device is needed.  mask_idx must be
+ * sorted and distinct in [0, K).
+ * hif4_ptq_state_bytes   record size (0 for invalid sizes).
+ * hif4_ptq_state_pack    writes the record into out (>= that size; else
+ *                        WORKSPACE); SHAPE if K % 64, INVALID_ARG otherwise.
+ * hif4_ptq_state_info    checks a record (magic, version, sizes, checksum,
+ *                        indices; FORMAT when any fails) and reports N, K,
+ *                        n_masked (each output pointer may be NULL).
+ * hif4_ptq_state_unpack  checks the record as info does and copies its
+ *                        sections into caller buffers of those sizes.
+ */
+size_t hif4_ptq_state_bytes(int64_t N, int64_t K, int32_t n_masked);
+hif4_status hif4_ptq_state_pack(int64_t N, int64_t K, const uint8_t *codes, const uint32_t *meta,
+                                const int32_t *mask_idx, int32_t n_masked, const void *w_masked,
+                                void *out, size_t out_bytes);
+hif4_status hif4_ptq_state_info(const void *buf, size_t bytes, int64_t *N, int64_t *K,
+                                int32_t *n_masked);
+hif4_status hif4_ptq_state_unpack(const void *buf, size_t bytes, uint8_t *codes, uint32_t *meta,
+                                  int32_t *mask_idx, void *w_masked);
 
 /* Synchronizes `stream`, reads the device status word and maps its bits:
  * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX -> HIF4_ERR_INVALID_ARG,

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_status_strings_and_version(L):
     assert L.hif4_version() >= 100
-    for code in range(9):
+    for code in range(10):
         assert L.hif4_status_string(code)
 
 
