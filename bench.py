@@ -46,7 +46,11 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 # DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
 # hex digits) of the kernel source it was taken on; stale entries read as null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # bench FFN step, 57600 tokens: GEMM 1 (fused fake-quant epilogue) read 4.71 GB + wrote 1.59 GB,
+    # GEMM 2 read 9.21 GB + wrote 0.58 GB (one ncu pass, dram__bytes_read/write.sum); mean per launch
+    ("gemm", "4cfff8d3be964f4f"): 8.045e9,
+}
 
 
 def parse():
@@ -350,7 +354,7 @@ def main():
     gemm_ms = max_over_ranks((stage_ms["gemm_1_gelu_fq"] + stage_ms["gemm_2"]) / 2)
     achieved = flop_gemm / (gemm_ms * 1e-3) / 1e12
     peak = P["bf16_tflops_sustained"]
-    gh = src_hash("hif4_linear.cu", "hif4_sm100.cuh")
+    gh = src_hash("hif4_linear.cu", "hif4_sm100.cuh", "hif4_encode.cuh", "hif4_internal.cuh")
     traffic = NCU_TRAFFIC.get(("gemm", gh))
     roofline = {"kernel": "k_gemm (hif4_gemm_bf16_fq, hif4_gemm_bf16)", "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
