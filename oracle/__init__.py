@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.orc_weight_hat.argtypes = [P, P, i64, i64, P, ctypes.c_int, P, P]
             L.orc_gelu_tanh.restype = ctypes.c_double
             L.orc_gelu_tanh.argtypes = [ctypes.c_double]
+            L.orc_gptq_factor.restype = ctypes.c_int
+            L.orc_gptq_factor.argtypes = [P, i64, ctypes.c_double, P, P]
+            L.orc_higptq1.restype = i64
+            L.orc_higptq1.argtypes = [P, i64, i64, P, P, P, i64, P, P, P, P]
             L.orc_round_bf16.restype = ctypes.c_uint16
             L.orc_round_bf16.argtypes = [ctypes.c_double]
             L.orc_round_bf16_array.restype = None
@@ -179,6 +183,47 @@ def weight_hat(codes, meta, N, K, mask_idx=None, w_masked_bf16=None) -> np.ndarr
 
 def gelu_tanh(x: float) -> float:
     return lib().orc_gelu_tanh(float(x))
+
+
+def gptq_factor(H: np.ndarray, damp: float = 0.01):
+    """-> (U upper K x K with (H + damp mean(diag H) I)^{-1} = U^T U, dead flags K)."""
+    H = np.ascontiguousarray(H, dtype=np.float64)
+    K = H.shape[0]
+    U = np.zeros((K, K), np.float64)
+    dead = np.zeros(K, np.uint8)
+    if lib().orc_gptq_factor(_p(H), K, float(damp), _p(U), _p(dead)) != 0:
+        raise ValueError("Hessian is not positive definite after damping")
+    return U, dead
+
+
+def higptq1(w_bf16: np.ndarray, H: np.ndarray, chan_mask=None, damp: float = 0.01, blocksize: int = 128,
+            threads: int = 1, factor=None):
+    """HiGPTQ scheme one -> (codes N x K/2, meta N x K/64, wq N x K double,
+    w_masked N x n_masked BF16 bits or None).  Rows are independent given the
+    Hessian factor, so they are split over ``threads``."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    N, K = w.shape
+    U, dead = gptq_factor(H, damp) if factor is None else factor
+    cm = None if chan_mask is None else np.ascontiguousarray(chan_mask, dtype=np.uint8)
+    nm = 0 if cm is None else int(np.count_nonzero(cm))
+    codes = np.zeros((N, K // 2), np.uint8)
+    meta = np.zeros((N, K // 64), np.uint32)
+    wq = np.zeros((N, K), np.float64)
+    wm = np.zeros((N, nm), np.uint16) if nm else None
+    L = lib()
+
+    def run(r0, r1):
+        if r1 > r0:
+            off = ctypes.c_void_p
+            rc = L.orc_higptq1(off(w.ctypes.data + r0 * K * 2), r1 - r0, K, _p(U), _p(dead), _p(cm), blocksize,
+                               off(codes.ctypes.data + r0 * (K // 2)), off(meta.ctypes.data + r0 * (K // 64) * 4),
+                               off(wq.ctypes.data + r0 * K * 8),
+                               off(wm.ctypes.data + r0 * nm * 2) if nm else None)
+            if rc != 0:
+                raise ValueError("bad arguments for higptq1")
+
+    _split(N, threads, run)
+    return codes, meta, wq, wm
 
 
 def round_bf16(x) -> np.ndarray:

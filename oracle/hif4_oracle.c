@@ -422,3 +422,176 @@ long orc_channel_mask(const uint16_t *pct, long C, unsigned mask_num,
     free(items);
     return n_top;
 }
+
+/* ----------------------------------------------------------------- HiGPTQ */
+
+/* Upper-triangular error-feedback factor of GPTQ, as HiGPTQ uses it [HiF4
+ * article, section 3.1 (HiGPTQ is GPTQ adapted to the HiF4 unit); GPTQ's
+ * Hessian factor]:
+ *   Hd = H + damp * mean(diag H) * I, after a zero diagonal entry (an input
+ *        channel that never fires) is set to 1 and flagged dead;
+ *   Hd^{-1} = U^T U with U upper triangular.
+ * Steps as stated: Cholesky factor of Hd, the inverse from it, the Cholesky
+ * factor of that inverse.  H and U are K x K, row-major.  dead: K flags or
+ * NULL.  Returns 0, or -1 when Hd is not positive definite. */
+int orc_gptq_factor(const double *H, long K, double damp, double *U, unsigned char *dead)
+{
+    double *A = malloc(sizeof(double) * K * K);
+    double *Li = calloc((size_t)K * K, sizeof(double));
+    if (!A || !Li) {
+        free(A);
+        free(Li);
+        return -1;
+    }
+    memcpy(A, H, sizeof(double) * K * K);
+    double mean = 0.0;
+    for (long i = 0; i < K; ++i) {
+        int d = A[i * K + i] == 0.0;
+        if (d) A[i * K + i] = 1.0;
+        if (dead) dead[i] = (unsigned char)d;
+        mean += A[i * K + i];
+    }
+    mean /= (double)K;
+    for (long i = 0; i < K; ++i) A[i * K + i] += damp * mean;
+    int rc = 0;
+    /* 1. Hd = L L^T (lower L, in the lower triangle of A) */
+    for (long j = 0; j < K && rc == 0; ++j) {
+        double s = A[j * K + j];
+        for (long k = 0; k < j; ++k) s -= A[j * K + k] * A[j * K + k];
+        if (!(s > 0.0)) {
+            rc = -1;
+            break;
+        }
+        A[j * K + j] = sqrt(s);
+        for (long i = j + 1; i < K; ++i) {
+            double t = A[i * K + j];
+            for (long k = 0; k < j; ++k) t -= A[i * K + k] * A[j * K + k];
+            A[i * K + j] = t / A[j * K + j];
+        }
+    }
+    if (rc == 0) {
+        /* 2. L^{-1} (lower), then Hd^{-1} = L^{-T} L^{-1} into U's storage */
+        for (long j = 0; j < K; ++j) {
+            Li[j * K + j] = 1.0 / A[j * K + j];
+            for (long i = j + 1; i < K; ++i) {
+                double t = 0.0;
+                for (long k = j; k < i; ++k) t += A[i * K + k] * Li[k * K + j];
+                Li[i * K + j] = -t / A[i * K + i];
+            }
+        }
+        for (long i = 0; i < K; ++i)
+            for (long j = 0; j < K; ++j) {
+                double t = 0.0;
+                for (long k = i > j ? i : j; k < K; ++k) t += Li[k * K + i] * Li[k * K + j];
+                U[i * K + j] = t;
+            }
+        /* 3. Hd^{-1} = C C^T (lower C), U = C^T */
+        memcpy(A, U, sizeof(double) * K * K);
+        for (long j = 0; j < K && rc == 0; ++j) {
+            double s = A[j * K + j];
+            for (long k = 0; k < j; ++k) s -= A[j * K + k] * A[j * K + k];
+            if (!(s > 0.0)) {
+                rc = -1;
+                break;
+            }
+            A[j * K + j] = sqrt(s);
+            for (long i = j + 1; i < K; ++i) {
+                double t = A[i * K + j];
+                for (long k = 0; k < j; ++k) t -= A[i * K + k] * A[j * K + k];
+                A[i * K + j] = t / A[j * K + j];
+            }
+        }
+        for (long i = 0; i < K && rc == 0; ++i)
+            for (long j = 0; j < K; ++j) U[i * K + j] = j >= i ? A[j * K + i] : 0.0;
+    }
+    free(A);
+    free(Li);
+    return rc;
+}
+
+/* HiGPTQ, scheme one [HiF4 article, section 3.1, first scheme: 64 columns are
+ * quantized at a time; the level-1, level-2 and level-3 exponents of the
+ * group are fixed together, then the remaining weights of the block are
+ * updated].  W: N x K BF16 bits (row-major; a group of 64 columns is one HiF4
+ * unit per row).  U, dead: from orc_gptq_factor.  Per group g of the block
+ * [b0, b1) (blocksize a multiple of 64), for each row:
+ *   Q_g = the unit quantized from the row's current values (encode rule of
+ *         orc_quantize_unit, protected columns excluded from the scale);
+ *         a protected column's value is the BF16 rounding of its current
+ *         weight (what the product uses), since it is not HiF4-coded;
+ *   D   = W_g - Q_g,   E = D U_gg^{-1}   (E U_gg = D, U_gg upper),
+ *   W_c -= E U_{g,c} for the later columns c of the block;
+ * then, once per block, W_c -= E_block U_{block,c} for the columns after it
+ * [GPTQ's error feedback and its lazy blocked update, here per group].
+ * Dead input channels are zeroed first.  Outputs: codes (N x K/2), meta
+ * (N x K/64), wq (N x K quantized values, protected columns included) and
+ * w_masked (N x n_masked BF16 bits of the protected columns in ascending
+ * order; may be NULL).  Returns 0, or -1 on bad arguments. */
+long orc_higptq1(const uint16_t *w, long N, long K, const double *U, const unsigned char *dead,
+                 const unsigned char *chan_mask, long blocksize, unsigned char *codes, uint32_t *meta,
+                 double *wq, uint16_t *w_masked)
+{
+    if (N <= 0 || K <= 0 || K % ORC_UNIT || blocksize <= 0 || blocksize % ORC_UNIT) return -1;
+    double *W = malloc(sizeof(double) * K);
+    double *E = malloc(sizeof(double) * blocksize);
+    if (!W || !E) {
+        free(W);
+        free(E);
+        return -1;
+    }
+    for (long n = 0; n < N; ++n) {
+        for (long k = 0; k < K; ++k) W[k] = (dead && dead[k]) ? 0.0 : orc_bf16_to_double(w[n * K + k]);
+        for (long b0 = 0; b0 < K; b0 += blocksize) {
+            const long b1 = b0 + blocksize < K ? b0 + blocksize : K;
+            for (long g0 = b0; g0 < b1; g0 += ORC_UNIT) {
+                unsigned char nib[ORC_UNIT];
+                uint32_t m;
+                orc_quantize_unit(W + g0, chan_mask ? chan_mask + g0 : NULL, nib, &m);
+                double D[ORC_UNIT];
+                for (int i = 0; i < ORC_UNIT; ++i) {
+                    const long col = g0 + i;
+                    double q;
+                    if (chan_mask && chan_mask[col])
+                        q = orc_bf16_to_double(orc_round_bf16(W[col]));
+                    else
+                        q = orc_decode_element(nib[i], m, i);
+                    wq[n * K + col] = q;
+                    D[i] = W[col] - q;
+                    if (i % 2 == 0) codes[n * (K / 2) + col / 2] = 0;
+                    codes[n * (K / 2) + col / 2] |= (unsigned char)(nib[i] << (4 * (i % 2)));
+                }
+                meta[n * (K / ORC_UNIT) + g0 / ORC_UNIT] = m;
+                /* E U_gg = D, U_gg upper triangular: forward over the columns */
+                for (int j = 0; j < ORC_UNIT; ++j) {
+                    double t = D[j];
+                    for (int i = 0; i < j; ++i) t -= E[g0 - b0 + i] * U[(g0 + i) * K + g0 + j];
+                    E[g0 - b0 + j] = t / U[(g0 + j) * K + g0 + j];
+                }
+                /* the later columns of this block */
+                for (long c = g0 + ORC_UNIT; c < b1; ++c) {
+                    double t = 0.0;
+                    for (int j = 0; j < ORC_UNIT; ++j) t += E[g0 - b0 + j] * U[(g0 + j) * K + c];
+                    W[c] -= t;
+                }
+            }
+            /* the columns after the block, once */
+            for (long c = b1; c < K; ++c) {
+                double t = 0.0;
+                for (long j = b0; j < b1; ++j) t += E[j - b0] * U[j * K + c];
+                W[c] -= t;
+            }
+        }
+    }
+    free(W);
+    free(E);
+    if (w_masked && chan_mask) {
+        long nm = 0;
+        for (long k = 0; k < K; ++k) nm += chan_mask[k] != 0;
+        for (long n = 0; n < N; ++n) {
+            long j = 0;
+            for (long k = 0; k < K; ++k)
+                if (chan_mask[k]) w_masked[n * nm + j++] = orc_round_bf16(wq[n * K + k]);
+        }
+    }
+    return 0;
+}
