@@ -50,6 +50,11 @@ SIGNATURES = {
     "hif4_calib_noalloc_scratch_bytes": (_SZ, []),
     "hif4_calib_percentile_mask_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _U32, _U32, _U32, _U32, _P, _P,
                                                           _P, _P, _P]),
+    "hif4_hessian_workspace": (_SZ, [_I64, _I64]),
+    "hif4_hessian": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
+    "hif4_higptq1_workspace": (_SZ, [_I64, _I64, _I64]),
+    "hif4_higptq1": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, ctypes.c_double, _I64, _P, _P, _P, _P,
+                                    _SZ, _P, _P]),
     "hif4_ptq_state_bytes": (_SZ, [_I64, _I64, _I32]),
     "hif4_ptq_state_pack": (ctypes.c_int, [_I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ]),
     "hif4_ptq_state_info": (ctypes.c_int, [_P, _SZ, _P, _P, _P]),
@@ -314,6 +319,40 @@ def calib_percentile_mask(acts: torch.Tensor, q=(999, 1000), frac=(1, 100), *, w
         _ptr(acts), T, C, acts.stride(0), q[0], q[1], frac[0], frac[1], _ptr(pct), _ptr(ratio), _ptr(mask),
         _ptr(midx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return pct, ratio, mask, midx[:n_top]
+
+
+def hessian(x: torch.Tensor, *, out=None, workspace=None, status=None, stream=None):
+    """H = XᵀX (FP32 K x K) of BF16 activations X (T x K)."""
+    _dev(x, "x")
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    T, K = x.shape
+    if out is None:
+        out = torch.empty(K, K, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, int(lib().hif4_hessian_workspace(T, K))), dtype=torch.uint8, device=x.device)
+    _check("hif4_hessian", lib().hif4_hessian(_ptr(x), T, K, x.stride(0), _ptr(out), _ptr(workspace),
+                                              workspace.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def higptq1(w: torch.Tensor, H: torch.Tensor, mask_idx: torch.Tensor | None = None, damp: float = 0.01,
+            blocksize: int = 128, *, workspace=None, status=None, stream=None):
+    """HiGPTQ scheme one -> (codes u8 [N, K/2], meta i32 [N, K/64], w_masked bf16 [N, n] or None)."""
+    _dev(w, "w")
+    assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.stride(1) == 1
+    assert H.dtype == torch.float32 and H.is_contiguous()
+    N, K = w.shape
+    n = 0 if mask_idx is None else int(mask_idx.numel())
+    codes = torch.empty(N, K // 2, dtype=torch.uint8, device=w.device)
+    meta = torch.empty(N, K // 64, dtype=torch.int32, device=w.device)
+    wm = torch.empty(N, n, dtype=torch.bfloat16, device=w.device) if n else None
+    if workspace is None:
+        need = int(lib().hif4_higptq1_workspace(N, K, blocksize))
+        workspace = torch.empty(max(1, need), dtype=torch.uint8, device=w.device)
+    _check("hif4_higptq1", lib().hif4_higptq1(
+        _ptr(w), N, K, w.stride(0), _ptr(H), _ptr(mask_idx) if n else None, n, float(damp), blocksize,
+        _ptr(codes), _ptr(meta), _ptr(wm), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
+    return codes, meta, wm
 
 
 def ptq_state_pack(codes: torch.Tensor, meta: torch.Tensor, mask_idx: torch.Tensor | None = None,

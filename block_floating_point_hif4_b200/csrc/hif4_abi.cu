@@ -96,7 +96,7 @@ extern "C" hif4_status hif4_get_status(const uint32_t *status_word, hif4_stream_
         return HIF4_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return HIF4_ERR_CUDA;
     if (w & HIF4_FLAG_TIMEOUT) return HIF4_ERR_TIMEOUT;
-    if (w & HIF4_FLAG_BAD_INDEX) return HIF4_ERR_INVALID_ARG;
+    if (w & (HIF4_FLAG_BAD_INDEX | HIF4_FLAG_NOT_SPD)) return HIF4_ERR_INVALID_ARG;
     if (w & HIF4_FLAG_NONFINITE) return HIF4_ERR_NONFINITE;
     return HIF4_OK;
 }

@@ -67,6 +67,7 @@ typedef enum { HIF4_F32 = 0, HIF4_BF16 = 1 } hif4_dtype;
 #define HIF4_FLAG_NONFINITE 0x1u /* NaN -> 0, +-Inf -> +-FLT_MAX was applied */
 #define HIF4_FLAG_TIMEOUT 0x2u   /* a pipeline wait hit its iteration limit */
 #define HIF4_FLAG_BAD_INDEX 0x4u /* a mask index was out of range or unsorted */
+#define HIF4_FLAG_NOT_SPD 0x8u   /* a damped Hessian was not positive definite (HiGPTQ) */
 
 /* Flags of hif4_linear_w4a4 / hif4_gemm_bf16. */
 #define HIF4_LINEAR_GELU_TANH 0x1u /* y = gelu_tanh(acc + bias) */
@@ -305,6 +306,50 @@ hif4_status hif4_calib_percentile_mask_noalloc(const void *acts, int64_t tokens,
                                                hif4_stream_t stream);
 
 /*
+ * hif4_hessian — H = X^T X (FP32, K x K) of a layer's input activations X
+ * (BF16 T x K, ldx), the second-moment matrix HiGPTQ weighs the weight
+ * error with.  Tensor-core product with FP32 accumulation (the BF16 products
+ * are exact).  workspace >= hif4_hessian_workspace(T, K) bytes (X^T, rows
+ * padded to a multiple of 64), 256-byte aligned; H 16-byte aligned.
+ * Errors: SHAPE (K % 64, ldx < K), ALIGNMENT, WORKSPACE, INVALID_ARG.
+ */
+size_t hif4_hessian_workspace(int64_t T, int64_t K);
+hif4_status hif4_hessian(const void *x, int64_t T, int64_t K, int64_t ldx, float *H, void *workspace,
+                         size_t ws_bytes, uint32_t *status, hif4_stream_t stream);
+
+/*
+ * hif4_higptq1 — HiGPTQ, scheme one [HiF4 article, section 3.1: 64 columns
+ * (one HiF4 unit per row) are quantized at a time with the level-1, level-2
+ * and level-3 exponents fixed together; the remaining weights of the block
+ * are then updated; GPTQ's Hessian error feedback]:
+ *   Hd = H + damp * mean(diag H) * I (a zero diagonal entry -- a dead input
+ *        channel -- is set to 1 and its weights to 0); Hd^{-1} = U^T U;
+ *   for each block of `blocksize` columns and each 64-column group g in it,
+ *   per row:  Q_g = HiF4 quantization of the row's current values (encode
+ *   rule of hif4_quantize; protected columns are excluded from the scale and
+ *   take the BF16 rounding of their current value),  E = (W_g - Q_g) U_gg^-1,
+ *   W_c -= E U_{g,c} for the later columns of the block, and after the block
+ *   W_c -= E_block U_{block,c} for every later column.
+ * w       BF16 N x K (ldw), the layer weight.   H  FP32 K x K (symmetric).
+ * mask_idx  NULL or n_masked sorted distinct columns kept in BF16.
+ * damp    relative damping (>= 0; 0.01 is customary).
+ * blocksize  64, 128 (0 = 128), 192 or 256.
+ * codes / meta  out: HiF4 N x K/2 and N x K/64 (as hif4_quantize writes
+ *         them, protected columns coded 0), ready for hif4_linear_w4a4;
+ * w_masked  out: BF16 N x n_masked, the protected columns' final values.
+ * workspace >= hif4_higptq1_workspace(N, K, blocksize), 256-byte aligned.
+ * The factor runs in FP64, the group loop in FP32.  Device flags: NOT_SPD
+ * (Hd not positive definite), BAD_INDEX, NONFINITE (non-finite weights,
+ * mapped as hif4_quantize maps them).  Errors: SHAPE (K % 64, ldw < K),
+ * UNSUPPORTED (K > 32768), ALIGNMENT, WORKSPACE, INVALID_ARG.
+ */
+size_t hif4_higptq1_workspace(int64_t N, int64_t K, int64_t blocksize);
+hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t ldw, const float *H,
+                         const int32_t *mask_idx, int32_t n_masked, double damp, int64_t blocksize,
+                         uint8_t *codes, uint32_t *meta, void *w_masked, void *workspace, size_t ws_bytes,
+                         uint32_t *status, hif4_stream_t stream);
+
+/*
  * Compact PTQ state of one linear layer [TA summary, "Method overview":
  * compact deltas that restore the quantized behaviour are stored instead of
  * the full BF16 weights]: its HiF4 codes and metadata (as hif4_quantize
@@ -337,7 +382,7 @@ hif4_status hif4_ptq_state_unpack(const void *buf, size_t bytes, uint8_t *codes,
                                   int32_t *mask_idx, void *w_masked);
 
 /* Synchronizes `stream`, reads the device status word and maps its bits:
- * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX -> HIF4_ERR_INVALID_ARG,
+ * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX or NOT_SPD -> HIF4_ERR_INVALID_ARG,
  * NONFINITE -> HIF4_ERR_NONFINITE, none -> HIF4_OK.  The word is not cleared. */
 hif4_status hif4_get_status(const uint32_t *status_word, hif4_stream_t stream);
 /* Clears the device status word (asynchronously, on `stream`). */

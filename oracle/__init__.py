@@ -186,9 +186,22 @@ def gelu_tanh(x: float) -> float:
 
 
 def gptq_factor(H: np.ndarray, damp: float = 0.01):
-    """-> (U upper K x K with (H + damp mean(diag H) I)^{-1} = U^T U, dead flags K)."""
+    """-> (U upper K x K with (H + damp mean(diag H) I)^{-1} = U^T U, dead flags K).
+
+    Up to K = 1024 the C routine (textbook loops); beyond, the same three
+    steps with numpy's Cholesky and inverse (library primitives), which the
+    CPU tests pin against the C routine."""
     H = np.ascontiguousarray(H, dtype=np.float64)
     K = H.shape[0]
+    if K > 1024:
+        Hd = H.copy()
+        dead = (np.diag(Hd) == 0).astype(np.uint8)
+        Hd[np.diag_indices(K)] = np.where(dead == 1, 1.0, np.diag(Hd))
+        Hd[np.diag_indices(K)] += damp * np.mean(np.diag(Hd))
+        L = np.linalg.cholesky(Hd)
+        Li = np.linalg.inv(L)
+        U = np.linalg.cholesky(Li.T @ Li).T
+        return np.ascontiguousarray(U), dead
     U = np.zeros((K, K), np.float64)
     dead = np.zeros(K, np.uint8)
     if lib().orc_gptq_factor(_p(H), K, float(damp), _p(U), _p(dead)) != 0:

@@ -50,6 +50,22 @@ def test_factor_matches_numpy(K):
     assert np.array_equal(np.tril(U, -1), np.zeros_like(U))
 
 
+def test_large_k_factor_path_matches_the_c_routine():
+    """Above K = 1024 the factor uses numpy's Cholesky and inverse; at the
+    boundary both paths must agree."""
+    rng = np.random.default_rng(12)
+    H = _hessian(rng, 3000, 1088)
+    U_np, d_np = oracle.gptq_factor(H, 0.01)                       # K = 1088: numpy path
+    import ctypes
+    K = H.shape[0]
+    U_c = np.zeros((K, K))
+    dead = np.zeros(K, np.uint8)
+    rc = oracle.lib().orc_gptq_factor(H.ctypes.data_as(ctypes.c_void_p), K, 0.01,
+                                      U_c.ctypes.data_as(ctypes.c_void_p), dead.ctypes.data_as(ctypes.c_void_p))
+    assert rc == 0 and np.array_equal(dead, d_np)
+    assert np.allclose(U_np, U_c, rtol=1e-8, atol=1e-10 * np.abs(U_c).max())
+
+
 @pytest.mark.parametrize("kind", ["identity", "block_diagonal"])
 def test_no_cross_group_coupling_reduces_to_plain_quantization(kind):
     rng = np.random.default_rng(3)
