@@ -4,9 +4,11 @@ command to put under a profiler (ncu) or to time one kernel in isolation.
     python -m block_floating_point_hif4_b200.profile OP [--log2n N] [--tokens T] [--reps R]
 
 OP: quantize | dequantize | fake_quantize | gemm | gemm_gelu | gemm_fq | calib |
-linear | ffn.  gemm_fq is the FFN's first GEMM: bias-free, tanh-GELU and the
+linear | ffn | higptq.  gemm_fq is the FFN's first GEMM: bias-free, tanh-GELU and the
 HiF4 fake quantization of its output (1 % protected columns) in the epilogue;
-ffn is the whole W4A4 FFN block (hif4_ffn_w4a4, --n = hidden width).
+ffn is the whole W4A4 FFN block (hif4_ffn_w4a4, --n = hidden width);
+higptq times HiGPTQ scheme one on an --n x --channels weight with the
+Hessian of --tokens activation rows (the Hessian itself untimed).
 Sizes default to small cases that still exceed the 126 MB L2 (a few hundred
 MB on the device).  Prints the mean CUDA-event time per call.
 """
@@ -19,7 +21,7 @@ import sys
 def main(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "gemm", "gemm_gelu", "gemm_fq",
-                                  "calib", "linear", "ffn"])
+                                  "calib", "linear", "ffn", "higptq"])
     p.add_argument("--log2n", type=int, default=28, help="elements for quantize/dequantize/fake_quantize")
     p.add_argument("--tokens", type=int, default=57600)
     p.add_argument("--channels", type=int, default=5120)
@@ -43,6 +45,14 @@ def main(argv=None):
               "dequantize": lambda: H.dequantize(codes, meta, 1024, out=y),
               "fake_quantize": lambda: H.fake_quantize(x, out=y)}[a.op]
         nbytes = n * (4.0 if a.op == "fake_quantize" else 2.5625)
+    elif a.op == "higptq":
+        x, _ = wl.device_rows(a.tokens, a.channels, seed=3, device=dev)
+        w = wl.device_weight(a.n, a.channels, 0.015, seed=31, device=dev)
+        Hm = H.hessian(x)
+        del x
+        ws = torch.empty(H.lib().hif4_higptq1_workspace(a.n, a.channels, 128), dtype=torch.uint8, device=dev)
+        fn = lambda: H.higptq1(w, Hm, None, 0.01, 128, workspace=ws)  # noqa: E731
+        nbytes = 2.0 * a.n * a.channels * a.channels / 2        # FLOPs of the lazy updates (N K^2 / 2 FMA)
     elif a.op == "calib":
         x = wl.calib_torch(a.tokens, a.channels, dev)
         ws = torch.empty(H.calib_workspace(a.tokens, a.channels), dtype=torch.uint8, device=dev)
@@ -82,7 +92,7 @@ def main(argv=None):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.reps
-    unit = "TFLOP/s" if a.op in ("gemm", "gemm_gelu", "gemm_fq", "linear", "ffn") else "GB/s"
+    unit = "TFLOP/s" if a.op in ("gemm", "gemm_gelu", "gemm_fq", "linear", "ffn", "higptq") else "GB/s"
     rate = nbytes / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print("%s: %.4f ms per call, %.1f %s" % (a.op, ms, rate, unit))
     return 0

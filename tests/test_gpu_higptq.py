@@ -49,10 +49,6 @@ def _objective(w_bits, wq, Hd):
     return float(np.einsum("nk,kl,nl->", d, Hd, d))
 
 
-def _decode(codes, meta, K):
-    return oracle.dequantize(codes, meta.view(np.uint32) if meta.dtype != np.uint32 else meta, K)
-
-
 def run_gpu(Hm, w_bits, Hf32, idx, damp, bs):
     import torch
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
