@@ -107,17 +107,21 @@ __global__ void __launch_bounds__(256) k_potrf_tile(double *A, int64_t K, int kb
         }
         __syncthreads();
     }
-    // inverse of the lower factor, one column per thread
-    if (tid < TB) {
-        const int j = tid;
-        I[j][j] = 1.0 / T[j][j];
-        for (int i = j + 1; i < TB; ++i) {
-            double t = 0.0;
-            for (int k = j; k < i; ++k) t += T[i][k] * I[k][j];
-            I[i][j] = -t / T[i][i];
-        }
-    }
+    // inverse of the lower factor, row by row: I[i][j] = -(sum_{k=j}^{i-1}
+    // T[i][k] I[k][j]) / T[i][i] for j < i; four threads share each column's
+    // dot product (lanes 4j..4j+3 of the block, combined by shuffles)
+    if (tid < TB) I[tid][tid] = 1.0 / T[tid][tid];
     __syncthreads();
+    for (int i = 1; i < TB; ++i) {
+        const int j = tid >> 2, part = tid & 3;
+        double t = 0.0;
+        if (j < i)
+            for (int k = j + part; k < i; k += 4) t += T[i][k] * I[k][j];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        if (j < i && part == 0) I[i][j] = -t * I[i][i];
+        __syncthreads();
+    }
     for (int e = tid; e < TB * TB; e += 256) {
         const int r = e / TB, c = e % TB;
         if (c <= r) a0[(int64_t)r * K + c] = T[r][c];
@@ -214,45 +218,53 @@ __global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb)
         for (int j = 0; j < 4; ++j) c[(int64_t)(r0 + i) * K + c0 + j] -= acc[i][j];
 }
 
-// Block row i of Y = L^{-1} (lower): Y[i][i] = Linv_i and, for j < i,
-// Y[i][j] = -Linv_i sum_{k=j}^{i-1} L[i][k] Y[k][j].  One block per j <= i
-// (blockIdx.x = j); rows of Y above i are complete.
-__global__ void __launch_bounds__(256) k_trtri_row(const double *A, int64_t K, int i, const double *LinvAll,
-                                                   double *Y)
+// Y = L^{-1} (lower, tile rows), right-looking.  Y starts at zero and
+// accumulates S[i][j] = sum_{k<i} L[i][k] Y[k][j] in place; at step k block
+// row k is finalized (k_trtri_finalize: Y[k][k] = Linv_k, Y[k][j] =
+// -Linv_k S[k][j]) and its contribution is added to every later block row
+// (k_trtri_update: S[i][j] += L[i][k] Y[k][j], i > k >= j).
+__global__ void __launch_bounds__(256) k_trtri_finalize(int64_t K, int k, const double *LinvAll, double *Y)
 {
     extern __shared__ double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Z = X + TB;
-    Tile *Acc = Z + TB;
     const int j = blockIdx.x;
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
-    double *y = Y + (int64_t)i * TB * K + (int64_t)j * TB;
-    const double *li = LinvAll + (int64_t)i * TB * TB;
-    if (j == i) {
-        for (int e = threadIdx.x; e < TB * TB; e += 256) y[(int64_t)(e / TB) * K + e % TB] = li[e];
+    const double *lk = LinvAll + (int64_t)k * TB * TB;
+    double *y = Y + (int64_t)k * TB * K + (int64_t)j * TB;
+    if (j == k) {
+        for (int e = threadIdx.x; e < TB * TB; e += 256) y[(int64_t)(e / TB) * K + e % TB] = lk[e];
         return;
     }
-    double acc[4][4] = {};
-    for (int k = j; k < i; ++k) {
-        __syncthreads();
-        tile_load(X, A + (int64_t)i * TB * K + (int64_t)k * TB, K);          // L[i][k]
-        tile_load(Z, Y + (int64_t)k * TB * K + (int64_t)j * TB, K);          // Y[k][j]
-        __syncthreads();
-        tile_mma_nn(acc, X, Z);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) Acc[r0 + a][c0 + b] = acc[a][b];
-    tile_load(X, li, TB);
+    tile_load(X, lk, TB);
+    tile_load(Z, y, K);
     __syncthreads();
     double out[4][4] = {};
-    tile_mma_nn(out, X, Acc);
+    tile_mma_nn(out, X, Z);
+    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) y[(int64_t)(r0 + a) * K + c0 + b] = -out[a][b];
+}
+
+// grid (k + 1, nb - 1 - k): block (j, ii) updates S[k + 1 + ii][j]
+__global__ void __launch_bounds__(256) k_trtri_update(const double *A, int64_t K, int k, double *Y)
+{
+    extern __shared__ double smd[];
+    Tile *X = reinterpret_cast<Tile *>(smd);
+    Tile *Z = X + TB;
+    const int j = blockIdx.x, i = k + 1 + blockIdx.y;
+    tile_load(X, A + (int64_t)i * TB * K + (int64_t)k * TB, K);            // L[i][k]
+    tile_load(Z, Y + (int64_t)k * TB * K + (int64_t)j * TB, K);            // Y[k][j]
+    __syncthreads();
+    double acc[4][4] = {};
+    tile_mma_nn(acc, X, Z);
+    double *s = Y + (int64_t)i * TB * K + (int64_t)j * TB;
+    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) s[(int64_t)(r0 + a) * K + c0 + b] += acc[a][b];
 }
 
 // U[i][j] = Y[K-1-i][K-1-j] for j >= i (FP32, upper), 0 below; and the
@@ -643,13 +655,15 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     double *mean = reinterpret_cast<double *>(ws + L.mean);
     const int nb = (int)(K / TB);
 
-    static bool attr2[64] = {false}, attr2b[64] = {false}, attr2c[64] = {false}, attr3[64] = {false};
+    static bool attr2[64] = {false}, attr2b[64] = {false}, attr2c[64] = {false}, attr2d[64] = {false},
+                attr2e[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (!set_smem_once(k_potrf_tile, 2 * kTileBytes, attr2[dev & 63]) ||
         !set_smem_once(k_panel, 2 * kTileBytes, attr2b[dev & 63]) ||
         !set_smem_once(k_syrk, 2 * kTileBytes, attr2c[dev & 63]) ||
-        !set_smem_once(k_trtri_row, 3 * kTileBytes, attr3[dev & 63]))
+        !set_smem_once(k_trtri_finalize, 2 * kTileBytes, attr2d[dev & 63]) ||
+        !set_smem_once(k_trtri_update, 2 * kTileBytes, attr2e[dev & 63]))
         return HIF4_ERR_CUDA;
 
     // 1. protected columns, Hessian diagonal statistics, FP32 working weights
@@ -680,9 +694,12 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
         }
         if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     }
-    // 3. Y = L'^{-1} by block rows, then U = P Y P and the inverses of U's diagonal blocks
-    for (int i = 0; i < nb; ++i) {
-        k_trtri_row<<<i + 1, 256, 3 * kTileBytes, s>>>(A, K, i, Linv, Y);
+    // 3. Y = L'^{-1} (right-looking by block rows), then U = P Y P and the
+    //    inverses of U's diagonal blocks
+    if (cudaMemsetAsync(Y, 0, (size_t)K * K * 8, s) != cudaSuccess) return HIF4_ERR_CUDA;
+    for (int k = 0; k < nb; ++k) {
+        k_trtri_finalize<<<k + 1, 256, 2 * kTileBytes, s>>>(K, k, Linv, Y);
+        if (k + 1 < nb) k_trtri_update<<<dim3(k + 1, nb - 1 - k), 256, 2 * kTileBytes, s>>>(A, K, k, Y);
         if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     }
     k_build_u<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG);
