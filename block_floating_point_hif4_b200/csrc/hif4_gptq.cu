@@ -88,23 +88,31 @@ __global__ void __launch_bounds__(256) k_potrf_tile(double *A, int64_t K, int kb
     }
     if (tid == 0) bad = 0;
     __syncthreads();
+    // left-looking by columns: T[r][j] -= sum_{k<j} T[r][k] T[j][k] for r >= j
+    // (four threads per row share the dot product), then the pivot and the
+    // scaling of the column below it
+    __shared__ double rpiv;
     for (int j = 0; j < TB; ++j) {
+        const int r = tid >> 2, part = tid & 3;
+        double t = 0.0;
+        if (r >= j)
+            for (int k = part; k < j; k += 4) t += T[r][k] * T[j][k];
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        if (r >= j && part == 0) T[r][j] -= t;
+        __syncthreads();
         if (tid == 0) {
             double d = T[j][j];
             if (!(d > 0.0)) {
                 bad = 1;
                 d = 1.0;
             }
-            T[j][j] = sqrt(d);
+            d = sqrt(d);
+            T[j][j] = d;
+            rpiv = 1.0 / d;
         }
         __syncthreads();
-        for (int r = j + 1 + tid; r < TB; r += 256) T[r][j] /= T[j][j];
-        __syncthreads();
-        const int n = TB - 1 - j;                       // trailing (r, c), j < c <= r
-        for (int e = tid; e < n * n; e += 256) {
-            const int r = j + 1 + e / n, c = j + 1 + e % n;
-            if (c <= r) T[r][c] -= T[r][j] * T[c][j];
-        }
+        if (r > j && part == 0) T[r][j] *= rpiv;
         __syncthreads();
     }
     // inverse of the lower factor, row by row: I[i][j] = -(sum_{k=j}^{i-1}
@@ -451,58 +459,74 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
 }
 
 // C (M x Nc, ldc) -= A (M x Kd, lda) B (Kd x Nc, ldb) in FP32: 128 x 128
-// tiles, 256 threads with 8 x 8 outputs each, k in steps of 8 through shared
-// memory.  Kd is a multiple of 8; M and Nc are ragged (guarded).
-__global__ void __launch_bounds__(256) k_sgemm_sub(float *C, int64_t ldc, const float *A, int64_t lda,
+// tiles, 256 threads with 8 x 8 outputs each, k in steps of 8 through two
+// shared-memory buffers (the next step's tiles are loaded into registers
+// while the current one is multiplied, one barrier per step).  Kd, lda and
+// ldb are multiples of 4 and A, B 16-byte aligned (float4 loads); M and Nc
+// are ragged (guarded).
+__global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, const float *A, int64_t lda,
                                                    const float *B, int64_t ldb, int64_t M, int64_t Nc, int Kd)
 {
-    __shared__ float As[8][128 + 4];
-    __shared__ float Bs[8][128 + 4];
+    __shared__ __align__(16) float As[2][8][128 + 4];
+    __shared__ __align__(16) float Bs[2][8][128 + 4];
     const int tid = threadIdx.x;
     const int64_t m0 = blockIdx.y * 128ll, n0 = blockIdx.x * 128ll;
-    const int tr = tid / 16, tc = tid % 16;           // 16 x 16 threads, 8 x 8 each
+    const int tr = tid / 16, tc = tid % 16;           // 16 x 16 threads, 8 x 8 outputs each
+    const int ar = tid / 2, ak = 4 * (tid % 2);       // A: row ar, k columns ak..ak+3
+    const int bk = tid / 32, bc = 4 * (tid % 32);     // B: k row bk, columns bc..bc+3
+    const int64_t gm = m0 + ar, gn = n0 + bc;
+    float4 ra, rb;
+    auto gload = [&](int k0) {
+        ra = gm < M ? *reinterpret_cast<const float4 *>(A + gm * lda + k0 + ak) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *brow = B + (int64_t)(k0 + bk) * ldb;
+        if (gn + 3 < Nc) {
+            rb = *reinterpret_cast<const float4 *>(brow + gn);
+        } else {
+            rb.x = gn < Nc ? brow[gn] : 0.f;
+            rb.y = gn + 1 < Nc ? brow[gn + 1] : 0.f;
+            rb.z = gn + 2 < Nc ? brow[gn + 2] : 0.f;
+            rb.w = 0.f;
+        }
+    };
+    auto sstore = [&](int b) {
+        As[b][ak][ar] = ra.x;
+        As[b][ak + 1][ar] = ra.y;
+        As[b][ak + 2][ar] = ra.z;
+        As[b][ak + 3][ar] = ra.w;
+        *reinterpret_cast<float4 *>(&Bs[b][bk][bc]) = rb;
+    };
     float acc[8][8] = {};
-    for (int k0 = 0; k0 < Kd; k0 += 8) {
-        // A tile 128 x 8: thread loads 4 elements (row tid / 2, cols 4 (tid % 2) ..)
-        {
-            const int r = tid / 2, kk = 4 * (tid % 2);
-            const int64_t gm = m0 + r;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) As[kk + i][r] = gm < M ? A[gm * lda + k0 + kk + i] : 0.0f;
-        }
-        // B tile 8 x 128: thread loads 4 elements (row tid / 32, cols 4 (tid % 32) ..)
-        {
-            const int kk = tid / 32, c = 4 * (tid % 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int64_t gn = n0 + c + i;
-                Bs[kk][c + i] = gn < Nc ? B[(int64_t)(k0 + kk) * ldb + gn] : 0.0f;
-            }
-        }
-        __syncthreads();
+    gload(0);
+    sstore(0);
+    __syncthreads();
+    for (int k0 = 0, b = 0; k0 < Kd; k0 += 8, b ^= 1) {
+        const bool more = k0 + 8 < Kd;
+        if (more) gload(k0 + 8);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            float av[8], bv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                av[i] = As[kk][tr * 8 + i];
-                bv[i] = Bs[kk][tc * 8 + i];
-            }
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[b][kk][tr * 8]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[b][kk][tr * 8 + 4]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[b][kk][tc * 8]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[b][kk][tc * 8 + 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(av[i], bv[jj], acc[i][jj]);
         }
+        if (more) sstore(b ^ 1);
         __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t gm = m0 + tr * 8 + i;
-        if (gm >= M) continue;
+        const int64_t cm = m0 + tr * 8 + i;
+        if (cm >= M) continue;
+        float *crow = C + cm * ldc;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int64_t gn = n0 + tc * 8 + j;
-            if (gn < Nc) C[gm * ldc + gn] -= acc[i][j];
+        for (int jj = 0; jj < 8; ++jj) {
+            const int64_t cn = n0 + tc * 8 + jj;
+            if (cn < Nc) crow[cn] -= acc[i][jj];
         }
     }
 }
