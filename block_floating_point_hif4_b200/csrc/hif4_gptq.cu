@@ -70,12 +70,14 @@ __global__ void k_fill_reversed(const float *H, int64_t K, const uint8_t *dead, 
 
 // Cholesky factorization of diagonal tile kb of A (lower, in place) and the
 // inverse of the factor into Linv (64 x 64).  One block of 256 threads.
-typedef double Tile[TB + 1];                 // one row of a padded 64 x 64 FP64 tile
-constexpr size_t kTileBytes = sizeof(double) * TB * (TB + 1);
+// One row of a padded 64 x 64 FP64 tile: 66 doubles (528 bytes) keep rows
+// 16-byte aligned for paired loads and offset consecutive rows by 4 banks.
+typedef double Tile[TB + 2];
+constexpr size_t kTileBytes = sizeof(double) * TB * (TB + 2);
 
 __global__ void __launch_bounds__(256) k_potrf_tile(double *A, int64_t K, int kb, double *Linv, uint32_t *status)
 {
-    extern __shared__ double smd[];
+    extern __shared__ __align__(16) double smd[];
     Tile *T = reinterpret_cast<Tile *>(smd);
     Tile *I = T + TB;
     __shared__ int bad;
@@ -145,35 +147,25 @@ __device__ __forceinline__ void tile_load(Tile *S, const double *src, int64_t ld
     for (int e = threadIdx.x; e < TB * TB; e += 256) S[e / TB][e % TB] = src[(int64_t)(e / TB) * ld + e % TB];
 }
 
-// acc += X Y^T (X, Y: 64 x 64 in shared memory)
-__device__ __forceinline__ void tile_mma_nt(double (&acc)[4][4], const Tile *X, const Tile *Y)
+// S = src^T (S[k][c] = src[c][k]): the right operand of an X Y^T product
+// stored k-major, so that the product reads it like an X Y operand.
+__device__ __forceinline__ void tile_load_t(Tile *S, const double *src, int64_t ld)
 {
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
-    for (int k = 0; k < TB; ++k) {
-        double x[4], y[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[i] = X[r0 + i][k];
-            y[i] = Y[c0 + i][k];
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
-    }
+    for (int e = threadIdx.x; e < TB * TB; e += 256) S[e % TB][e / TB] = src[(int64_t)(e / TB) * ld + e % TB];
 }
 
-// acc += X Y (X, Y: 64 x 64 in shared memory)
+// acc += X Y (X, Y: 64 x 64 in shared memory; Y read as pairs along a row)
 __device__ __forceinline__ void tile_mma_nn(double (&acc)[4][4], const Tile *X, const Tile *Y)
 {
     const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
+#pragma unroll 4
     for (int k = 0; k < TB; ++k) {
-        double x[4], y[4];
+        double x[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[i] = X[r0 + i][k];
-            y[i] = Y[k][c0 + i];
-        }
+        for (int i = 0; i < 4; ++i) x[i] = X[r0 + i][k];
+        const double2 ya = *reinterpret_cast<const double2 *>(&Y[k][c0]);
+        const double2 yb = *reinterpret_cast<const double2 *>(&Y[k][c0 + 2]);
+        const double y[4] = {ya.x, ya.y, yb.x, yb.y};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -186,16 +178,16 @@ __device__ __forceinline__ void tile_mma_nn(double (&acc)[4][4], const Tile *X, 
 // before it is written).
 __global__ void __launch_bounds__(256) k_panel(double *A, int64_t K, int kb, const double *Linv)
 {
-    extern __shared__ double smd[];
+    extern __shared__ __align__(16) double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Y = X + TB;
     const int rt = kb + 1 + blockIdx.x;
     double *a = A + (int64_t)rt * TB * K + (int64_t)kb * TB;
     tile_load(X, a, K);
-    tile_load(Y, Linv, TB);
+    tile_load_t(Y, Linv, TB);
     __syncthreads();
     double acc[4][4] = {};
-    tile_mma_nt(acc, X, Y);
+    tile_mma_nn(acc, X, Y);
     const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -210,14 +202,14 @@ __global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb)
 {
     const int ti = kb + 1 + blockIdx.y, tj = kb + 1 + blockIdx.x;
     if (tj > ti) return;
-    extern __shared__ double smd[];
+    extern __shared__ __align__(16) double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Y = X + TB;
     tile_load(X, A + (int64_t)ti * TB * K + (int64_t)kb * TB, K);
-    tile_load(Y, A + (int64_t)tj * TB * K + (int64_t)kb * TB, K);
+    tile_load_t(Y, A + (int64_t)tj * TB * K + (int64_t)kb * TB, K);
     __syncthreads();
     double acc[4][4] = {};
-    tile_mma_nt(acc, X, Y);
+    tile_mma_nn(acc, X, Y);
     double *c = A + (int64_t)ti * TB * K + (int64_t)tj * TB;
     const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
 #pragma unroll
@@ -233,7 +225,7 @@ __global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb)
 // (k_trtri_update: S[i][j] += L[i][k] Y[k][j], i > k >= j).
 __global__ void __launch_bounds__(256) k_trtri_finalize(int64_t K, int k, const double *LinvAll, double *Y)
 {
-    extern __shared__ double smd[];
+    extern __shared__ __align__(16) double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Z = X + TB;
     const int j = blockIdx.x;
@@ -258,7 +250,7 @@ __global__ void __launch_bounds__(256) k_trtri_finalize(int64_t K, int k, const 
 // grid (k + 1, nb - 1 - k): block (j, ii) updates S[k + 1 + ii][j]
 __global__ void __launch_bounds__(256) k_trtri_update(const double *A, int64_t K, int k, double *Y)
 {
-    extern __shared__ double smd[];
+    extern __shared__ __align__(16) double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Z = X + TB;
     const int j = blockIdx.x, i = k + 1 + blockIdx.y;
