@@ -27,6 +27,7 @@ def main(argv=None):
     p.add_argument("--channels", type=int, default=5120)
     p.add_argument("--n", type=int, default=5120, help="output features for gemm/linear")
     p.add_argument("--reps", type=int, default=3)
+    p.add_argument("--blocksize", type=int, default=128, help="HiGPTQ block (64, 128, 192, 256)")
     a = p.parse_args(argv)
 
     import torch
@@ -50,8 +51,9 @@ def main(argv=None):
         w = wl.device_weight(a.n, a.channels, 0.015, seed=31, device=dev)
         Hm = H.hessian(x)
         del x
-        ws = torch.empty(H.lib().hif4_higptq1_workspace(a.n, a.channels, 128), dtype=torch.uint8, device=dev)
-        fn = lambda: H.higptq1(w, Hm, None, 0.01, 128, workspace=ws)  # noqa: E731
+        ws = torch.empty(H.lib().hif4_higptq1_workspace(a.n, a.channels, a.blocksize), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: H.higptq1(w, Hm, None, 0.01, a.blocksize, workspace=ws)  # noqa: E731
         nbytes = 2.0 * a.n * a.channels * a.channels / 2        # FLOPs of the lazy updates (N K^2 / 2 FMA)
     elif a.op == "calib":
         x = wl.calib_torch(a.tokens, a.channels, dev)
