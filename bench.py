@@ -14,7 +14,9 @@ max-over-ranks step time.
 The same JSON line carries the other rows of the path, each timed the same
 way: the quantizer sweep's largest size (quantize, dequantize; 2^30 BF16
 values) and the calibration workload (16 x 14400 tokens x 5120 channels),
-as GB/s of algorithmic bytes and a fraction of HBM roofline.
+as GB/s of algorithmic bytes and a fraction of HBM roofline; and HiGPTQ
+scheme one on W1 (13824 x 5120, Hessian of the step's activations), as
+TFLOP/s of its FP32 error-feedback updates against the FP32 ALU peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hif4|reference]
 
@@ -42,7 +44,7 @@ METRIC = "W4A4 HiF4 linear TFLOP/s & quantizer GB/s at Wan2.2 shapes, % of roofl
 TOKENS, D_MODEL, D_FFN = 57600, 5120, 13824
 QUANT_N = 1 << 30
 CALIB_T, CALIB_C = 16 * 14400, 5120
-FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 # DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
 # hex digits) of the kernel source it was taken on; stale entries read as null.
@@ -73,7 +75,7 @@ def peaks():
         d = json.load(open(path))
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "source": "measured"}
+                "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)), "source": "measured"}
     except Exception:
         return dict(FALLBACK, source="fallback")
 
@@ -455,6 +457,26 @@ def main():
         comps["calib_percentile_mask"]["workload"] = \
             "calib 230400 x 5120 BF16, 2 B/elem read once (algorithmic); two radix passes read it twice"
         del acts
+        torch.cuda.empty_cache()
+        # HiGPTQ scheme one on the FFN's W1 with the Hessian of the layer input
+        xg, _ = wl.device_rows(M, D, seed=sharding.rank_seed(3, rank), device=dev)
+        w1g = wl.device_weight(F, D, 0.015, seed=31, device=dev)
+        Hg = H.hessian(xg)
+        del xg
+        gws = torch.empty(H.lib().hif4_higptq1_workspace(F, D, 128), dtype=torch.uint8, device=dev)
+        r = time_op(lambda: H.higptq1(w1g, Hg, idx1, 0.01, 128, workspace=gws), args, stream, barrier,
+                    max_over_ranks, world, 0.0, P)
+        fp32_peak = 148 * 128 * 2 * P["sm_max_mhz"] * 1e6 / 1e12
+        flop = float(F) * D * D                       # FP32 error-feedback updates: 2 x N K^2 / 2
+        tf = world * flop / (r["ms"] * 1e-3) / 1e12
+        comps["higptq1"] = {"value": tf, "unit": "TFLOP/s", "ms": r["ms"], "bound": "alu", "peak": fp32_peak,
+                            "frac": tf / world / fp32_peak,
+                            "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x %.0f MHz" % P["sm_max_mhz"],
+                            "workload": "HiGPTQ scheme one, W1 %d x %d (Wan2.2 FFN), Hessian of %d x %d "
+                                        "activations, block 128, 1%% protected; FLOPs counted: the FP32 "
+                                        "error-feedback updates (N K^2), the FP64 factor (2 K^3 / 3) on top"
+                                        % (F, D, M, D)}
+        del w1g, Hg, gws
         line["components"] = comps
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
