@@ -737,19 +737,22 @@ extern "C" hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_
 
 // ---------------------------------------------- FFN block on host activations
 //
-// The tokens stream through the GPU in chunks of C rows.  Two copy streams
-// run beside the caller's stream: chunk i+1 is copied in while chunk i
-// computes and chunk i-1 is copied out, with double-buffered device staging
-// (xs[2], ys[2]) ordered by events:
-//   h2d:     wait x_free[s]  -> copy x rows into xs[s]  -> record x_ready[s]
-//   compute: wait x_ready[s] -> fake-quant xs[s]        -> record x_free[s]
-//            GEMM 1 (+ fake quant of H)  -> wait y_free[s] -> GEMM 2 into ys[s]
-//            -> record y_ready[s]
-//   d2h:     wait y_ready[s] -> copy ys[s] out          -> record y_free[s]
-// with s = i % 2.  The weights are decoded once per call.  The streams and
-// events are created per call and released once their work completes.
-// Workspace: what1 F x D | what2 D x F | mask1 D | mask2 F | xhat1 C x D |
-// hhat C x F | xs 2 x C x D | ys 2 x C x D (x 2 for FP32 output).
+// The tokens stream through the GPU in chunks of at most C rows.  Two copy
+// streams run beside two compute streams (the caller's and one more): chunk
+// i is copied in, computed on compute stream i % 2 and copied out, so the
+// copies of neighbouring chunks overlap its compute and the next chunk's
+// kernels fill the SMs that the tail of chunk i's GEMMs leaves idle.
+// Staging (xs, ys) and scratch (xhat1, hhat) are double-buffered by slot
+// s = i % 2 and ordered by events:
+//   h2d:       wait x_free[s]  -> copy x rows into xs[s]  -> record x_ready[s]
+//   compute s: wait x_ready[s] -> fake-quant xs[s]        -> record x_free[s]
+//              GEMM 1 (+ fake quant of H) -> wait y_free[s] -> GEMM 2 into
+//              ys[s] -> record y_ready[s]
+//   d2h:       wait y_ready[s] -> copy ys[s] out          -> record y_free[s]
+// The weights are decoded once per call.  The streams and events are created
+// per call and released once their work completes.
+// Workspace: what1 F x D | what2 D x F | mask1 D | mask2 F | xhat1 2 x C x D |
+// hhat 2 x C x F | xs 2 x C x D | ys 2 x C x D (x 2 for FP32 output).
 
 namespace hif4 {
 namespace {
@@ -759,8 +762,8 @@ size_t ffn_host_layout(int64_t C, int64_t D, int64_t F, uint32_t flags, size_t *
     const size_t ysz = (flags & HIF4_LINEAR_OUT_F32) ? 4 : 2;
     size_t o = 0;
     const size_t sizes[8] = {(size_t)F * D * 2, (size_t)D * F * 2, (size_t)D, (size_t)F,
-                             (size_t)C * D * 2, (size_t)C * F * 2, 2 * align256((size_t)C * D * 2),
-                             2 * align256((size_t)C * D * ysz)};
+                             2 * align256((size_t)C * D * 2), 2 * align256((size_t)C * F * 2),
+                             2 * align256((size_t)C * D * 2), 2 * align256((size_t)C * D * ysz)};
     for (int i = 0; i < 8; ++i) {
         if (off) off[i] = o;
         o += align256(sizes[i]);
@@ -821,14 +824,15 @@ void ffn_host_schedule(int64_t M, int64_t chunk_rows, int64_t C, int64_t *starts
 }
 
 struct HostPipe {
-    cudaStream_t h2d = nullptr, d2h = nullptr;
-    cudaEvent_t start = nullptr, done = nullptr;
+    cudaStream_t h2d = nullptr, d2h = nullptr, cs1 = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr, prepared = nullptr;
     cudaEvent_t x_ready[2] = {}, x_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
     bool make()
     {
         if (cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
         if (cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
-        cudaEvent_t *all[10] = {&start, &done, &x_ready[0], &x_ready[1], &x_free[0],
+        if (cudaStreamCreateWithFlags(&cs1, cudaStreamNonBlocking) != cudaSuccess) return false;
+        cudaEvent_t *all[11] = {&start, &done, &prepared, &x_ready[0], &x_ready[1], &x_free[0],
                                 &x_free[1], &y_ready[0], &y_ready[1], &y_free[0], &y_free[1]};
         for (cudaEvent_t *e : all)
             if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
@@ -838,12 +842,13 @@ struct HostPipe {
     {
         // Destroying a stream or an event with work pending is allowed: its
         // resources are released once that work completes.
-        cudaEvent_t all[10] = {start, done, x_ready[0], x_ready[1], x_free[0],
+        cudaEvent_t all[11] = {start, done, prepared, x_ready[0], x_ready[1], x_free[0],
                                x_free[1], y_ready[0], y_ready[1], y_free[0], y_free[1]};
         for (cudaEvent_t e : all)
             if (e) cudaEventDestroy(e);
         if (h2d) cudaStreamDestroy(h2d);
         if (d2h) cudaStreamDestroy(d2h);
+        if (cs1) cudaStreamDestroy(cs1);
     }
 };
 
@@ -886,8 +891,10 @@ extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t
     uint16_t *what2 = reinterpret_cast<uint16_t *>(ws + off[1]);
     uint8_t *mask1 = ws + off[2];
     uint8_t *mask2 = ws + off[3];
-    uint16_t *xhat1 = reinterpret_cast<uint16_t *>(ws + off[4]);
-    uint16_t *hhat = reinterpret_cast<uint16_t *>(ws + off[5]);
+    uint16_t *xhat1[2] = {reinterpret_cast<uint16_t *>(ws + off[4]),
+                          reinterpret_cast<uint16_t *>(ws + off[4] + align256((size_t)C * D * 2))};
+    uint16_t *hhat[2] = {reinterpret_cast<uint16_t *>(ws + off[5]),
+                         reinterpret_cast<uint16_t *>(ws + off[5] + align256((size_t)C * F * 2))};
     uint8_t *xs[2] = {ws + off[6], ws + off[6] + align256((size_t)C * D * 2)};
     uint8_t *ys[2] = {ws + off[7], ws + off[7] + align256((size_t)C * D * ysz)};
 
@@ -897,17 +904,21 @@ extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t
     if (cudaEventRecord(P.start, s) != cudaSuccess || cudaStreamWaitEvent(P.h2d, P.start, 0) != cudaSuccess ||
         cudaStreamWaitEvent(P.d2h, P.start, 0) != cudaSuccess)
         return HIF4_ERR_CUDA;
-    st = ffn_prepare(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, w2_codes, w2_meta, mask2_idx,
-                     n_mask2, w2_masked, what1, what2, mask1, mask2, status, s);
-    if (st != HIF4_OK) return st;
-
-    // On any failure below, the caller's stream still waits for the copies
-    // already queued, so no buffer is released under a running copy.
+    // On any failure below, the caller's stream still waits for the work
+    // already queued on the other streams, so no buffer is released under it.
     auto join = [&](hif4_status result) {
         if (cudaEventRecord(P.done, P.h2d) == cudaSuccess) cudaStreamWaitEvent(s, P.done, 0);
+        if (cudaEventRecord(P.done, P.cs1) == cudaSuccess) cudaStreamWaitEvent(s, P.done, 0);
         if (cudaEventRecord(P.done, P.d2h) == cudaSuccess) cudaStreamWaitEvent(s, P.done, 0);
         return result;
     };
+    st = ffn_prepare(D, F, w1_codes, w1_meta, mask1_idx, n_mask1, w1_masked, w2_codes, w2_meta, mask2_idx,
+                     n_mask2, w2_masked, what1, what2, mask1, mask2, status, s);
+    if (st != HIF4_OK) return join(st);
+    // the second compute stream starts after the masks and decoded weights
+    if (cudaEventRecord(P.prepared, s) != cudaSuccess || cudaStreamWaitEvent(P.cs1, P.prepared, 0) != cudaSuccess)
+        return join(HIF4_ERR_CUDA);
+    cudaStream_t cs[2] = {s, P.cs1};
     const uint8_t *xh = static_cast<const uint8_t *>(x_host);
     uint8_t *yh = static_cast<uint8_t *>(y_host);
     // at most ceil(M / C) + 7 chunks: equal chunks, or the ramped schedule
@@ -925,18 +936,19 @@ extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t
                               (size_t)rows, cudaMemcpyHostToDevice, P.h2d) != cudaSuccess ||
             cudaEventRecord(P.x_ready[sl], P.h2d) != cudaSuccess)
             return join(HIF4_ERR_CUDA);
-        // compute
-        if (cudaStreamWaitEvent(s, P.x_ready[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
-        st = fake_quantize_bf16(xs[sl], rows, D, D, n_mask1 > 0 ? mask1 : nullptr, xhat1, D, status, s);
+        // compute on stream sl
+        cudaStream_t c = cs[sl];
+        if (cudaStreamWaitEvent(c, P.x_ready[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = fake_quantize_bf16(xs[sl], rows, D, D, n_mask1 > 0 ? mask1 : nullptr, xhat1[sl], D, status, c);
         if (st != HIF4_OK) return join(st);
-        if (cudaEventRecord(P.x_free[sl], s) != cudaSuccess) return join(HIF4_ERR_CUDA);
-        st = launch_gemm(xhat1, rows, D, D, what1, F, D, b1, n_mask2 > 0 ? mask2 : nullptr, hhat, F,
-                         HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, s);
+        if (cudaEventRecord(P.x_free[sl], c) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = launch_gemm(xhat1[sl], rows, D, D, what1, F, D, b1, n_mask2 > 0 ? mask2 : nullptr, hhat[sl], F,
+                         HIF4_LINEAR_GELU_TANH | HIF4_LINEAR_FAKE_QUANT_OUT, status, c);
         if (st != HIF4_OK) return join(st);
-        if (i >= 2 && cudaStreamWaitEvent(s, P.y_free[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
-        st = launch_gemm(hhat, rows, F, F, what2, D, F, b2, nullptr, ys[sl], D, flags, status, s);
+        if (i >= 2 && cudaStreamWaitEvent(c, P.y_free[sl], 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        st = launch_gemm(hhat[sl], rows, F, F, what2, D, F, b2, nullptr, ys[sl], D, flags, status, c);
         if (st != HIF4_OK) return join(st);
-        if (cudaEventRecord(P.y_ready[sl], s) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        if (cudaEventRecord(P.y_ready[sl], c) != cudaSuccess) return join(HIF4_ERR_CUDA);
         // copy out
         if (cudaStreamWaitEvent(P.d2h, P.y_ready[sl], 0) != cudaSuccess ||
             cudaMemcpy2DAsync(yh + (size_t)r0 * ldy * ysz, (size_t)ldy * ysz, ys[sl], (size_t)D * ysz,
@@ -944,8 +956,10 @@ extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t
             cudaEventRecord(P.y_free[sl], P.d2h) != cudaSuccess)
             return join(HIF4_ERR_CUDA);
     }
-    // the caller's stream completes only after the last row has landed on the host
-    if (cudaEventRecord(P.done, P.d2h) != cudaSuccess || cudaStreamWaitEvent(s, P.done, 0) != cudaSuccess)
+    // the caller's stream completes only after the second compute stream and
+    // the last row has landed on the host
+    if (cudaEventRecord(P.done, P.cs1) != cudaSuccess || cudaStreamWaitEvent(s, P.done, 0) != cudaSuccess ||
+        cudaEventRecord(P.done, P.d2h) != cudaSuccess || cudaStreamWaitEvent(s, P.done, 0) != cudaSuccess)
         return join(HIF4_ERR_CUDA);
     return HIF4_OK;
 }

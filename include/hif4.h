@@ -226,10 +226,13 @@ hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_t ldx,
  * hif4_ffn_w4a4_host — hif4_ffn_w4a4 on HOST activations: x_host (BF16
  * M x D, ldx) and y_host (BF16, or FP32 with HIF4_LINEAR_OUT_F32, M x D,
  * ldy) are host buffers.  The rows stream through the GPU in chunks of
- * chunk_rows (0 = automatic: at most 8192, whole 128-row tiles), the copy of
- * chunk i+1 to the device and of chunk i-1 back to the host overlapping the
- * compute of chunk i (two internal copy streams, double-buffered staging in
- * the workspace).  The results equal hif4_ffn_w4a4 on the same rows.
+ * chunk_rows (0 = automatic: at most 8192 rows in whole 128-row tiles,
+ * ramping 1024 / 2048 / 4096 rows up at the start and down at the end), the
+ * copies of neighbouring chunks overlapping the compute of chunk i.  Chunks
+ * alternate between `stream` and one internal compute stream, so a chunk's
+ * kernels can start on the SMs the previous chunk's last GEMM wave leaves
+ * idle; two internal copy streams; staging and scratch double-buffered in
+ * the workspace.  The results equal hif4_ffn_w4a4 on the same rows.
  * Page-locked host buffers (cudaHostAlloc / cudaHostRegister) are needed for
  * the overlap; pageable ones give the same results with serialized copies.
  * Asynchronous on `stream`: when `stream` completes, y_host holds the
