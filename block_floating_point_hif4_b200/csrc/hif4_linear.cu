@@ -771,41 +771,43 @@ size_t ffn_host_layout(int64_t C, int64_t D, int64_t F, uint32_t flags, size_t *
     return o;
 }
 
-// Largest chunk: the caller's chunk_rows, or (0) at most 8192 rows in whole
-// 128-row GEMM tiles.
+// Largest chunk: the caller's chunk_rows, or (0) at most 4096 rows in whole
+// 128-row GEMM tiles.  Host copies and compute run at about the same rate
+// here (PCIe both ways vs the power-capped GEMMs), so the pipeline gains
+// nothing from longer chunks and loses their longer fill and drain.
 int64_t ffn_host_chunk(int64_t M, int64_t chunk_rows)
 {
     if (chunk_rows > 0) return chunk_rows < M ? chunk_rows : M;
-    const int64_t n = (M + 8191) / 8192;
+    const int64_t n = (M + 4095) / 4096;
     int64_t c = (M + n - 1) / n;
     c = (c + 127) / 128 * 128;
     return c < M ? c : M;
 }
 
 // Row ranges of the chunks.  An explicit chunk_rows gives equal chunks.  The
-// automatic schedule ramps up (1024, 2048, 4096 rows) and back down at the
-// end, so that the copy in of the first chunk and the copy out of the last
-// one, which nothing overlaps, stay short; the middle runs in chunks of at
-// most C rows.
+// automatic schedule ramps up (1024, 2048 rows) and back down at the end, so
+// that the copy in of the first chunk and the copy out of the last one,
+// which nothing overlaps, stay short; the middle runs in chunks of at most C
+// rows.
 void ffn_host_schedule(int64_t M, int64_t chunk_rows, int64_t C, int64_t *starts, int64_t *counts, int &n)
 {
     n = 0;
-    if (chunk_rows > 0 || M < 4 * C) {
+    const int64_t ramp[2] = {1024, 2048};
+    const int64_t ends = 2 * (ramp[0] + ramp[1]);
+    if (chunk_rows > 0 || M < ends + 2 * C) {
         for (int64_t r = 0; r < M; r += C) {
             starts[n] = r;
             counts[n++] = M - r < C ? M - r : C;
         }
         return;
     }
-    const int64_t ramp[3] = {1024, 2048, 4096};
     int64_t r = 0;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 2; ++i) {
         starts[n] = r;
         counts[n++] = ramp[i];
         r += ramp[i];
     }
-    const int64_t tail = 4096 + 2048 + 1024;
-    const int64_t mid = M - r - tail;
+    const int64_t mid = M - ends;
     const int64_t pieces = (mid + C - 1) / C;
     int64_t per = (mid + pieces - 1) / pieces;
     per = (per + 127) / 128 * 128;
@@ -816,7 +818,7 @@ void ffn_host_schedule(int64_t M, int64_t chunk_rows, int64_t C, int64_t *starts
         r += c;
         left -= c;
     }
-    for (int i = 2; i >= 0; --i) {
+    for (int i = 1; i >= 0; --i) {
         starts[n] = r;
         counts[n++] = ramp[i];
         r += ramp[i];
@@ -921,8 +923,8 @@ extern "C" hif4_status hif4_ffn_w4a4_host(const void *x_host, int64_t M, int64_t
     cudaStream_t cs[2] = {s, P.cs1};
     const uint8_t *xh = static_cast<const uint8_t *>(x_host);
     uint8_t *yh = static_cast<uint8_t *>(y_host);
-    // at most ceil(M / C) + 7 chunks: equal chunks, or the ramped schedule
-    const int64_t max_chunks = (M + C - 1) / C + 7;
+    // at most ceil(M / C) + 5 chunks: equal chunks, or the ramped schedule
+    const int64_t max_chunks = (M + C - 1) / C + 5;
     std::vector<int64_t> starts((size_t)max_chunks), counts((size_t)max_chunks);
     int nchunks = 0;
     ffn_host_schedule(M, chunk_rows, C, starts.data(), counts.data(), nchunks);

@@ -226,8 +226,8 @@ hif4_status hif4_ffn_w4a4(const void *x, int64_t M, int64_t D, int64_t ldx,
  * hif4_ffn_w4a4_host — hif4_ffn_w4a4 on HOST activations: x_host (BF16
  * M x D, ldx) and y_host (BF16, or FP32 with HIF4_LINEAR_OUT_F32, M x D,
  * ldy) are host buffers.  The rows stream through the GPU in chunks of
- * chunk_rows (0 = automatic: at most 8192 rows in whole 128-row tiles,
- * ramping 1024 / 2048 / 4096 rows up at the start and down at the end), the
+ * chunk_rows (0 = automatic: at most 4096 rows in whole 128-row tiles,
+ * ramping 1024 / 2048 rows up at the start and down at the end), the
  * copies of neighbouring chunks overlapping the compute of chunk i.  Chunks
  * alternate between `stream` and one internal compute stream, so a chunk's
  * kernels can start on the SMs the previous chunk's last GEMM wave leaves

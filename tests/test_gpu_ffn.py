@@ -195,8 +195,8 @@ def test_ffn_host_pipeline_equals_device_call(H, M, chunk):
     compute) gives exactly the rows hif4_ffn_w4a4 gives on device buffers:
     per-row work and per-element accumulation order do not depend on the
     chunking.  Strided host rows, a ragged last chunk, the automatic ramped
-    schedule (40000 rows: 1024, 2048, 4096, 4 middle chunks, 4096, 2048,
-    1024) and FP32 output."""
+    schedule (40000 rows: 1024, 2048, ten middle chunks, 2048, 1024) and
+    FP32 output."""
     import torch
     D, F = 256, 512
     rng = np.random.default_rng(M + chunk)
