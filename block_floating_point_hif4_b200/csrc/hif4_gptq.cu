@@ -197,11 +197,13 @@ __global__ void __launch_bounds__(256) k_panel(double *A, int64_t K, int kb, con
 
 // Trailing update after tile kb: A[ti][tj] -= L[ti][kb] L[tj][kb]^T for
 // kb < tj <= ti.  Grid (n, n) with n the trailing tile count; blocks above
-// the diagonal exit at once.
-__global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb)
+// the diagonal exit at once, and so does tile (kb + 1, kb + 1) when
+// skip_next_diag is set (it is updated first, by a one-block launch, so that
+// its factorization can overlap the rest of this update).
+__global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb, int skip_next_diag)
 {
     const int ti = kb + 1 + blockIdx.y, tj = kb + 1 + blockIdx.x;
-    if (tj > ti) return;
+    if (tj > ti || (skip_next_diag && blockIdx.x == 0 && blockIdx.y == 0)) return;
     extern __shared__ __align__(16) double smd[];
     Tile *X = reinterpret_cast<Tile *>(smd);
     Tile *Y = X + TB;
@@ -510,15 +512,25 @@ __global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, con
         if (more) sstore(b ^ 1);
         __syncthreads();
     }
+    // C -= acc, two float4 per row where the 8 columns are inside (C, ldc
+    // and the column offset are multiples of 4 floats)
+    const int64_t cn0 = n0 + tc * 8;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t cm = m0 + tr * 8 + i;
         if (cm >= M) continue;
-        float *crow = C + cm * ldc;
+        float *crow = C + cm * ldc + cn0;
+        if (cn0 + 7 < Nc) {
+            float4 *c4 = reinterpret_cast<float4 *>(crow);
+            float4 u = c4[0], v = c4[1];
+            u.x -= acc[i][0]; u.y -= acc[i][1]; u.z -= acc[i][2]; u.w -= acc[i][3];
+            v.x -= acc[i][4]; v.y -= acc[i][5]; v.z -= acc[i][6]; v.w -= acc[i][7];
+            c4[0] = u;
+            c4[1] = v;
+        } else {
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            const int64_t cn = n0 + tc * 8 + jj;
-            if (cn < Nc) crow[cn] -= acc[i][jj];
+            for (int jj = 0; jj < 8; ++jj)
+                if (cn0 + jj < Nc) crow[jj] -= acc[i][jj];
         }
     }
 }
@@ -587,6 +599,25 @@ bool set_smem_once(F *kernel, size_t bytes, bool &done)
     done = true;
     return true;
 }
+
+// Second stream and events of the factorization look-ahead (created per call,
+// released once their work completes).
+struct Aux {
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t ev_diag = nullptr, ev_factored = nullptr;
+    bool make()
+    {
+        return cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaEventCreateWithFlags(&ev_diag, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&ev_factored, cudaEventDisableTiming) == cudaSuccess;
+    }
+    ~Aux()
+    {
+        if (ev_diag) cudaEventDestroy(ev_diag);
+        if (ev_factored) cudaEventDestroy(ev_factored);
+        if (s2) cudaStreamDestroy(s2);
+    }
+};
 
 template <int NG>
 hif4_status launch_gptq_block(const GptqArgs &a, cudaStream_t s)
@@ -701,15 +732,33 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     k_fill_reversed<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(
         H, K, dead, mean, damp, A);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    //    Look-ahead: after panel kb, diagonal tile kb + 1 is updated first and
+    //    factored on a second stream while the rest of the trailing update
+    //    runs (disjoint tiles); panel kb + 1 waits for it.
+    Aux X;
+    if (!X.make()) return HIF4_ERR_CUDA;
+    auto join = [&](hif4_status r) {
+        if (cudaEventRecord(X.ev_factored, X.s2) == cudaSuccess) cudaStreamWaitEvent(s, X.ev_factored, 0);
+        return r;
+    };
+    k_potrf_tile<<<1, 256, 2 * kTileBytes, s>>>(A, K, 0, Linv, status);
+    if (launch_status() != HIF4_OK) return join(HIF4_ERR_CUDA);
     for (int kb = 0; kb < nb; ++kb) {
-        k_potrf_tile<<<1, 256, 2 * kTileBytes, s>>>(A, K, kb, Linv + (size_t)kb * TB * TB, status);
         const int n = nb - 1 - kb;
-        if (n > 0) {
-            k_panel<<<n, 256, 2 * kTileBytes, s>>>(A, K, kb, Linv + (size_t)kb * TB * TB);
-            k_syrk<<<dim3(n, n), 256, 2 * kTileBytes, s>>>(A, K, kb);
-        }
-        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+        if (n == 0) break;
+        if (kb > 0 && cudaStreamWaitEvent(s, X.ev_factored, 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
+        k_panel<<<n, 256, 2 * kTileBytes, s>>>(A, K, kb, Linv + (size_t)kb * TB * TB);
+        k_syrk<<<1, 256, 2 * kTileBytes, s>>>(A, K, kb, 0);                   // tile (kb + 1, kb + 1)
+        if (launch_status() != HIF4_OK || cudaEventRecord(X.ev_diag, s) != cudaSuccess ||
+            cudaStreamWaitEvent(X.s2, X.ev_diag, 0) != cudaSuccess)
+            return join(HIF4_ERR_CUDA);
+        k_potrf_tile<<<1, 256, 2 * kTileBytes, X.s2>>>(A, K, kb + 1, Linv + (size_t)(kb + 1) * TB * TB, status);
+        if (launch_status() != HIF4_OK || cudaEventRecord(X.ev_factored, X.s2) != cudaSuccess)
+            return join(HIF4_ERR_CUDA);
+        if (n > 1) k_syrk<<<dim3(n, n), 256, 2 * kTileBytes, s>>>(A, K, kb, 1);
+        if (launch_status() != HIF4_OK) return join(HIF4_ERR_CUDA);
     }
+    if (nb > 1 && cudaStreamWaitEvent(s, X.ev_factored, 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
     // 3. Y = L'^{-1} (right-looking by block rows), then U = P Y P and the
     //    inverses of U's diagonal blocks
     if (cudaMemsetAsync(Y, 0, (size_t)K * K * 8, s) != cudaSuccess) return HIF4_ERR_CUDA;
