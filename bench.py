@@ -45,6 +45,7 @@ TOKENS, D_MODEL, D_FFN = 57600, 5120, 13824
 QUANT_N = 1 << 30
 CALIB_T, CALIB_C = 16 * 14400, 5120
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}                # B200 datasheet figures, for context
 
 # DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
 # hex digits) of the kernel source it was taken on; stale entries read as null.
@@ -363,7 +364,7 @@ def main():
                 "peak_source": "%s bf16 sustained (burst %.1f, frac %.3f)" % (P["source"], P["bf16_tflops"],
                                                                             achieved / P["bf16_tflops"]),
                 "algorithmic_per_launch": "2*M*N*K = %.4g FLOP" % flop_gemm,
-                "avg_launch_ms": gemm_ms}
+                "avg_launch_ms": gemm_ms, "frac_datasheet": achieved / DATASHEET["bf16_tflops"]}
 
     share = {s: v / sum(stage_ms.values()) for s, v in stage_ms.items()}
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -477,7 +478,32 @@ def main():
                                         "error-feedback updates (N K^2), the FP64 factor (2 K^3 / 3) on top"
                                         % (F, D, M, D)}
         del w1g, Hg, gws
+        torch.cuda.empty_cache()
+        # the attention projection (57600 x 5120 -> 5120, bias, 51 protected
+        # channels) through the public linear call, device buffers
+        xa, _ = wl.device_rows(M, D, seed=sharding.rank_seed(2, rank), device=dev)
+        wa = wl.device_weight(D, D, 0.015, seed=21, device=dev)
+        _, _, ma, ia = H.calib_percentile_mask(xa)
+        wac, wam = H.quantize(wa, ma)
+        wak = wa[:, ia.long()].contiguous()
+        ba = wl.device_weight(1, D, 0.01, seed=22, device=dev).view(D).contiguous()
+        ya = torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+        aws = torch.empty(H.linear_w4a4_workspace(M, D, D), dtype=torch.uint8, device=dev)
+        r = time_op(lambda: H.linear_w4a4(xa, wac, wam, D, ia, wak, ba, out=ya, workspace=aws), args, stream,
+                    barrier, max_over_ranks, world, 0.0, P)
+        aflop = 2.0 * M * D * D
+        atf = world * aflop / (r["ms"] * 1e-3) / 1e12
+        comps["linear_attn_proj"] = {"value": atf, "unit": "TFLOP/s", "ms": r["ms"], "bound": "tensor",
+                                     "peak": P["bf16_tflops"], "frac": atf / world / P["bf16_tflops"],
+                                     "frac_datasheet": atf / world / DATASHEET["bf16_tflops"],
+                                     "peak_source": "%s bf16 burst" % P["source"],
+                                     "workload": "hif4_linear_w4a4 57600 x 5120 -> 5120, bias, 51 protected "
+                                                 "channels; activation fake-quant, weight decode and GEMM all "
+                                                 "timed"}
+        del xa, wa, wac, wam, wak, ba, ya, aws
         line["components"] = comps
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            add_cpu_component_rates(comps)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
@@ -497,6 +523,31 @@ def main():
     return 0
 
 
+def add_cpu_component_rates(comps):
+    """The CPU oracle's rate on a bounded sample of each component workload,
+    beside the GPU line (kind "oracle"; not a target)."""
+    import numpy as np
+
+    import oracle
+    from block_floating_point_hif4_b200 import workloads as wl
+    thr = max(1, len(os.sched_getaffinity(0)))
+    n = 1 << 22
+    xb = wl.quant_sweep(n, seed=1)
+    rows = np.ascontiguousarray(xb[: n // 1024 * 1024].reshape(-1, 1024))
+    codes, meta, _ = oracle.quantize(rows)
+    q = cpu_rate(lambda: oracle.quantize(rows), n * 2.5625) / 1e9
+    d = cpu_rate(lambda: oracle.dequantize(codes, meta, 1024), n * 2.5625) / 1e9
+    acts, _ = wl.calib(T=14400, C=512, seed=4)
+    c = cpu_rate(lambda: oracle.percentile(acts, threads=thr), acts.size * 2.0) / 1e9
+    comps["quantize"]["cpu_baseline"] = {"value": q, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                         "sample": "2^22 elements of the quantizer sweep"}
+    comps["dequantize"]["cpu_baseline"] = {"value": d, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                           "sample": "2^22 elements of the quantizer sweep"}
+    comps["calib_percentile_mask"]["cpu_baseline"] = {"value": c, "unit": "GB/s", "cores": thr, "kind": "oracle",
+                                                      "sample": "14400 tokens x 512 channels of the calibration "
+                                                                "recipe, percentiles (sort per channel)"}
+
+
 def time_op(fn, args, stream, barrier, max_over_ranks, world, bytes_per_call, P):
     import torch
     for _ in range(args.warmup):
@@ -512,8 +563,19 @@ def time_op(fn, args, stream, barrier, max_over_ranks, world, bytes_per_call, P)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     gbs = world * bytes_per_call / (ms * 1e-3) / 1e9
     return {"value": gbs, "unit": "GB/s", "ms": ms, "bound": "hbm", "peak": P["hbm_gbs"],
-            "frac": gbs / world / P["hbm_gbs"], "peak_source": P["source"],
-            "l2": "inputs larger than L2"}
+            "frac": gbs / world / P["hbm_gbs"], "frac_datasheet": gbs / world / DATASHEET["hbm_gbs"],
+            "peak_source": P["source"], "l2": "inputs larger than L2"}
+
+
+def cpu_rate(fn, units, reps=2):
+    """Best-of-`reps` wall-clock rate (units per second) of a CPU oracle call."""
+    best = None
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn()
+        dt = time.perf_counter() - t0
+        best = dt if best is None else min(best, dt)
+    return units / best
 
 
 if __name__ == "__main__":
