@@ -357,7 +357,7 @@ def main():
     gemm_ms = max_over_ranks((stage_ms["gemm_1_gelu_fq"] + stage_ms["gemm_2"]) / 2)
     achieved = flop_gemm / (gemm_ms * 1e-3) / 1e12
     peak = P["bf16_tflops_sustained"]
-    gh = src_hash("hif4_linear.cu", "hif4_sm100.cuh", "hif4_encode.cuh", "hif4_internal.cuh")
+    gh = src_hash("hif4_gemm.cuh", "hif4_sm100.cuh", "hif4_encode.cuh", "hif4_internal.cuh")
     traffic = NCU_TRAFFIC.get(("gemm", gh))
     roofline = {"kernel": "k_gemm (hif4_gemm_bf16_fq, hif4_gemm_bf16)", "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
