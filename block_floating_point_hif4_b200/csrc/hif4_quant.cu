@@ -818,9 +818,51 @@ struct DequantArgs {
     uint32_t total_units;
 };
 
+// BF16 output by byte-permute lookups.  Element value m S 2^(E-2) with
+// S = 2^(e6-31) (1 + f/4) equals [m (4 + f)] 2^-35 2^(e6 + E): the BF16 bits
+// of the first factor (small integers scaled by 2^-35, exact) form one
+// 8-entry table per f, split into low and high bytes; one prmt looks up 4
+// elements' bytes at once, and adding (e6 + E) << 7 to a BF16 pair word
+// scales both halves (every result is a normal number, no carry crosses the
+// halves).  m = 0 entries are masked to zero; the sign bit is the code's.
+__device__ __forceinline__ void dequant8_bf16(uint32_t cw, uint32_t e6, uint32_t Elo, uint32_t Ehi, uint4 T,
+                                              uint32_t (&out)[4])
+{
+    const uint32_t n8 = ((cw & 0x77777777u) + 0x77777777u) & 0x88888888u;   // bit 3 of nibble: m != 0
+    const uint32_t nA = n8 << 4, sA = cw << 4;                              // byte MSBs: even nibbles
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint32_t sel = (cw >> (16 * half)) & 0x7777u;
+        const uint32_t lo4 = prmt(T.x, T.y, sel), hi4 = prmt(T.z, T.w, sel);
+        const uint32_t add = imad((e6 + (half ? Ehi : Elo)) << 7, 0x10001u, 0u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int k = 2 * half + j;
+            const uint32_t v = prmt(lo4, hi4, j ? 0x7362u : 0x5140u);
+            const uint32_t msk = prmt(nA, n8, 0xCC88u + 0x1111u * k);      // 0xFFFF halves where m != 0
+            const uint32_t sg = prmt(sA, cw, 0xC888u + 0x1111u * k) & 0x80008000u;
+            out[k] = ((v + add) & msk) | sg;
+        }
+    }
+}
+
 template <bool F32OUT, bool CONTIG>
 __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
 {
+    __shared__ __align__(16) uint32_t tab[4][4];       // [f] = {low bytes m 0-3, 4-7, high bytes m 0-3, 4-7}
+    if (!F32OUT) {
+        if (threadIdx.x < 16) {
+            const uint32_t f = threadIdx.x >> 2, which = threadIdx.x & 3u;
+            uint32_t v = 0;
+            for (uint32_t k = 0; k < 4; ++k) {
+                const uint32_t m = (which & 1u) * 4u + k;
+                const uint32_t t = m ? f_bits((float)(m * (4u + f)) * 0x1p-35f) >> 16 : 0u;
+                v |= ((which >> 1) ? (t >> 8) : (t & 0xFFu)) << (8 * k);
+            }
+            tab[f][which] = v;
+        }
+        __syncthreads();
+    }
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t lane8 = lane & 7u;
     const uint32_t nquads = (a.total_units + 3u) >> 2;
@@ -848,19 +890,25 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
             if (q >= nquads) break;
             if (unit[u] >= a.total_units) continue;
             const uint32_t w = mw[u];
-            const float S = e6m2_value(w & 0xFFu);
             const uint32_t e2 = (w >> (8 + lane8)) & 1u;
             const uint32_t e3lo = (w >> (16 + 2 * lane8)) & 1u;
             const uint32_t e3hi = (w >> (17 + 2 * lane8)) & 1u;
-            const float step_lo = ldexp_small(S, (int)(e2 + e3lo) - 2);
-            const float step_hi = ldexp_small(S, (int)(e2 + e3hi) - 2);
             float o[8];
+            uint32_t ob[4];
+            if (F32OUT) {
+                const float S = e6m2_value(w & 0xFFu);
+                const float step_lo = ldexp_small(S, (int)(e2 + e3lo) - 2);
+                const float step_hi = ldexp_small(S, (int)(e2 + e3hi) - 2);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t nib = (cw[u] >> (4 * i)) & 15u;
-                const float mf = bits_f(0x4B000000u | (nib & 7u)) - 8388608.0f;   // exact m
-                const float q = mf * (i < 4 ? step_lo : step_hi);
-                o[i] = bits_f(f_bits(q) | ((nib >> 3) << 31));
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t nib = (cw[u] >> (4 * i)) & 15u;
+                    const float mf = bits_f(0x4B000000u | (nib & 7u)) - 8388608.0f;   // exact m
+                    const float q = mf * (i < 4 ? step_lo : step_hi);
+                    o[i] = bits_f(f_bits(q) | ((nib >> 3) << 31));
+                }
+            } else {
+                const uint4 T = *reinterpret_cast<const uint4 *>(tab[w & 3u]);
+                dequant8_bf16(cw[u], (w & 0xFFu) >> 2, e2 + e3lo, e2 + e3hi, T, ob);
             }
             int64_t off;
             if (CONTIG) {
@@ -875,9 +923,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
                 p[0] = make_float4(o[0], o[1], o[2], o[3]);
                 p[1] = make_float4(o[4], o[5], o[6], o[7]);
             } else {
-                *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.y) + off) =
-                    make_uint4(pack_bf16_exact(o[0], o[1]), pack_bf16_exact(o[2], o[3]),
-                               pack_bf16_exact(o[4], o[5]), pack_bf16_exact(o[6], o[7]));
+                *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.y) + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
             }
         }
     }
