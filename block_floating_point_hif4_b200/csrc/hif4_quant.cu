@@ -30,6 +30,10 @@ using namespace enc;
 
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
+#ifndef HIF4_DQ_UNROLL
+#define HIF4_DQ_UNROLL 4
+#endif
+constexpr int kDqUnroll = HIF4_DQ_UNROLL;            // units in flight per dequantize lane
 
 struct QuantArgs {
     const void *x;
@@ -869,10 +873,10 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
     const uint32_t gwarp = (blockIdx.x * kThreads + threadIdx.x) >> 5;
     const uint32_t nwarps = (gridDim.x * kThreads) >> 5;
 
-    for (uint32_t q0 = gwarp; q0 < nquads; q0 += nwarps * kUnroll) {
-        uint32_t cw[kUnroll], mw[kUnroll], unit[kUnroll];
+    for (uint32_t q0 = gwarp; q0 < nquads; q0 += nwarps * kDqUnroll) {
+        uint32_t cw[kDqUnroll], mw[kDqUnroll], unit[kDqUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kDqUnroll; ++u) {
             const uint32_t q = q0 + (uint32_t)u * nwarps;
             unit[u] = q * 4u + (lane >> 3);
             if (q < nquads && unit[u] < a.total_units) {
@@ -885,7 +889,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kDqUnroll; ++u) {
             const uint32_t q = q0 + (uint32_t)u * nwarps;
             if (q >= nquads) break;
             if (unit[u] >= a.total_units) continue;
@@ -930,11 +934,11 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a)
 }
 
 template <typename K>
-int grid_for(K kernel, uint32_t total_units)
+int grid_for(K kernel, uint32_t total_units, int unroll = kUnroll)
 {
     const int per_sm = blocks_per_sm(reinterpret_cast<const void *>(kernel), kThreads, 0);
     const uint64_t quads = (total_units + 3ull) / 4ull;
-    const uint64_t warps_needed = (quads + kUnroll - 1) / kUnroll;
+    const uint64_t warps_needed = (quads + unroll - 1) / unroll;
     const uint64_t blocks_needed = (warps_needed + kThreads / 32 - 1) / (kThreads / 32);
     uint64_t g = (uint64_t)per_sm * (uint64_t)sm_count();
     if (blocks_needed < g) g = blocks_needed;
@@ -1094,11 +1098,11 @@ extern "C" hif4_status hif4_dequantize(const uint8_t *codes, const uint32_t *met
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool contig = ldy == cols;
     if (out_dtype == HIF4_F32) {
-        if (contig) { auto k = k_dequant<true, true>; k<<<grid_for(k, da.total_units), kThreads, 0, s>>>(da); }
-        else { auto k = k_dequant<true, false>; k<<<grid_for(k, da.total_units), kThreads, 0, s>>>(da); }
+        if (contig) { auto k = k_dequant<true, true>; k<<<grid_for(k, da.total_units, kDqUnroll), kThreads, 0, s>>>(da); }
+        else { auto k = k_dequant<true, false>; k<<<grid_for(k, da.total_units, kDqUnroll), kThreads, 0, s>>>(da); }
     } else {
-        if (contig) { auto k = k_dequant<false, true>; k<<<grid_for(k, da.total_units), kThreads, 0, s>>>(da); }
-        else { auto k = k_dequant<false, false>; k<<<grid_for(k, da.total_units), kThreads, 0, s>>>(da); }
+        if (contig) { auto k = k_dequant<false, true>; k<<<grid_for(k, da.total_units, kDqUnroll), kThreads, 0, s>>>(da); }
+        else { auto k = k_dequant<false, false>; k<<<grid_for(k, da.total_units, kDqUnroll), kThreads, 0, s>>>(da); }
     }
     return launch_status();
 }
