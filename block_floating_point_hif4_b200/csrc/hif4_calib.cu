@@ -613,27 +613,63 @@ __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int 
     const uint32_t need_eq = n_top - above;            // ties at tau taken by lowest index
     const float med = __uint_as_float(med_key << 16);
 
-    uint32_t eq_base = 0, m_base = 0;
-    for (int c0 = 0; c0 < C; c0 += kMaskThreads) {
-        const int c = c0 + threadIdx.x;
-        const bool in = c < C;
+    // Mask and indices in three passes over contiguous per-warp channel
+    // ranges (warp w owns [w chunk, (w+1) chunk)), with ballots inside a warp
+    // and one prefix over the 32 warp totals between passes: ties at tau go
+    // to the lowest channel indices, and mask_idx lists the masked channels
+    // in ascending order.
+    constexpr int kWarps = kMaskThreads / 32;
+    __shared__ uint32_t wsum[kWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int chunk = ((C + kWarps - 1) / kWarps + 31) & ~31;
+    const int cbeg = warp * chunk, cend = min(C, cbeg + chunk);
+    // pass 1: channels tied at tau, per warp
+    uint32_t n_eq = 0;
+    for (int c0 = cbeg; c0 < cend; c0 += 32) {
+        const int c = c0 + lane;
+        n_eq += __popc(__ballot_sync(0xffffffffu, c < cend && n_top && (pct[c] & 0x7FFFu) == tau));
+    }
+    if (lane == 0) wsum[warp] = n_eq;
+    __syncthreads();
+    uint32_t eq_base = 0;
+    for (int w = 0; w < warp; ++w) eq_base += wsum[w];
+    __syncthreads();
+    // pass 2: masked channels, per warp
+    uint32_t n_m = 0;
+    for (int c0 = cbeg, er = (int)eq_base; c0 < cend; c0 += 32) {
+        const int c = c0 + lane;
+        const bool in = c < cend;
         const uint32_t key = in ? (pct[c] & 0x7FFFu) : 0u;
-        const uint32_t eq = in && n_top && key == tau;
-        uint32_t tot_eq;
-        const uint32_t eq_rank = eq_base + block_excl_scan(eq, scratch, tot_eq);
-        const uint32_t m = in && n_top && (key > tau || (eq && eq_rank < need_eq));
-        uint32_t tot_m;
-        const uint32_t m_pos = m_base + block_excl_scan(m, scratch, tot_m);
+        const bool eq = in && n_top && key == tau;
+        const uint32_t be = __ballot_sync(0xffffffffu, eq);
+        const bool m = in && n_top && (key > tau || (eq && (uint32_t)er + __popc(be & lt) < need_eq));
+        n_m += __popc(__ballot_sync(0xffffffffu, m));
+        er += __popc(be);
+    }
+    if (lane == 0) wsum[warp] = n_m;
+    __syncthreads();
+    uint32_t m_base = 0;
+    for (int w = 0; w < warp; ++w) m_base += wsum[w];
+    // pass 3: outputs
+    for (int c0 = cbeg, er = (int)eq_base, mr = (int)m_base; c0 < cend; c0 += 32) {
+        const int c = c0 + lane;
+        const bool in = c < cend;
+        const uint32_t key = in ? (pct[c] & 0x7FFFu) : 0u;
+        const bool eq = in && n_top && key == tau;
+        const uint32_t be = __ballot_sync(0xffffffffu, eq);
+        const bool m = in && n_top && (key > tau || (eq && (uint32_t)er + __popc(be & lt) < need_eq));
+        const uint32_t bm = __ballot_sync(0xffffffffu, m);
         if (in) {
             mask[c] = (uint8_t)m;
             float rt;
             if (med_key == 0) rt = key ? __int_as_float(0x7F800000) : 0.0f;
             else rt = __fdiv_rn(__uint_as_float(key << 16), med);
             ratio[c] = rt;
-            if (m && mask_idx) mask_idx[m_pos] = c;
+            if (m && mask_idx) mask_idx[mr + __popc(bm & lt)] = c;
         }
-        eq_base += tot_eq;
-        m_base += tot_m;
+        er += __popc(be);
+        mr += __popc(bm);
     }
 }
 
