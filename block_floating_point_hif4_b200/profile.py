@@ -8,7 +8,9 @@ linear | ffn | higptq.  gemm_fq is the FFN's first GEMM: bias-free, tanh-GELU an
 HiF4 fake quantization of its output (1 % protected columns) in the epilogue;
 ffn is the whole W4A4 FFN block (hif4_ffn_w4a4, --n = hidden width);
 higptq times HiGPTQ scheme one on an --n x --channels weight with the
-Hessian of --tokens activation rows (the Hessian itself untimed).
+Hessian of --tokens activation rows (the Hessian itself untimed);
+fake_quantize_x is the FFN step's first call: --tokens x --channels
+activations with 1 % protected channels.
 Sizes default to small cases that still exceed the 126 MB L2 (a few hundred
 MB on the device).  Prints the mean CUDA-event time per call.
 """
@@ -20,8 +22,8 @@ import sys
 
 def main(argv=None):
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "gemm", "gemm_gelu", "gemm_fq",
-                                  "calib", "linear", "ffn", "higptq"])
+    p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "fake_quantize_x", "gemm", "gemm_gelu",
+                                  "gemm_fq", "calib", "linear", "ffn", "higptq"])
     p.add_argument("--log2n", type=int, default=28, help="elements for quantize/dequantize/fake_quantize")
     p.add_argument("--tokens", type=int, default=57600)
     p.add_argument("--channels", type=int, default=5120)
@@ -46,6 +48,14 @@ def main(argv=None):
               "dequantize": lambda: H.dequantize(codes, meta, 1024, out=y),
               "fake_quantize": lambda: H.fake_quantize(x, out=y)}[a.op]
         nbytes = n * (4.0 if a.op == "fake_quantize" else 2.5625)
+    elif a.op == "fake_quantize_x":
+        x, _ = wl.device_rows(a.tokens, a.channels, seed=3, device=dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        cm = (torch.rand(a.channels, device=dev, generator=g) < 0.01).to(torch.uint8)
+        y = torch.empty_like(x)
+        fn = lambda: H.fake_quantize(x, cm, out=y)  # noqa: E731
+        nbytes = 4.0 * a.tokens * a.channels
     elif a.op == "higptq":
         x, _ = wl.device_rows(a.tokens, a.channels, seed=3, device=dev)
         w = wl.device_weight(a.n, a.channels, 0.015, seed=31, device=dev)
