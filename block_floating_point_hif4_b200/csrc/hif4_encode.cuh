@@ -171,7 +171,9 @@ __device__ __forceinline__ void plan_quarter(uint32_t A01, uint32_t A23, uint32_
 }
 
 // Fake-quantized BF16 pairs of one quarter (fast path): w = the 8 input
-// words, mw = protected halves (MASK only; passed through unchanged).
+// words, mw = protected halves (MASK only; passed through unchanged).  The
+// two halves of a pair are computed independently and a protected half's
+// result is replaced by its input, so the products run on w unmasked.
 template <bool MASK>
 __device__ __forceinline__ void fq_quarter(const uint32_t *w, const uint32_t *mw, const Quarter &p, float S,
                                            uint32_t *out)
@@ -187,8 +189,7 @@ __device__ __forceinline__ void fq_quarter(const uint32_t *w, const uint32_t *mw
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        const uint32_t wz = MASK ? (w[q] & ~mw[q]) : w[q];
-        const u64 x = pk(bits_f(wz << 16), bits_f(wz & 0xFFFF0000u));
+        const u64 x = pk(bits_f(w[q] << 16), bits_f(w[q] & 0xFFFF0000u));
         const u64 r = ffma2(x, p.HH[q >> 1], fmul2(x, p.LL[q >> 1]));
         const u64 mf = fadd2(fadd2(r, MAGIC2), NMAGIC2);   // signed RNE(r), +0 when 0
         float ml, mh;

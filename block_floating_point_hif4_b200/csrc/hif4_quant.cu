@@ -513,9 +513,16 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
     uint32_t bad = 0, i = 0;
     for (; i < my_n; ++i) {
         const uint32_t st = i % kStages;
-        const bool ok = mbar_wait_bounded(&full[st], (i / kStages) & 1u, &abort_flag, kWaitNs);
         const uint32_t unit = (blockIdx.x + i * gridDim.x) * kChunkUnits + (tid >> 2);
         const bool active = unit < a.total_units;
+        // the mask bytes do not depend on the stage: their load overlaps the wait
+        uint32_t mraw[4] = {0, 0, 0, 0};
+        if (MASK && active) {
+            const uint32_t cu = unit - a.upr_div.div(unit) * a.upr;
+            const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + q4 * 16));
+            mraw[0] = m4.x; mraw[1] = m4.y; mraw[2] = m4.z; mraw[3] = m4.w;
+        }
+        const bool ok = mbar_wait_bounded(&full[st], (i / kStages) & 1u, &abort_flag, kWaitNs);
         uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (ok && active) {
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + (size_t)st * kChunkBytes + tid * 32u);
@@ -526,13 +533,6 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
         // stage st consumed by every thread; leave together if any wait gave up
         if (__syncthreads_or(!ok)) break;
         if (tid == 0 && i + kStages < my_n) issue(i + kStages);
-        uint32_t mraw[4] = {0, 0, 0, 0};
-        uint32_t cu = 0;
-        if (MASK && active) {
-            cu = unit - a.upr_div.div(unit) * a.upr;
-            const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + q4 * 16));
-            mraw[0] = m4.x; mraw[1] = m4.y; mraw[2] = m4.z; mraw[3] = m4.w;
-        }
         uint32_t out[8], meta;
         encode16<MASK, MODE>(w, mraw, q4, bad, out, meta);
         if (!active) continue;

@@ -25,6 +25,8 @@ def main(argv=None):
     p.add_argument("op", choices=["quantize", "dequantize", "fake_quantize", "fake_quantize_x", "gemm", "gemm_gelu",
                                   "gemm_fq", "calib", "linear", "ffn", "higptq"])
     p.add_argument("--log2n", type=int, default=28, help="elements for quantize/dequantize/fake_quantize")
+    p.add_argument("--protect", type=float, default=0.01,
+                   help="fake_quantize_x: fraction of protected channels (0 = no mask)")
     p.add_argument("--tokens", type=int, default=57600)
     p.add_argument("--channels", type=int, default=5120)
     p.add_argument("--n", type=int, default=5120, help="output features for gemm/linear")
@@ -52,7 +54,7 @@ def main(argv=None):
         x, _ = wl.device_rows(a.tokens, a.channels, seed=3, device=dev)
         g = torch.Generator(device=dev)
         g.manual_seed(5)
-        cm = (torch.rand(a.channels, device=dev, generator=g) < 0.01).to(torch.uint8)
+        cm = (torch.rand(a.channels, device=dev, generator=g) < a.protect).to(torch.uint8) if a.protect > 0 else None
         y = torch.empty_like(x)
         fn = lambda: H.fake_quantize(x, cm, out=y)  # noqa: E731
         nbytes = 4.0 * a.tokens * a.channels
