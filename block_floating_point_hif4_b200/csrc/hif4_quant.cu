@@ -330,19 +330,16 @@ __device__ __forceinline__ void slow_lane16(const uint32_t (&w)[8], const uint32
     }
 }
 
+// mw: the protected halves of the 8 input words as 16-bit lane masks (all
+// ones where the channel is protected; read only with MASK).
 template <bool MASK, int MODE>
-__device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t (&mraw)[4], uint32_t q4,
+__device__ __forceinline__ void encode16(const uint32_t (&w)[8], const uint32_t (&mw)[8], uint32_t q4,
                                          uint32_t &bad, uint32_t (&out)[8], uint32_t &meta)
 {
     const u64 MAGIC2 = pk(12582912.0f, 12582912.0f);
-    // protected columns: 16-bit lane masks (all ones where the mask byte is nonzero)
-    uint32_t mw[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mw[i] = 0;
-    if (MASK) mask_words16(mraw, mw);
     uint32_t mk[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) mk[i] = w[i] & ~mw[i] & 0x7FFF7FFFu;
+    for (int i = 0; i < 8; ++i) mk[i] = (MASK ? (w[i] & ~mw[i]) : w[i]) & 0x7FFF7FFFu;
     uint32_t A01, A23, A8;
     quarter_max(mk, A01, A23, A8);
     uint32_t ak = max(A8 & 0xFFFFu, A8 >> 16);
@@ -442,8 +439,10 @@ __global__ void __launch_bounds__(kThreads, 3) k_quant_bf16(QuantArgs a)
             if (o >= nocts) break;                                      // warp-uniform
             const bool active = unit[u] < a.total_units;
             const uint32_t (&w)[8] = raw[u];
+            uint32_t mw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (MASK) mask_words16(mraw[u], mw);
             uint32_t out[8], meta;
-            encode16<MASK, MODE>(w, mraw[u], q4, bad, out, meta);
+            encode16<MASK, MODE>(w, mw, q4, bad, out, meta);
             if (!active) continue;
             if (MODE == 0) {
                 asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(a.codes + (size_t)unit[u] * 32 + q4 * 8),
@@ -481,7 +480,11 @@ constexpr uint32_t kChunkBytes = kChunkUnits * HIF4_UNIT * 2;   // 8 KB
 constexpr size_t kTmaSmem = (size_t)kStages * kChunkBytes + 128;
 constexpr uint64_t kWaitNs = 2000000000ull;               // 2 s: far above any chunk
 
-template <bool MASK, int MODE>
+// FIXED (with MASK): the grid is a multiple of upr / gcd(upr, 64), so the
+// chunk stride gridDim.x * 64 units is a whole number of rows and a thread's
+// channels are the same in every chunk: its protected-lane masks are built
+// once, before the loop.
+template <bool MASK, int MODE, bool FIXED>
 __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs a)
 {
     using namespace sm100;
@@ -510,6 +513,15 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
     if (tid == 0)
         for (uint32_t i = 0; i < my_n && i < (uint32_t)kStages; ++i) issue(i);
 
+    uint32_t mw_fixed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (MASK && FIXED) {
+        const uint32_t unit0 = blockIdx.x * kChunkUnits + (tid >> 2);
+        const uint32_t cu0 = unit0 - a.upr_div.div(unit0) * a.upr;
+        const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu0 * HIF4_UNIT + q4 * 16));
+        const uint32_t mraw[4] = {m4.x, m4.y, m4.z, m4.w};
+        mask_words16(mraw, mw_fixed);
+    }
+
     uint32_t bad = 0, i = 0;
     for (; i < my_n; ++i) {
         const uint32_t st = i % kStages;
@@ -517,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
         const bool active = unit < a.total_units;
         // the mask bytes do not depend on the stage: their load overlaps the wait
         uint32_t mraw[4] = {0, 0, 0, 0};
-        if (MASK && active) {
+        if (MASK && !FIXED && active) {
             const uint32_t cu = unit - a.upr_div.div(unit) * a.upr;
             const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + q4 * 16));
             mraw[0] = m4.x; mraw[1] = m4.y; mraw[2] = m4.z; mraw[3] = m4.w;
@@ -533,8 +545,15 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
         // stage st consumed by every thread; leave together if any wait gave up
         if (__syncthreads_or(!ok)) break;
         if (tid == 0 && i + kStages < my_n) issue(i + kStages);
+        uint32_t mw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (MASK && FIXED) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mw[j] = mw_fixed[j];
+        } else if (MASK) {
+            mask_words16(mraw, mw);
+        }
         uint32_t out[8], meta;
-        encode16<MASK, MODE>(w, mraw, q4, bad, out, meta);
+        encode16<MASK, MODE>(w, mw, q4, bad, out, meta);
         if (!active) continue;
         if (MODE == 0) {
             asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(a.codes + (size_t)unit * 32 + q4 * 8), "r"(out[0]),
@@ -957,23 +976,52 @@ int grid_for16(K kernel, uint32_t total_units)
     return (int)(g < 1 ? 1 : g);
 }
 
-template <bool MASK, int MODE>
-hif4_status launch_quant_tma(const QuantArgs &qa, cudaStream_t s)
+// Opts the kernel into kTmaSmem of dynamic shared memory (once per device).
+template <bool MASK, int MODE, bool FIXED>
+bool quant_tma_attr()
 {
-    auto k = k_quant_tma<MASK, MODE>;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr[dev & 63]) {
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTmaSmem) != cudaSuccess)
-            return HIF4_ERR_CUDA;
+        if (cudaFuncSetAttribute(k_quant_tma<MASK, MODE, FIXED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kTmaSmem) != cudaSuccess)
+            return false;
         attr[dev & 63] = true;
     }
-    const uint32_t nchunks = (qa.total_units + kChunkUnits - 1) / kChunkUnits;
-    int grid = blocks_per_sm(reinterpret_cast<const void *>(k), kThreads, kTmaSmem) * sm_count();
-    if ((uint32_t)grid > nchunks) grid = (int)nchunks;
-    k<<<grid, kThreads, kTmaSmem, s>>>(qa);
+    return true;
+}
+
+template <bool MASK, int MODE, bool FIXED>
+hif4_status launch_quant_tma_grid(const QuantArgs &qa, int grid, cudaStream_t s)
+{
+    if (!quant_tma_attr<MASK, MODE, FIXED>()) return HIF4_ERR_CUDA;
+    k_quant_tma<MASK, MODE, FIXED><<<grid, kThreads, kTmaSmem, s>>>(qa);
     return launch_status();
+}
+
+template <bool MASK, int MODE>
+hif4_status launch_quant_tma(const QuantArgs &qa, cudaStream_t s)
+{
+    if (!quant_tma_attr<MASK, MODE, false>()) return HIF4_ERR_CUDA;
+    const uint32_t nchunks = (qa.total_units + kChunkUnits - 1) / kChunkUnits;
+    int grid = blocks_per_sm(reinterpret_cast<const void *>(k_quant_tma<MASK, MODE, false>), kThreads, kTmaSmem) *
+               sm_count();
+    if ((uint32_t)grid > nchunks) grid = (int)nchunks;
+    if (MASK) {
+        // the largest grid whose chunk stride is a whole number of rows, if
+        // it keeps at least 7/8 of the blocks
+        uint32_t g = qa.upr, b = (uint32_t)kChunkUnits;
+        while (b) {
+            const uint32_t r = g % b;
+            g = b;
+            b = r;
+        }
+        const uint32_t step = qa.upr / g;
+        const uint32_t gf = ((uint32_t)grid / step) * step;
+        if (gf >= 1 && gf * 8 >= (uint32_t)grid * 7) return launch_quant_tma_grid<MASK, MODE, MASK>(qa, (int)gf, s);
+    }
+    return launch_quant_tma_grid<MASK, MODE, false>(qa, grid, s);
 }
 
 template <bool BF16, bool MASK, int MODE>

@@ -201,6 +201,31 @@ def test_fake_quantize_matches_oracle(H):
     assert np.array_equal(got0, wl.f32_to_bf16_bits(ref0.astype(np.float32)))
 
 
+@pytest.mark.parametrize("rows,cols", [
+    (4001, 640),        # chunk stride a whole number of rows: lane masks built once; ragged last chunk
+    (20000, 5120),      # the same with ~57 chunks per block (Wan2.2 channel count)
+    (50, 64 * 997),     # no such grid (997 units per row): masks per chunk
+])
+def test_masked_fake_quantize_chunk_strides(H, rows, cols):
+    """Masked fake quantization over many chunks per block, in both launch
+    forms of the streaming kernel; rows are independent, so a spread sample
+    of rows is checked against the oracle."""
+    torch = _torch()
+    rng = np.random.default_rng(rows + cols)
+    x = rng.standard_normal((rows, cols), dtype=np.float32)
+    x *= rng.lognormal(0, 0.5, cols).astype(np.float32)
+    x = wl.f32_to_bf16_bits(x)
+    idx = np.sort(rng.choice(cols, max(1, cols // 100), replace=False)).astype(np.int32)
+    mask = np.zeros(cols, np.uint8)
+    mask[idx] = 7                                           # any nonzero byte protects
+    got = to_host_bits(H.fake_quantize(to_dev_bf16(x), torch.from_numpy(mask).cuda()))
+    sample = np.unique(np.concatenate([np.arange(min(rows, 64)), rng.choice(rows, min(rows, 192), replace=False),
+                                       [rows - 1]]))
+    ref = oracle.fake_quantize(np.ascontiguousarray(x[sample]), idx)
+    assert np.array_equal(got[sample], wl.f32_to_bf16_bits(ref.astype(np.float32)))
+    assert np.array_equal(got[:, idx], x[:, idx])           # every protected channel passes through
+
+
 def test_gpu_idempotence(H):
     torch = _torch()
     x = to_dev_bf16(wl.quant_sweep(1 << 20).reshape(-1, 1024))
