@@ -50,9 +50,9 @@ DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}                # B200 dat
 # DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
 # hex digits) of the kernel source it was taken on; stale entries read as null.
 NCU_TRAFFIC = {
-    # bench FFN step, 57600 tokens: GEMM 1 (fused fake-quant epilogue) read 4.70 GB + wrote 1.58 GB,
+    # bench FFN step, 57600 tokens: GEMM 1 (fused fake-quant epilogue) read 4.71 GB + wrote 1.59 GB,
     # GEMM 2 read 9.21 GB + wrote 0.58 GB (one ncu pass, dram__bytes_read/write.sum); mean per launch
-    ("gemm", "9577a0791310727e"): 8.035e9,
+    ("gemm", "35fde63dfbb6ccaf"): 8.046e9,
 }
 
 
