@@ -18,9 +18,9 @@
 // U = P L'^{-1} P (upper, positive diagonal: the Cholesky factor of Hd^{-1}),
 // so one Cholesky factorization and one triangular inverse suffice, and the
 // inverse of U's 64 x 64 diagonal block g is the reversed diagonal block of
-// L' itself.  Both run in FP64 as 64 x 64 tile kernels (a single-block tile
-// factorization, then tile products for the panel, the trailing update and
-// the inverse's block rows).  The group loop runs in FP32: one warp per row
+// L' itself.  Both run in FP64 by one recursion over halves whose products
+// are tiled FP64 GEMMs (section "Factor" below).  The group loop runs in
+// FP32: one warp per row
 // quantizes with the exact FP32 encode rule of the streaming quantizer, and
 // the lazy update after each block is an FP32 tile GEMM.
 #include <cuda_bf16.h>
@@ -68,205 +68,234 @@ __global__ void k_fill_reversed(const float *H, int64_t K, const uint8_t *dead, 
     A[i * K + j] = v;
 }
 
-// Cholesky factorization of diagonal tile kb of A (lower, in place) and the
-// inverse of the factor into Linv (64 x 64).  One block of 256 threads.
-// One row of a padded 64 x 64 FP64 tile: 66 doubles (528 bytes) keep rows
-// 16-byte aligned for paired loads and offset consecutive rows by 4 banks.
-typedef double Tile[TB + 2];
-constexpr size_t kTileBytes = sizeof(double) * TB * (TB + 2);
+// The factor and its inverse, recursively.  For a diagonal block of n rows
+// at offset o (n a multiple of 64), split n = n1 + n2 and
+//   (L11, L11^{-1}) of A11                    recursively
+//   T   = A21 L11^{-T}                         (= L21)
+//   A22 = A22 - T T^T                          (lower tiles)
+//   Y21 = T L11^{-1}
+//   (L22, L22^{-1}) of A22                    recursively (T is reused there)
+//   Y21 = -L22^{-1} Y21                        (into T, then copied back)
+// with Y holding L^{-1}: [[L11, 0], [L21, L22]]^{-1} has the off-diagonal
+// block -L22^{-1} L21 L11^{-1}.  A 64-row block is a leaf: one thread block
+// factors it and inverts its factor.  Only the diagonal tiles of L are kept
+// (in A); every product is an FP64 GEMM that skips the tiles in which a
+// triangular operand is zero, so the whole factor costs K^3/3 + K^3/3 FLOP.
 
-__global__ void __launch_bounds__(256) k_potrf_tile(double *A, int64_t K, int kb, double *Linv, uint32_t *status)
+constexpr int LP = TB + 2;              // padded smem row of a leaf tile (doubles)
+constexpr size_t kLeafSmem = sizeof(double) * 3 * TB * LP;
+
+// One 64 x 64 diagonal block: Cholesky (lower, in place in A, right-looking
+// by columns) and the inverse of the factor into Y (zeros above the
+// diagonal).  A pivot that is not positive is replaced by 1 and reported as
+// HIF4_FLAG_NOT_SPD.  256 threads.
+__global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
 {
     extern __shared__ __align__(16) double smd[];
-    Tile *T = reinterpret_cast<Tile *>(smd);
-    Tile *I = T + TB;
+    double(*T)[LP] = reinterpret_cast<double(*)[LP]>(smd);      // the factor
+    double(*R)[LP] = T + TB;                                     // right-hand sides of L X = I
+    double(*X)[LP] = R + TB;                                     // the inverse
+    __shared__ double col[TB], piv[TB], rpiv[TB];
     __shared__ int bad;
-    const int tid = threadIdx.x;
-    double *a0 = A + (int64_t)kb * TB * K + (int64_t)kb * TB;
-    for (int e = tid; e < TB * TB; e += 256) {
-        const int r = e / TB, c = e % TB;
-        T[r][c] = c <= r ? a0[(int64_t)r * K + c] : 0.0;
-        I[r][c] = 0.0;
-    }
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;  // 16 x 16 thread grid
+    for (int r = ty; r < TB; r += 16)
+        for (int c = tx; c < TB; c += 16) {
+            T[r][c] = c <= r ? A[(int64_t)r * lda + c] : 0.0;
+            R[r][c] = r == c ? 1.0 : 0.0;
+            X[r][c] = 0.0;
+        }
     if (tid == 0) bad = 0;
     __syncthreads();
-    // left-looking by columns: T[r][j] -= sum_{k<j} T[r][k] T[j][k] for r >= j
-    // (four threads per row share the dot product), then the pivot and the
-    // scaling of the column below it
-    __shared__ double rpiv;
     for (int j = 0; j < TB; ++j) {
-        const int r = tid >> 2, part = tid & 3;
-        double t = 0.0;
-        if (r >= j)
-            for (int k = part; k < j; k += 4) t += T[r][k] * T[j][k];
-        t += __shfl_xor_sync(0xffffffffu, t, 1);
-        t += __shfl_xor_sync(0xffffffffu, t, 2);
-        if (r >= j && part == 0) T[r][j] -= t;
-        __syncthreads();
-        if (tid == 0) {
+        // column j: the pivot, then the scaled entries below it (thread r
+        // owns row r); one reciprocal square root per column
+        if (tid < TB) {
             double d = T[j][j];
-            if (!(d > 0.0)) {
-                bad = 1;
-                d = 1.0;
+            const bool ok = d > 0.0;
+            if (!ok) d = 1.0;
+            const double rs = rsqrt(d);
+            if (tid > j) {
+                const double l = T[tid][j] * rs;
+                col[tid] = l;
+                T[tid][j] = l;
+            } else if (tid == j) {
+                piv[j] = d * rs;
+                rpiv[j] = rs;
+                if (!ok) bad = 1;
             }
-            d = sqrt(d);
-            T[j][j] = d;
-            rpiv = 1.0 / d;
         }
         __syncthreads();
-        if (r > j && part == 0) T[r][j] *= rpiv;
+        // rank-1 update of the trailing lower triangle, 4 x 4 candidates per
+        // thread (the pivot itself is written after the loop: every thread
+        // above read it before the sync)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = j + 1 + ty + 16 * a;
+            if (r < TB) {
+                const double lr = col[r];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int c = j + 1 + tx + 16 * b;
+                    if (c <= r) T[r][c] -= lr * col[c];
+                }
+            }
+        }
         __syncthreads();
     }
-    // inverse of the lower factor, row by row: I[i][j] = -(sum_{k=j}^{i-1}
-    // T[i][k] I[k][j]) / T[i][i] for j < i; four threads share each column's
-    // dot product (lanes 4j..4j+3 of the block, combined by shuffles)
-    if (tid < TB) I[tid][tid] = 1.0 / T[tid][tid];
+    if (tid < TB) T[tid][tid] = piv[tid];
     __syncthreads();
-    for (int i = 1; i < TB; ++i) {
-        const int j = tid >> 2, part = tid & 3;
-        double t = 0.0;
-        if (j < i)
-            for (int k = j + part; k < i; k += 4) t += T[i][k] * I[k][j];
-        t += __shfl_xor_sync(0xffffffffu, t, 1);
-        t += __shfl_xor_sync(0xffffffffu, t, 2);
-        if (j < i && part == 0) I[i][j] = -t * I[i][i];
+    // L X = I by rows: at step r row r of X is R[r][:] / L[r][r], and its
+    // contribution leaves the rows below (row r of R is final at step r and
+    // nobody writes it during that step)
+    for (int r = 0; r < TB; ++r) {
+        const double rd = rpiv[r];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int i = r + 1 + ty + 16 * a;
+            if (i < TB) {
+                const double lir = T[i][r] * rd;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int c = tx + 16 * b;
+                    if (c <= r) R[i][c] -= lir * R[r][c];
+                }
+            }
+        }
+        if (tid <= r) X[r][tid] = R[r][tid] * rd;
         __syncthreads();
     }
-    for (int e = tid; e < TB * TB; e += 256) {
-        const int r = e / TB, c = e % TB;
-        if (c <= r) a0[(int64_t)r * K + c] = T[r][c];
-        Linv[e] = I[r][c];
-    }
+    for (int r = ty; r < TB; r += 16)
+        for (int c = tx; c < TB; c += 16) {
+            if (c <= r) A[(int64_t)r * lda + c] = T[r][c];
+            Y[(int64_t)r * ldy + c] = c <= r ? X[r][c] : 0.0;
+        }
     if (tid == 0 && bad && status) atomicOr(status, HIF4_FLAG_NOT_SPD);
 }
 
-// 64 x 64 FP64 tile product helpers: 256 threads, each a 4 x 4 sub-block
-// (rows 4 (tid / 16) + i, cols 4 (tid % 16) + j).
-__device__ __forceinline__ void tile_load(Tile *S, const double *src, int64_t ld)
-{
-    for (int e = threadIdx.x; e < TB * TB; e += 256) S[e / TB][e % TB] = src[(int64_t)(e / TB) * ld + e % TB];
-}
+// FP64 GEMM on whole 64 x 64 tiles: C = alpha op(A) op(B) (+ C if beta),
+// one 64 x 64 tile of C per 128-thread block (8 rows x 4 columns per
+// thread), the K loop in 32-deep stages double-buffered through registers
+// and shared memory; the A stage is stored k-major so that a thread's 8 A
+// values and 4 B values of one k are 6 paired loads for 32 FMAs.  A is M x K
+// row-major; B is K x N row-major, or (BT) N x K row-major holding B^T.
+// Triangular operands skip their zero tiles: tri_a (A lower) ends the K loop
+// after tile ti; tri_b with B lower starts it at tile tj, with B^T lower
+// (BT) ends it after tile tj.  lower_c computes only the tiles tj <= ti.
+// M, N, K are multiples of 64; pointers and leading dimensions keep 16-byte
+// alignment.
+constexpr int KC = 32;                    // K per stage
+constexpr int SP = TB + 2;                // padded smem row of a stage (doubles; 16-byte multiple)
+constexpr int kStageD = 2 * KC * SP;      // A^T and B stages, KC x 64 each
+constexpr size_t kGemmSmem = sizeof(double) * 2 * kStageD;
+constexpr int kGemmThreads = 128;
 
-// S = src^T (S[k][c] = src[c][k]): the right operand of an X Y^T product
-// stored k-major, so that the product reads it like an X Y operand.
-__device__ __forceinline__ void tile_load_t(Tile *S, const double *src, int64_t ld)
-{
-    for (int e = threadIdx.x; e < TB * TB; e += 256) S[e % TB][e / TB] = src[(int64_t)(e / TB) * ld + e % TB];
-}
+struct Dgemm {
+    const double *A;
+    int64_t lda;
+    const double *B;
+    int64_t ldb;
+    double *C;
+    int64_t ldc;
+    int M, N, K;
+    double alpha;
+    int beta, tri_a, tri_b, lower_c;
+};
 
-// acc += X Y (X, Y: 64 x 64 in shared memory; Y read as pairs along a row)
-__device__ __forceinline__ void tile_mma_nn(double (&acc)[4][4], const Tile *X, const Tile *Y)
+template <bool BT>
+__global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
 {
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
+    const int tj = blockIdx.x, ti = blockIdx.y;
+    if (g.lower_c && tj > ti) return;
+    extern __shared__ __align__(16) double smd[];
+    int k0 = 0, k1 = g.K;
+    if (g.tri_a) k1 = min(k1, TB * (ti + 1));
+    if (g.tri_b) {
+        if (BT)
+            k1 = min(k1, TB * (tj + 1));
+        else
+            k0 = max(k0, TB * tj);
+    }
+    const int tid = threadIdx.x, r0 = 8 * (tid >> 4), c0 = 4 * (tid & 15);
+    const double *Ab = g.A + (int64_t)ti * TB * g.lda;
+    const double *Bb = BT ? g.B + (int64_t)tj * TB * g.ldb : g.B + (int64_t)tj * TB;
+    double2 ra[8], rb[8];
+    // a stage: 64 rows x 32 k of A and 32 k x 64 columns of B, 8 pairs each per thread
+    auto load = [&](int k) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int idx = tid + kGemmThreads * q;                  // 0 .. 1023
+            ra[q] = *reinterpret_cast<const double2 *>(Ab + (int64_t)(idx >> 4) * g.lda + k + 2 * (idx & 15));
+            if (BT)
+                rb[q] = *reinterpret_cast<const double2 *>(Bb + (int64_t)(idx >> 4) * g.ldb + k + 2 * (idx & 15));
+            else
+                rb[q] = *reinterpret_cast<const double2 *>(Bb + (int64_t)(k + (idx >> 5)) * g.ldb + 2 * (idx & 31));
+        }
+    };
+    auto store = [&](int buf) {
+        double *As = smd + buf * kStageD, *Bs = As + KC * SP;       // As[k][row], Bs[k][col]
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int idx = tid + kGemmThreads * q;
+            As[(2 * (idx & 15)) * SP + (idx >> 4)] = ra[q].x;
+            As[(2 * (idx & 15) + 1) * SP + (idx >> 4)] = ra[q].y;
+            if (BT) {
+                Bs[(2 * (idx & 15)) * SP + (idx >> 4)] = rb[q].x;
+                Bs[(2 * (idx & 15) + 1) * SP + (idx >> 4)] = rb[q].y;
+            } else {
+                *reinterpret_cast<double2 *>(Bs + (idx >> 5) * SP + 2 * (idx & 31)) = rb[q];
+            }
+        }
+    };
+    double acc[8][4] = {};
+    if (k0 < k1) {
+        load(k0);
+        store(0);
+        __syncthreads();
+        int buf = 0;
+        for (int k = k0; k < k1; k += KC) {
+            const bool more = k + KC < k1;
+            if (more) load(k + KC);
+            const double *As = smd + buf * kStageD, *Bs = As + KC * SP;
 #pragma unroll 4
-    for (int k = 0; k < TB; ++k) {
-        double x[4];
+            for (int kk = 0; kk < KC; ++kk) {
+                double x[8], y[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = X[r0 + i][k];
-        const double2 ya = *reinterpret_cast<const double2 *>(&Y[k][c0]);
-        const double2 yb = *reinterpret_cast<const double2 *>(&Y[k][c0 + 2]);
-        const double y[4] = {ya.x, ya.y, yb.x, yb.y};
+                for (int h = 0; h < 4; ++h) {
+                    const double2 v = *reinterpret_cast<const double2 *>(As + kk * SP + r0 + 2 * h);
+                    x[2 * h] = v.x;
+                    x[2 * h + 1] = v.y;
+                }
+                const double2 ya = *reinterpret_cast<const double2 *>(Bs + kk * SP + c0);
+                const double2 yb = *reinterpret_cast<const double2 *>(Bs + kk * SP + c0 + 2);
+                y[0] = ya.x;
+                y[1] = ya.y;
+                y[2] = yb.x;
+                y[3] = yb.y;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
+            }
+            if (more) store(buf ^ 1);
+            __syncthreads();
+            buf ^= 1;
+        }
     }
-}
-
-// Panel below diagonal tile kb: L[r, kb] = A[r, kb] Linv^T for the row
-// tiles r > kb.  One block per row tile (in place: the tile is read whole
-// before it is written).
-__global__ void __launch_bounds__(256) k_panel(double *A, int64_t K, int kb, const double *Linv)
-{
-    extern __shared__ __align__(16) double smd[];
-    Tile *X = reinterpret_cast<Tile *>(smd);
-    Tile *Y = X + TB;
-    const int rt = kb + 1 + blockIdx.x;
-    double *a = A + (int64_t)rt * TB * K + (int64_t)kb * TB;
-    tile_load(X, a, K);
-    tile_load_t(Y, Linv, TB);
-    __syncthreads();
-    double acc[4][4] = {};
-    tile_mma_nn(acc, X, Y);
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) a[(int64_t)(r0 + i) * K + c0 + j] = acc[i][j];
-}
-
-// Trailing update after tile kb: A[ti][tj] -= L[ti][kb] L[tj][kb]^T for
-// kb < tj <= ti.  Grid (n, n) with n the trailing tile count; blocks above
-// the diagonal exit at once, and so does tile (kb + 1, kb + 1) when
-// skip_next_diag is set (it is updated first, by a one-block launch, so that
-// its factorization can overlap the rest of this update).
-__global__ void __launch_bounds__(256) k_syrk(double *A, int64_t K, int kb, int skip_next_diag)
-{
-    const int ti = kb + 1 + blockIdx.y, tj = kb + 1 + blockIdx.x;
-    if (tj > ti || (skip_next_diag && blockIdx.x == 0 && blockIdx.y == 0)) return;
-    extern __shared__ __align__(16) double smd[];
-    Tile *X = reinterpret_cast<Tile *>(smd);
-    Tile *Y = X + TB;
-    tile_load(X, A + (int64_t)ti * TB * K + (int64_t)kb * TB, K);
-    tile_load_t(Y, A + (int64_t)tj * TB * K + (int64_t)kb * TB, K);
-    __syncthreads();
-    double acc[4][4] = {};
-    tile_mma_nn(acc, X, Y);
-    double *c = A + (int64_t)ti * TB * K + (int64_t)tj * TB;
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) c[(int64_t)(r0 + i) * K + c0 + j] -= acc[i][j];
-}
-
-// Y = L^{-1} (lower, tile rows), right-looking.  Y starts at zero and
-// accumulates S[i][j] = sum_{k<i} L[i][k] Y[k][j] in place; at step k block
-// row k is finalized (k_trtri_finalize: Y[k][k] = Linv_k, Y[k][j] =
-// -Linv_k S[k][j]) and its contribution is added to every later block row
-// (k_trtri_update: S[i][j] += L[i][k] Y[k][j], i > k >= j).
-__global__ void __launch_bounds__(256) k_trtri_finalize(int64_t K, int k, const double *LinvAll, double *Y)
-{
-    extern __shared__ __align__(16) double smd[];
-    Tile *X = reinterpret_cast<Tile *>(smd);
-    Tile *Z = X + TB;
-    const int j = blockIdx.x;
-    const double *lk = LinvAll + (int64_t)k * TB * TB;
-    double *y = Y + (int64_t)k * TB * K + (int64_t)j * TB;
-    if (j == k) {
-        for (int e = threadIdx.x; e < TB * TB; e += 256) y[(int64_t)(e / TB) * K + e % TB] = lk[e];
-        return;
+    for (int i = 0; i < 8; ++i) {
+        double2 *cp = reinterpret_cast<double2 *>(g.C + (int64_t)(ti * TB + r0 + i) * g.ldc + tj * TB + c0);
+        double2 u = make_double2(g.alpha * acc[i][0], g.alpha * acc[i][1]);
+        double2 v = make_double2(g.alpha * acc[i][2], g.alpha * acc[i][3]);
+        if (g.beta) {
+            const double2 cu = cp[0], cv = cp[1];
+            u.x += cu.x;
+            u.y += cu.y;
+            v.x += cv.x;
+            v.y += cv.y;
+        }
+        cp[0] = u;
+        cp[1] = v;
     }
-    tile_load(X, lk, TB);
-    tile_load(Z, y, K);
-    __syncthreads();
-    double out[4][4] = {};
-    tile_mma_nn(out, X, Z);
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) y[(int64_t)(r0 + a) * K + c0 + b] = -out[a][b];
-}
-
-// grid (k + 1, nb - 1 - k): block (j, ii) updates S[k + 1 + ii][j]
-__global__ void __launch_bounds__(256) k_trtri_update(const double *A, int64_t K, int k, double *Y)
-{
-    extern __shared__ __align__(16) double smd[];
-    Tile *X = reinterpret_cast<Tile *>(smd);
-    Tile *Z = X + TB;
-    const int j = blockIdx.x, i = k + 1 + blockIdx.y;
-    tile_load(X, A + (int64_t)i * TB * K + (int64_t)k * TB, K);            // L[i][k]
-    tile_load(Z, Y + (int64_t)k * TB * K + (int64_t)j * TB, K);            // Y[k][j]
-    __syncthreads();
-    double acc[4][4] = {};
-    tile_mma_nn(acc, X, Z);
-    double *s = Y + (int64_t)i * TB * K + (int64_t)j * TB;
-    const int r0 = 4 * (threadIdx.x / 16), c0 = 4 * (threadIdx.x % 16);
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) s[(int64_t)(r0 + a) * K + c0 + b] += acc[a][b];
 }
 
 // U[i][j] = Y[K-1-i][K-1-j] for j >= i (FP32, upper), 0 below; and the
@@ -563,7 +592,7 @@ size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace sections of hif4_higptq1.
 struct GptqLayout {
-    size_t A, Y, Linv, U, UinvG, W, Err, mask, rank, dead, mean, total;
+    size_t A, Y, T, U, UinvG, W, Err, mask, rank, dead, mean, total;
 };
 
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
@@ -577,7 +606,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     };
     take(L.A, k * k * 8);
     take(L.Y, k * k * 8);
-    take(L.Linv, nb * TB * TB * 8);
+    // the factor's scratch: the root split's n2 x n1 block (nested splits are smaller)
+    take(L.T, (nb - nb / 2) * (nb / 2 > 0 ? nb / 2 : 1) * TB * TB * 8);
     take(L.U, k * k * 4);
     take(L.UinvG, nb * TB * TB * 4);
     take(L.W, (size_t)N * k * 4);
@@ -600,22 +630,47 @@ bool set_smem_once(F *kernel, size_t bytes, bool &done)
     return true;
 }
 
-// Second stream and events of the factorization look-ahead (created per call,
-// released once their work completes).
-struct Aux {
-    cudaStream_t s2 = nullptr;
-    cudaEvent_t ev_diag = nullptr, ev_factored = nullptr;
-    bool make()
+// The factor of section "Factor": A (lower triangle of P Hd P on entry) and
+// Y = L^{-1}, both K x K; T the scratch block.
+struct Factor {
+    double *A, *Y, *T;
+    int64_t K;
+    uint32_t *status;
+    cudaStream_t s;
+
+    hif4_status gemm(bool bt, const double *a, int64_t lda, const double *b, int64_t ldb, double *c, int64_t ldc,
+                     int64_t M, int64_t N, int64_t Kd, double alpha, int beta, int tri_a, int tri_b, int lower_c)
     {
-        return cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking) == cudaSuccess &&
-               cudaEventCreateWithFlags(&ev_diag, cudaEventDisableTiming) == cudaSuccess &&
-               cudaEventCreateWithFlags(&ev_factored, cudaEventDisableTiming) == cudaSuccess;
+        Dgemm g{a, lda, b, ldb, c, ldc, (int)M, (int)N, (int)Kd, alpha, beta, tri_a, tri_b, lower_c};
+        const dim3 grid((unsigned)(N / TB), (unsigned)(M / TB));
+        if (bt)
+            k_dgemm<true><<<grid, kGemmThreads, kGemmSmem, s>>>(g);
+        else
+            k_dgemm<false><<<grid, kGemmThreads, kGemmSmem, s>>>(g);
+        return launch_status();
     }
-    ~Aux()
+
+    // rows [o, o + n) of the factor and of its inverse
+    hif4_status run(int64_t o, int64_t n)
     {
-        if (ev_diag) cudaEventDestroy(ev_diag);
-        if (ev_factored) cudaEventDestroy(ev_factored);
-        if (s2) cudaStreamDestroy(s2);
+        if (n == TB) {
+            k_leaf<<<1, 256, kLeafSmem, s>>>(A + o * K + o, K, Y + o * K + o, K, status);
+            return launch_status();
+        }
+        const int64_t n1 = n / TB / 2 * TB, n2 = n - n1, a = o, b = o + n1;
+        hif4_status st = run(a, n1);
+        if (st != HIF4_OK) return st;
+        double *A21 = A + b * K + a, *A22 = A + b * K + b, *Y11 = Y + a * K + a, *Y21 = Y + b * K + a,
+               *Y22 = Y + b * K + b;
+        if ((st = gemm(true, A21, K, Y11, K, T, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
+        if ((st = gemm(true, T, n1, T, n1, A22, K, n2, n2, n1, -1.0, 1, 0, 0, 1)) != HIF4_OK) return st;
+        if ((st = gemm(false, T, n1, Y11, K, Y21, K, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
+        if ((st = run(b, n2)) != HIF4_OK) return st;
+        if ((st = gemm(false, Y22, K, Y21, K, T, n1, n2, n1, n2, -1.0, 0, 1, 0, 0)) != HIF4_OK) return st;
+        if (cudaMemcpy2DAsync(Y21, (size_t)K * 8, T, (size_t)n1 * 8, (size_t)n1 * 8, (size_t)n2,
+                              cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return HIF4_ERR_CUDA;
+        return HIF4_OK;
     }
 };
 
@@ -691,7 +746,7 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     double *A = reinterpret_cast<double *>(ws + L.A);
     double *Y = reinterpret_cast<double *>(ws + L.Y);
-    double *Linv = reinterpret_cast<double *>(ws + L.Linv);
+    double *T = reinterpret_cast<double *>(ws + L.T);
     float *U = reinterpret_cast<float *>(ws + L.U);
     float *UinvG = reinterpret_cast<float *>(ws + L.UinvG);
     float *W = reinterpret_cast<float *>(ws + L.W);
@@ -700,17 +755,13 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
     uint8_t *dead = ws + L.dead;
     double *mean = reinterpret_cast<double *>(ws + L.mean);
-    const int nb = (int)(K / TB);
 
-    static bool attr2[64] = {false}, attr2b[64] = {false}, attr2c[64] = {false}, attr2d[64] = {false},
-                attr2e[64] = {false};
+    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!set_smem_once(k_potrf_tile, 2 * kTileBytes, attr2[dev & 63]) ||
-        !set_smem_once(k_panel, 2 * kTileBytes, attr2b[dev & 63]) ||
-        !set_smem_once(k_syrk, 2 * kTileBytes, attr2c[dev & 63]) ||
-        !set_smem_once(k_trtri_finalize, 2 * kTileBytes, attr2d[dev & 63]) ||
-        !set_smem_once(k_trtri_update, 2 * kTileBytes, attr2e[dev & 63]))
+    if (!set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
+        !set_smem_once(k_dgemm<false>, kGemmSmem, attr_g0[dev & 63]) ||
+        !set_smem_once(k_dgemm<true>, kGemmSmem, attr_g1[dev & 63]))
         return HIF4_ERR_CUDA;
 
     // 1. protected columns, Hessian diagonal statistics, FP32 working weights
@@ -728,48 +779,17 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
         k_w_to_f32<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W, status);
         if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     }
-    // 2. P Hd P = L' L'^T (FP64, 64 x 64 tiles, right-looking)
+    // 2. P Hd P = L' L'^T and Y = L'^{-1} (FP64, recursive), then U = P Y P
+    //    and the inverses of U's diagonal blocks
     k_fill_reversed<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(
         H, K, dead, mean, damp, A);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    //    Look-ahead: after panel kb, diagonal tile kb + 1 is updated first and
-    //    factored on a second stream while the rest of the trailing update
-    //    runs (disjoint tiles); panel kb + 1 waits for it.
-    Aux X;
-    if (!X.make()) return HIF4_ERR_CUDA;
-    auto join = [&](hif4_status r) {
-        if (cudaEventRecord(X.ev_factored, X.s2) == cudaSuccess) cudaStreamWaitEvent(s, X.ev_factored, 0);
-        return r;
-    };
-    k_potrf_tile<<<1, 256, 2 * kTileBytes, s>>>(A, K, 0, Linv, status);
-    if (launch_status() != HIF4_OK) return join(HIF4_ERR_CUDA);
-    for (int kb = 0; kb < nb; ++kb) {
-        const int n = nb - 1 - kb;
-        if (n == 0) break;
-        if (kb > 0 && cudaStreamWaitEvent(s, X.ev_factored, 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
-        k_panel<<<n, 256, 2 * kTileBytes, s>>>(A, K, kb, Linv + (size_t)kb * TB * TB);
-        k_syrk<<<1, 256, 2 * kTileBytes, s>>>(A, K, kb, 0);                   // tile (kb + 1, kb + 1)
-        if (launch_status() != HIF4_OK || cudaEventRecord(X.ev_diag, s) != cudaSuccess ||
-            cudaStreamWaitEvent(X.s2, X.ev_diag, 0) != cudaSuccess)
-            return join(HIF4_ERR_CUDA);
-        k_potrf_tile<<<1, 256, 2 * kTileBytes, X.s2>>>(A, K, kb + 1, Linv + (size_t)(kb + 1) * TB * TB, status);
-        if (launch_status() != HIF4_OK || cudaEventRecord(X.ev_factored, X.s2) != cudaSuccess)
-            return join(HIF4_ERR_CUDA);
-        if (n > 1) k_syrk<<<dim3(n, n), 256, 2 * kTileBytes, s>>>(A, K, kb, 1);
-        if (launch_status() != HIF4_OK) return join(HIF4_ERR_CUDA);
-    }
-    if (nb > 1 && cudaStreamWaitEvent(s, X.ev_factored, 0) != cudaSuccess) return join(HIF4_ERR_CUDA);
-    // 3. Y = L'^{-1} (right-looking by block rows), then U = P Y P and the
-    //    inverses of U's diagonal blocks
-    if (cudaMemsetAsync(Y, 0, (size_t)K * K * 8, s) != cudaSuccess) return HIF4_ERR_CUDA;
-    for (int k = 0; k < nb; ++k) {
-        k_trtri_finalize<<<k + 1, 256, 2 * kTileBytes, s>>>(K, k, Linv, Y);
-        if (k + 1 < nb) k_trtri_update<<<dim3(k + 1, nb - 1 - k), 256, 2 * kTileBytes, s>>>(A, K, k, Y);
-        if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    }
+    Factor F{A, Y, T, K, status, s};
+    const hif4_status fst = F.run(0, K);
+    if (fst != HIF4_OK) return fst;
     k_build_u<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    // 4. the group loop: per block, the groups with their in-block feedback,
+    // 3. the group loop: per block, the groups with their in-block feedback,
     //    then the lazy update of every later column
     for (int64_t b0 = 0; b0 < K; b0 += B) {
         const int64_t b1 = b0 + B < K ? b0 + B : K;
