@@ -27,6 +27,7 @@
 
 #include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
+#include "hif4_sm100.cuh"
 
 namespace hif4 {
 namespace {
@@ -82,110 +83,195 @@ __global__ void k_fill_reversed(const float *H, int64_t K, const uint8_t *dead, 
 // (in A); every product is an FP64 GEMM that skips the tiles in which a
 // triangular operand is zero, so the whole factor costs K^3/3 + K^3/3 FLOP.
 
-constexpr int LP = TB + 2;              // padded smem row of a leaf tile (doubles)
-constexpr size_t kLeafSmem = sizeof(double) * 3 * TB * LP;
+constexpr int HB = TB / 2;               // half leaf: one warp's block
+constexpr int HP = HB + 1;               // padded smem row of a half block (doubles)
+constexpr size_t kLeafSmem = sizeof(double) * 7 * HB * HP;
 
-// One 64 x 64 diagonal block: Cholesky (lower, in place in A, right-looking
-// by columns) and the inverse of the factor into Y (zeros above the
-// diagonal).  A pivot that is not positive is replaced by 1 and reported as
+// Cholesky of a 32 x 32 block held by one warp, lane r holding row r in
+// a[0..31] (a[c] for c <= r is read; the rest must be 0).  On return a is
+// row r of the factor.  Pivots that are not positive are replaced by 1 and
+// counted in *bad.
+__device__ __forceinline__ void warp_chol32(double (&a)[HB], int &bad)
+{
+    const int r = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < HB; ++j) {
+        double d = __shfl_sync(0xffffffffu, a[j], j);
+        const bool ok = d > 0.0;
+        if (!ok) d = 1.0;
+        const double rs = rsqrt(d);
+        const double l = a[j] * rs;                   // lane j: the pivot d rs; below it: the column
+        if (r >= j) a[j] = l;
+        bad |= (int)(!ok && r == j);
+#pragma unroll
+        for (int c = j + 1; c < HB; ++c) {
+            const double lc = __shfl_sync(0xffffffffu, l, c);
+            if (r >= c) a[c] -= l * lc;
+        }
+    }
+}
+
+// Inverse of the 32 x 32 lower factor held by rows (lane r: row r in a[]),
+// returned by columns: lane c gets column c of L^{-1} in x[0..31] (0 above
+// the diagonal).  Forward substitution, row r of L broadcast from lane r.
+__device__ __forceinline__ void warp_inv32(const double (&a)[HB], double (&x)[HB])
+{
+    const int c = threadIdx.x & 31;
+    double dg = 1.0;                                 // lane c: L[c][c] (static indexing keeps a[] in registers)
+#pragma unroll
+    for (int k = 0; k < HB; ++k)
+        if (k == c) dg = a[k];
+    const double rdiag = 1.0 / dg;
+#pragma unroll
+    for (int r = 0; r < HB; ++r) {
+        double sum = 0.0;
+#pragma unroll
+        for (int k = 0; k < r; ++k) sum = fma(__shfl_sync(0xffffffffu, a[k], r), x[k], sum);
+        x[r] = ((r == c ? 1.0 : 0.0) - sum) * __shfl_sync(0xffffffffu, rdiag, r);
+    }
+}
+
+// One 64 x 64 diagonal block: its Cholesky factor (lower, in place in A)
+// and the factor's inverse into Y (zeros above the diagonal), as two halves:
+// warp 0 factors and inverts the 32 x 32 diagonal blocks in registers, all
+// 8 warps form L21 = A21 L11^{-T}, A22 - L21 L21^T and
+// Y21 = -L22^{-1} L21 L11^{-1} as 32 x 32 x 32 shared-memory products.  A
+// pivot that is not positive is replaced by 1 and reported as
 // HIF4_FLAG_NOT_SPD.  256 threads.
 __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
 {
     extern __shared__ __align__(16) double smd[];
-    double(*T)[LP] = reinterpret_cast<double(*)[LP]>(smd);      // the factor
-    double(*R)[LP] = T + TB;                                     // right-hand sides of L X = I
-    double(*X)[LP] = R + TB;                                     // the inverse
-    __shared__ double col[TB], piv[TB], rpiv[TB];
-    __shared__ int bad;
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;  // 16 x 16 thread grid
-    for (int r = ty; r < TB; r += 16)
-        for (int c = tx; c < TB; c += 16) {
-            T[r][c] = c <= r ? A[(int64_t)r * lda + c] : 0.0;
-            R[r][c] = r == c ? 1.0 : 0.0;
-            X[r][c] = 0.0;
-        }
-    if (tid == 0) bad = 0;
-    __syncthreads();
-    for (int j = 0; j < TB; ++j) {
-        // column j: the pivot, then the scaled entries below it (thread r
-        // owns row r); one reciprocal square root per column
-        if (tid < TB) {
-            double d = T[j][j];
-            const bool ok = d > 0.0;
-            if (!ok) d = 1.0;
-            const double rs = rsqrt(d);
-            if (tid > j) {
-                const double l = T[tid][j] * rs;
-                col[tid] = l;
-                T[tid][j] = l;
-            } else if (tid == j) {
-                piv[j] = d * rs;
-                rpiv[j] = rs;
-                if (!ok) bad = 1;
-            }
-        }
-        __syncthreads();
-        // rank-1 update of the trailing lower triangle, 4 x 4 candidates per
-        // thread (the pivot itself is written after the loop: every thread
-        // above read it before the sync)
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = j + 1 + ty + 16 * a;
-            if (r < TB) {
-                const double lr = col[r];
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int c = j + 1 + tx + 16 * b;
-                    if (c <= r) T[r][c] -= lr * col[c];
-                }
-            }
-        }
-        __syncthreads();
+    double(*A11)[HP] = reinterpret_cast<double(*)[HP]>(smd);    // A11, then L11
+    double(*A21)[HP] = A11 + HB;                                 // A21
+    double(*A22)[HP] = A21 + HB;                                 // A22, then L22
+    double(*L21)[HP] = A22 + HB;
+    double(*X11)[HP] = L21 + HB;                                 // L11^{-1}
+    double(*X22)[HP] = X11 + HB;                                 // L22^{-1}
+    double(*T)[HP] = X22 + HB;                                   // L21 L11^{-1}, then Y21
+    __shared__ int bad_all;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll 16
+    for (int e = tid; e < TB * TB; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        const double v = c <= r ? A[(int64_t)r * lda + c] : 0.0;
+        if (r < HB) {
+            if (c < HB) A11[r][c] = v;
+        } else if (c < HB)
+            A21[r - HB][c] = v;
+        else
+            A22[r - HB][c - HB] = v;
     }
-    if (tid < TB) T[tid][tid] = piv[tid];
+    if (tid == 0) bad_all = 0;
     __syncthreads();
-    // L X = I by rows: at step r row r of X is R[r][:] / L[r][r], and its
-    // contribution leaves the rows below (row r of R is final at step r and
-    // nobody writes it during that step)
-    for (int r = 0; r < TB; ++r) {
-        const double rd = rpiv[r];
+    // each thread's four outputs of a 32 x 32 product: rows ro + 8 i, column lane
+    const int ro = warp;
+    int bad = 0;
+    if (warp == 0) {
+        double a[HB], x[HB];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int i = r + 1 + ty + 16 * a;
-            if (i < TB) {
-                const double lir = T[i][r] * rd;
+        for (int c = 0; c < HB; ++c) a[c] = A11[lane][c];
+        warp_chol32(a, bad);
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int c = tx + 16 * b;
-                    if (c <= r) R[i][c] -= lir * R[r][c];
-                }
-            }
-        }
-        if (tid <= r) X[r][tid] = R[r][tid] * rd;
-        __syncthreads();
+        for (int c = 0; c < HB; ++c) A11[lane][c] = c <= lane ? a[c] : 0.0;
+        warp_inv32(a, x);
+#pragma unroll
+        for (int r = 0; r < HB; ++r) X11[r][lane] = x[r];
     }
-    for (int r = ty; r < TB; r += 16)
-        for (int c = tx; c < TB; c += 16) {
-            if (c <= r) A[(int64_t)r * lda + c] = T[r][c];
-            Y[(int64_t)r * ldy + c] = c <= r ? X[r][c] : 0.0;
+    __syncthreads();
+    // L21 = A21 X11^T   (X11 lower: k <= c)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = ro + 8 * i;
+        double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+        for (int k = 0; k < HB; k += 2) {                       // X11[lane][k] = 0 for k > lane
+            s0 = fma(A21[r][k], X11[lane][k], s0);
+            s1 = fma(A21[r][k + 1], X11[lane][k + 1], s1);
         }
-    if (tid == 0 && bad && status) atomicOr(status, HIF4_FLAG_NOT_SPD);
+        L21[r][lane] = s0 + s1;
+    }
+    __syncthreads();
+    // A22 -= L21 L21^T (lower half), T = L21 X11 (X11 lower: k >= c)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = ro + 8 * i;
+        double s0 = 0.0, s1 = 0.0, t0 = 0.0, t1 = 0.0;
+#pragma unroll
+        for (int k = 0; k < HB; k += 2) {                       // X11[k][lane] = 0 for k < lane
+            s0 = fma(L21[r][k], L21[lane][k], s0);
+            s1 = fma(L21[r][k + 1], L21[lane][k + 1], s1);
+            t0 = fma(L21[r][k], X11[k][lane], t0);
+            t1 = fma(L21[r][k + 1], X11[k + 1][lane], t1);
+        }
+        if (lane <= r) A22[r][lane] -= s0 + s1;
+        T[r][lane] = t0 + t1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        double a[HB], x[HB];
+#pragma unroll
+        for (int c = 0; c < HB; ++c) a[c] = A22[lane][c];
+        warp_chol32(a, bad);
+#pragma unroll
+        for (int c = 0; c < HB; ++c) A22[lane][c] = c <= lane ? a[c] : 0.0;
+        warp_inv32(a, x);
+#pragma unroll
+        for (int r = 0; r < HB; ++r) X22[r][lane] = x[r];
+        if (bad) atomicOr(&bad_all, 1);
+    }
+    __syncthreads();
+    // Y21 = -X22 T   (X22 lower: k <= r); results kept in registers until all reads of T are done
+    double y21[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = ro + 8 * i;
+        double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+        for (int k = 0; k < HB; k += 2) {                       // X22[r][k] = 0 for k > r
+            s0 = fma(X22[r][k], T[k][lane], s0);
+            s1 = fma(X22[r][k + 1], T[k + 1][lane], s1);
+        }
+        y21[i] = -(s0 + s1);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) T[ro + 8 * i][lane] = y21[i];
+    __syncthreads();
+    for (int e = tid; e < TB * TB; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        double l, y;
+        if (r < HB) {
+            l = c < HB ? A11[r][c] : 0.0;
+            y = c < HB ? X11[r][c] : 0.0;
+        } else if (c < HB) {
+            l = L21[r - HB][c];
+            y = T[r - HB][c];
+        } else {
+            l = A22[r - HB][c - HB];
+            y = X22[r - HB][c - HB];
+        }
+        if (c <= r) A[(int64_t)r * lda + c] = l;
+        Y[(int64_t)r * ldy + c] = y;
+    }
+    if (tid == 0 && bad_all && status) atomicOr(status, HIF4_FLAG_NOT_SPD);
 }
 
 // FP64 GEMM on whole 64 x 64 tiles: C = alpha op(A) op(B) (+ C if beta),
-// one 64 x 64 tile of C per 128-thread block (8 rows x 4 columns per
-// thread), the K loop in 32-deep stages double-buffered through registers
-// and shared memory; the A stage is stored k-major so that a thread's 8 A
-// values and 4 B values of one k are 6 paired loads for 32 FMAs.  A is M x K
-// row-major; B is K x N row-major, or (BT) N x K row-major holding B^T.
-// Triangular operands skip their zero tiles: tri_a (A lower) ends the K loop
-// after tile ti; tri_b with B lower starts it at tile tj, with B^T lower
-// (BT) ends it after tile tj.  lower_c computes only the tiles tj <= ti.
-// M, N, K are multiples of 64; pointers and leading dimensions keep 16-byte
-// alignment.
+// on the FP64 tensor-core MMA (m8n8k4).  One 64 x 64 tile of C per
+// 128-thread block, a 32 x 32 quarter per warp (4 x 4 MMA tiles); the K loop
+// runs in 32-deep stages that cp.async copies double-buffer into shared
+// memory in the operands' own layouts: A row-major, B k-major (B row-major)
+// or n-major (BT, B^T row-major), whose fragments the MMA reads directly.  A
+// is M x K row-major; B is K x N row-major, or (BT) N x K row-major holding
+// B^T.  Triangular operands skip their zero tiles: tri_a (A lower) ends the
+// K loop after tile ti; tri_b with B lower starts it at tile tj, with B^T
+// lower (BT) ends it after tile tj.  lower_c computes only the tiles
+// tj <= ti.  M, N, K are multiples of 64; pointers and leading dimensions
+// keep 16-byte alignment.
 constexpr int KC = 32;                    // K per stage
-constexpr int SP = TB + 2;                // padded smem row of a stage (doubles; 16-byte multiple)
-constexpr int kStageD = 2 * KC * SP;      // A^T and B stages, KC x 64 each
+constexpr int AS = KC + 4;                // smem row of an n- or m-major stage (doubles; 16-byte multiple)
+constexpr int BS = TB + 4;                // smem row of a k-major B stage
+constexpr int kStageD = 2 * TB * AS;      // A stage + the larger B stage (64 x 36 >= 32 x 68)
 constexpr size_t kGemmSmem = sizeof(double) * 2 * kStageD;
 constexpr int kGemmThreads = 128;
 
@@ -201,6 +287,21 @@ struct Dgemm {
     int beta, tri_a, tri_b, lower_c;
 };
 
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_addr(smem_dst)), "l"(gmem_src)
+                 : "memory");
+}
+
+// d (8 x 8, two per lane: row lane / 4, columns 2 (lane % 4) + {0, 1}) +=
+// a (8 x 4, row lane / 4, column lane % 4) b (4 x 8, row lane % 4, column lane / 4)
+__device__ __forceinline__ void dmma884(double (&d)[2], double a, double b)
+{
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
+}
+
 template <bool BT>
 __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
 {
@@ -215,87 +316,68 @@ __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
         else
             k0 = max(k0, TB * tj);
     }
-    const int tid = threadIdx.x, r0 = 8 * (tid >> 4), c0 = 4 * (tid & 15);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int wm = 32 * (warp >> 1), wn = 32 * (warp & 1), gid = lane >> 2, tig = lane & 3;
     const double *Ab = g.A + (int64_t)ti * TB * g.lda;
     const double *Bb = BT ? g.B + (int64_t)tj * TB * g.ldb : g.B + (int64_t)tj * TB;
-    double2 ra[8], rb[8];
-    // a stage: 64 rows x 32 k of A and 32 k x 64 columns of B, 8 pairs each per thread
-    auto load = [&](int k) {
+    // one stage: 64 x 32 of A and 32 x 64 of B as 16-byte chunks, 8 + 8 per thread
+    auto issue = [&](int k, int st) {
+        double *As = smd + st * kStageD, *Bs = As + TB * AS;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int idx = tid + kGemmThreads * q;                  // 0 .. 1023
-            ra[q] = *reinterpret_cast<const double2 *>(Ab + (int64_t)(idx >> 4) * g.lda + k + 2 * (idx & 15));
+            cp_async16(As + (idx >> 4) * AS + 2 * (idx & 15), Ab + (int64_t)(idx >> 4) * g.lda + k + 2 * (idx & 15));
             if (BT)
-                rb[q] = *reinterpret_cast<const double2 *>(Bb + (int64_t)(idx >> 4) * g.ldb + k + 2 * (idx & 15));
+                cp_async16(Bs + (idx >> 4) * AS + 2 * (idx & 15),
+                           Bb + (int64_t)(idx >> 4) * g.ldb + k + 2 * (idx & 15));
             else
-                rb[q] = *reinterpret_cast<const double2 *>(Bb + (int64_t)(k + (idx >> 5)) * g.ldb + 2 * (idx & 31));
+                cp_async16(Bs + (idx >> 5) * BS + 2 * (idx & 31), Bb + (int64_t)(k + (idx >> 5)) * g.ldb + 2 * (idx & 31));
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    auto store = [&](int buf) {
-        double *As = smd + buf * kStageD, *Bs = As + KC * SP;       // As[k][row], Bs[k][col]
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int idx = tid + kGemmThreads * q;
-            As[(2 * (idx & 15)) * SP + (idx >> 4)] = ra[q].x;
-            As[(2 * (idx & 15) + 1) * SP + (idx >> 4)] = ra[q].y;
-            if (BT) {
-                Bs[(2 * (idx & 15)) * SP + (idx >> 4)] = rb[q].x;
-                Bs[(2 * (idx & 15) + 1) * SP + (idx >> 4)] = rb[q].y;
-            } else {
-                *reinterpret_cast<double2 *>(Bs + (idx >> 5) * SP + 2 * (idx & 31)) = rb[q];
-            }
-        }
-    };
-    double acc[8][4] = {};
+    double acc[4][4][2] = {};
     if (k0 < k1) {
-        load(k0);
-        store(0);
-        __syncthreads();
-        int buf = 0;
-        for (int k = k0; k < k1; k += KC) {
-            const bool more = k + KC < k1;
-            if (more) load(k + KC);
-            const double *As = smd + buf * kStageD, *Bs = As + KC * SP;
-#pragma unroll 4
-            for (int kk = 0; kk < KC; ++kk) {
-                double x[8], y[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const double2 v = *reinterpret_cast<const double2 *>(As + kk * SP + r0 + 2 * h);
-                    x[2 * h] = v.x;
-                    x[2 * h + 1] = v.y;
-                }
-                const double2 ya = *reinterpret_cast<const double2 *>(Bs + kk * SP + c0);
-                const double2 yb = *reinterpret_cast<const double2 *>(Bs + kk * SP + c0 + 2);
-                y[0] = ya.x;
-                y[1] = ya.y;
-                y[2] = yb.x;
-                y[3] = yb.y;
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fma(x[i], y[j], acc[i][j]);
+        issue(k0, 0);
+        int st = 0;
+        for (int k = k0; k < k1; k += KC, st ^= 1) {
+            if (k + KC < k1) {
+                issue(k + KC, st ^ 1);
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
             }
-            if (more) store(buf ^ 1);
             __syncthreads();
-            buf ^= 1;
+            const double *As = smd + st * kStageD, *Bs = As + TB * AS;
+#pragma unroll
+            for (int kk = 0; kk < KC; kk += 4) {
+                double a[4], b[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = As[(wm + 8 * i + gid) * AS + kk + tig];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    b[j] = BT ? Bs[(wn + 8 * j + gid) * AS + kk + tig] : Bs[(kk + tig) * BS + wn + 8 * j + gid];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) dmma884(acc[i][j], a[i], b[j]);
+            }
+            __syncthreads();                                         // stage st is refilled two steps on
         }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        double2 *cp = reinterpret_cast<double2 *>(g.C + (int64_t)(ti * TB + r0 + i) * g.ldc + tj * TB + c0);
-        double2 u = make_double2(g.alpha * acc[i][0], g.alpha * acc[i][1]);
-        double2 v = make_double2(g.alpha * acc[i][2], g.alpha * acc[i][3]);
-        if (g.beta) {
-            const double2 cu = cp[0], cv = cp[1];
-            u.x += cu.x;
-            u.y += cu.y;
-            v.x += cv.x;
-            v.y += cv.y;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            double2 *cp = reinterpret_cast<double2 *>(g.C + (int64_t)(ti * TB + wm + 8 * i + gid) * g.ldc + tj * TB +
+                                                      wn + 8 * j + 2 * tig);
+            double2 u = make_double2(g.alpha * acc[i][j][0], g.alpha * acc[i][j][1]);
+            if (g.beta) {
+                const double2 cu = *cp;
+                u.x += cu.x;
+                u.y += cu.y;
+            }
+            *cp = u;
         }
-        cp[0] = u;
-        cp[1] = v;
-    }
 }
 
 // U[i][j] = Y[K-1-i][K-1-j] for j >= i (FP32, upper), 0 below; and the
