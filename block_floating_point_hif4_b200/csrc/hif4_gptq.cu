@@ -100,7 +100,7 @@ __device__ __forceinline__ void warp_chol32(double (&a)[HB], int &bad)
         const bool ok = d > 0.0;
         if (!ok) d = 1.0;
         const double rs = rsqrt(d);
-        const double l = a[j] * rs;                   // lane j: the pivot d rs; below it: the column
+        const double l = r == j ? d * rs : a[j] * rs; // lane j: the pivot; below it: the column
         if (r >= j) a[j] = l;
         bad |= (int)(!ok && r == j);
 #pragma unroll
