@@ -19,10 +19,11 @@
 // so one Cholesky factorization and one triangular inverse suffice, and the
 // inverse of U's 64 x 64 diagonal block g is the reversed diagonal block of
 // L' itself.  Both run in FP64 by one recursion over halves whose products
-// are tiled FP64 GEMMs (section "Factor" below).  The group loop runs in
-// FP32: one warp per row
-// quantizes with the exact FP32 encode rule of the streaming quantizer, and
-// the lazy update after each block is an FP32 tile GEMM.
+// are FP64 tensor-core GEMMs (the factor section below).  The group loop
+// runs in FP32: one warp per row quantizes with the exact FP32 encode rule
+// of the streaming quantizer, and the lazy update after each block is a GEMM
+// on the TF32 tensor cores with split operands (three TF32 products per
+// FP32 product, FP32 accumulation).
 #include <cuda_bf16.h>
 
 #include "hif4_encode.cuh"
@@ -563,87 +564,131 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
     }
 }
 
-// C (M x Nc, ldc) -= A (M x Kd, lda) B (Kd x Nc, ldb) in FP32: 128 x 128
-// tiles, 256 threads with 8 x 8 outputs each, k in steps of 8 through two
-// shared-memory buffers (the next step's tiles are loaded into registers
-// while the current one is multiplied, one barrier per step).  Kd, lda and
-// ldb are multiples of 4 and A, B 16-byte aligned (float4 loads); M and Nc
-// are ragged (guarded).
+// C (M x Nc, ldc) -= A (M x Kd, lda) B (Kd x Nc, ldb), FP32 operands and
+// accumulation, on the TF32 tensor-core MMA (m16n8k8) with each operand
+// split as x = hi + lo (hi = x rounded to TF32, lo = the rest rounded to
+// TF32) and the product taken as lo hi + hi lo + hi hi: the dropped lo lo
+// term and the TF32 rounding of lo leave an error of the order of FP32
+// rounding.  64 x 128 tiles, 8 warps of 32 x 32 (2 x 4 MMA tiles); the K
+// loop in 32-deep stages that cp.async copies double-buffer into shared
+// memory (rows past M and columns past Nc are zero-filled and not stored).
+// Kd is a multiple of 32, Nc of 4; lda, ldb, ldc multiples of 4 floats and
+// A, B, C 16-byte aligned.
+constexpr int SGM = 64, SGN = 128, SGK = 32;
+constexpr int SAS = SGK + 4;              // smem row of the A stage (floats): conflict-free fragment loads
+constexpr int SBS = SGN + 8;              // smem row of the B stage
+constexpr int kSgStage = SGM * SAS + SGK * SBS;
+constexpr size_t kSgSmem = sizeof(float) * 2 * kSgStage;
+
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_addr(smem_dst)), "l"(gmem_src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t tf32_rna(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    hi = tf32_rna(x);
+    lo = tf32_rna(x - __uint_as_float(hi));
+}
+
+// d (16 x 8: rows g, g + 8, columns 2 t + {0, 1}) += a (16 x 8) b (8 x 8), TF32 in, FP32 out
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 __global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, const float *A, int64_t lda,
                                                    const float *B, int64_t ldb, int64_t M, int64_t Nc, int Kd)
 {
-    __shared__ __align__(16) float As[2][8][128 + 4];
-    __shared__ __align__(16) float Bs[2][8][128 + 4];
-    const int tid = threadIdx.x;
-    const int64_t m0 = blockIdx.y * 128ll, n0 = blockIdx.x * 128ll;
-    const int tr = tid / 16, tc = tid % 16;           // 16 x 16 threads, 8 x 8 outputs each
-    const int ar = tid / 2, ak = 4 * (tid % 2);       // A: row ar, k columns ak..ak+3
-    const int bk = tid / 32, bc = 4 * (tid % 32);     // B: k row bk, columns bc..bc+3
-    const int64_t gm = m0 + ar, gn = n0 + bc;
-    float4 ra, rb;
-    auto gload = [&](int k0) {
-        ra = gm < M ? *reinterpret_cast<const float4 *>(A + gm * lda + k0 + ak) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float *brow = B + (int64_t)(k0 + bk) * ldb;
-        if (gn + 3 < Nc) {
-            rb = *reinterpret_cast<const float4 *>(brow + gn);
+    extern __shared__ __align__(16) float sgs[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+    const int wm = 32 * (warp >> 2), wn = 32 * (warp & 3);
+    const int64_t m0 = (int64_t)blockIdx.y * SGM, n0 = (int64_t)blockIdx.x * SGN;
+    auto issue = [&](int k, int st) {
+        float *As = sgs + st * kSgStage, *Bs = As + SGM * SAS;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {                                // A: 64 rows x 8 chunks
+            const int idx = tid + 256 * q, r = idx >> 3, ch = idx & 7;
+            const bool ok = m0 + r < M;
+            cp_async16_zfill(As + r * SAS + 4 * ch, ok ? A + (m0 + r) * lda + k + 4 * ch : A, ok);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                                // B: 32 rows x 32 chunks
+            const int idx = tid + 256 * q, r = idx >> 5, ch = idx & 31;
+            const bool ok = n0 + 4 * ch < Nc;
+            cp_async16_zfill(Bs + r * SBS + 4 * ch, ok ? B + (int64_t)(k + r) * ldb + n0 + 4 * ch : B, ok);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    float acc[2][4][4] = {};
+    issue(0, 0);
+    int st = 0;
+    for (int k = 0; k < Kd; k += SGK, st ^= 1) {
+        if (k + SGK < Kd) {
+            issue(k + SGK, st ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
-            rb.x = gn < Nc ? brow[gn] : 0.f;
-            rb.y = gn + 1 < Nc ? brow[gn + 1] : 0.f;
-            rb.z = gn + 2 < Nc ? brow[gn + 2] : 0.f;
-            rb.w = 0.f;
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-    };
-    auto sstore = [&](int b) {
-        As[b][ak][ar] = ra.x;
-        As[b][ak + 1][ar] = ra.y;
-        As[b][ak + 2][ar] = ra.z;
-        As[b][ak + 3][ar] = ra.w;
-        *reinterpret_cast<float4 *>(&Bs[b][bk][bc]) = rb;
-    };
-    float acc[8][8] = {};
-    gload(0);
-    sstore(0);
-    __syncthreads();
-    for (int k0 = 0, b = 0; k0 < Kd; k0 += 8, b ^= 1) {
-        const bool more = k0 + 8 < Kd;
-        if (more) gload(k0 + 8);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&As[b][kk][tr * 8]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&As[b][kk][tr * 8 + 4]);
-            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[b][kk][tc * 8]);
-            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[b][kk][tc * 8 + 4]);
-            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(av[i], bv[jj], acc[i][jj]);
-        }
-        if (more) sstore(b ^ 1);
         __syncthreads();
-    }
-    // C -= acc, two float4 per row where the 8 columns are inside (C, ldc
-    // and the column offset are multiples of 4 floats)
-    const int64_t cn0 = n0 + tc * 8;
+        const float *As = sgs + st * kSgStage, *Bs = As + SGM * SAS;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int64_t cm = m0 + tr * 8 + i;
-        if (cm >= M) continue;
-        float *crow = C + cm * ldc + cn0;
-        if (cn0 + 7 < Nc) {
-            float4 *c4 = reinterpret_cast<float4 *>(crow);
-            float4 u = c4[0], v = c4[1];
-            u.x -= acc[i][0]; u.y -= acc[i][1]; u.z -= acc[i][2]; u.w -= acc[i][3];
-            v.x -= acc[i][4]; v.y -= acc[i][5]; v.z -= acc[i][6]; v.w -= acc[i][7];
-            c4[0] = u;
-            c4[1] = v;
-        } else {
+        for (int kk = 0; kk < SGK; kk += 8) {
+            uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                if (cn0 + jj < Nc) crow[jj] -= acc[i][jj];
+            for (int i = 0; i < 2; ++i) {
+                const float *ar = As + (wm + 16 * i + g) * SAS + kk + t;
+                split_tf32(ar[0], ah[i][0], al[i][0]);
+                split_tf32(ar[8 * SAS], ah[i][1], al[i][1]);
+                split_tf32(ar[4], ah[i][2], al[i][2]);
+                split_tf32(ar[8 * SAS + 4], ah[i][3], al[i][3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float *bc = Bs + (kk + t) * SBS + wn + 8 * j + g;
+                split_tf32(bc[0], bh[j][0], bl[j][0]);
+                split_tf32(bc[4 * SBS], bh[j][1], bl[j][1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_tf32(acc[i][j], al[i], bh[j]);
+                    mma_tf32(acc[i][j], ah[i], bl[j]);
+                    mma_tf32(acc[i][j], ah[i], bh[j]);
+                }
         }
+        __syncthreads();                                             // stage st is refilled two steps on
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t c = n0 + wn + 8 * j + 2 * t;
+            if (c >= Nc) continue;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t r = m0 + wm + 16 * i + g + 8 * h;
+                if (r >= M) continue;
+                float2 *cp = reinterpret_cast<float2 *>(C + r * ldc + c);
+                float2 v = *cp;
+                v.x -= acc[i][j][2 * h];
+                v.y -= acc[i][j][2 * h + 1];
+                *cp = v;
+            }
+        }
 }
 
 // Xt (K x Tp, BF16) = X^T with the rows past T zero-filled.  32 x 32 tiles.
@@ -838,10 +883,11 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     uint8_t *dead = ws + L.dead;
     double *mean = reinterpret_cast<double *>(ws + L.mean);
 
-    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false};
+    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false}, attr_sg[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
+    if (!set_smem_once(k_sgemm_sub, kSgSmem, attr_sg[dev & 63]) ||
+        !set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
         !set_smem_once(k_dgemm<false>, kGemmSmem, attr_g0[dev & 63]) ||
         !set_smem_once(k_dgemm<true>, kGemmSmem, attr_g1[dev & 63]))
         return HIF4_ERR_CUDA;
@@ -896,7 +942,7 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
                                  : launch_gptq_block<4>(a, s);
         if (st != HIF4_OK) return st;
         if (b1 < K) {
-            k_sgemm_sub<<<dim3((unsigned)((K - b1 + 127) / 128), (unsigned)((N + 127) / 128)), 256, 0, s>>>(
+            k_sgemm_sub<<<dim3((unsigned)((K - b1 + SGN - 1) / SGN), (unsigned)((N + SGM - 1) / SGM)), 256, kSgSmem, s>>>(
                 W + b1, K, Err, 64 * NG, U + b0 * K + b1, K, N, K - b1, 64 * NG);
             if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
         }
