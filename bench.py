@@ -467,15 +467,26 @@ def main():
         gws = torch.empty(H.lib().hif4_higptq1_workspace(F, D, 128), dtype=torch.uint8, device=dev)
         r = time_op(lambda: H.higptq1(w1g, Hg, idx1, 0.01, 128, workspace=gws), args, stream, barrier,
                     max_over_ranks, world, 0.0, P)
-        fp32_peak = 148 * 128 * 2 * P["sm_max_mhz"] * 1e6 / 1e12
-        flop = float(F) * D * D                       # FP32 error-feedback updates: 2 x N K^2 / 2
+        # Composite roofline of the call: the FP32 error-feedback updates
+        # (N K^2 FLOP) at the split-TF32 tensor rate (three TF32 products per
+        # FP32 product) plus the FP64 factor (2 K^3 / 3 FLOP) at the FP64
+        # peak.  TF32 peak = the bf16 peak x the nominal 1.1 / 2.25 ratio.
+        fp64_peak = 148 * 64 * 2 * P["sm_max_mhz"] * 1e6 / 1e12
+        tf32x3_peak = P["bf16_tflops"] * (1.1 / 2.25) / 3.0
+        upd_flop, fac_flop = float(F) * D * D, 2.0 * float(D) ** 3 / 3.0
+        t_min_ms = (upd_flop / (tf32x3_peak * 1e12) + fac_flop / (fp64_peak * 1e12)) * 1e3
+        flop = upd_flop + fac_flop
         tf = world * flop / (r["ms"] * 1e-3) / 1e12
-        comps["higptq1"] = {"value": tf, "unit": "TFLOP/s", "ms": r["ms"], "bound": "alu", "peak": fp32_peak,
-                            "frac": tf / world / fp32_peak,
-                            "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x %.0f MHz" % P["sm_max_mhz"],
+        comp_peak = flop / (t_min_ms * 1e-3) / 1e12
+        comps["higptq1"] = {"value": tf, "unit": "TFLOP/s", "ms": r["ms"], "bound": "tensor (FP64 + split TF32)",
+                            "peak": comp_peak, "frac": tf / world / comp_peak, "roofline_ms": t_min_ms,
+                            "peak_source": "composite: N K^2 at %.0f TFLOP/s (TF32 = %s bf16 burst x 1.1/2.25, "
+                                           "/3 for the split products) + 2 K^3/3 at %.1f TFLOP/s FP64 (derived: "
+                                           "148 SMs x 64 FP64 lanes x 2 x %.0f MHz)"
+                                           % (tf32x3_peak, P["source"], fp64_peak, P["sm_max_mhz"]),
                             "workload": "HiGPTQ scheme one, W1 %d x %d (Wan2.2 FFN), Hessian of %d x %d "
                                         "activations, block 128, 1%% protected; FLOPs counted: the FP32 "
-                                        "error-feedback updates (N K^2), the FP64 factor (2 K^3 / 3) on top"
+                                        "error-feedback updates (N K^2) plus the FP64 factor (2 K^3 / 3)"
                                         % (F, D, M, D)}
         del w1g, Hg, gws
         torch.cuda.empty_cache()

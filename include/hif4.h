@@ -341,7 +341,9 @@ hif4_status hif4_hessian(const void *x, int64_t T, int64_t K, int64_t ldx, float
  *         them, protected columns coded 0), ready for hif4_linear_w4a4;
  * w_masked  out: BF16 N x n_masked, the protected columns' final values.
  * workspace >= hif4_higptq1_workspace(N, K, blocksize), 256-byte aligned.
- * The factor runs in FP64, the group loop in FP32.  Device flags: NOT_SPD
+ * The factor runs in FP64, the group loop in FP32 (its lazy update on the
+ * TF32 tensor cores with each operand split in two TF32 parts: three
+ * products per FP32 product, FP32 accumulation).  Device flags: NOT_SPD
  * (Hd not positive definite), BAD_INDEX, NONFINITE (non-finite weights,
  * mapped as hif4_quantize maps them).  Errors: SHAPE (K % 64, ldw < K),
  * UNSUPPORTED (K > 32768), ALIGNMENT, WORKSPACE, INVALID_ARG.
