@@ -132,6 +132,24 @@ __device__ __forceinline__ void warp_inv32(const double (&a)[HB], double (&x)[HB
     }
 }
 
+// One warp: the 32 x 32 lower block S (shared memory) -> its factor in S (0
+// above the diagonal) and the factor's inverse in X.  Not inlined: the leaf
+// calls it twice and its unrolled body is large, so one copy of the code
+// halves what the leaf fetches.
+__device__ __noinline__ void warp_factor_half(double (*S)[HP], double (*X)[HP], int &bad)
+{
+    const int lane = threadIdx.x & 31;
+    double a[HB], x[HB];
+#pragma unroll
+    for (int c = 0; c < HB; ++c) a[c] = S[lane][c];
+    warp_chol32(a, bad);
+#pragma unroll
+    for (int c = 0; c < HB; ++c) S[lane][c] = c <= lane ? a[c] : 0.0;
+    warp_inv32(a, x);
+#pragma unroll
+    for (int r = 0; r < HB; ++r) X[r][lane] = x[r];
+}
+
 // One 64 x 64 diagonal block: its Cholesky factor (lower, in place in A)
 // and the factor's inverse into Y (zeros above the diagonal), as two halves:
 // warp 0 factors and inverts the 32 x 32 diagonal blocks in registers, all
@@ -167,17 +185,7 @@ __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y,
     // each thread's four outputs of a 32 x 32 product: rows ro + 8 i, column lane
     const int ro = warp;
     int bad = 0;
-    if (warp == 0) {
-        double a[HB], x[HB];
-#pragma unroll
-        for (int c = 0; c < HB; ++c) a[c] = A11[lane][c];
-        warp_chol32(a, bad);
-#pragma unroll
-        for (int c = 0; c < HB; ++c) A11[lane][c] = c <= lane ? a[c] : 0.0;
-        warp_inv32(a, x);
-#pragma unroll
-        for (int r = 0; r < HB; ++r) X11[r][lane] = x[r];
-    }
+    if (warp == 0) warp_factor_half(A11, X11, bad);
     __syncthreads();
     // L21 = A21 X11^T   (X11 lower: k <= c)
 #pragma unroll
@@ -209,15 +217,7 @@ __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y,
     }
     __syncthreads();
     if (warp == 0) {
-        double a[HB], x[HB];
-#pragma unroll
-        for (int c = 0; c < HB; ++c) a[c] = A22[lane][c];
-        warp_chol32(a, bad);
-#pragma unroll
-        for (int c = 0; c < HB; ++c) A22[lane][c] = c <= lane ? a[c] : 0.0;
-        warp_inv32(a, x);
-#pragma unroll
-        for (int r = 0; r < HB; ++r) X22[r][lane] = x[r];
+        warp_factor_half(A22, X22, bad);
         if (bad) atomicOr(&bad_all, 1);
     }
     __syncthreads();
