@@ -570,15 +570,17 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
 // TF32) and the product taken as lo hi + hi lo + hi hi: the dropped lo lo
 // term and the TF32 rounding of lo leave an error of the order of FP32
 // rounding.  64 x 128 tiles, 8 warps of 32 x 32 (2 x 4 MMA tiles); the K
-// loop in 32-deep stages that cp.async copies double-buffer into shared
-// memory (rows past M and columns past Nc are zero-filled and not stored).
-// Kd is a multiple of 32, Nc of 4; lda, ldb, ldc multiples of 4 floats and
-// A, B, C 16-byte aligned.
-constexpr int SGM = 64, SGN = 128, SGK = 32;
+// loop in 32-deep stages that cp.async copies triple-buffer into shared
+// memory, and the C tile itself is fetched into shared memory first, so
+// that its read-modify-write waits on nothing at the end (rows past M and
+// columns past Nc are zero-filled and not stored).  Kd is a multiple of 32,
+// Nc of 4; lda, ldb, ldc multiples of 4 floats and A, B, C 16-byte aligned.
+constexpr int SGM = 64, SGN = 128, SGK = 32, SGST = 3;
 constexpr int SAS = SGK + 4;              // smem row of the A stage (floats): conflict-free fragment loads
 constexpr int SBS = SGN + 8;              // smem row of the B stage
+constexpr int SCS = SGN + 4;              // smem row of the C tile
 constexpr int kSgStage = SGM * SAS + SGK * SBS;
-constexpr size_t kSgSmem = sizeof(float) * 2 * kSgStage;
+constexpr size_t kSgSmem = sizeof(float) * (SGST * kSgStage + SGM * SCS);
 
 __device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid)
 {
@@ -632,28 +634,39 @@ __global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, con
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    float acc[2][4][4] = {};
+    // the C tile (64 x 128: 8 chunks per thread) first, in its own group
+    float *Cs = sgs + SGST * kSgStage;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int idx = tid + 256 * q, r = idx >> 5, ch = idx & 31;
+        const bool ok = m0 + r < M && n0 + 4 * ch < Nc;
+        cp_async16_zfill(Cs + r * SCS + 4 * ch, ok ? C + (m0 + r) * ldc + n0 + 4 * ch : C, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const int nk = Kd / SGK;
     issue(0, 0);
-    int st = 0;
-    for (int k = 0; k < Kd; k += SGK, st ^= 1) {
-        if (k + SGK < Kd) {
-            issue(k + SGK, st ^ 1);
+    if (nk > 1) issue(SGK, 1);
+    float acc[2][4][4] = {};
+    for (int i = 0; i < nk; ++i) {
+        // stage i has landed once at most the one group issued after it is pending
+        if (i + 1 < nk)
             asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
+        else
             asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
         __syncthreads();
-        const float *As = sgs + st * kSgStage, *Bs = As + SGM * SAS;
+        // every thread is past stage i - 1, whose buffer now takes stage i + 2
+        if (i + 2 < nk) issue((i + 2) * SGK, (i + 2) % SGST);
+        const float *As = sgs + (i % SGST) * kSgStage, *Bs = As + SGM * SAS;
 #pragma unroll
         for (int kk = 0; kk < SGK; kk += 8) {
             uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const float *ar = As + (wm + 16 * i + g) * SAS + kk + t;
-                split_tf32(ar[0], ah[i][0], al[i][0]);
-                split_tf32(ar[8 * SAS], ah[i][1], al[i][1]);
-                split_tf32(ar[4], ah[i][2], al[i][2]);
-                split_tf32(ar[8 * SAS + 4], ah[i][3], al[i][3]);
+            for (int ii = 0; ii < 2; ++ii) {
+                const float *ar = As + (wm + 16 * ii + g) * SAS + kk + t;
+                split_tf32(ar[0], ah[ii][0], al[ii][0]);
+                split_tf32(ar[8 * SAS], ah[ii][1], al[ii][1]);
+                split_tf32(ar[4], ah[ii][2], al[ii][2]);
+                split_tf32(ar[8 * SAS + 4], ah[ii][3], al[ii][3]);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -662,31 +675,31 @@ __global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, con
                 split_tf32(bc[4 * SBS], bh[j][1], bl[j][1]);
             }
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    mma_tf32(acc[i][j], al[i], bh[j]);
-                    mma_tf32(acc[i][j], ah[i], bl[j]);
-                    mma_tf32(acc[i][j], ah[i], bh[j]);
+                    mma_tf32(acc[ii][j], al[ii], bh[j]);
+                    mma_tf32(acc[ii][j], ah[ii], bl[j]);
+                    mma_tf32(acc[ii][j], ah[ii], bh[j]);
                 }
         }
-        __syncthreads();                                             // stage st is refilled two steps on
     }
+    // C tile: landed with the first group; each thread reads back only what it owns
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int64_t c = n0 + wn + 8 * j + 2 * t;
+            const int cl = wn + 8 * j + 2 * t;
+            const int64_t c = n0 + cl;
             if (c >= Nc) continue;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int64_t r = m0 + wm + 16 * i + g + 8 * h;
+                const int rl = wm + 16 * ii + g + 8 * h;
+                const int64_t r = m0 + rl;
                 if (r >= M) continue;
-                float2 *cp = reinterpret_cast<float2 *>(C + r * ldc + c);
-                float2 v = *cp;
-                v.x -= acc[i][j][2 * h];
-                v.y -= acc[i][j][2 * h + 1];
-                *cp = v;
+                const float2 cv = *reinterpret_cast<const float2 *>(Cs + rl * SCS + cl);
+                *reinterpret_cast<float2 *>(C + r * ldc + c) =
+                    make_float2(cv.x - acc[ii][j][2 * h], cv.y - acc[ii][j][2 * h + 1]);
             }
         }
 }
