@@ -26,11 +26,17 @@
 // FP32 product, FP32 accumulation).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
 #include "hif4_sm100.cuh"
 
 namespace hif4 {
+
+bool make_tensor_map_f32_2d_sw128(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
 namespace {
 
 constexpr int TB = 64;            // factorization tile
@@ -564,31 +570,7 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
     }
 }
 
-// C (M x Nc, ldc) -= A (M x Kd, lda) B (Kd x Nc, ldb), FP32 operands and
-// accumulation, on the TF32 tensor-core MMA (m16n8k8) with each operand
-// split as x = hi + lo (hi = x rounded to TF32, lo = the rest rounded to
-// TF32) and the product taken as lo hi + hi lo + hi hi: the dropped lo lo
-// term and the TF32 rounding of lo leave an error of the order of FP32
-// rounding.  64 x 128 tiles, 8 warps of 32 x 32 (2 x 4 MMA tiles); the K
-// loop in 32-deep stages that cp.async copies triple-buffer into shared
-// memory, and the C tile itself is fetched into shared memory first, so
-// that its read-modify-write waits on nothing at the end (rows past M and
-// columns past Nc are zero-filled and not stored).  Kd is a multiple of 32,
-// Nc of 4; lda, ldb, ldc multiples of 4 floats and A, B, C 16-byte aligned.
-constexpr int SGM = 64, SGN = 128, SGK = 32, SGST = 3;
-constexpr int SAS = SGK + 4;              // smem row of the A stage (floats): conflict-free fragment loads
-constexpr int SBS = SGN + 8;              // smem row of the B stage
-constexpr int SCS = SGN + 4;              // smem row of the C tile
-constexpr int kSgStage = SGM * SAS + SGK * SBS;
-constexpr size_t kSgSmem = sizeof(float) * (SGST * kSgStage + SGM * SCS);
-
-__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_addr(smem_dst)), "l"(gmem_src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
-}
-
+// FP32 -> TF32 (round to nearest, ties away): the low 13 mantissa bits cleared.
 __device__ __forceinline__ uint32_t tf32_rna(float x)
 {
     uint32_t r;
@@ -596,112 +578,242 @@ __device__ __forceinline__ uint32_t tf32_rna(float x)
     return r;
 }
 
-__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+// The lazy update C (M x Nc, ldc) -= E B after each block, on the tcgen05
+// tensor cores, kind::tf32, as a persistent kernel: one CTA per SM walks
+// 128 x 128 tiles of C, each accumulated in
+// FP32 in one of two 128-column TMEM accumulators, so that the epilogue of a
+// tile (C -= accumulator, read-modify-write in global memory) overlaps the
+// loads and MMAs of the next.  Both operands come pre-split (x = hi + lo,
+// hi = x rounded to TF32, lo = the rest rounded to TF32; A = the block's
+// error E as E_hi, E_lo, N x Kd; B = U^T as U^T_hi, U^T_lo, K x K, so that a
+// 128-column tile of C reads 128 K-major rows) and each 8-deep k-step issues
+// lo hi + hi lo + hi hi (the dropped lo lo term and the TF32 rounding of lo
+// leave an error of the order of FP32 rounding).  A 3-stage ring of four 128 x 32 FP32 tiles (64 KB
+// each, 128-byte swizzle) is filled by TMA.  Warp 0: TMA producer; warp 1:
+// TMEM allocation and the single MMA-issuing thread; warps 2-5: epilogue,
+// thread = row.  Every wait is bounded; a time-out sets the abort flag, lets
+// the copies in flight land, and reports HIF4_FLAG_TIMEOUT.
+constexpr int UBM = 128, UBN = 128, UBK = 32, USTG = 3;
+constexpr uint32_t kUTile = UBM * UBK * 4;                // one 128 x 32 FP32 tile: 16 KB
+constexpr uint32_t kUStage = 4 * kUTile;                  // E_hi, E_lo, U^T_hi, U^T_lo
+constexpr size_t kUSmem = USTG * kUStage + 1024 + 256;
+constexpr int kUThreads = 192;
+constexpr uint32_t kUTmemCols = 2 * UBN;
+constexpr uint64_t kUWaitNs = 2000000000ull;
+
+struct UpdArgs {
+    float *W;                // C = W[:, b1:], row-major, ld ldw
+    int64_t ldw, M, Nc;      // rows of W; columns after the block (a multiple of 64)
+    int b0, b1, nkb;         // the block [b0, b1) of K; 32-deep k-blocks
+    int num_m, num_tiles;    // 128-row tiles of W; all tiles
+    uint32_t *status;
+};
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (FP32 in smem read as TF32, FP32 accumulate).
+__device__ __forceinline__ void mma_tf32_tc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate)
 {
-    hi = tf32_rna(x);
-    lo = tf32_rna(x - __uint_as_float(hi));
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
-// d (16 x 8: rows g, g + 8, columns 2 t + {0, 1}) += a (16 x 8) b (8 x 8), TF32 in, FP32 out
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+// Instruction descriptor, kind::tf32: D = F32 (bits 4-5 = 1), A = B = TF32
+// (2 in bits 7-9 and 10-12), both K-major, N >> 3 in bits 17-22, M >> 4 in
+// bits 24-28.
+constexpr uint32_t idesc_tf32_f32(uint32_t M, uint32_t N)
 {
-    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                 "{%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(256, 2) k_sgemm_sub(float *C, int64_t ldc, const float *A, int64_t lda,
-                                                   const float *B, int64_t ldb, int64_t M, int64_t Nc, int Kd)
+__global__ void __launch_bounds__(kUThreads, 1)
+k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
+              const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmBl, UpdArgs g)
 {
-    extern __shared__ __align__(16) float sgs[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
-    const int wm = 32 * (warp >> 2), wn = 32 * (warp & 3);
-    const int64_t m0 = (int64_t)blockIdx.y * SGM, n0 = (int64_t)blockIdx.x * SGN;
-    auto issue = [&](int k, int st) {
-        float *As = sgs + st * kSgStage, *Bs = As + SGM * SAS;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {                                // A: 64 rows x 8 chunks
-            const int idx = tid + 256 * q, r = idx >> 3, ch = idx & 7;
-            const bool ok = m0 + r < M;
-            cp_async16_zfill(As + r * SAS + 4 * ch, ok ? A + (m0 + r) * lda + k + 4 * ch : A, ok);
+    using namespace sm100;
+    extern __shared__ uint8_t usm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(usm_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + USTG * kUStage);
+    uint64_t *full = bars, *empty = bars + USTG, *tfull = bars + 2 * USTG, *tempty = tfull + 2, *drain = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *abort_flag = tmem_holder + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < USTG; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {                                // B: 32 rows x 32 chunks
-            const int idx = tid + 256 * q, r = idx >> 5, ch = idx & 31;
-            const bool ok = n0 + 4 * ch < Nc;
-            cp_async16_zfill(Bs + r * SBS + 4 * ch, ok ? B + (int64_t)(k + r) * ldb + n0 + 4 * ch : B, ok);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    // the C tile (64 x 128: 8 chunks per thread) first, in its own group
-    float *Cs = sgs + SGST * kSgStage;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const int idx = tid + 256 * q, r = idx >> 5, ch = idx & 31;
-        const bool ok = m0 + r < M && n0 + 4 * ch < Nc;
-        cp_async16_zfill(Cs + r * SCS + 4 * ch, ok ? C + (m0 + r) * ldc + n0 + 4 * ch : C, ok);
+        mbar_init(drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    const int nk = Kd / SGK;
-    issue(0, 0);
-    if (nk > 1) issue(SGK, 1);
-    float acc[2][4][4] = {};
-    for (int i = 0; i < nk; ++i) {
-        // stage i has landed once at most the one group issued after it is pending
-        if (i + 1 < nk)
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();
-        // every thread is past stage i - 1, whose buffer now takes stage i + 2
-        if (i + 2 < nk) issue((i + 2) * SGK, (i + 2) % SGST);
-        const float *As = sgs + (i % SGST) * kSgStage, *Bs = As + SGM * SAS;
-#pragma unroll
-        for (int kk = 0; kk < SGK; kk += 8) {
-            uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
-#pragma unroll
-            for (int ii = 0; ii < 2; ++ii) {
-                const float *ar = As + (wm + 16 * ii + g) * SAS + kk + t;
-                split_tf32(ar[0], ah[ii][0], al[ii][0]);
-                split_tf32(ar[8 * SAS], ah[ii][1], al[ii][1]);
-                split_tf32(ar[4], ah[ii][2], al[ii][2]);
-                split_tf32(ar[8 * SAS + 4], ah[ii][3], al[ii][3]);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float *bc = Bs + (kk + t) * SBS + wn + 8 * j + g;
-                split_tf32(bc[0], bh[j][0], bl[j][0]);
-                split_tf32(bc[4 * SBS], bh[j][1], bl[j][1]);
-            }
-#pragma unroll
-            for (int ii = 0; ii < 2; ++ii)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    mma_tf32(acc[ii][j], al[ii], bh[j]);
-                    mma_tf32(acc[ii][j], ah[ii], bl[j]);
-                    mma_tf32(acc[ii][j], ah[ii], bh[j]);
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmAh);
+        prefetch_tensormap(&tmAl);
+        prefetch_tensormap(&tmBh);
+        prefetch_tensormap(&tmBl);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, kUTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- producer
+            uint32_t stage = 0, phase = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
+                const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * UBN;
+                for (int kb = 0; kb < g.nkb; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kUWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = sm + stage * kUStage;
+                    mbar_arrive_expect_tx(&full[stage], kUStage);
+                    tma_load_2d(st, &tmAh, kb * UBK, m0, &full[stage]);
+                    tma_load_2d(st + kUTile, &tmAl, kb * UBK, m0, &full[stage]);
+                    tma_load_2d(st + 2 * kUTile, &tmBh, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
+                    tma_load_2d(st + 3 * kUTile, &tmBl, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
+                    ++issued;
+                    if (++stage == USTG) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
-        }
-    }
-    // C tile: landed with the first group; each thread reads back only what it owns
-#pragma unroll
-    for (int ii = 0; ii < 2; ++ii)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int cl = wn + 8 * j + 2 * t;
-            const int64_t c = n0 + cl;
-            if (c >= Nc) continue;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int rl = wm + 16 * ii + g + 8 * h;
-                const int64_t r = m0 + rl;
-                if (r >= M) continue;
-                const float2 cv = *reinterpret_cast<const float2 *>(Cs + rl * SCS + cl);
-                *reinterpret_cast<float2 *>(C + r * ldc + c) =
-                    make_float2(cv.x - acc[ii][j][2 * h], cv.y - acc[ii][j][2 * h + 1]);
+            }
+            if (!ok) {
+                // let our own copies land: the most recent phase of every stage loaded
+                for (uint32_t i = 0; i < USTG && i < issued; ++i) {
+                    const uint32_t st = (stage + USTG - 1 - i) % USTG;
+                    const uint32_t ph = (st < stage) ? phase : (phase ^ 1u);
+                    mbar_wait_bounded(&full[st], ph, nullptr, 100000000ull);
+                }
             }
         }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------- MMA issuer
+            const uint32_t idesc = idesc_tf32_f32(UBM, UBN);
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
+                if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kUWaitNs)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + acc * UBN;
+                for (int kb = 0; kb < g.nkb; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kUWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ah = smem_addr(sm + stage * kUStage), al = ah + kUTile, bh = ah + 2 * kUTile,
+                                   bl = ah + 3 * kUTile;
+#pragma unroll
+                    for (int k = 0; k < UBK / 8; ++k) {                // 8 TF32 = 32 bytes per step
+                        mma_tf32_tc(d, smem_desc_sw128(al + 32 * k), smem_desc_sw128(bh + 32 * k), idesc,
+                                    (kb | k) != 0);
+                        mma_tf32_tc(d, smem_desc_sw128(ah + 32 * k), smem_desc_sw128(bl + 32 * k), idesc, 1u);
+                        mma_tf32_tc(d, smem_desc_sw128(ah + 32 * k), smem_desc_sw128(bh + 32 * k), idesc, 1u);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == USTG) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                acc ^= 1u;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            // no MMA may still be running when TMEM is released
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0, nullptr, 100000000ull);
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int q = warp & 3;                                        // TMEM lane quarter of this warp
+        uint32_t acc = 0, acc_phase = 0;
+        for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
+            const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * UBN;
+            if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kUWaitNs)) break;
+            tc_fence_after();
+            const int64_t row = (int64_t)m0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < UBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * UBN + 32 * c, r);
+                tmem_ld_wait();
+                const int64_t col = (int64_t)n0 + 32 * c;              // 32 columns: all inside Nc or all past it
+                if (row < g.M && col < g.Nc) {
+                    float4 *p = reinterpret_cast<float4 *>(g.W + row * g.ldw + g.b1 + col);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        float4 w = p[v];
+                        w.x -= __uint_as_float(r[4 * v]);
+                        w.y -= __uint_as_float(r[4 * v + 1]);
+                        w.z -= __uint_as_float(r[4 * v + 2]);
+                        w.w -= __uint_as_float(r[4 * v + 3]);
+                        p[v] = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            acc ^= 1u;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kUTmemCols);
+    if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
+}
+
+// hi / lo TF32 parts of n floats.
+__global__ void k_split_tf32(const float *x, int64_t n, float *hi, float *lo)
+{
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = x[i];
+        const uint32_t h = tf32_rna(v);
+        hi[i] = __uint_as_float(h);
+        lo[i] = __uint_as_float(tf32_rna(v - __uint_as_float(h)));
+    }
+}
+
+// U^T split into TF32 parts (K x K, K a multiple of 32), 32 x 32 tiles through
+// shared memory so that both the reads of U and the writes of U^T coalesce.
+__global__ void k_ut_split(const float *U, int64_t K, float *UTh, float *UTl)
+{
+    __shared__ float t[32][33];
+    const int64_t i0 = blockIdx.y * 32ll, j0 = blockIdx.x * 32ll;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) t[threadIdx.y + 8 * q][threadIdx.x] = U[(i0 + threadIdx.y + 8 * q) * K + j0 + threadIdx.x];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float v = t[threadIdx.x][threadIdx.y + 8 * q];
+        const uint32_t h = tf32_rna(v);
+        const int64_t o = (j0 + threadIdx.y + 8 * q) * K + i0 + threadIdx.x;
+        UTh[o] = __uint_as_float(h);
+        UTl[o] = __uint_as_float(tf32_rna(v - __uint_as_float(h)));
+    }
 }
 
 // Xt (K x Tp, BF16) = X^T with the rows past T zero-filled.  32 x 32 tiles.
@@ -732,7 +844,7 @@ size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace sections of hif4_higptq1.
 struct GptqLayout {
-    size_t A, Y, T, U, UinvG, W, Err, mask, rank, dead, mean, total;
+    size_t A, Y, T, U, UinvG, UTh, UTl, W, Err, Eh, El, mask, rank, dead, mean, total;
 };
 
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
@@ -750,8 +862,12 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     take(L.T, (nb - nb / 2) * (nb / 2 > 0 ? nb / 2 : 1) * TB * TB * 8);
     take(L.U, k * k * 4);
     take(L.UinvG, nb * TB * TB * 4);
+    take(L.UTh, k * k * 4);
+    take(L.UTl, k * k * 4);
     take(L.W, (size_t)N * k * 4);
     take(L.Err, (size_t)N * (size_t)B * 4);
+    take(L.Eh, (size_t)N * (size_t)B * 4);
+    take(L.El, (size_t)N * (size_t)B * 4);
     take(L.mask, k);
     take(L.rank, k * 4);
     take(L.dead, k);
@@ -891,15 +1007,20 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     float *UinvG = reinterpret_cast<float *>(ws + L.UinvG);
     float *W = reinterpret_cast<float *>(ws + L.W);
     float *Err = reinterpret_cast<float *>(ws + L.Err);
+    float *UTh = reinterpret_cast<float *>(ws + L.UTh);
+    float *UTl = reinterpret_cast<float *>(ws + L.UTl);
+    float *Eh = reinterpret_cast<float *>(ws + L.Eh);
+    float *El = reinterpret_cast<float *>(ws + L.El);
     uint8_t *mask = ws + L.mask;
     int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
     uint8_t *dead = ws + L.dead;
     double *mean = reinterpret_cast<double *>(ws + L.mean);
 
-    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false}, attr_sg[64] = {false};
+    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!set_smem_once(k_sgemm_sub, kSgSmem, attr_sg[dev & 63]) ||
+    static bool attr_up[64] = {false};
+    if (!set_smem_once(k_update_tf32, kUSmem, attr_up[dev & 63]) ||
         !set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
         !set_smem_once(k_dgemm<false>, kGemmSmem, attr_g0[dev & 63]) ||
         !set_smem_once(k_dgemm<true>, kGemmSmem, attr_g1[dev & 63]))
@@ -930,6 +1051,13 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     if (fst != HIF4_OK) return fst;
     k_build_u<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    // U^T in TF32 parts: the K-major B operand of the lazy update
+    k_ut_split<<<dim3((unsigned)(K / 32), (unsigned)(K / 32)), dim3(32, 8), 0, s>>>(U, K, UTh, UTl);
+    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    CUtensorMap mBh, mBl;
+    if (!make_tensor_map_f32_2d_sw128(&mBh, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN) ||
+        !make_tensor_map_f32_2d_sw128(&mBl, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN))
+        return HIF4_ERR_CUDA;
     // 3. the group loop: per block, the groups with their in-block feedback,
     //    then the lazy update of every later column
     for (int64_t b0 = 0; b0 < K; b0 += B) {
@@ -955,8 +1083,18 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
                                  : launch_gptq_block<4>(a, s);
         if (st != HIF4_OK) return st;
         if (b1 < K) {
-            k_sgemm_sub<<<dim3((unsigned)((K - b1 + SGN - 1) / SGN), (unsigned)((N + SGM - 1) / SGM)), 256, kSgSmem, s>>>(
-                W + b1, K, Err, 64 * NG, U + b0 * K + b1, K, N, K - b1, 64 * NG);
+            const int64_t kd = 64 * NG, ne = N * kd;
+            k_split_tf32<<<(unsigned)std::min<int64_t>((ne + 255) / 256, 8 * (int64_t)sm_count()), 256, 0, s>>>(
+                Err, ne, Eh, El);
+            if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+            CUtensorMap mAh, mAl;
+            if (!make_tensor_map_f32_2d_sw128(&mAh, Eh, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM) ||
+                !make_tensor_map_f32_2d_sw128(&mAl, El, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM))
+                return HIF4_ERR_CUDA;
+            const int num_m = (int)((N + UBM - 1) / UBM), num_n = (int)((K - b1 + UBN - 1) / UBN);
+            UpdArgs ua{W, K, N, K - b1, (int)b0, (int)b1, (int)(kd / UBK), num_m, num_m * num_n, status};
+            const int grid = std::min(num_m * num_n, sm_count());
+            k_update_tf32<<<grid, kUThreads, kUSmem, s>>>(mAh, mAl, mBh, mBl, ua);
             if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
         }
     }
