@@ -474,16 +474,21 @@ def main():
         fp64_peak = 148 * 64 * 2 * P["sm_max_mhz"] * 1e6 / 1e12
         tf32x3_peak = P["bf16_tflops"] * (1.1 / 2.25) / 3.0
         upd_flop, fac_flop = float(F) * D * D, 2.0 * float(D) ** 3 / 3.0
-        t_min_ms = (upd_flop / (tf32x3_peak * 1e12) + fac_flop / (fp64_peak * 1e12)) * 1e3
+        # the updates also read and write W's remaining columns once per block
+        upd_bytes = 8.0 * F * sum(D - b1 for b1 in range(128, D, 128))
+        t_upd_ms = max(upd_flop / (tf32x3_peak * 1e12), upd_bytes / (P["hbm_gbs"] * 1e9)) * 1e3
+        t_min_ms = t_upd_ms + fac_flop / (fp64_peak * 1e12) * 1e3
         flop = upd_flop + fac_flop
         tf = world * flop / (r["ms"] * 1e-3) / 1e12
         comp_peak = flop / (t_min_ms * 1e-3) / 1e12
         comps["higptq1"] = {"value": tf, "unit": "TFLOP/s", "ms": r["ms"], "bound": "tensor (FP64 + split TF32)",
                             "peak": comp_peak, "frac": tf / world / comp_peak, "roofline_ms": t_min_ms,
-                            "peak_source": "composite: N K^2 at %.0f TFLOP/s (TF32 = %s bf16 burst x 1.1/2.25, "
-                                           "/3 for the split products) + 2 K^3/3 at %.1f TFLOP/s FP64 (derived: "
-                                           "148 SMs x 64 FP64 lanes x 2 x %.0f MHz)"
-                                           % (tf32x3_peak, P["source"], fp64_peak, P["sm_max_mhz"]),
+                            "peak_source": "composite: the updates at max(N K^2 at %.0f TFLOP/s (TF32 = %s bf16 "
+                                           "burst x 1.1/2.25, /3 for the split products), %.2f GB of W read and "
+                                           "written at %.0f GB/s) + 2 K^3/3 at %.1f TFLOP/s FP64 (derived: 148 SMs "
+                                           "x 64 FP64 lanes x 2 x %.0f MHz)"
+                                           % (tf32x3_peak, P["source"], upd_bytes / 1e9, P["hbm_gbs"], fp64_peak,
+                                              P["sm_max_mhz"]),
                             "workload": "HiGPTQ scheme one, W1 %d x %d (Wan2.2 FFN), Hessian of %d x %d "
                                         "activations, block 128, 1%% protected; FLOPs counted: the FP32 "
                                         "error-feedback updates (N K^2) plus the FP64 factor (2 K^3 / 3)"
