@@ -142,6 +142,23 @@ def test_dead_channel_and_non_positive_definite(H):
     assert H.get_status(status) == 1                            # HIF4_ERR_INVALID_ARG (NOT_SPD)
 
 
+def test_many_tiles_ragged_rows(H):
+    """N = 3000 rows (not a multiple of the update's 128-row tiles) and K =
+    1024: each lazy update has 24 x up to 7 tiles, more than there are SMs,
+    so every persistent update CTA walks several tiles and both TMEM
+    accumulators; 128 sampled rows against the oracle."""
+    rng = np.random.default_rng(11)
+    N, K = 3000, 1024
+    w = _bf16(rng, (N, K), 0.02)
+    x = _factor_x(rng, 3000, K)
+    Hf = (x.T @ x).astype(np.float32)
+    idx = np.array([5, 300, 301, 1023], np.int32)
+    got = run_gpu(H, w, Hf, idx, 0.01, 128)
+    factor = oracle.gptq_factor(Hf.astype(np.float64), 0.01)
+    rows = np.unique(np.concatenate([wl.sample_rows(N, 120), [0, 2943, 2944, N - 1]]))
+    compare(w, Hf, idx, 0.01, 128, got, factor=factor, rows=rows)
+
+
 @pytest.mark.slow
 def test_wan22_w1_sampled_rows(H):
     """W1 of the Wan2.2 FFN (13824 x 5120) with the Hessian of 8192 tokens of
