@@ -41,6 +41,33 @@ namespace {
 
 constexpr int TB = 64;            // factorization tile
 
+// Programmatic dependent launch along the factor's chain of dependent
+// kernels: each waits for the previous grid (completion and memory) before
+// its first global access, then lets the next one launch, so that only the
+// launch and block set-up overlap.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_enter()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+hif4_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) return HIF4_ERR_CUDA;
+    return launch_status();
+}
+
 // ---------------------------------------------------------------- factor
 
 // dead[i] = (H_ii == 0); mean of the fixed diagonal -> *mean (one block).
@@ -165,6 +192,7 @@ __device__ __noinline__ void warp_factor_half(double (*S)[HP], double (*X)[HP], 
 // HIF4_FLAG_NOT_SPD.  256 threads.
 __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
 {
+    pdl_enter();
     extern __shared__ __align__(16) double smd[];
     double(*A11)[HP] = reinterpret_cast<double(*)[HP]>(smd);    // A11, then L11
     double(*A21)[HP] = A11 + HB;                                 // A21
@@ -312,6 +340,7 @@ __device__ __forceinline__ void dmma884(double (&d)[2], double a, double b)
 template <bool BT>
 __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
 {
+    pdl_enter();
     const int tj = blockIdx.x, ti = blockIdx.y;
     if (g.lower_c && tj > ti) return;
     extern __shared__ __align__(16) double smd[];
@@ -576,6 +605,17 @@ __device__ __forceinline__ uint32_t tf32_rna(float x)
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
     return r;
+}
+
+// dst (rows x cols, ld ldd) = src (ld lds), FP64; cols a multiple of 2.
+__global__ void k_copy2d(double *dst, int64_t ldd, const double *src, int64_t lds, int64_t rows, int64_t cols)
+{
+    pdl_enter();
+    const int64_t pairs = cols / 2, n = rows * pairs;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / pairs, c = 2 * (i - r * pairs);
+        *reinterpret_cast<double2 *>(dst + r * ldd + c) = *reinterpret_cast<const double2 *>(src + r * lds + c);
+    }
 }
 
 // The lazy update C (M x Nc, ldc) -= E B after each block, on the tcgen05
@@ -899,20 +939,14 @@ struct Factor {
     {
         Dgemm g{a, lda, b, ldb, c, ldc, (int)M, (int)N, (int)Kd, alpha, beta, tri_a, tri_b, lower_c};
         const dim3 grid((unsigned)(N / TB), (unsigned)(M / TB));
-        if (bt)
-            k_dgemm<true><<<grid, kGemmThreads, kGemmSmem, s>>>(g);
-        else
-            k_dgemm<false><<<grid, kGemmThreads, kGemmSmem, s>>>(g);
-        return launch_status();
+        return bt ? launch_pdl(k_dgemm<true>, grid, dim3(kGemmThreads), kGemmSmem, s, g)
+                  : launch_pdl(k_dgemm<false>, grid, dim3(kGemmThreads), kGemmSmem, s, g);
     }
 
     // rows [o, o + n) of the factor and of its inverse
     hif4_status run(int64_t o, int64_t n)
     {
-        if (n == TB) {
-            k_leaf<<<1, 256, kLeafSmem, s>>>(A + o * K + o, K, Y + o * K + o, K, status);
-            return launch_status();
-        }
+        if (n == TB) return launch_pdl(k_leaf, dim3(1), dim3(256), kLeafSmem, s, A + o * K + o, K, Y + o * K + o, K, status);
         const int64_t n1 = n / TB / 2 * TB, n2 = n - n1, a = o, b = o + n1;
         hif4_status st = run(a, n1);
         if (st != HIF4_OK) return st;
@@ -923,10 +957,9 @@ struct Factor {
         if ((st = gemm(false, T, n1, Y11, K, Y21, K, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
         if ((st = run(b, n2)) != HIF4_OK) return st;
         if ((st = gemm(false, Y22, K, Y21, K, T, n1, n2, n1, n2, -1.0, 0, 1, 0, 0)) != HIF4_OK) return st;
-        if (cudaMemcpy2DAsync(Y21, (size_t)K * 8, T, (size_t)n1 * 8, (size_t)n1 * 8, (size_t)n2,
-                              cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-            return HIF4_ERR_CUDA;
-        return HIF4_OK;
+        const int64_t pairs = n2 * n1 / 2;
+        const unsigned cb = (unsigned)std::min<int64_t>((pairs + 255) / 256, 4 * (int64_t)sm_count());
+        return launch_pdl(k_copy2d, dim3(cb), dim3(256), 0, s, Y21, K, (const double *)T, n1, n2, n1);
     }
 };
 
