@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "hif4_internal.cuh"
+#include "hif4_pdl.cuh"
 #include "hif4_sm100.cuh"
 
 namespace hif4 {
@@ -131,6 +132,7 @@ __device__ __forceinline__ void load4(const uint16_t *p, bool all4, int valid, u
 template <int MODE, bool V8>
 __global__ void __launch_bounds__(kThreads) k_pass(PassArgs a)
 {
+    pdl_enter();
     constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
     extern __shared__ uint32_t h[];                    // [NB][kSlab / 2]
     __shared__ uint32_t par[kSlab];                    // MODE 2: target bin; MODE 3: window start
@@ -247,6 +249,7 @@ __global__ void __launch_bounds__(kThreads) k_pass(PassArgs a)
 // Bin of the first radix histogram that holds rank k (one warp per channel).
 __global__ void k_select1(const uint32_t *hist1, int C, uint32_t k, uint16_t *tbin, const uint8_t *failed)
 {
+    pdl_enter();
     const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (c >= C) return;
     if (failed && !failed[c]) return;
@@ -341,6 +344,7 @@ __device__ __forceinline__ bool row_candidate(uint32_t w01, uint32_t w23, uint32
 template <int MODE>
 __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_constant__ CUtensorMap tm, PassArgs a)
 {
+    pdl_enter();
     using namespace sm100;
     constexpr int NB = MODE == 1 ? kBins1 : MODE == 2 ? kBins2 : kWinBins;
     extern __shared__ __align__(128) uint8_t smraw[];
@@ -489,6 +493,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
 __global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, uint32_t k, uint16_t *out,
                            const uint8_t *failed)
 {
+    pdl_enter();
     const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (c >= C) return;
     if (failed && !failed[c]) return;
@@ -504,6 +509,7 @@ __global__ void k_finalize(const uint32_t *hist1, const uint32_t *hist2, int C, 
 __global__ void k_window_final(uint32_t *whist, const uint32_t *ge, const uint16_t *lo, int C, uint64_t T, uint32_t k,
                                uint16_t *pct, uint8_t *failed, uint32_t *needed)
 {
+    pdl_enter();
     const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (c >= C) return;
@@ -568,6 +574,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratc
 __global__ void __launch_bounds__(kMaskThreads) k_mask(const uint16_t *pct, int C, uint32_t n_top, float *ratio,
                                                       uint8_t *mask, int32_t *mask_idx, const uint32_t *timed_out)
 {
+    pdl_enter();
     extern __shared__ uint32_t hist[];                 // [kKeySlots]
     if (*timed_out) {                                  // block-uniform
         for (int c = threadIdx.x; c < C; c += kMaskThreads) {
@@ -739,9 +746,10 @@ hif4_status launch_pass_tma(const PassArgs &a0, cudaStream_t s, bool &done)
     if (share < 4 * kTmaRows) share = 4 * kTmaRows;
     if (share > kMaxRowsPerBlock) share = kMaxRowsPerBlock;
     a.rows_per_split = share;
-    k<<<(int)((total + share - 1) / share), kTmaThreads, smem, s>>>(tm, a);
-    done = true;
-    return launch_status();
+    const hif4_status st = launch_pdl(k, dim3((unsigned)((total + share - 1) / share)), dim3(kTmaThreads), smem, s,
+                                      tm, a);
+    done = st == HIF4_OK;
+    return st;
 }
 
 template <int MODE>
@@ -770,9 +778,8 @@ hif4_status launch_pass(const PassArgs &a0, bool v8, bool tma, cudaStream_t s)
     const int64_t splits = splits_for(a.T, a.nslab, per_sm);
     a.rows_per_split = (a.T + splits - 1) / splits;
     const int grid = (int)(a.nslab * splits);
-    if (v8) kt<<<grid, kThreads, smem, s>>>(a);
-    else kf<<<grid, kThreads, smem, s>>>(a);
-    return launch_status();
+    return v8 ? launch_pdl(kt, dim3(grid), dim3(kThreads), smem, s, a)
+              : launch_pdl(kf, dim3(grid), dim3(kThreads), smem, s, a);
 }
 
 } // namespace
@@ -845,11 +852,13 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     // TMA needs a 16-byte aligned base and row stride (the box is 256 bytes wide)
     const bool tmas = aligned16(acts) && ((lda * R * 2) % 16 == 0);
     if ((st = launch_pass<1>(sa, v8s, tmas, s)) != HIF4_OK) return st;
-    k_select1<<<fgrid, 256, 0, s>>>(hs, (int)channels, r_lo, tbin, nullptr);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (launch_pdl(k_select1, dim3(fgrid), dim3(256), 0, s, (const uint32_t *)hs, (int)channels, r_lo, tbin,
+                   (const uint8_t *)nullptr) != HIF4_OK)
+        return HIF4_ERR_CUDA;
     if ((st = launch_pass<2>(sa, v8s, tmas, s)) != HIF4_OK) return st;
-    k_finalize<<<fgrid, 256, 0, s>>>(hs, hs2, (int)channels, r_lo, lo, nullptr);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (launch_pdl(k_finalize, dim3(fgrid), dim3(256), 0, s, (const uint32_t *)hs, (const uint32_t *)hs2,
+                   (int)channels, r_lo, lo, (const uint8_t *)nullptr) != HIF4_OK)
+        return HIF4_ERR_CUDA;
 
     // 2-3. windowed pass over every token, then the key where rank k falls
     const bool v8 = aligned_to(acts, 8) && (lda % 4 == 0);
@@ -865,9 +874,10 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.whist = whist;
     a.timed_out = timed_out;
     if ((st = launch_pass<3>(a, v8, tma, s)) != HIF4_OK) return st;
-    k_window_final<<<fgrid, 256, 0, s>>>(whist, ge, lo, (int)channels, (uint64_t)tokens, (uint32_t)kk,
-                                         static_cast<uint16_t *>(pct), failed, needed);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (launch_pdl(k_window_final, dim3(fgrid), dim3(256), 0, s, whist, (const uint32_t *)ge, (const uint16_t *)lo,
+                   (int)channels, (uint64_t)tokens, (uint32_t)kk, static_cast<uint16_t *>(pct), failed,
+                   needed) != HIF4_OK)
+        return HIF4_ERR_CUDA;
 
     // 4. exact two-pass radix select for the channels outside their window
     a.hist1 = whist;
@@ -876,11 +886,13 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
     a.tbin = tbin;
     a.needed = needed;
     if ((st = launch_pass<1>(a, v8, tma, s)) != HIF4_OK) return st;
-    k_select1<<<fgrid, 256, 0, s>>>(whist, (int)channels, (uint32_t)kk, tbin, failed);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (launch_pdl(k_select1, dim3(fgrid), dim3(256), 0, s, (const uint32_t *)whist, (int)channels, (uint32_t)kk,
+                   tbin, (const uint8_t *)failed) != HIF4_OK)
+        return HIF4_ERR_CUDA;
     if ((st = launch_pass<2>(a, v8, tma, s)) != HIF4_OK) return st;
-    k_finalize<<<fgrid, 256, 0, s>>>(whist, hist2, (int)channels, (uint32_t)kk, static_cast<uint16_t *>(pct), failed);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    if (launch_pdl(k_finalize, dim3(fgrid), dim3(256), 0, s, (const uint32_t *)whist, (const uint32_t *)hist2,
+                   (int)channels, (uint32_t)kk, static_cast<uint16_t *>(pct), (const uint8_t *)failed) != HIF4_OK)
+        return HIF4_ERR_CUDA;
 
     // 5. median over channels, ratios, top-n mask
     static bool mattr[64] = {false};
@@ -892,7 +904,7 @@ extern "C" hif4_status hif4_calib_percentile_mask(const void *acts, int64_t toke
         mattr[dev & 63] = true;
     }
     const uint32_t n_top = (uint32_t)(((uint64_t)channels * mask_num) / mask_den);
-    k_mask<<<1, kMaskThreads, kKeySlots * 4, s>>>(static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask,
-                                             mask_idx_out, timed_out);
-    return launch_status();
+    return launch_pdl(k_mask, dim3(1), dim3(kMaskThreads), (size_t)kKeySlots * 4, s,
+                      static_cast<const uint16_t *>(pct), (int)channels, n_top, ratio, mask, mask_idx_out,
+                      (const uint32_t *)timed_out);
 }

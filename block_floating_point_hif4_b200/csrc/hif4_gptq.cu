@@ -30,6 +30,7 @@
 
 #include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
+#include "hif4_pdl.cuh"
 #include "hif4_sm100.cuh"
 
 namespace hif4 {
@@ -40,33 +41,6 @@ bool make_tensor_map_f32_2d_sw128(CUtensorMap *map, const void *base, uint64_t i
 namespace {
 
 constexpr int TB = 64;            // factorization tile
-
-// Programmatic dependent launch along the factor's chain of dependent
-// kernels: each waits for the previous grid (completion and memory) before
-// its first global access, then lets the next one launch, so that only the
-// launch and block set-up overlap.  Both are no-ops for a normal launch.
-__device__ __forceinline__ void pdl_enter()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-template <typename... KArgs, typename... Args>
-hif4_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) return HIF4_ERR_CUDA;
-    return launch_status();
-}
 
 // ---------------------------------------------------------------- factor
 
