@@ -407,7 +407,9 @@ __global__ void k_build_u(const double *Y, const double *A, int64_t K, float *U,
 
 // ------------------------------------------------------------ group loop
 
-constexpr int kRowsPerBlock = 8;            // one warp per weight row
+constexpr int kWarpsPerBlock = 8;           // one warp per weight row at a time
+constexpr int kRowsPerWarp = 4;             // rows a warp takes in turn (amortizes the U tiles' load)
+constexpr int kRowsPerBlock = kWarpsPerBlock * kRowsPerWarp;
 
 // u8 mask and column -> protected rank (-1 when not protected) from the
 // sorted indices; flags bad indices.
@@ -465,18 +467,19 @@ struct GptqArgs {
     float *Err;              // N x 64 NG
 };
 
-// One block of NG groups (64 NG columns) for kRowsPerBlock rows, a warp per
+// One block of NG groups (64 NG columns) for kRowsPerBlock rows (each warp
+// takes kRowsPerWarp of them in turn, after one load of the U tiles), a warp per
 // row; lane l holds elements 2l, 2l+1 of each group.  Per group: the exact
 // FP32 unit quantization (encode rule of the streaming quantizer), D = W - Q,
 // E = D Uinv_g (Uinv_g upper), feedback into the block's later groups.
 template <int NG>
-__global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
+__global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
 {
     constexpr int NP = NG * (NG - 1) / 2;     // U tiles (g, h), g < h
     extern __shared__ float smf[];
     float *Ui = smf;                          // NG x 64 x 64
     float *Uo = Ui + NG * 4096;               // NP x 64 x 64
-    float *Dsh = Uo + NP * 4096;              // kRowsPerBlock x 64
+    float *Dsh = Uo + NP * 4096;              // kWarpsPerBlock x 64
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g0 = a.b0 / 64;
     for (int e = threadIdx.x; e < NG * 4096; e += blockDim.x) Ui[e] = a.UinvG[(g0 + e / 4096) * 4096 + e % 4096];
@@ -485,89 +488,92 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock) k_gptq_block(GptqArgs a)
             for (int e = threadIdx.x; e < 4096; e += blockDim.x)
                 Uo[p * 4096 + e] = a.U[(a.b0 + 64 * g + e / 64) * a.K + a.b0 + 64 * h + e % 64];
     __syncthreads();
-    const int64_t n = blockIdx.x * (int64_t)kRowsPerBlock + warp;
-    if (n >= a.N) return;                     // no block-wide barrier below
     float *dsh = Dsh + warp * 64;
-    float x[NG][2];
+#pragma unroll 1
+    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+        const int64_t n = blockIdx.x * (int64_t)kRowsPerBlock + rr * kWarpsPerBlock + warp;
+        if (n >= a.N) break;                      // no block-wide barrier below
+        float x[NG][2];
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const float2 v = *reinterpret_cast<const float2 *>(a.W + n * a.K + a.b0 + 64 * g + 2 * lane);
-        x[g][0] = v.x;
-        x[g][1] = v.y;
-    }
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const int64_t col = a.b0 + 64 * g + 2 * lane;
-        const bool m0 = a.mask && a.mask[col], m1 = a.mask && a.mask[col + 1];
-        const float v0 = m0 ? 0.0f : x[g][0], v1 = m1 ? 0.0f : x[g][1];
-        // level 1: unit maximum -> scale code
-        float am = fmaxf(fabsf(v0), fabsf(v1));
-        float a4 = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));       // 4-element group: lanes 2k, 2k+1
-        am = a4;
-#pragma unroll
-        for (int o = 2; o < 32; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        const uint32_t c = select_scale_code(am);
-        const float S = e6m2_value(c);
-        const uint32_t t = a4 <= 1.75f * S ? 0u : a4 <= 3.5f * S ? 1u : 2u;
-        const uint32_t tm = max(t, __shfl_xor_sync(0xffffffffu, t, 2));  // 8-element group: lanes 4j..4j+3
-        const uint32_t e2 = tm == 2u, e3 = t > e2 ? t - e2 : 0u;
-        const int E = (int)(e2 + e3);
-        const float step = ldexp_small(S, E - 2), inv = ldexp_small(__frcp_rn(S), 2 - E);
-        const uint32_t q0m = enc::round_exact(fabsf(v0), inv, step), q1m = enc::round_exact(fabsf(v1), inv, step);
-        const uint32_t s0 = q0m ? f_bits(v0) >> 31 : 0u, s1 = q1m ? f_bits(v1) >> 31 : 0u;
-        const float b0v = __bfloat162float(__float2bfloat16_rn(x[g][0]));
-        const float b1v = __bfloat162float(__float2bfloat16_rn(x[g][1]));
-        const float q0 = m0 ? b0v : bits_f(f_bits((float)q0m * step) | (s0 << 31));
-        const float q1 = m1 ? b1v : bits_f(f_bits((float)q1m * step) | (s1 << 31));
-        const uint32_t nib0 = m0 ? 0u : (q0m | (s0 << 3)), nib1 = m1 ? 0u : (q1m | (s1 << 3));
-        a.codes[n * (a.K / 2) + col / 2] = (uint8_t)(nib0 | (nib1 << 4));
-        const uint32_t b2 = __ballot_sync(0xffffffffu, e2 && (lane & 3) == 0);
-        const uint32_t b3 = __ballot_sync(0xffffffffu, e3 && (lane & 1) == 0);
-        if (lane == 0) {
-            uint32_t mw = c;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mw |= ((b2 >> (4 * j)) & 1u) << (8 + j);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) mw |= ((b3 >> (2 * k)) & 1u) << (16 + k);
-            a.meta[n * (a.K / 64) + col / 64] = mw;
+        for (int g = 0; g < NG; ++g) {
+            const float2 v = *reinterpret_cast<const float2 *>(a.W + n * a.K + a.b0 + 64 * g + 2 * lane);
+            x[g][0] = v.x;
+            x[g][1] = v.y;
         }
-        if (m0) a.w_masked[n * a.n_masked + a.rank[col]] = (uint16_t)(f_bits(b0v) >> 16);
-        if (m1) a.w_masked[n * a.n_masked + a.rank[col + 1]] = (uint16_t)(f_bits(b1v) >> 16);
-        // E = D Uinv_g
-        __syncwarp();
-        dsh[2 * lane] = x[g][0] - q0;
-        dsh[2 * lane + 1] = x[g][1] - q1;
-        __syncwarp();
-        const float *ui = Ui + g * 4096 + 2 * lane;
-        float e0 = 0.0f, e1 = 0.0f;
-        for (int i = 0; i < 64; ++i) {
-            const float d = dsh[i];
-            const float2 u = *reinterpret_cast<const float2 *>(ui + i * 64);
-            e0 = fmaf(d, u.x, e0);
-            e1 = fmaf(d, u.y, e1);
-        }
-        *reinterpret_cast<float2 *>(a.Err + n * (64 * NG) + 64 * g + 2 * lane) = make_float2(e0, e1);
-        // feedback into the later groups of the block
-        if (g + 1 < NG) {
-            __syncwarp();
-            dsh[2 * lane] = e0;
-            dsh[2 * lane + 1] = e1;
-            __syncwarp();
 #pragma unroll
-            for (int h = g + 1; h < NG; ++h) {
-                int p = 0;
-                for (int gg = 0; gg < g; ++gg) p += NG - 1 - gg;
-                p += h - g - 1;
-                const float *uo = Uo + p * 4096 + 2 * lane;
-                float d0 = 0.0f, d1 = 0.0f;
-                for (int i = 0; i < 64; ++i) {
-                    const float ei = dsh[i];
-                    const float2 u = *reinterpret_cast<const float2 *>(uo + i * 64);
-                    d0 = fmaf(ei, u.x, d0);
-                    d1 = fmaf(ei, u.y, d1);
+        for (int g = 0; g < NG; ++g) {
+            const int64_t col = a.b0 + 64 * g + 2 * lane;
+            const bool m0 = a.mask && a.mask[col], m1 = a.mask && a.mask[col + 1];
+            const float v0 = m0 ? 0.0f : x[g][0], v1 = m1 ? 0.0f : x[g][1];
+            // level 1: unit maximum -> scale code
+            float am = fmaxf(fabsf(v0), fabsf(v1));
+            float a4 = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));       // 4-element group: lanes 2k, 2k+1
+            am = a4;
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            const uint32_t c = select_scale_code(am);
+            const float S = e6m2_value(c);
+            const uint32_t t = a4 <= 1.75f * S ? 0u : a4 <= 3.5f * S ? 1u : 2u;
+            const uint32_t tm = max(t, __shfl_xor_sync(0xffffffffu, t, 2));  // 8-element group: lanes 4j..4j+3
+            const uint32_t e2 = tm == 2u, e3 = t > e2 ? t - e2 : 0u;
+            const int E = (int)(e2 + e3);
+            const float step = ldexp_small(S, E - 2), inv = ldexp_small(__frcp_rn(S), 2 - E);
+            const uint32_t q0m = enc::round_exact(fabsf(v0), inv, step), q1m = enc::round_exact(fabsf(v1), inv, step);
+            const uint32_t s0 = q0m ? f_bits(v0) >> 31 : 0u, s1 = q1m ? f_bits(v1) >> 31 : 0u;
+            const float b0v = __bfloat162float(__float2bfloat16_rn(x[g][0]));
+            const float b1v = __bfloat162float(__float2bfloat16_rn(x[g][1]));
+            const float q0 = m0 ? b0v : bits_f(f_bits((float)q0m * step) | (s0 << 31));
+            const float q1 = m1 ? b1v : bits_f(f_bits((float)q1m * step) | (s1 << 31));
+            const uint32_t nib0 = m0 ? 0u : (q0m | (s0 << 3)), nib1 = m1 ? 0u : (q1m | (s1 << 3));
+            a.codes[n * (a.K / 2) + col / 2] = (uint8_t)(nib0 | (nib1 << 4));
+            const uint32_t b2 = __ballot_sync(0xffffffffu, e2 && (lane & 3) == 0);
+            const uint32_t b3 = __ballot_sync(0xffffffffu, e3 && (lane & 1) == 0);
+            if (lane == 0) {
+                uint32_t mw = c;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mw |= ((b2 >> (4 * j)) & 1u) << (8 + j);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) mw |= ((b3 >> (2 * k)) & 1u) << (16 + k);
+                a.meta[n * (a.K / 64) + col / 64] = mw;
+            }
+            if (m0) a.w_masked[n * a.n_masked + a.rank[col]] = (uint16_t)(f_bits(b0v) >> 16);
+            if (m1) a.w_masked[n * a.n_masked + a.rank[col + 1]] = (uint16_t)(f_bits(b1v) >> 16);
+            // E = D Uinv_g
+            __syncwarp();
+            dsh[2 * lane] = x[g][0] - q0;
+            dsh[2 * lane + 1] = x[g][1] - q1;
+            __syncwarp();
+            const float *ui = Ui + g * 4096 + 2 * lane;
+            float e0 = 0.0f, e1 = 0.0f;
+            for (int i = 0; i < 64; ++i) {
+                const float d = dsh[i];
+                const float2 u = *reinterpret_cast<const float2 *>(ui + i * 64);
+                e0 = fmaf(d, u.x, e0);
+                e1 = fmaf(d, u.y, e1);
+            }
+            *reinterpret_cast<float2 *>(a.Err + n * (64 * NG) + 64 * g + 2 * lane) = make_float2(e0, e1);
+            // feedback into the later groups of the block
+            if (g + 1 < NG) {
+                __syncwarp();
+                dsh[2 * lane] = e0;
+                dsh[2 * lane + 1] = e1;
+                __syncwarp();
+#pragma unroll
+                for (int h = g + 1; h < NG; ++h) {
+                    int p = 0;
+                    for (int gg = 0; gg < g; ++gg) p += NG - 1 - gg;
+                    p += h - g - 1;
+                    const float *uo = Uo + p * 4096 + 2 * lane;
+                    float d0 = 0.0f, d1 = 0.0f;
+                    for (int i = 0; i < 64; ++i) {
+                        const float ei = dsh[i];
+                        const float2 u = *reinterpret_cast<const float2 *>(uo + i * 64);
+                        d0 = fmaf(ei, u.x, d0);
+                        d1 = fmaf(ei, u.y, d1);
+                    }
+                    x[h][0] -= d0;
+                    x[h][1] -= d1;
                 }
-                x[h][0] -= d0;
-                x[h][1] -= d1;
             }
         }
     }
@@ -941,12 +947,12 @@ template <int NG>
 hif4_status launch_gptq_block(const GptqArgs &a, cudaStream_t s)
 {
     constexpr int NP = NG * (NG - 1) / 2;
-    const size_t smem = sizeof(float) * ((NG + NP) * 4096 + kRowsPerBlock * 64);
+    const size_t smem = sizeof(float) * ((NG + NP) * 4096 + kWarpsPerBlock * 64);
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (!set_smem_once(k_gptq_block<NG>, smem, attr[dev & 63])) return HIF4_ERR_CUDA;
-    k_gptq_block<NG><<<(unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock), 32 * kRowsPerBlock, smem, s>>>(a);
+    k_gptq_block<NG><<<(unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock), 32 * kWarpsPerBlock, smem, s>>>(a);
     return launch_status();
 }
 
