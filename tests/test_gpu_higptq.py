@@ -111,7 +111,7 @@ def test_identity_hessian_is_plain_quantization(H):
     assert np.array_equal(wm, w[:, idx])
 
 
-@pytest.mark.parametrize("bs", [64, 128, 256])
+@pytest.mark.parametrize("bs", [64, 128, 192, 256])
 def test_small_layer_vs_oracle(H, bs):
     rng = np.random.default_rng(bs)
     N, K = 96, 512
