@@ -95,66 +95,81 @@ constexpr int HB = TB / 2;               // half leaf: one warp's block
 constexpr int HP = HB + 1;               // padded smem row of a half block (doubles)
 constexpr size_t kLeafSmem = sizeof(double) * 7 * HB * HP;
 
-// Cholesky of a 32 x 32 block held by one warp, lane r holding row r in
-// a[0..31] (a[c] for c <= r is read; the rest must be 0).  On return a is
-// row r of the factor.  Pivots that are not positive are replaced by 1 and
-// counted in *bad.
-__device__ __forceinline__ void warp_chol32(double (&a)[HB], int &bad)
+// Cholesky of the 32 x 32 lower block S (shared memory) by one warp, lane r
+// owning row r, in four panels of 8 columns: the row is held in a register
+// window whose position w is column 8 p + w, and after each panel the 8
+// finished columns go to S and the window shifts by 8.  One unrolled panel
+// body serves all four panels (the leaf runs once per 64 rows, so code size
+// - instruction fetch - matters more than the predicated work on the dead
+// window positions of the later panels).  On return S holds the factor, 0
+// above the diagonal.  Pivots that are not positive are replaced by 1 and
+// counted in bad.
+__device__ __forceinline__ void warp_chol32(double (*S)[HP], int &bad)
 {
     const int r = threadIdx.x & 31;
+    double a[HB];
 #pragma unroll
-    for (int j = 0; j < HB; ++j) {
-        double d = __shfl_sync(0xffffffffu, a[j], j);
-        const bool ok = d > 0.0;
-        if (!ok) d = 1.0;
-        const double rs = rsqrt(d);
-        const double l = r == j ? d * rs : a[j] * rs; // lane j: the pivot; below it: the column
-        if (r >= j) a[j] = l;
-        bad |= (int)(!ok && r == j);
+    for (int c = 0; c < HB; ++c) a[c] = c <= r ? S[r][c] : 0.0;
+#pragma unroll 1
+    for (int p = 0; p < HB; p += 8) {
 #pragma unroll
-        for (int c = j + 1; c < HB; ++c) {
-            const double lc = __shfl_sync(0xffffffffu, l, c);
-            if (r >= c) a[c] -= l * lc;
+        for (int j = 0; j < 8; ++j) {
+            const int J = p + j;                                     // column
+            double d = __shfl_sync(0xffffffffu, a[j], J);
+            const bool ok = d > 0.0;
+            if (!ok) d = 1.0;
+            const double rs = rsqrt(d);
+            const double l = r == J ? d * rs : a[j] * rs;           // lane J: the pivot; below it: the column
+            if (r >= J) a[j] = l;
+            bad |= (int)(!ok && r == J);
+#pragma unroll
+            for (int w = j + 1; w < HB; ++w) {
+                const int C = p + w;                                 // column of window position w
+                const double lc = __shfl_sync(0xffffffffu, l, C & 31);
+                if (C < HB && r >= C) a[w] -= l * lc;
+            }
         }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) S[r][p + j] = p + j <= r ? a[j] : 0.0;
+#pragma unroll
+        for (int w = 0; w < HB - 8; ++w) a[w] = a[w + 8];
     }
+    __syncwarp();
 }
 
-// Inverse of the 32 x 32 lower factor held by rows (lane r: row r in a[]),
-// returned by columns: lane c gets column c of L^{-1} in x[0..31] (0 above
-// the diagonal).  Forward substitution, row r of L broadcast from lane r.
-__device__ __forceinline__ void warp_inv32(const double (&a)[HB], double (&x)[HB])
+// Inverse of the 32 x 32 lower factor L (shared memory) into X (0 above the
+// diagonal), one warp: lane c computes column c by forward substitution,
+// L's rows read from shared memory as broadcasts.
+__device__ __forceinline__ void warp_inv32(const double (*L)[HP], double (*X)[HP])
 {
+    __shared__ double rdiag[HB];
     const int c = threadIdx.x & 31;
-    double dg = 1.0;                                 // lane c: L[c][c] (static indexing keeps a[] in registers)
-#pragma unroll
-    for (int k = 0; k < HB; ++k)
-        if (k == c) dg = a[k];
-    const double rdiag = 1.0 / dg;
+    rdiag[c] = 1.0 / L[c][c];
+    __syncwarp();
+    double x[HB];
 #pragma unroll
     for (int r = 0; r < HB; ++r) {
-        double sum = 0.0;
+        double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-        for (int k = 0; k < r; ++k) sum = fma(__shfl_sync(0xffffffffu, a[k], r), x[k], sum);
-        x[r] = ((r == c ? 1.0 : 0.0) - sum) * __shfl_sync(0xffffffffu, rdiag, r);
+        for (int k = 0; k + 1 < r; k += 2) {
+            s0 = fma(L[r][k], x[k], s0);
+            s1 = fma(L[r][k + 1], x[k + 1], s1);
+        }
+        if (r & 1) s0 = fma(L[r][r - 1], x[r - 1], s0);
+        x[r] = ((r == c ? 1.0 : 0.0) - (s0 + s1)) * rdiag[r];
     }
+#pragma unroll
+    for (int r = 0; r < HB; ++r) X[r][c] = x[r];
+    __syncwarp();
 }
 
 // One warp: the 32 x 32 lower block S (shared memory) -> its factor in S (0
 // above the diagonal) and the factor's inverse in X.  Not inlined: the leaf
-// calls it twice and its unrolled body is large, so one copy of the code
-// halves what the leaf fetches.
+// calls it twice, so one copy of the code halves what the leaf fetches.
 __device__ __noinline__ void warp_factor_half(double (*S)[HP], double (*X)[HP], int &bad)
 {
-    const int lane = threadIdx.x & 31;
-    double a[HB], x[HB];
-#pragma unroll
-    for (int c = 0; c < HB; ++c) a[c] = S[lane][c];
-    warp_chol32(a, bad);
-#pragma unroll
-    for (int c = 0; c < HB; ++c) S[lane][c] = c <= lane ? a[c] : 0.0;
-    warp_inv32(a, x);
-#pragma unroll
-    for (int r = 0; r < HB; ++r) X[r][lane] = x[r];
+    warp_chol32(S, bad);
+    warp_inv32(S, X);
 }
 
 // One 64 x 64 diagonal block: its Cholesky factor (lower, in place in A)
