@@ -294,10 +294,21 @@ __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y,
 // keep 16-byte alignment.
 constexpr int KC = 32;                    // K per stage
 constexpr int AS = KC + 4;                // smem row of an n- or m-major stage (doubles; 16-byte multiple)
-constexpr int BS = TB + 4;                // smem row of a k-major B stage
-constexpr int kStageD = 2 * TB * AS;      // A stage + the larger B stage (64 x 36 >= 32 x 68)
-constexpr size_t kGemmSmem = sizeof(double) * 2 * kStageD;
 constexpr int kGemmThreads = 128;
+
+// Tile T x T of C per block (T = 64, or 32 for products with few tiles, so
+// that they still spread over the SMs): the A stage (T x 32) and the larger
+// of the B stages (T x 32 n-major, 32 x (T + 4) k-major).
+template <int T>
+constexpr int stage_doubles()
+{
+    return T * AS + (T * AS > KC * (T + 4) ? T * AS : KC * (T + 4));
+}
+template <int T>
+constexpr size_t gemm_smem()
+{
+    return sizeof(double) * 2 * stage_doubles<T>();
+}
 
 struct Dgemm {
     const double *A;
@@ -326,41 +337,46 @@ __device__ __forceinline__ void dmma884(double (&d)[2], double a, double b)
                  : "d"(a), "d"(b));
 }
 
-template <bool BT>
+template <bool BT, int T>
 __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
 {
     pdl_enter();
+    constexpr int BS = T + 4;                 // smem row of a k-major B stage
+    constexpr int SD = stage_doubles<T>();
+    constexpr int F = T / 16;                 // MMA tiles per warp side (warp tile T/2 x T/2)
+    constexpr int CH = T * KC / 2;            // 16-byte chunks of one operand stage
     const int tj = blockIdx.x, ti = blockIdx.y;
     if (g.lower_c && tj > ti) return;
     extern __shared__ __align__(16) double smd[];
     int k0 = 0, k1 = g.K;
-    if (g.tri_a) k1 = min(k1, TB * (ti + 1));
+    if (g.tri_a) k1 = min(k1, T * (ti + 1));
     if (g.tri_b) {
         if (BT)
-            k1 = min(k1, TB * (tj + 1));
+            k1 = min(k1, T * (tj + 1));
         else
-            k0 = max(k0, TB * tj);
+            k0 = max(k0, T * tj);
     }
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int wm = 32 * (warp >> 1), wn = 32 * (warp & 1), gid = lane >> 2, tig = lane & 3;
-    const double *Ab = g.A + (int64_t)ti * TB * g.lda;
-    const double *Bb = BT ? g.B + (int64_t)tj * TB * g.ldb : g.B + (int64_t)tj * TB;
-    // one stage: 64 x 32 of A and 32 x 64 of B as 16-byte chunks, 8 + 8 per thread
+    const int wm = (T / 2) * (warp >> 1), wn = (T / 2) * (warp & 1), gid = lane >> 2, tig = lane & 3;
+    const double *Ab = g.A + (int64_t)ti * T * g.lda;
+    const double *Bb = BT ? g.B + (int64_t)tj * T * g.ldb : g.B + (int64_t)tj * T;
+    // one stage: T x 32 of A and 32 x T of B as 16-byte chunks
     auto issue = [&](int k, int st) {
-        double *As = smd + st * kStageD, *Bs = As + TB * AS;
+        double *As = smd + st * SD, *Bs = As + T * AS;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int idx = tid + kGemmThreads * q;                  // 0 .. 1023
+        for (int q = 0; q < CH / kGemmThreads; ++q) {
+            const int idx = tid + kGemmThreads * q;                  // 0 .. CH - 1
             cp_async16(As + (idx >> 4) * AS + 2 * (idx & 15), Ab + (int64_t)(idx >> 4) * g.lda + k + 2 * (idx & 15));
             if (BT)
                 cp_async16(Bs + (idx >> 4) * AS + 2 * (idx & 15),
                            Bb + (int64_t)(idx >> 4) * g.ldb + k + 2 * (idx & 15));
             else
-                cp_async16(Bs + (idx >> 5) * BS + 2 * (idx & 31), Bb + (int64_t)(k + (idx >> 5)) * g.ldb + 2 * (idx & 31));
+                cp_async16(Bs + (idx / (T / 2)) * BS + 2 * (idx % (T / 2)),
+                           Bb + (int64_t)(k + idx / (T / 2)) * g.ldb + 2 * (idx % (T / 2)));
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    double acc[4][4][2] = {};
+    double acc[F][F][2] = {};
     if (k0 < k1) {
         issue(k0, 0);
         int st = 0;
@@ -372,28 +388,28 @@ __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
                 asm volatile("cp.async.wait_group 0;" ::: "memory");
             }
             __syncthreads();
-            const double *As = smd + st * kStageD, *Bs = As + TB * AS;
+            const double *As = smd + st * SD, *Bs = As + T * AS;
 #pragma unroll
             for (int kk = 0; kk < KC; kk += 4) {
-                double a[4], b[4];
+                double a[F], b[F];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) a[i] = As[(wm + 8 * i + gid) * AS + kk + tig];
+                for (int i = 0; i < F; ++i) a[i] = As[(wm + 8 * i + gid) * AS + kk + tig];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < F; ++j)
                     b[j] = BT ? Bs[(wn + 8 * j + gid) * AS + kk + tig] : Bs[(kk + tig) * BS + wn + 8 * j + gid];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < F; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) dmma884(acc[i][j], a[i], b[j]);
+                    for (int j = 0; j < F; ++j) dmma884(acc[i][j], a[i], b[j]);
             }
             __syncthreads();                                         // stage st is refilled two steps on
         }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < F; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            double2 *cp = reinterpret_cast<double2 *>(g.C + (int64_t)(ti * TB + wm + 8 * i + gid) * g.ldc + tj * TB +
+        for (int j = 0; j < F; ++j) {
+            double2 *cp = reinterpret_cast<double2 *>(g.C + (int64_t)(ti * T + wm + 8 * i + gid) * g.ldc + tj * T +
                                                       wn + 8 * j + 2 * tig);
             double2 u = make_double2(g.alpha * acc[i][j][0], g.alpha * acc[i][j][1]);
             if (g.beta) {
@@ -933,9 +949,15 @@ struct Factor {
                      int64_t M, int64_t N, int64_t Kd, double alpha, int beta, int tri_a, int tri_b, int lower_c)
     {
         Dgemm g{a, lda, b, ldb, c, ldc, (int)M, (int)N, (int)Kd, alpha, beta, tri_a, tri_b, lower_c};
-        const dim3 grid((unsigned)(N / TB), (unsigned)(M / TB));
-        return bt ? launch_pdl(k_dgemm<true>, grid, dim3(kGemmThreads), kGemmSmem, s, g)
-                  : launch_pdl(k_dgemm<false>, grid, dim3(kGemmThreads), kGemmSmem, s, g);
+        const int64_t mt = M / TB, nt = N / TB, tiles = lower_c ? mt * (mt + 1) / 2 : mt * nt;
+        if (tiles < sm_count()) {                 // few tiles: 32 x 32 ones, four times as many blocks
+            const dim3 grid((unsigned)(N / 32), (unsigned)(M / 32));
+            return bt ? launch_pdl(k_dgemm<true, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g)
+                      : launch_pdl(k_dgemm<false, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g);
+        }
+        const dim3 grid((unsigned)nt, (unsigned)mt);
+        return bt ? launch_pdl(k_dgemm<true, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), s, g)
+                  : launch_pdl(k_dgemm<false, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), s, g);
     }
 
     // rows [o, o + n) of the factor and of its inverse
@@ -1044,14 +1066,17 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     uint8_t *dead = ws + L.dead;
     double *mean = reinterpret_cast<double *>(ws + L.mean);
 
-    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false};
+    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false}, attr_g2[64] = {false},
+                attr_g3[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     static bool attr_up[64] = {false};
     if (!set_smem_once(k_update_tf32, kUSmem, attr_up[dev & 63]) ||
         !set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
-        !set_smem_once(k_dgemm<false>, kGemmSmem, attr_g0[dev & 63]) ||
-        !set_smem_once(k_dgemm<true>, kGemmSmem, attr_g1[dev & 63]))
+        !set_smem_once(k_dgemm<false, 64>, gemm_smem<64>(), attr_g0[dev & 63]) ||
+        !set_smem_once(k_dgemm<true, 64>, gemm_smem<64>(), attr_g1[dev & 63]) ||
+        !set_smem_once(k_dgemm<false, 32>, gemm_smem<32>(), attr_g2[dev & 63]) ||
+        !set_smem_once(k_dgemm<true, 32>, gemm_smem<32>(), attr_g3[dev & 63]))
         return HIF4_ERR_CUDA;
 
     // 1. protected columns, Hessian diagonal statistics, FP32 working weights
