@@ -950,7 +950,7 @@ struct Factor {
     {
         Dgemm g{a, lda, b, ldb, c, ldc, (int)M, (int)N, (int)Kd, alpha, beta, tri_a, tri_b, lower_c};
         const int64_t mt = M / TB, nt = N / TB, tiles = lower_c ? mt * (mt + 1) / 2 : mt * nt;
-        if (tiles < sm_count()) {                 // few tiles: 32 x 32 ones, four times as many blocks
+        if (tiles < 3 * sm_count()) {             // few tiles: 32 x 32 ones, four times as many blocks
             const dim3 grid((unsigned)(N / 32), (unsigned)(M / 32));
             return bt ? launch_pdl(k_dgemm<true, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g)
                       : launch_pdl(k_dgemm<false, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g);
