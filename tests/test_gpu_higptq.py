@@ -123,6 +123,20 @@ def test_small_layer_vs_oracle(H, bs):
     compare(w, Hf, idx, 0.01, bs, got)
 
 
+@pytest.mark.parametrize("K", [64, 128, 320])
+def test_factor_recursion_shapes(H, K):
+    """The factor's recursion at its edges: one 64-column leaf (K = 64), one
+    split (128), and uneven splits of an odd tile count (320 = 2 + 3 tiles,
+    then 1 + 2)."""
+    rng = np.random.default_rng(K + 7)
+    N = 70
+    w = _bf16(rng, (N, K), 0.02)
+    x = _factor_x(rng, 1500, K, rank=8)
+    Hf = (x.T @ x).astype(np.float32)
+    got = run_gpu(H, w, Hf, [], 0.01, 64)
+    compare(w, Hf, [], 0.01, 64, got)
+
+
 def test_dead_channel_and_non_positive_definite(H):
     import torch
     rng = np.random.default_rng(4)
