@@ -483,6 +483,14 @@ __global__ void k_w_to_f32(const uint16_t *w, int64_t ldw, int64_t N, int64_t K,
     if (bad && status) atomicOr(status, HIF4_FLAG_NONFINITE);
 }
 
+// FP32 -> TF32 (round to nearest, ties away): the low 13 mantissa bits cleared.
+__device__ __forceinline__ uint32_t tf32_rna(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
 struct GptqArgs {
     const float *W;          // N x K current weights (FP32)
     int64_t N, K;
@@ -495,7 +503,7 @@ struct GptqArgs {
     uint8_t *codes;          // N x K/2
     uint32_t *meta;          // N x K/64
     uint16_t *w_masked;      // N x n_masked
-    float *Err;              // N x 64 NG
+    float *Eh, *El;          // N x 64 NG: the block's error E = D U_gg^{-1} as TF32 parts (hi + lo)
 };
 
 // One block of NG groups (64 NG columns) for kRowsPerBlock rows (each warp
@@ -582,7 +590,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
                 e0 = fmaf(d, u.x, e0);
                 e1 = fmaf(d, u.y, e1);
             }
-            *reinterpret_cast<float2 *>(a.Err + n * (64 * NG) + 64 * g + 2 * lane) = make_float2(e0, e1);
+            {
+                // E in two TF32 parts: the lazy update's split operand
+                const uint32_t h0 = tf32_rna(e0), h1 = tf32_rna(e1);
+                const int64_t o = n * (64 * NG) + 64 * g + 2 * lane;
+                *reinterpret_cast<float2 *>(a.Eh + o) = make_float2(__uint_as_float(h0), __uint_as_float(h1));
+                *reinterpret_cast<float2 *>(a.El + o) = make_float2(__uint_as_float(tf32_rna(e0 - __uint_as_float(h0))),
+                                                                  __uint_as_float(tf32_rna(e1 - __uint_as_float(h1))));
+            }
             // feedback into the later groups of the block
             if (g + 1 < NG) {
                 __syncwarp();
@@ -608,14 +623,6 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
             }
         }
     }
-}
-
-// FP32 -> TF32 (round to nearest, ties away): the low 13 mantissa bits cleared.
-__device__ __forceinline__ uint32_t tf32_rna(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
 }
 
 // dst (rows x cols, ld ldd) = src (ld lds), FP64; cols a multiple of 2.
@@ -837,17 +844,6 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
     if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
 }
 
-// hi / lo TF32 parts of n floats.
-__global__ void k_split_tf32(const float *x, int64_t n, float *hi, float *lo)
-{
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const float v = x[i];
-        const uint32_t h = tf32_rna(v);
-        hi[i] = __uint_as_float(h);
-        lo[i] = __uint_as_float(tf32_rna(v - __uint_as_float(h)));
-    }
-}
-
 // U^T split into TF32 parts (K x K, K a multiple of 32), 32 x 32 tiles through
 // shared memory so that both the reads of U and the writes of U^T coalesce.
 __global__ void k_ut_split(const float *U, int64_t K, float *UTh, float *UTl)
@@ -895,7 +891,7 @@ size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace sections of hif4_higptq1.
 struct GptqLayout {
-    size_t A, Y, T, U, UinvG, UTh, UTl, W, Err, Eh, El, mask, rank, dead, mean, total;
+    size_t A, Y, T, U, UinvG, UTh, UTl, W, Eh, El, mask, rank, dead, mean, total;
 };
 
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
@@ -916,7 +912,6 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     take(L.UTh, k * k * 4);
     take(L.UTl, k * k * 4);
     take(L.W, (size_t)N * k * 4);
-    take(L.Err, (size_t)N * (size_t)B * 4);
     take(L.Eh, (size_t)N * (size_t)B * 4);
     take(L.El, (size_t)N * (size_t)B * 4);
     take(L.mask, k);
@@ -1056,7 +1051,6 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     float *U = reinterpret_cast<float *>(ws + L.U);
     float *UinvG = reinterpret_cast<float *>(ws + L.UinvG);
     float *W = reinterpret_cast<float *>(ws + L.W);
-    float *Err = reinterpret_cast<float *>(ws + L.Err);
     float *UTh = reinterpret_cast<float *>(ws + L.UTh);
     float *UTl = reinterpret_cast<float *>(ws + L.UTl);
     float *Eh = reinterpret_cast<float *>(ws + L.Eh);
@@ -1129,17 +1123,15 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
         a.codes = codes;
         a.meta = meta;
         a.w_masked = static_cast<uint16_t *>(w_masked);
-        a.Err = Err;
+        a.Eh = Eh;
+        a.El = El;
         hif4_status st = NG == 1 ? launch_gptq_block<1>(a, s)
                        : NG == 2 ? launch_gptq_block<2>(a, s)
                        : NG == 3 ? launch_gptq_block<3>(a, s)
                                  : launch_gptq_block<4>(a, s);
         if (st != HIF4_OK) return st;
         if (b1 < K) {
-            const int64_t kd = 64 * NG, ne = N * kd;
-            k_split_tf32<<<(unsigned)std::min<int64_t>((ne + 255) / 256, 8 * (int64_t)sm_count()), 256, 0, s>>>(
-                Err, ne, Eh, El);
-            if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+            const int64_t kd = 64 * NG;
             CUtensorMap mAh, mAl;
             if (!make_tensor_map_f32_2d_sw128(&mAh, Eh, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM) ||
                 !make_tensor_map_f32_2d_sw128(&mAl, El, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM))
