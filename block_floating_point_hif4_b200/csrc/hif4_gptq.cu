@@ -174,7 +174,7 @@ __device__ __noinline__ void warp_factor_half(double (*S)[HP], double (*X)[HP], 
 
 // One 64 x 64 diagonal block: its Cholesky factor (lower, in place in A)
 // and the factor's inverse into Y (zeros above the diagonal), as two halves:
-// warp 0 factors and inverts the 32 x 32 diagonal blocks in registers, all
+// warp 0 factors and inverts the 32 x 32 diagonal blocks (warp_factor_half), all
 // 8 warps form L21 = A21 L11^{-T}, A22 - L21 L21^T and
 // Y21 = -L22^{-1} L21 L11^{-1} as 32 x 32 x 32 shared-memory products.  A
 // pivot that is not positive is replaced by 1 and reported as
@@ -280,9 +280,9 @@ __global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y,
     if (tid == 0 && bad_all && status) atomicOr(status, HIF4_FLAG_NOT_SPD);
 }
 
-// FP64 GEMM on whole 64 x 64 tiles: C = alpha op(A) op(B) (+ C if beta),
-// on the FP64 tensor-core MMA (m8n8k4).  One 64 x 64 tile of C per
-// 128-thread block, a 32 x 32 quarter per warp (4 x 4 MMA tiles); the K loop
+// FP64 GEMM on whole tiles: C = alpha op(A) op(B) (+ C if beta), on the FP64
+// tensor-core MMA (m8n8k4).  One T x T tile of C per 128-thread block (T =
+// 64, or 32 below), a T/2 x T/2 quarter per warp (T/16 x T/16 MMA tiles); the K loop
 // runs in 32-deep stages that cp.async copies double-buffer into shared
 // memory in the operands' own layouts: A row-major, B k-major (B row-major)
 // or n-major (BT, B^T row-major), whose fragments the MMA reads directly.  A
