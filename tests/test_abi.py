@@ -109,3 +109,53 @@ def test_argument_errors_return_before_any_launch(L):
     assert ffn(fake, 4, 64, 64, fake, fake, 128, None, 0, None, None, fake, fake, None, 2, None, None, fake, 64,
                0, fake, 1 << 30, None, None) == 1
     assert L.hif4_get_status(None, None) == 1
+
+
+def test_higptq_hessian_and_host_ffn_argument_errors(L):
+    P = ctypes.c_void_p
+    fake = P(0x1000)          # never dereferenced: every call below fails validation first
+    # HiGPTQ workspace: K % 64 and unsupported block sizes give 0; it grows with N
+    assert L.hif4_higptq1_workspace(16, 100, 128) == 0
+    assert L.hif4_higptq1_workspace(16, 512, 100) == 0
+    assert L.hif4_higptq1_workspace(16, 512, 320) == 0
+    assert 0 < L.hif4_higptq1_workspace(16, 512, 0) == L.hif4_higptq1_workspace(16, 512, 128)
+    assert L.hif4_higptq1_workspace(1024, 512, 128) > L.hif4_higptq1_workspace(16, 512, 128)
+    ws = L.hif4_higptq1_workspace(16, 512, 128)
+
+    def gptq(w=fake, N=16, K=512, ldw=512, H=fake, idx=None, nm=0, damp=0.01, bs=128, codes=fake, meta=fake,
+             wm=None, work=fake, wsb=ws):
+        return L.hif4_higptq1(w, N, K, ldw, H, idx, nm, damp, bs, codes, meta, wm, work, wsb, None, None)
+
+    assert gptq(K=100, ldw=100) == 3     # K not a multiple of 64
+    assert gptq(ldw=256) == 3            # ldw < K
+    assert gptq(bs=100) == 1             # block size not a multiple of 64
+    assert gptq(bs=320) == 1             # block size above 256
+    assert gptq(damp=-1.0) == 1          # negative damping
+    assert gptq(N=0) == 1
+    assert gptq(K=32832, ldw=32832) == 8  # K above the supported 32768
+    assert gptq(nm=3) == 1               # protected count without indices
+    assert gptq(H=None) == 1
+    assert gptq(meta=P(0x1002)) == 2     # misaligned metadata
+    assert gptq(wsb=ws - 1) == 4         # workspace too small
+    assert gptq(work=P(0x1010)) == 2     # workspace not 256-byte aligned
+    # Hessian
+    assert L.hif4_hessian_workspace(3001, 256) > 0
+    hs = L.hif4_hessian_workspace(3001, 256)
+    assert L.hif4_hessian(fake, 3001, 100, 100, fake, fake, hs, None, None) == 3
+    assert L.hif4_hessian(fake, 3001, 256, 128, fake, fake, hs, None, None) == 3
+    assert L.hif4_hessian(None, 3001, 256, 256, fake, fake, hs, None, None) == 1
+    assert L.hif4_hessian(fake, 3001, 256, 256, P(0x1004), fake, hs, None, None) == 2
+    assert L.hif4_hessian(fake, 3001, 256, 256, fake, fake, hs - 1, None, None) == 4
+    # FFN on host buffers: unknown flag, null host input, ldx < D, workspace too small
+    fh = L.hif4_ffn_w4a4_host
+
+    def ffn_host(x=fake, M=64, D=64, ldx=64, F=128, y=fake, ldy=64, flags=0, work=fake, wsb=1 << 30):
+        return fh(x, M, D, ldx, fake, fake, F, None, 0, None, None, fake, fake, None, 0, None, None, y, ldy, 0,
+                  flags, work, wsb, None, None)
+
+    assert ffn_host(flags=0x10) == 1     # no such flag
+    assert ffn_host(x=None) == 1
+    assert ffn_host(ldx=32) == 3
+    assert ffn_host(F=100) == 3
+    assert ffn_host(wsb=64) == 4
+    assert ffn_host(M=0) == 0            # nothing to do
