@@ -53,12 +53,14 @@ SIGNATURES = {
     "hif4_hessian_workspace": (_SZ, [_I64, _I64]),
     "hif4_hessian": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
     "hif4_higptq1_workspace": (_SZ, [_I64, _I64, _I64]),
+    "hif4_higptq1_group_inputs_offset": (_SZ, [_I64, _I64, _I64]),
     "hif4_higptq1": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, ctypes.c_double, _I64, _P, _P, _P, _P,
                                     _SZ, _P, _P]),
     "hif4_ptq_state_bytes": (_SZ, [_I64, _I64, _I32]),
     "hif4_ptq_state_pack": (ctypes.c_int, [_I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ]),
     "hif4_ptq_state_info": (ctypes.c_int, [_P, _SZ, _P, _P, _P]),
     "hif4_ptq_state_unpack": (ctypes.c_int, [_P, _SZ, _P, _P, _P, _P]),
+    "hif4_debug_wait_test": (None, [ctypes.c_uint32, ctypes.c_uint64]),
     "hif4_get_status": (ctypes.c_int, [_P, _P]),
     "hif4_reset_status": (ctypes.c_int, [_P, _P]),
     "hif4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -353,6 +355,16 @@ def higptq1(w: torch.Tensor, H: torch.Tensor, mask_idx: torch.Tensor | None = No
         _ptr(w), N, K, w.stride(0), _ptr(H), _ptr(mask_idx) if n else None, n, float(damp), blocksize,
         _ptr(codes), _ptr(meta), _ptr(wm), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
     return codes, meta, wm
+
+
+def higptq1_group_inputs(workspace: torch.Tensor, N: int, K: int, blocksize: int = 128) -> torch.Tensor:
+    """FP32 [N, K] view of a hif4_higptq1 workspace: after the call, the
+    weights each 64-column group was quantized from (stream-ordered)."""
+    off = int(lib().hif4_higptq1_group_inputs_offset(N, K, blocksize))
+    if off == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid HiGPTQ shape")
+    assert workspace.dtype == torch.uint8 and workspace.numel() >= off + N * K * 4
+    return workspace[off:off + N * K * 4].view(torch.float32).view(N, K)
 
 
 def ptq_state_pack(codes: torch.Tensor, meta: torch.Tensor, mask_idx: torch.Tensor | None = None,

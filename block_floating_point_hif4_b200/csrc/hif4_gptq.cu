@@ -492,7 +492,8 @@ __device__ __forceinline__ uint32_t tf32_rna(float x)
 }
 
 struct GptqArgs {
-    const float *W;          // N x K current weights (FP32)
+    float *W;                // N x K current weights (FP32); each group's columns get the values
+                             // that group is quantized from
     int64_t N, K;
     int64_t b0;              // first column of the block
     const float *U;          // K x K upper factor
@@ -510,7 +511,11 @@ struct GptqArgs {
 // takes kRowsPerWarp of them in turn, after one load of the U tiles), a warp per
 // row; lane l holds elements 2l, 2l+1 of each group.  Per group: the exact
 // FP32 unit quantization (encode rule of the streaming quantizer), D = W - Q,
-// E = D Uinv_g (Uinv_g upper), feedback into the block's later groups.
+// E = D Uinv_g (Uinv_g upper), feedback into the block's later groups.  The
+// values a later group is quantized from (after the in-block feedback) are
+// written back over its columns of W, so that on return W holds, for every
+// group, exactly the weights that group was quantized from (later blocks
+// never touch earlier columns).
 template <int NG>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
 {
@@ -542,6 +547,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             const int64_t col = a.b0 + 64 * g + 2 * lane;
+            if (g > 0) *reinterpret_cast<float2 *>(a.W + n * a.K + col) = make_float2(x[g][0], x[g][1]);
             const bool m0 = a.mask && a.mask[col], m1 = a.mask && a.mask[col + 1];
             const float v0 = m0 ? 0.0f : x[g][0], v1 = m1 ? 0.0f : x[g][1];
             // level 1: unit maximum -> scale code
@@ -1023,6 +1029,12 @@ extern "C" size_t hif4_higptq1_workspace(int64_t N, int64_t K, int64_t blocksize
     const int64_t B = blocksize == 0 ? 128 : blocksize;
     if (B % HIF4_UNIT != 0 || B > 256 || B <= 0) return 0;
     return gptq_layout(N, K, B).total;
+}
+
+extern "C" size_t hif4_higptq1_group_inputs_offset(int64_t N, int64_t K, int64_t blocksize)
+{
+    if (hif4_higptq1_workspace(N, K, blocksize) == 0) return (size_t)-1;
+    return gptq_layout(N, K, blocksize == 0 ? 128 : blocksize).W;
 }
 
 extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t ldw, const float *H,

@@ -295,7 +295,10 @@ hif4_status hif4_calib_percentile_mask(const void *acts, int64_t tokens, int64_t
  *     current histogram layout: channels <= 5445).
  *   - The first call on a device looks up the array's device address once
  *     (that device must be current); make that first call before any stream
- *     capture begins.
+ *     capture begins.  The address stays cached for the life of the
+ *     process: after cudaDeviceReset, or anything else that tears down and
+ *     re-creates the device's primary context, it is stale, so do not use
+ *     this call on that device again in the same process.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents: calls whose execution overlaps on the GPU (different streams
  *     without ordering) race and give wrong results.  Order them.
@@ -353,6 +356,19 @@ hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t ldw, const
                          const int32_t *mask_idx, int32_t n_masked, double damp, int64_t blocksize,
                          uint8_t *codes, uint32_t *meta, void *w_masked, void *workspace, size_t ws_bytes,
                          uint32_t *status, hif4_stream_t stream);
+/*
+ * hif4_higptq1_group_inputs_offset — byte offset, inside a hif4_higptq1
+ * workspace of the same N, K and blocksize, of an FP32 N x K array (row
+ * stride K) that, once the call has completed on its stream, holds for every
+ * 64-column group the weights that group was quantized from: the layer
+ * weight after the error feedback of every earlier group (dead input
+ * channels zeroed) [HiF4 article, section 3.1: each group is quantized from
+ * its current, updated values].  Lets a caller inspect the feedback, or check
+ * each group's codes against a plain quantization of those values.  The array
+ * stays valid until the workspace is reused.  Returns (size_t)-1 for shapes
+ * hif4_higptq1_workspace refuses.
+ */
+size_t hif4_higptq1_group_inputs_offset(int64_t N, int64_t K, int64_t blocksize);
 
 /*
  * Compact PTQ state of one linear layer [TA summary, "Method overview":
@@ -385,6 +401,23 @@ hif4_status hif4_ptq_state_info(const void *buf, size_t bytes, int64_t *N, int64
                                 int32_t *n_masked);
 hif4_status hif4_ptq_state_unpack(const void *buf, size_t bytes, uint8_t *codes, uint32_t *meta,
                                   int32_t *mask_idx, void *w_masked);
+
+/*
+ * hif4_debug_wait_test — failure-handling diagnostic; off by default and not
+ * meant for production runs.  Every wait of the TMA-fed kernels on an
+ * asynchronous copy is bounded by wall time (4 s in the tcgen05 GEMM, 2 s in
+ * the quantizers and the calibration passes): a block whose wait runs out
+ * stops, lets the copies it issued land (and, in the GEMM, its MMAs
+ * complete before the tensor memory is freed), and reports
+ * HIF4_FLAG_TIMEOUT in the status word; the calibration then poisons its
+ * outputs (ratios NaN, mask 0, indices -1).  While `withhold` is nonzero,
+ * block 0 of every later launch of those kernels from this process leaves
+ * its first copy un-issued, so the wait on it can only end at its limit;
+ * `limit_ns` (0 = the defaults) replaces every such limit.  Call
+ * hif4_debug_wait_test(0, 0) to return to normal operation.  Process-wide,
+ * not thread-safe against concurrent launches; no device work.
+ */
+void hif4_debug_wait_test(uint32_t withhold, uint64_t limit_ns);
 
 /* Synchronizes `stream`, reads the device status word and maps its bits:
  * TIMEOUT -> HIF4_ERR_TIMEOUT, BAD_INDEX or NOT_SPD -> HIF4_ERR_INVALID_ARG,

@@ -121,6 +121,12 @@ def test_higptq_hessian_and_host_ffn_argument_errors(L):
     assert 0 < L.hif4_higptq1_workspace(16, 512, 0) == L.hif4_higptq1_workspace(16, 512, 128)
     assert L.hif4_higptq1_workspace(1024, 512, 128) > L.hif4_higptq1_workspace(16, 512, 128)
     ws = L.hif4_higptq1_workspace(16, 512, 128)
+    # the group-inputs array lies inside the workspace, 256-byte aligned; refused shapes give (size_t)-1
+    for N, K, bs in ((16, 512, 128), (3000, 1024, 64), (70, 320, 0), (13824, 5120, 128)):
+        off = L.hif4_higptq1_group_inputs_offset(N, K, bs)
+        assert off % 256 == 0 and off + N * K * 4 <= L.hif4_higptq1_workspace(N, K, bs)
+    assert L.hif4_higptq1_group_inputs_offset(16, 100, 128) == ctypes.c_size_t(-1).value
+    assert L.hif4_higptq1_group_inputs_offset(16, 512, 320) == ctypes.c_size_t(-1).value
 
     def gptq(w=fake, N=16, K=512, ldw=512, H=fake, idx=None, nm=0, damp=0.01, bs=128, codes=fake, meta=fake,
              wm=None, work=fake, wsb=ws):

@@ -4,7 +4,22 @@
 The oracle runs in FP64, the GPU group loop in FP32, so the error feedback
 differs in the last bits and a quantization decision that sits next to a
 rounding boundary can go the other way; the differences then feed forward.
-The bars, fixed here:
+So the GPU result is checked as a sequence of correct HiGPTQ steps, from
+the values each 64-column group was quantized from (which the call leaves
+in its workspace, hif4_higptq1_group_inputs_offset):
+  * step validity, every group of every checked row: its codes and metadata
+    equal the oracle's plain quantization of those FP32 values, bit for bit,
+    and a protected column holds their BF16 rounding;
+  * feedback: those values equal, within FP32 rounding, the FP64 GPTQ update
+    W0_h - sum_{g<h} E_g U_{g,h}, with E_g = (W_g - Q_g) U_gg^-1 computed in
+    FP64 from the GPU's own W_g and Q_g and U the oracle's FP64 factor.  The
+    bound is 2^-14 x (|W0| + (|D| |U_gg^-1|) |U_{g,h}|) summed in absolute
+    values: twice the worst case of the GPU's arithmetic (FP32 rounding of U,
+    <= 384-term FP32 accumulations of split-TF32 products per update launch
+    and <= 64-term ones for E, one rounding of W per block: about 2^-15 of
+    that sum).  A dropped term, a wrong sign or a wrong index moves some
+    element by a sizeable fraction of the sum itself.
+And against the oracle's own FP64 run, end to end:
   * the first 64-column group of every row has received no feedback: its
     codes and metadata are bit-exact;
   * with no cross-group coupling (identity Hessian) everything is bit-exact;
@@ -18,6 +33,7 @@ import pytest
 
 import oracle
 from block_floating_point_hif4_b200 import workloads as wl
+from tests._gptq_check import check_group_steps
 from tests._util import THREADS, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
@@ -49,16 +65,21 @@ def _objective(w_bits, wq, Hd):
     return float(np.einsum("nk,kl,nl->", d, Hd, d))
 
 
-def run_gpu(Hm, w_bits, Hf32, idx, damp, bs):
+def run_gpu(Hm, w_bits, Hf32, idx, damp, bs, w_dev=None):
+    """-> (codes, meta, w_masked bits or None, group inputs FP32 N x K)."""
     import torch
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     i_dev = torch.from_numpy(np.asarray(idx, np.int32)).cuda() if len(idx) else None
-    codes, meta, wm = Hm.higptq1(to_dev_bf16(w_bits), torch.from_numpy(Hf32).cuda(), i_dev, damp, bs,
+    w_dev = to_dev_bf16(w_bits) if w_dev is None else w_dev
+    N, K = w_dev.shape
+    ws = torch.empty(Hm.lib().hif4_higptq1_workspace(N, K, bs), dtype=torch.uint8, device="cuda")
+    codes, meta, wm = Hm.higptq1(w_dev, torch.from_numpy(Hf32).cuda(), i_dev, damp, bs, workspace=ws,
                                  status=status)
     torch.cuda.synchronize()
     assert Hm.get_status(status) == 0
+    gin = Hm.higptq1_group_inputs(ws, N, K, bs).cpu().numpy()
     return (codes.cpu().numpy(), meta.cpu().numpy().view(np.uint32),
-            None if wm is None else wm.view(torch.int16).cpu().numpy().view(np.uint16))
+            None if wm is None else wm.view(torch.int16).cpu().numpy().view(np.uint16), gin)
 
 
 def compare(w_bits, Hf32, idx, damp, bs, got, factor=None, rows=None):
@@ -69,6 +90,8 @@ def compare(w_bits, Hf32, idx, damp, bs, got, factor=None, rows=None):
     wr = np.ascontiguousarray(w_bits[rows])
     c_o, m_o, wq_o, wm_o = oracle.higptq1(wr, Hf32.astype(np.float64), mask if len(idx) else None, damp, bs,
                                           threads=THREADS, factor=factor)
+    check_group_steps(w_bits, idx, got, factor if factor is not None else oracle.gptq_factor(
+        Hf32.astype(np.float64), damp), rows)
     c_g, m_g, wm_g = got[0][rows], got[1][rows], None if got[2] is None else got[2][rows]
     # the first group of every row: no feedback yet, bit-exact
     assert np.array_equal(c_g[:, :32], c_o[:, :32]) and np.array_equal(m_g[:, 0], m_o[:, 0])
@@ -105,7 +128,7 @@ def test_identity_hessian_is_plain_quantization(H):
     idx = np.array([1, 64, 200, 511], np.int32)
     mask = np.zeros(K, np.uint8)
     mask[idx] = 1
-    codes, meta, wm = run_gpu(H, w, np.eye(K, dtype=np.float32), idx, 0.01, 128)
+    codes, meta, wm, _ = run_gpu(H, w, np.eye(K, dtype=np.float32), idx, 0.01, 128)
     rc, rm, _ = oracle.quantize(w, mask)
     assert np.array_equal(codes, rc) and np.array_equal(meta, rm)
     assert np.array_equal(wm, w[:, idx])
@@ -175,18 +198,21 @@ def test_many_tiles_ragged_rows(H):
 
 @pytest.mark.slow
 def test_wan22_w1_sampled_rows(H):
-    """W1 of the Wan2.2 FFN (13824 x 5120) with the Hessian of 8192 tokens of
-    the attention-projection input recipe; 128 sampled rows against the
-    oracle (rows are independent given the Hessian factor)."""
-    d = wl.attn_proj(M=8192, seed=2)
-    x = d["x"]
-    x64 = wl.bf16_bits_to_f32(x).astype(np.float64)
+    """W1 of the Wan2.2 FFN (13824 x 5120, the bench's seeded weight) with the
+    Hessian of the bench's 57600 activation tokens (the attention-projection
+    input recipe, seed 3) and its 51 seeded outlier channels protected; 128
+    sampled rows against the oracle, every group of them step-checked (rows
+    are independent given the Hessian factor)."""
+    import torch
+    xd, outl = wl.device_rows(57600, 5120, seed=3, device="cuda")
+    x64 = wl.bf16_bits_to_f32(xd.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+    del xd
     Hf = (x64.T @ x64).astype(np.float32)
-    w1 = wl.ffn(seed=3, with_x=False)["w1"]
-    p = oracle.percentile(d["x"], threads=THREADS)
-    _, m, _ = oracle.channel_mask(p)
-    idx = np.nonzero(m)[0].astype(np.int32)
-    got = run_gpu(H, w1, Hf, idx, 0.01, 128)
+    del x64
+    w1d = wl.device_weight(13824, 5120, 0.015, seed=31, device="cuda")
+    w1 = w1d.view(torch.int16).cpu().numpy().view(np.uint16)
+    idx = outl.cpu().numpy().astype(np.int32)
+    got = run_gpu(H, w1, Hf, idx, 0.01, 128, w_dev=w1d)
     factor = oracle.gptq_factor(Hf.astype(np.float64), 0.01)
     rows = wl.sample_rows(w1.shape[0], 128)
     compare(w1, Hf, idx, 0.01, 128, got, factor=factor, rows=rows)

@@ -13,12 +13,15 @@ Each pin compares the oracle with something other than itself:
   * on inputs whose channels are correlated across groups (a few shared
     factors) the layer-output error tr((W - Q) H (W - Q)^T) is well below
     that of plain rounding to the nearest HiF4 values.
+The per-group step check that the GPU tests apply passes on the oracle's
+own run and fails on one with a group's error left out of the feedback.
 """
 import numpy as np
 import pytest
 
 import oracle
 from block_floating_point_hif4_b200 import workloads as wl
+from tests._gptq_check import check_group_steps
 
 
 def _weights(rng, N, K, scale=0.02):
@@ -140,3 +143,38 @@ def test_output_error_is_well_below_plain_rounding():
         d = w64 - q
         return float(np.einsum("nk,kl,nl->", d, H, d))
     assert err(wq) < 0.5 * err(w_rtn)
+
+
+def test_group_step_check_catches_a_wrong_feedback():
+    """The per-group check fails on a result whose feedback skipped one
+    group's error (made on the CPU by running the oracle's steps on a
+    perturbed copy), and passes on the oracle's own FP64 run."""
+    rng = np.random.default_rng(21)
+    N, K = 16, 256
+    w = _weights(rng, N, K)
+    Hd = _hessian(rng, 1000, K)
+    factor = oracle.gptq_factor(Hd, 0.01)
+    U = factor[0]
+    c, m, wq, _ = oracle.higptq1(w, Hd, None, 0.01, 64, factor=factor)
+    # the oracle's group inputs, rebuilt from its own output: W_h = W0_h - sum_{g<h} E_g U_{g,h}
+    w0 = wl.bf16_bits_to_f32(w).astype(np.float64)
+    gin = w0.copy()
+    for h in range(1, K // 64):
+        s = slice(64 * h, 64 * h + 64)
+        acc = np.zeros((N, 64))
+        for g in range(h):
+            t = slice(64 * g, 64 * g + 64)
+            e = (gin[:, t] - wq[:, t]) @ np.linalg.inv(U[t, t])
+            acc += e @ U[t, s]
+        gin[:, s] = w0[:, s] - acc
+    ok = (c, m, None, gin.astype(np.float32))
+    c2, m2, _ = oracle.quantize(gin.astype(np.float32))
+    assert np.array_equal(c2, c) and np.array_equal(m2, m)     # the rebuilt inputs reproduce the codes
+    check_group_steps(w, [], ok, factor)
+    # group 2 never received group 0's error: its inputs (and codes) are those of a wrong feedback
+    bad = gin.copy()
+    e0 = (gin[:, :64] - wq[:, :64]) @ np.linalg.inv(U[:64, :64])
+    bad[:, 128:192] += e0 @ U[:64, 128:192]
+    cb, mb, _ = oracle.quantize(bad.astype(np.float32))
+    with pytest.raises(AssertionError):
+        check_group_steps(w, [], (cb, mb, None, bad.astype(np.float32)), factor)
