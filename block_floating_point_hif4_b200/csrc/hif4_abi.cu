@@ -1,4 +1,5 @@
 // hif4_abi.cu — status handling and per-device caches of libhif4.
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -20,6 +21,19 @@ struct OccEntry {
 OccEntry g_occ[256];
 int g_nocc = 0;
 } // namespace
+
+namespace {
+std::atomic<uint32_t> g_withhold{0};
+std::atomic<uint64_t> g_wait_limit{0};
+} // namespace
+
+uint32_t wait_test_withhold() { return g_withhold.load(std::memory_order_relaxed); }
+
+uint64_t wait_limit_ns(uint64_t dflt)
+{
+    const uint64_t v = g_wait_limit.load(std::memory_order_relaxed);
+    return v ? v : dflt;
+}
 
 int sm_count()
 {
@@ -151,3 +165,9 @@ extern "C" const char *hif4_status_string(hif4_status s)
 }
 
 extern "C" int hif4_version(void) { return 100; }
+
+extern "C" void hif4_debug_wait_test(uint32_t withhold, uint64_t limit_ns)
+{
+    hif4::g_withhold.store(withhold ? 1u : 0u);
+    hif4::g_wait_limit.store(limit_ns);
+}

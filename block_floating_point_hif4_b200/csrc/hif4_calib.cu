@@ -66,6 +66,8 @@ struct PassArgs {
     uint32_t *ge;            // window pass: [C]
     uint32_t *whist;         // window pass: [C][256]
     uint32_t *timed_out;     // set to 1 when a TMA transfer never lands
+    uint32_t withhold;       // TMA passes: block 0 withholds its first copy (failure-handling test)
+    uint64_t wait_ns;        // TMA passes: limit of every bounded wait
 };
 
 // Bin holding ascending rank k of a histogram of `nbins` (multiple of 32)
@@ -399,10 +401,11 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
                 for (; issued < nchunks; ++issued) {
                     const uint32_t gi = g + (uint32_t)issued, st = gi % kTmaStages;
                     if (gi >= (uint32_t)kTmaStages &&
-                        !mbar_wait_bounded(&empty[st], (gi / kTmaStages - 1u) & 1u, &abort_flag, kWaitNs)) {
+                        !mbar_wait_bounded(&empty[st], (gi / kTmaStages - 1u) & 1u, &abort_flag, a.wait_ns)) {
                         ok = false;
                         break;
                     }
+                    if (a.withhold && blockIdx.x == 0 && gi == 0) continue;   // its wait can only run out
                     mbar_arrive_expect_tx(&full[st], kTileBytes);
                     tma_load_2d(tiles + st * kTileBytes, &tm, c0, (int32_t)(t0 + (int64_t)issued * kTmaRows),
                                 &full[st]);
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) k_pass_tma(const __grid_consta
             for (int ci = 0; ci < nchunks; ++ci) {
                 const uint32_t gi = g + (uint32_t)ci, st = gi % kTmaStages;
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait_bounded(&full[st], (gi / kTmaStages) & 1u, &abort_flag, kWaitNs));
+                                mbar_wait_bounded(&full[st], (gi / kTmaStages) & 1u, &abort_flag, a.wait_ns));
                 if (!ok) break;
                 // rows warp + 16 i of this tile that lie inside the segment
                 const int64_t left = t1 - (t0 + (int64_t)ci * kTmaRows);
@@ -738,6 +741,8 @@ hif4_status launch_pass_tma(const PassArgs &a0, cudaStream_t s, bool &done)
         attr[dev & 63] = true;
     }
     PassArgs a = a0;
+    a.withhold = wait_test_withhold();
+    a.wait_ns = wait_limit_ns(kWaitNs);
     // equal shares of the slab-major (slab, row) space, one block per
     // resident slot, 4..65535 tiles' worth of rows each
     const int64_t slots = (int64_t)blocks_per_sm(reinterpret_cast<const void *>(k), kTmaThreads, smem) * sm_count();

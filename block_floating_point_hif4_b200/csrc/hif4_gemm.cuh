@@ -36,6 +36,7 @@ struct Args {
     const uint8_t *out_mask;  // HIF4_LINEAR_FAKE_QUANT_OUT: u8 [N] protected output columns, or null
     uint32_t *status;
     uint64_t timeout_ns;
+    uint32_t withhold;      // block 0 withholds its first copy (failure-handling test)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Args &g, int &mb, int &nb)
@@ -154,10 +155,12 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
-                    tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
-                    ++issued;
+                    if (!(g.withhold && t == 0 && kb == 0)) {      // else its wait can only run out
+                        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                        tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, mb * BM, &full[stage]);
+                        tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+                        ++issued;
+                    }
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;

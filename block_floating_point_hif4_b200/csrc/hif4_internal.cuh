@@ -31,6 +31,11 @@ inline hif4_status launch_status()
 
 // Number of SMs of the current device (cached per device ordinal).
 int sm_count();
+// Failure-handling diagnostics (hif4_debug_wait_test): whether TMA-fed
+// launches withhold the first copy of their block 0, and the limit of their
+// bounded waits (dflt unless a test set one).
+uint32_t wait_test_withhold();
+uint64_t wait_limit_ns(uint64_t dflt);
 // Resident blocks per SM for `kernel` at this block size (cached per kernel
 // and device).
 int blocks_per_sm(const void *kernel, int threads, size_t dyn_smem);

@@ -108,7 +108,8 @@ hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const 
     g.flags = flags;
     g.out_mask = out_mask;
     g.status = status;
-    g.timeout_ns = TIMEOUT_NS;
+    g.timeout_ns = wait_limit_ns(TIMEOUT_NS);
+    g.withhold = wait_test_withhold();
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);

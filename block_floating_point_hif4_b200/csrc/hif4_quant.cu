@@ -47,6 +47,8 @@ struct QuantArgs {
     FastDiv upr_div;
     uint32_t total_units;
     uint32_t *status;
+    uint32_t withhold;         // TMA kernels: block 0 withholds its first copy (failure-handling test)
+    uint64_t wait_ns;          // TMA kernels: limit of every bounded wait
 };
 
 // Loads the 8 elements of lane vector `e` (element offset) as FP32.
@@ -503,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
     }
     __syncthreads();
     auto issue = [&](uint32_t i) {
+        if (a.withhold && blockIdx.x == 0 && i == 0) return;   // its wait can only run out
         const uint32_t chunk = blockIdx.x + i * gridDim.x;
         const uint32_t u0 = chunk * kChunkUnits;
         const uint32_t nu = min((uint32_t)kChunkUnits, a.total_units - u0);
@@ -534,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, HIF4_QT_MINB) k_quant_tma(QuantArgs 
             const uint4 m4 = __ldg(reinterpret_cast<const uint4 *>(a.chan_mask + (size_t)cu * HIF4_UNIT + q4 * 16));
             mraw[0] = m4.x; mraw[1] = m4.y; mraw[2] = m4.z; mraw[3] = m4.w;
         }
-        const bool ok = mbar_wait_bounded(&full[st], (i / kStages) & 1u, &abort_flag, kWaitNs);
+        const bool ok = mbar_wait_bounded(&full[st], (i / kStages) & 1u, &abort_flag, a.wait_ns);
         uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (ok && active) {
             const uint4 *src = reinterpret_cast<const uint4 *>(sm + (size_t)st * kChunkBytes + tid * 32u);
@@ -753,6 +756,7 @@ __global__ void __launch_bounds__(kThreads, HIF4_Q32_MINB) k_quant32(const __gri
     }
     __syncthreads();
     auto issue = [&](uint32_t i) {
+        if (a.withhold && blockIdx.x == 0 && i == 0) return;   // its wait can only run out
         const uint32_t st = i % kQ32Stages;
         mbar_arrive_expect_tx(&full[st], kQ32Bytes);
         tma_load_2d(sm + (size_t)st * kQ32Bytes, &tm, 0, (int32_t)((blockIdx.x + i * gridDim.x) * kQ32Units),
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, HIF4_Q32_MINB) k_quant32(const __gri
     uint32_t bad = 0, i = 0;
     for (; i < my_n; ++i) {
         const uint32_t st = i % kQ32Stages;
-        const bool ok = mbar_wait_bounded(&full[st], (i / kQ32Stages) & 1u, &abort_flag, kWaitNs);
+        const bool ok = mbar_wait_bounded(&full[st], (i / kQ32Stages) & 1u, &abort_flag, a.wait_ns);
         const uint32_t unit = (blockIdx.x + i * gridDim.x) * kQ32Units + r;
         const bool active = unit < a.total_units;
         uint32_t w[16];
@@ -1025,8 +1029,11 @@ hif4_status launch_quant_tma(const QuantArgs &qa, cudaStream_t s)
 }
 
 template <bool BF16, bool MASK, int MODE>
-hif4_status launch_quant(const QuantArgs &qa, bool contig, bool fast, cudaStream_t s)
+hif4_status launch_quant(const QuantArgs &qa0, bool contig, bool fast, cudaStream_t s)
 {
+    QuantArgs qa = qa0;
+    qa.withhold = wait_test_withhold();
+    qa.wait_ns = wait_limit_ns(kWaitNs);
     if (BF16 && MODE == 0 && fast && contig) {
         bool done = false;
         const hif4_status st = launch_quant32<MASK>(qa, s, done);
