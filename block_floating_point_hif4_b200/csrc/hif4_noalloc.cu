@@ -25,7 +25,9 @@ void *g_scratch_ptr[64] = {nullptr};
 
 // Device address of g_calib_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached for the life of the
+// process; a device reset (a new primary context) would leave the cached
+// address stale, which the header tells callers.
 hif4_status scratch_for_current_device(void **out)
 {
     int dev = 0;

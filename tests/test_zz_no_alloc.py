@@ -40,7 +40,9 @@ def test_noalloc_matches_allocating_entry_point():
     L = binding.lib()
     assert L.hif4_calib_noalloc_scratch_bytes() == 16 << 20
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    cases = [(14400, 320, (999, 1000), (1, 100), 5), (3001, 130, (1, 2), (1, 10), 6)]
+    # the last two cases sit at the Wan2.2 width and at the widest input the array admits
+    cases = [(14400, 320, (999, 1000), (1, 100), 5), (3001, 130, (1, 2), (1, 10), 6),
+             (4096, 5120, (999, 1000), (1, 100), 7), (4096, 5445, (999, 1000), (1, 100), 8)]
     for T, C, q, frac, seed in cases:
         acts_host, _ = wl.calib(T=T, C=C, seed=seed)
         acts = torch.from_numpy(acts_host.view(np.int16)).view(torch.bfloat16).cuda()
@@ -67,10 +69,13 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
 
     from block_floating_point_hif4_b200 import binding
     L = binding.lib()
-    C = 1 << 15
-    assert L.hif4_calib_workspace(16, C) > L.hif4_calib_noalloc_scratch_bytes()
+    cap = L.hif4_calib_noalloc_scratch_bytes()
+    # 5445 channels is the widest input whose scratch fits; one more does not
+    assert L.hif4_calib_workspace(4096, 5445) <= cap < L.hif4_calib_workspace(4096, 5446)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     dummy = torch.zeros(16, dtype=torch.int32, device="cuda")
-    rc = L.hif4_calib_percentile_mask_noalloc(_p(dummy), 16, C, C, 999, 1000, 1, 100, _p(dummy), _p(dummy),
-                                              _p(dummy), None, stream)
-    assert rc == 4                                           # HIF4_ERR_WORKSPACE, nothing launched
+    for T, C in ((4096, 5446), (16, 1 << 15)):
+        assert L.hif4_calib_workspace(T, C) > cap
+        rc = L.hif4_calib_percentile_mask_noalloc(_p(dummy), T, C, C, 999, 1000, 1, 100, _p(dummy), _p(dummy),
+                                                  _p(dummy), None, stream)
+        assert rc == 4                                       # HIF4_ERR_WORKSPACE, nothing launched
