@@ -60,10 +60,14 @@ SIGNATURES = {
     "hif4_ptq_state_pack": (ctypes.c_int, [_I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ]),
     "hif4_ptq_state_info": (ctypes.c_int, [_P, _SZ, _P, _P, _P]),
     "hif4_ptq_state_unpack": (ctypes.c_int, [_P, _SZ, _P, _P, _P, _P]),
+    "hif4_to_e4m3": (ctypes.c_int, [_P, _P, _I64, _I64, _P, _I64, _P, _I64, _P]),
+    "hif4_gemm_f8": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I64, _P, _I64, _P, _I64, _U32, _P,
+                                    _P]),
     "hif4_debug_wait_test": (None, [ctypes.c_uint32, ctypes.c_uint64]),
     "hif4_get_status": (ctypes.c_int, [_P, _P]),
     "hif4_reset_status": (ctypes.c_int, [_P, _P]),
     "hif4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "hif4_last_cuda_error": (ctypes.c_char_p, []),
     "hif4_version": (ctypes.c_int, []),
 }
 
@@ -75,6 +79,8 @@ class Hif4Error(RuntimeError):
     def __init__(self, fn, code):
         self.code = code
         msg = lib().hif4_status_string(code).decode()
+        if code == ERR_CUDA:
+            msg += ": " + lib().hif4_last_cuda_error().decode()
         super().__init__("%s failed: status %d (%s)" % (fn, code, msg))
 
 
@@ -213,6 +219,37 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None
     _check("hif4_gemm_bf16", lib().hif4_gemm_bf16(
         _ptr(a), M, K, a.stride(0), _ptr(b), N, b.stride(0), _ptr(bias), _ptr(out), out.stride(0),
         flags, _ptr(status), _stream(stream)))
+    return out
+
+
+def to_e4m3(codes: torch.Tensor, meta: torch.Tensor, cols: int, *, pad_rows: int = 1, out=None, stream=None):
+    """HiF4 codes -> (E4M3 bytes uint8 [rows, cols], unit scales FP32 [cols/64, lds]),
+    lds = rows rounded up to `pad_rows` (128 for the FP8 GEMM's A, 256 for its B)."""
+    _dev(codes, "codes")
+    rows = codes.shape[0]
+    lds = -(-rows // pad_rows) * pad_rows
+    if out is None:
+        out = (torch.empty(rows, cols, dtype=torch.uint8, device=codes.device),
+               torch.zeros(cols // 64, lds, dtype=torch.float32, device=codes.device))
+    q8, sc = out
+    _check("hif4_to_e4m3", lib().hif4_to_e4m3(_ptr(codes), _ptr(meta), rows, cols, _ptr(q8), q8.stride(0),
+                                              _ptr(sc), sc.stride(0), _stream(stream)))
+    return q8, sc
+
+
+def gemm_f8(a: torch.Tensor, sa: torch.Tensor, b: torch.Tensor, sb: torch.Tensor, *, out=None, out_f32=False,
+            status=None, stream=None):
+    """y = sum over units of sa sb (a_u · b_uᵀ) on the FP8 tensor cores (E4M3
+    operands from to_e4m3, FP32 unit scales, FP32 promotion)."""
+    _dev(a, "a")
+    M, K = a.shape
+    N = b.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32 if out_f32 else torch.bfloat16, device=a.device)
+    flags = LINEAR_OUT_F32 if out.dtype == torch.float32 else 0
+    _check("hif4_gemm_f8", lib().hif4_gemm_f8(_ptr(a), M, K, a.stride(0), _ptr(sa), sa.stride(0), _ptr(b), N,
+                                              b.stride(0), _ptr(sb), sb.stride(0), _ptr(out), out.stride(0), flags,
+                                              _ptr(status), _stream(stream)))
     return out
 
 

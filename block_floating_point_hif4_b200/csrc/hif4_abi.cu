@@ -80,6 +80,30 @@ bool make_tensor_map_bf16_2d(CUtensorMap *map, const void *base, uint64_t inner,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 8-bit 2-D tensor map with 128-byte swizzle (the FP8 GEMM's operands).
+bool make_tensor_map_u8_2d_sw128(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_encode) {
+            void *p = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                g_encode = reinterpret_cast<EncodeTiledFn>(p);
+        }
+    }
+    if (!g_encode) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)row_stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // FP32 2-D tensor map with 128-byte swizzle (the HiGPTQ update's operands).
 bool make_tensor_map_f32_2d_sw128(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer)
@@ -145,6 +169,23 @@ extern "C" hif4_status hif4_reset_status(uint32_t *status_word, hif4_stream_t st
     if (cudaMemsetAsync(status_word, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return HIF4_ERR_CUDA;
     return HIF4_OK;
+}
+
+namespace hif4 {
+namespace {
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+} // namespace
+
+hif4_status cuda_failed(cudaError_t e)
+{
+    t_last_cuda_error = e;
+    return HIF4_ERR_CUDA;
+}
+} // namespace hif4
+
+extern "C" const char *hif4_last_cuda_error(void)
+{
+    return hif4::t_last_cuda_error == cudaSuccess ? "" : cudaGetErrorName(hif4::t_last_cuda_error);
 }
 
 extern "C" const char *hif4_status_string(hif4_status s)

@@ -23,10 +23,14 @@ namespace hif4 {
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned_to(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Records the CUDA runtime error behind an HIF4_ERR_CUDA return (per host
+// thread; hif4_last_cuda_error reports it) and returns HIF4_ERR_CUDA.
+hif4_status cuda_failed(cudaError_t e);
+
 inline hif4_status launch_status()
 {
     cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? HIF4_OK : HIF4_ERR_CUDA;
+    return e == cudaSuccess ? HIF4_OK : cuda_failed(e);
 }
 
 // Number of SMs of the current device (cached per device ordinal).

@@ -195,6 +195,45 @@ hif4_status hif4_gemm_bf16_fq(const void *a, int64_t M, int64_t K, int64_t lda, 
                               int64_t ldy, uint32_t flags, uint32_t *status, hif4_stream_t stream);
 
 /*
+ * hif4_to_e4m3 — exact remap of HiF4 codes onto FP8 E4M3 plus one FP32 scale
+ * per 64-element unit [HiF4 format: an element is (-1)^s (m/4) 2^(e2+e3) S;
+ * m/4 2^E with m <= 7, E <= 2 has at most three significant bits]:
+ *   q8[r][c]          = E4M3 byte of (-1)^s (m/4) 2^E (0x00 for m = 0),
+ *   scale[u * lds + r] = S, the E6M2 value of unit u of row r (FP32, exact),
+ * so that q8 * scale is hif4_dequantize's value, bit for bit.  codes / meta
+ * as hif4_quantize writes them (rows x cols/2, rows x cols/64, dense).
+ * q8 rows x cols bytes (ldq, a multiple of 8; 8-byte aligned); scale is
+ * K-unit-major, (cols/64) x lds FP32, lds >= rows, 4-byte aligned; entries
+ * of rows >= `rows` are left untouched.
+ * Errors: SHAPE (cols % 64, ldq < cols, lds < rows), ALIGNMENT, INVALID_ARG.
+ */
+hif4_status hif4_to_e4m3(const uint8_t *codes, const uint32_t *meta, int64_t rows, int64_t cols, uint8_t *q8,
+                         int64_t ldq, float *scale, int64_t lds, hif4_stream_t stream);
+
+/*
+ * hif4_gemm_f8 — the W4A4 HiF4 product on the FP8 tensor cores [HiF4 format;
+ * TA abstract: W4A4 fake-quantized linears]:
+ *   y[m][n] = sum over units u of  sa[u][m] sb[u][n] sum_{k in u} a[m][k] b[n][k]
+ * with a, b E4M3 operands (hif4_to_e4m3 of HiF4 codes) and the unit scales
+ * applied in FP32 after each unit's 64-deep FP8 product (tcgen05 kind::f8f6f4,
+ * FP32 accumulation; exact for HiF4 operands, see the source), FP32 or BF16
+ * (round to nearest even) out.  Protected channels are not covered: they are
+ * the BF16 linear's job (hif4_gemm_bf16).
+ * a  M x K E4M3 bytes (lda >= K, a multiple of 16), sa (K/64) x lds_a FP32,
+ *    lds_a >= M rounded up to 128 (rows past M are read, never affect y);
+ * b  N x K E4M3 bytes (ldb), sb (K/64) x lds_b FP32, lds_b >= N rounded up to
+ *    256; all 16-byte aligned, lds_a and lds_b multiples of 4.
+ * flags  0 (BF16 y) or HIF4_LINEAR_OUT_F32.
+ * Errors: SHAPE (K % 64, K < 128, leading dimensions), ALIGNMENT,
+ * INVALID_ARG, UNSUPPORTED (sizes, or a layout the driver's tensor-map
+ * encoder refuses).  Bounded waits raise HIF4_FLAG_TIMEOUT as
+ * hif4_gemm_bf16.
+ */
+hif4_status hif4_gemm_f8(const uint8_t *a, int64_t M, int64_t K, int64_t lda, const float *sa, int64_t lds_a,
+                         const uint8_t *b, int64_t N, int64_t ldb, const float *sb, int64_t lds_b, void *y,
+                         int64_t ldy, uint32_t flags, uint32_t *status, hif4_stream_t stream);
+
+/*
  * hif4_ffn_w4a4 — the W4A4 HiF4 feed-forward block of a DiT layer [TA
  * abstract: fake-quantized main linears, protected channels in BF16; the
  * tanh-form GELU between them is the library's reading]:
@@ -427,6 +466,10 @@ hif4_status hif4_get_status(const uint32_t *status_word, hif4_stream_t stream);
 hif4_status hif4_reset_status(uint32_t *status_word, hif4_stream_t stream);
 
 const char *hif4_status_string(hif4_status s);
+/* Name of the last CUDA runtime error that made a call of this host thread
+ * return HIF4_ERR_CUDA where the call records it (every kernel launch; ""
+ * when none was recorded): a diagnostic beside the status code. */
+const char *hif4_last_cuda_error(void);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int hif4_version(void);
 
