@@ -514,6 +514,9 @@ def main():
                                                  "channels; activation fake-quant, weight decode and GEMM all "
                                                  "timed"}
         del xa, wa, wac, wam, wak, ba, ya, aws
+        torch.cuda.empty_cache()
+        comps["fp8_remap_gemm"] = fp8_remap_vs_bf16(H, wl, dev, rank, args, stream, barrier, max_over_ranks,
+                                                     world, P)
         line["components"] = comps
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             add_cpu_component_rates(comps)
@@ -562,6 +565,36 @@ def add_cpu_component_rates(comps):
     comps["calib_percentile_mask"]["cpu_baseline"] = {"value": c, "unit": "GB/s", "cores": thr, "kind": "oracle",
                                                       "sample": "14400 tokens x 512 channels of the calibration "
                                                                 "recipe, percentiles (sort per channel)"}
+
+
+def fp8_remap_vs_bf16(H, wl, dev, rank, args, stream, barrier, max_over_ranks, world, P):
+    """The first FFN GEMM's product (57600 x 13824 x 5120, no protected
+    channels) on the FP8 tensor cores with the exact E4M3 remap and per-unit
+    FP32 promotion (hif4_gemm_f8), timed beside the BF16 tcgen05 GEMM on the
+    same dequantized operands (hif4_gemm_bf16); both write BF16."""
+    import torch
+
+    from block_floating_point_hif4_b200 import sharding
+    M, D, F = args.tokens, D_MODEL, D_FFN
+    x, _ = wl.device_rows(M, D, seed=sharding.rank_seed(3, rank), device=dev)
+    w = wl.device_weight(F, D, 0.015, seed=31, device=dev)
+    ca, ma = H.quantize(x)
+    cb, mb = H.quantize(w)
+    del x, w
+    qa, sa = H.to_e4m3(ca, ma, D, pad_rows=128)
+    qb, sb = H.to_e4m3(cb, mb, D, pad_rows=256)
+    ah, bh = H.dequantize(ca, ma, D), H.dequantize(cb, mb, D)
+    y = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+    flop = 2.0 * M * F * D
+    r8 = time_op(lambda: H.gemm_f8(qa, sa, qb, sb, out=y), args, stream, barrier, max_over_ranks, world, 0.0, P)
+    r16 = time_op(lambda: H.gemm_bf16(ah, bh, out=y), args, stream, barrier, max_over_ranks, world, 0.0, P)
+    del ca, ma, cb, mb, qa, sa, qb, sb, ah, bh, y
+    torch.cuda.empty_cache()
+    tf8, tf16 = world * flop / (r8["ms"] * 1e-3) / 1e12, world * flop / (r16["ms"] * 1e-3) / 1e12
+    return {"value": tf8, "unit": "TFLOP/s", "ms": r8["ms"], "bound": "alu (per-unit FP32 promotion)",
+            "bf16_ms": r16["ms"], "bf16_value": tf16, "speedup_vs_bf16": r16["ms"] / r8["ms"],
+            "workload": "hif4_gemm_f8 57600 x 13824 x 5120 (E4M3 remap, per-unit FP32 scales, BF16 out) "
+                        "beside hif4_gemm_bf16 on the dequantized operands"}
 
 
 def quant_sweep(H, wl, dev, stream, args, barrier, max_over_ranks, world, P):

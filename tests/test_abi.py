@@ -165,3 +165,28 @@ def test_higptq_hessian_and_host_ffn_argument_errors(L):
     assert ffn_host(F=100) == 3
     assert ffn_host(wsb=64) == 4
     assert ffn_host(M=0) == 0            # nothing to do
+
+
+def test_fp8_remap_and_gemm_argument_errors(L):
+    P = ctypes.c_void_p
+    fake = P(0x1000)          # never dereferenced: every call below fails validation first
+    assert L.hif4_to_e4m3(fake, fake, 4, 100, fake, 128, fake, 4, None) == 3      # cols % 64
+    assert L.hif4_to_e4m3(fake, fake, 4, 128, fake, 64, fake, 4, None) == 3       # ldq < cols
+    assert L.hif4_to_e4m3(fake, fake, 4, 128, fake, 128, fake, 3, None) == 3      # lds < rows
+    assert L.hif4_to_e4m3(P(0x1001), fake, 4, 128, fake, 128, fake, 4, None) == 2  # codes misaligned
+    assert L.hif4_to_e4m3(fake, fake, 0, 128, fake, 128, fake, 0, None) == 0      # nothing to do
+
+    def f8(M=200, K=256, lda=256, sa=fake, lds_a=256, N=300, ldb=256, sb=fake, lds_b=512, y=fake, ldy=300,
+           flags=0):
+        return L.hif4_gemm_f8(fake, M, K, lda, sa, lds_a, fake, N, ldb, sb, lds_b, y, ldy, flags, None, None)
+
+    assert f8(K=100, lda=128, ldb=128) == 3      # K % 64
+    assert f8(K=64, lda=64, ldb=64) == 3         # K below the 128-byte operand box
+    assert f8(lds_a=200) == 3                    # row scales not padded to 128 rows
+    assert f8(lds_b=300) == 3                    # column scales not padded to 256 columns
+    assert f8(lda=200) == 3                      # lda < K
+    assert f8(lda=264) == 2                      # lda not a multiple of 16 bytes
+    assert f8(sa=P(0x1004)) == 2                 # scales not 16-byte aligned
+    assert f8(flags=1) == 1                      # GELU is not an option of this product
+    assert f8(y=None) == 1
+    assert f8(M=0) == 0
