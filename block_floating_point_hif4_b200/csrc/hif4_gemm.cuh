@@ -37,14 +37,15 @@ struct Args {
     uint32_t *status;
     uint64_t timeout_ns;
     uint32_t withhold;      // block 0 withholds its first copy (failure-handling test)
+    int group_m;            // m-tiles per rasterization group
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Args &g, int &mb, int &nb)
 {
-    const int per_group = GROUP_M * g.num_n;
+    const int per_group = g.group_m * g.num_n;
     const int gi = t / per_group;
-    const int first_m = gi * GROUP_M;
-    const int gm = min(g.num_m - first_m, GROUP_M);
+    const int first_m = gi * g.group_m;
+    const int gm = min(g.num_m - first_m, g.group_m);
     const int r = t - gi * per_group;
     mb = first_m + r % gm;
     nb = r / gm;
@@ -93,6 +94,135 @@ __device__ __forceinline__ void epi_pack32(const uint32_t (&r)[32], const uint16
     for (int j = 0; j < 16; ++j) {
         __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
         w[j] = *reinterpret_cast<uint32_t *>(&h2);
+    }
+}
+
+// One accumulator's rows of this warp's TMEM lane quarter (tacc: lane
+// quarter and accumulator column base) -> output row `row` (stored only if
+// row < M), columns nb * BN ... + BN - 1: + bias, optional tanh-GELU, FP32,
+// or BF16 (round to nearest even) with optional HiF4 fake quantization of
+// the row's 64-column units.
+__device__ __forceinline__ void store_tile_rows(const Args &g, uint32_t tacc, int row, int nb, uint32_t &nonfinite)
+{
+    using namespace sm100;
+    const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
+    const bool out_f32 = (g.flags & HIF4_LINEAR_OUT_F32) != 0;
+    const bool fq_out = (g.flags & HIF4_LINEAR_FAKE_QUANT_OUT) != 0;
+    uint16_t *yrow = static_cast<uint16_t *>(g.y) + (int64_t)row * g.ldy;
+    float *yrow32 = static_cast<float *>(g.y) + (int64_t)row * g.ldy;
+    // HiF4 fake-quant of the output along N: a thread holds whole
+    // 64-column units of its row (N % 64 == 0), so every unit
+    // decision is thread-local.
+#pragma unroll 1
+    for (int u = 0; fq_out && u < BN / 64; ++u) {
+        const int n0 = nb * BN + u * 64;
+        if (n0 >= g.N) break;                          // warp-uniform
+        uint32_t w[32];
+        {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tacc + u * 64, r);
+            tmem_ld_wait();
+            epi_pack32(r, g.bias ? g.bias + n0 : nullptr, gelu, w);
+            tmem_ld_32x32b_x32(tacc + u * 64 + 32, r);
+            tmem_ld_wait();
+            epi_pack32(r, g.bias ? g.bias + n0 + 32 : nullptr, gelu, w + 16);
+        }
+        uint32_t out[32];
+        uint32_t mraw[16];
+        uint32_t any = 0;
+        if (g.out_mask) {
+            const uint4 *mp = reinterpret_cast<const uint4 *>(g.out_mask + n0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 m = __ldg(mp + i);
+                mraw[4 * i] = m.x;
+                mraw[4 * i + 1] = m.y;
+                mraw[4 * i + 2] = m.z;
+                mraw[4 * i + 3] = m.w;
+                any |= m.x | m.y | m.z | m.w;
+            }
+        }
+        if (any) {                                     // warp-uniform: same columns
+            uint32_t mw[32];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) enc::mask_words16(mraw + 4 * i, mw + 8 * i);
+            enc::fq_unit64<true>(w, mw, out, nonfinite);
+        } else {
+            enc::fq_unit64<false>(w, w, out, nonfinite);
+        }
+        if (row < g.M) {
+            uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+        }
+    }
+#pragma unroll 1
+    for (int c = 0; !fq_out && c < BN / 32; ++c) {
+        const int n0 = nb * BN + c * 32;
+        if (n0 >= g.N) break;                          // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tacc + c * 32, r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (g.bias) {
+            if (n0 + 32 <= g.N) {
+                const uint4 *bp = reinterpret_cast<const uint4 *>(g.bias + n0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 b = __ldg(bp + i);
+                    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        v[8 * i + 2 * h] += __uint_as_float(bw[h] << 16);
+                        v[8 * i + 2 * h + 1] += __uint_as_float(bw[h] & 0xFFFF0000u);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (n0 + j < g.N) v[j] += __uint_as_float((uint32_t)g.bias[n0 + j] << 16);
+            }
+        }
+        if (gelu) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+        }
+        if (out_f32) {
+            if (row < g.M) {
+                if (n0 + 32 <= g.N) {
+                    float4 *dst = reinterpret_cast<float4 *>(yrow32 + n0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (n0 + j < g.N) yrow32[n0 + j] = v[j];
+                }
+            }
+            continue;
+        }
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            packed[j] = *reinterpret_cast<uint32_t *>(&h2);
+        }
+        if (row < g.M) {
+            if (n0 + 32 <= g.N) {
+                uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (n0 + j < g.N) yrow[n0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
+            }
+        }
     }
 }
 
@@ -218,9 +348,6 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     } else {
         // -------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
-        const bool out_f32 = (g.flags & HIF4_LINEAR_OUT_F32) != 0;
-        const bool fq_out = (g.flags & HIF4_LINEAR_FAKE_QUANT_OUT) != 0;
         uint32_t nonfinite = 0;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
@@ -228,124 +355,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             tile_coords(t, g, mb, nb);
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, g.timeout_ns)) break;
             tc_fence_after();
-            const int row = mb * BM + q * 32 + lane;
-            uint16_t *yrow = static_cast<uint16_t *>(g.y) + (int64_t)row * g.ldy;
-            float *yrow32 = static_cast<float *>(g.y) + (int64_t)row * g.ldy;
-            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            // HiF4 fake-quant of the output along N: a thread holds whole
-            // 64-column units of its row (N % 64 == 0), so every unit
-            // decision is thread-local.
-#pragma unroll 1
-            for (int u = 0; fq_out && u < BN / 64; ++u) {
-                const int n0 = nb * BN + u * 64;
-                if (n0 >= g.N) break;                          // warp-uniform
-                uint32_t w[32];
-                {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tacc + u * 64, r);
-                    tmem_ld_wait();
-                    epi_pack32(r, g.bias ? g.bias + n0 : nullptr, gelu, w);
-                    tmem_ld_32x32b_x32(tacc + u * 64 + 32, r);
-                    tmem_ld_wait();
-                    epi_pack32(r, g.bias ? g.bias + n0 + 32 : nullptr, gelu, w + 16);
-                }
-                uint32_t out[32];
-                uint32_t mraw[16];
-                uint32_t any = 0;
-                if (g.out_mask) {
-                    const uint4 *mp = reinterpret_cast<const uint4 *>(g.out_mask + n0);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 m = __ldg(mp + i);
-                        mraw[4 * i] = m.x;
-                        mraw[4 * i + 1] = m.y;
-                        mraw[4 * i + 2] = m.z;
-                        mraw[4 * i + 3] = m.w;
-                        any |= m.x | m.y | m.z | m.w;
-                    }
-                }
-                if (any) {                                     // warp-uniform: same columns
-                    uint32_t mw[32];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) enc::mask_words16(mraw + 4 * i, mw + 8 * i);
-                    enc::fq_unit64<true>(w, mw, out, nonfinite);
-                } else {
-                    enc::fq_unit64<false>(w, w, out, nonfinite);
-                }
-                if (row < g.M) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
-                }
-            }
-#pragma unroll 1
-            for (int c = 0; !fq_out && c < BN / 32; ++c) {
-                const int n0 = nb * BN + c * 32;
-                if (n0 >= g.N) break;                          // warp-uniform
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
-                tmem_ld_wait();
-                float v[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                if (g.bias) {
-                    if (n0 + 32 <= g.N) {
-                        const uint4 *bp = reinterpret_cast<const uint4 *>(g.bias + n0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint4 b = __ldg(bp + i);
-                            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                v[8 * i + 2 * h] += __uint_as_float(bw[h] << 16);
-                                v[8 * i + 2 * h + 1] += __uint_as_float(bw[h] & 0xFFFF0000u);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (n0 + j < g.N) v[j] += __uint_as_float((uint32_t)g.bias[n0 + j] << 16);
-                    }
-                }
-                if (gelu) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
-                }
-                if (out_f32) {
-                    if (row < g.M) {
-                        if (n0 + 32 <= g.N) {
-                            float4 *dst = reinterpret_cast<float4 *>(yrow32 + n0);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (n0 + j < g.N) yrow32[n0 + j] = v[j];
-                        }
-                    }
-                    continue;
-                }
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-                    packed[j] = *reinterpret_cast<uint32_t *>(&h2);
-                }
-                if (row < g.M) {
-                    if (n0 + 32 <= g.N) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + n0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (n0 + j < g.N) yrow[n0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
-                    }
-                }
-            }
+            store_tile_rows(g, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, mb * BM + q * 32 + lane, nb,
+                            nonfinite);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -361,6 +372,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
     if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
 }
+
 
 // ----------------------------------------------------------- host helpers
 

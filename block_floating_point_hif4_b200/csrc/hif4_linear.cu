@@ -92,16 +92,12 @@ hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const 
                         uint32_t *status, cudaStream_t s)
 {
     using namespace gemm;
-    CUtensorMap tmA, tmB;
-    if (!make_map(&tmA, a, M, K, lda, BM) || !make_map(&tmB, b, N, K, ldb, BN)) return HIF4_ERR_CUDA;
     Args g{};
     g.M = (int)M;
     g.N = (int)N;
     g.K = (int)K;
-    g.num_m = (int)((M + BM - 1) / BM);
     g.num_n = (int)((N + BN - 1) / BN);
     g.num_k = (int)(K / BK);
-    g.num_tiles = g.num_m * g.num_n;
     g.bias = static_cast<const uint16_t *>(bias);
     g.y = y;
     g.ldy = ldy;
@@ -110,12 +106,17 @@ hif4_status launch_gemm(const void *a, int64_t M, int64_t K, int64_t lda, const 
     g.status = status;
     g.timeout_ns = wait_limit_ns(TIMEOUT_NS);
     g.withhold = wait_test_withhold();
-    static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
+    static bool attr_set[64] = {false};
+    CUtensorMap tmA, tmB;
+    if (!make_map(&tmA, a, M, K, lda, BM) || !make_map(&tmB, b, N, K, ldb, BN)) return HIF4_ERR_CUDA;
+    g.num_m = (int)((M + BM - 1) / BM);
+    g.num_tiles = g.num_m * g.num_n;
+    g.group_m = GROUP_M;
     if (!attr_set[dev & 63]) {
-        if (cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
-            return HIF4_ERR_CUDA;
+        const cudaError_t e = cudaFuncSetAttribute(k_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_failed(e);
         attr_set[dev & 63] = true;
     }
     int grid = sm_count();
