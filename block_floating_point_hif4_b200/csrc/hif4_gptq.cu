@@ -504,7 +504,9 @@ struct GptqArgs {
     uint8_t *codes;          // N x K/2
     uint32_t *meta;          // N x K/64
     uint16_t *w_masked;      // N x n_masked
-    float *Eh, *El;          // N x 64 NG: the block's error E = D U_gg^{-1} as TF32 parts (hi + lo)
+    float *Eh, *El;          // the block's error E = D U_gg^{-1} as TF32 parts (hi + lo): its 64 NG
+                             // columns start at column e0 of N x ldE arrays (one per super-block)
+    int64_t ldE, e0;
 };
 
 // One block of NG groups (64 NG columns) for kRowsPerBlock rows (each warp
@@ -599,7 +601,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
             {
                 // E in two TF32 parts: the lazy update's split operand
                 const uint32_t h0 = tf32_rna(e0), h1 = tf32_rna(e1);
-                const int64_t o = n * (64 * NG) + 64 * g + 2 * lane;
+                const int64_t o = n * a.ldE + a.e0 + 64 * g + 2 * lane;
                 *reinterpret_cast<float2 *>(a.Eh + o) = make_float2(__uint_as_float(h0), __uint_as_float(h1));
                 *reinterpret_cast<float2 *>(a.El + o) = make_float2(__uint_as_float(tf32_rna(e0 - __uint_as_float(h0))),
                                                                   __uint_as_float(tf32_rna(e1 - __uint_as_float(h1))));
@@ -666,11 +668,13 @@ constexpr uint32_t kUTmemCols = 2 * UBN;
 constexpr uint64_t kUWaitNs = 2000000000ull;
 
 struct UpdArgs {
-    float *W;                // C = W[:, b1:], row-major, ld ldw
-    int64_t ldw, M, Nc;      // rows of W; columns after the block (a multiple of 64)
-    int b0, b1, nkb;         // the block [b0, b1) of K; 32-deep k-blocks
+    float *W;                // C = W[:, b1 : b1 + Nc], row-major, ld ldw
+    int64_t ldw, M, Nc;      // rows of W; columns updated (a multiple of 64)
+    int b0, b1, nkb;         // the error's rows of U start at b0 (its columns of K); first column of C;
+                             // 32-deep k-blocks
     int num_m, num_tiles;    // 128-row tiles of W; all tiles
     uint32_t *status;
+    int a0;                  // first column of the error in the E arrays
 };
 
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::tf32 (FP32 in smem read as TF32, FP32 accumulate).
@@ -748,8 +752,8 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
                     }
                     uint8_t *st = sm + stage * kUStage;
                     mbar_arrive_expect_tx(&full[stage], kUStage);
-                    tma_load_2d(st, &tmAh, kb * UBK, m0, &full[stage]);
-                    tma_load_2d(st + kUTile, &tmAl, kb * UBK, m0, &full[stage]);
+                    tma_load_2d(st, &tmAh, g.a0 + kb * UBK, m0, &full[stage]);
+                    tma_load_2d(st + kUTile, &tmAl, g.a0 + kb * UBK, m0, &full[stage]);
                     tma_load_2d(st + 2 * kUTile, &tmBh, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
                     tma_load_2d(st + 3 * kUTile, &tmBl, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
                     ++issued;
@@ -900,6 +904,10 @@ struct GptqLayout {
     size_t A, Y, T, U, UinvG, UTh, UTl, W, Eh, El, mask, rank, dead, mean, total;
 };
 
+// Columns of a super-block of the two-level lazy update: whole blocks, 512
+// columns when the block divides it (64, 128, 256), 576 for 192.
+int64_t super_cols(int64_t B) { return B * (512 / B > 1 ? 512 / B : 1); }
+
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
 {
     GptqLayout L{};
@@ -918,8 +926,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     take(L.UTh, k * k * 4);
     take(L.UTl, k * k * 4);
     take(L.W, (size_t)N * k * 4);
-    take(L.Eh, (size_t)N * (size_t)B * 4);
-    take(L.El, (size_t)N * (size_t)B * 4);
+    take(L.Eh, (size_t)N * (size_t)super_cols(B) * 4);
+    take(L.El, (size_t)N * (size_t)super_cols(B) * 4);
     take(L.mask, k);
     take(L.rank, k * 4);
     take(L.dead, k);
@@ -1117,42 +1125,59 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     if (!make_tensor_map_f32_2d_sw128(&mBh, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN) ||
         !make_tensor_map_f32_2d_sw128(&mBl, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN))
         return HIF4_ERR_CUDA;
-    // 3. the group loop: per block, the groups with their in-block feedback,
-    //    then the lazy update of every later column
-    for (int64_t b0 = 0; b0 < K; b0 += B) {
-        const int64_t b1 = b0 + B < K ? b0 + B : K;
-        const int NG = (int)((b1 - b0) / HIF4_UNIT);
-        GptqArgs a{};
-        a.W = W;
-        a.N = N;
-        a.K = K;
-        a.b0 = b0;
-        a.U = U;
-        a.UinvG = UinvG;
-        a.mask = n_masked > 0 ? mask : nullptr;
-        a.rank = rank;
-        a.n_masked = n_masked;
-        a.codes = codes;
-        a.meta = meta;
-        a.w_masked = static_cast<uint16_t *>(w_masked);
-        a.Eh = Eh;
-        a.El = El;
-        hif4_status st = NG == 1 ? launch_gptq_block<1>(a, s)
-                       : NG == 2 ? launch_gptq_block<2>(a, s)
-                       : NG == 3 ? launch_gptq_block<3>(a, s)
-                                 : launch_gptq_block<4>(a, s);
-        if (st != HIF4_OK) return st;
-        if (b1 < K) {
-            const int64_t kd = 64 * NG;
-            CUtensorMap mAh, mAl;
-            if (!make_tensor_map_f32_2d_sw128(&mAh, Eh, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM) ||
-                !make_tensor_map_f32_2d_sw128(&mAl, El, (uint64_t)kd, (uint64_t)N, (uint64_t)kd * 4, UBK, UBM))
-                return HIF4_ERR_CUDA;
-            const int num_m = (int)((N + UBM - 1) / UBM), num_n = (int)((K - b1 + UBN - 1) / UBN);
-            UpdArgs ua{W, K, N, K - b1, (int)b0, (int)b1, (int)(kd / UBK), num_m, num_m * num_n, status};
-            const int grid = std::min(num_m * num_n, sm_count());
-            k_update_tf32<<<grid, kUThreads, kUSmem, s>>>(mAh, mAl, mBh, mBl, ua);
-            if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    // 3. the group loop, a two-level lazy update: within a super-block of
+    //    S columns (whole blocks), each block's groups (with their in-block
+    //    feedback), then the rest of the super-block updated by the block's
+    //    error; after the super-block, every later column updated once by
+    //    the super-block's whole error.  The same sum as GPTQ's per-block
+    //    update, reordered; W's later columns are read and written once per
+    //    super-block instead of once per block.
+    const int64_t S = super_cols(B);
+    CUtensorMap mAh, mAl;
+    if (!make_tensor_map_f32_2d_sw128(&mAh, Eh, (uint64_t)S, (uint64_t)N, (uint64_t)S * 4, UBK, UBM) ||
+        !make_tensor_map_f32_2d_sw128(&mAl, El, (uint64_t)S, (uint64_t)N, (uint64_t)S * 4, UBK, UBM))
+        return HIF4_ERR_CUDA;
+    auto update = [&](int64_t a0, int64_t k0, int64_t k1, int64_t c0, int64_t c1) -> hif4_status {
+        // W[:, c0:c1] -= E[:, a0 : a0 + k1 - k0] U[k0:k1, c0:c1]
+        const int num_m = (int)((N + UBM - 1) / UBM), num_n = (int)((c1 - c0 + UBN - 1) / UBN);
+        UpdArgs ua{W, K, N, c1 - c0, (int)k0, (int)c0, (int)((k1 - k0) / UBK), num_m, num_m * num_n, status,
+                   (int)a0};
+        const int grid = std::min(num_m * num_n, sm_count());
+        k_update_tf32<<<grid, kUThreads, kUSmem, s>>>(mAh, mAl, mBh, mBl, ua);
+        return launch_status();
+    };
+    for (int64_t s0 = 0; s0 < K; s0 += S) {
+        const int64_t s1 = s0 + S < K ? s0 + S : K;
+        for (int64_t b0 = s0; b0 < s1; b0 += B) {
+            const int64_t b1 = b0 + B < s1 ? b0 + B : s1;
+            const int NG = (int)((b1 - b0) / HIF4_UNIT);
+            GptqArgs a{};
+            a.W = W;
+            a.N = N;
+            a.K = K;
+            a.b0 = b0;
+            a.U = U;
+            a.UinvG = UinvG;
+            a.mask = n_masked > 0 ? mask : nullptr;
+            a.rank = rank;
+            a.n_masked = n_masked;
+            a.codes = codes;
+            a.meta = meta;
+            a.w_masked = static_cast<uint16_t *>(w_masked);
+            a.Eh = Eh;
+            a.El = El;
+            a.ldE = S;
+            a.e0 = b0 - s0;
+            hif4_status st = NG == 1 ? launch_gptq_block<1>(a, s)
+                           : NG == 2 ? launch_gptq_block<2>(a, s)
+                           : NG == 3 ? launch_gptq_block<3>(a, s)
+                                     : launch_gptq_block<4>(a, s);
+            if (st != HIF4_OK) return st;
+            if (b1 < s1 && (st = update(b0 - s0, b0, b1, b1, s1)) != HIF4_OK) return st;
+        }
+        if (s1 < K) {
+            const hif4_status st = update(0, s0, s1, s1, K);
+            if (st != HIF4_OK) return st;
         }
     }
     return HIF4_OK;

@@ -13,12 +13,12 @@ in its workspace, hif4_higptq1_group_inputs_offset):
   * feedback: those values equal, within FP32 rounding, the FP64 GPTQ update
     W0_h - sum_{g<h} E_g U_{g,h}, with E_g = (W_g - Q_g) U_gg^-1 computed in
     FP64 from the GPU's own W_g and Q_g and U the oracle's FP64 factor.  The
-    bound is 2^-14 x (|W0| + (|D| |U_gg^-1|) |U_{g,h}|) summed in absolute
-    values: twice the worst case of the GPU's arithmetic (FP32 rounding of U,
-    <= 384-term FP32 accumulations of split-TF32 products per update launch
-    and <= 64-term ones for E, one rounding of W per block: about 2^-15 of
-    that sum).  A dropped term, a wrong sign or a wrong index moves some
-    element by a sizeable fraction of the sum itself.
+    bound is 2^-12 x (|W0| + (|D| |U_gg^-1|) |U_{g,h}|) summed in absolute
+    values: about twice the worst case of the GPU's arithmetic (FP32 rounding
+    of U, <= 1536-term FP32 accumulations of split-TF32 products per update
+    launch, <= 64-term ones for E, one rounding of W per update: about
+    2^-13.3 of that sum).  A dropped term, a wrong sign or a wrong index
+    moves some element by a sizeable fraction of the sum itself.
 And against the oracle's own FP64 run, end to end:
   * the first 64-column group of every row has received no feedback: its
     codes and metadata are bit-exact;
