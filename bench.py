@@ -51,9 +51,11 @@ DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}                # B200 dat
 # DRAM traffic per launch from an ncu capture, keyed by the SHA-256 (first 16
 # hex digits) of the kernel source it was taken on; stale entries read as null.
 NCU_TRAFFIC = {
-    # bench FFN step, 57600 tokens: GEMM 1 (fused fake-quant epilogue) read 4.71 GB + wrote 1.59 GB,
-    # GEMM 2 read 9.21 GB + wrote 0.58 GB (one ncu pass, dram__bytes_read/write.sum); mean per launch
-    ("gemm", "35fde63dfbb6ccaf"): 8.046e9,
+    # the FFN's two GEMMs on 8192 of the 57600 tokens (one ncu pass, dram__bytes_read/write.sum):
+    # GEMM 1 (fused fake-quant epilogue) read 664 MB + wrote 207 MB, GEMM 2 read 1283 MB + wrote 81 MB;
+    # every term grows with the rows (A and C once, the weight once per 2048 rows), so x 57600 / 8192:
+    # 6.13 and 9.59 GB, mean per launch
+    ("gemm", "b9d6f95439ebc864"): 7.859e9,
 }
 
 
