@@ -27,6 +27,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <mutex>
+#include <vector>
 
 #include "hif4_encode.cuh"
 #include "hif4_internal.cuh"
@@ -470,8 +472,43 @@ __global__ void k_mask_rank(const int32_t *idx, int n, int64_t K, uint8_t *mask,
 
 // W32 = BF16 w widened (dead input channels zeroed; NaN -> 0, +-Inf ->
 // +-FLT_MAX as the quantizer maps them, flagged).
+// W32 = BF16 w widened (dead input channels zeroed; NaN -> 0, +-Inf ->
+// +-FLT_MAX as the quantizer maps them, flagged).  A thread converts 8
+// consecutive elements of a row (one 16-byte load, two 16-byte stores; K and
+// ldw are multiples of 8 and w 16-byte aligned on this path), rows and
+// column octets in a grid-stride loop with one 32-bit division per octet.
 __global__ void k_w_to_f32(const uint16_t *w, int64_t ldw, int64_t N, int64_t K, const uint8_t *dead, float *W,
                            uint32_t *status)
+{
+    uint32_t bad = 0;
+    const uint32_t opr = (uint32_t)(K / 8);
+    const int64_t total = N * (int64_t)opr;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / opr;
+        const int64_t k = (i - n * opr) * 8;
+        const uint4 v = *reinterpret_cast<const uint4 *>(w + n * ldw + k);
+        const uint2 dk = *reinterpret_cast<const uint2 *>(dead + k);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            f[2 * j] = sanitize(bf16_lo(vw[j]), bad);
+            f[2 * j + 1] = sanitize(bf16_hi(vw[j]), bad);
+        }
+        const uint32_t dw[2] = {dk.x, dk.y};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if ((dw[j >> 2] >> (8 * (j & 3))) & 0xFFu) f[j] = 0.0f;
+        float4 *o = reinterpret_cast<float4 *>(W + n * K + k);
+        o[0] = make_float4(f[0], f[1], f[2], f[3]);
+        o[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    if (bad && status) atomicOr(status, HIF4_FLAG_NONFINITE);
+}
+
+// Any layout (2-byte aligned w, any ldw): one element per thread.
+__global__ void k_w_to_f32_any(const uint16_t *w, int64_t ldw, int64_t N, int64_t K, const uint8_t *dead, float *W,
+                               uint32_t *status)
 {
     uint32_t bad = 0;
     const int64_t total = N * K;
@@ -509,23 +546,25 @@ struct GptqArgs {
     int64_t ldE, e0;
 };
 
-// One block of NG groups (64 NG columns) for kRowsPerBlock rows (each warp
-// takes kRowsPerWarp of them in turn, after one load of the U tiles), a warp per
-// row; lane l holds elements 2l, 2l+1 of each group.  Per group: the exact
-// FP32 unit quantization (encode rule of the streaming quantizer), D = W - Q,
-// E = D Uinv_g (Uinv_g upper), feedback into the block's later groups.  The
-// values a later group is quantized from (after the in-block feedback) are
-// written back over its columns of W, so that on return W holds, for every
-// group, exactly the weights that group was quantized from (later blocks
-// never touch earlier columns).
+// One block of NG groups (64 NG columns) for kRowsPerBlock rows, a warp per
+// kRowsPerWarp consecutive rows taken in lockstep (each U tile element read
+// from shared memory serves all of them); lane l holds elements 2l, 2l+1 of
+// each group of each row.  Per group: the exact FP32 unit quantization
+// (encode rule of the streaming quantizer), D = W - Q, E = D Uinv_g (Uinv_g
+// upper), feedback into the block's later groups.  The values a later group
+// is quantized from (after the in-block feedback) are written back over its
+// columns of W, so that on return W holds, for every group, exactly the
+// weights that group was quantized from (later blocks never touch earlier
+// columns).
 template <int NG>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
 {
     constexpr int NP = NG * (NG - 1) / 2;     // U tiles (g, h), g < h
+    constexpr int R = kRowsPerWarp;
     extern __shared__ float smf[];
     float *Ui = smf;                          // NG x 64 x 64
     float *Uo = Ui + NG * 4096;               // NP x 64 x 64
-    float *Dsh = Uo + NP * 4096;              // kWarpsPerBlock x 64
+    float *Dsh = Uo + NP * 4096;              // kWarpsPerBlock x R x 64
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g0 = a.b0 / 64;
     for (int e = threadIdx.x; e < NG * 4096; e += blockDim.x) Ui[e] = a.UinvG[(g0 + e / 4096) * 4096 + e % 4096];
@@ -534,24 +573,56 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
             for (int e = threadIdx.x; e < 4096; e += blockDim.x)
                 Uo[p * 4096 + e] = a.U[(a.b0 + 64 * g + e / 64) * a.K + a.b0 + 64 * h + e % 64];
     __syncthreads();
-    float *dsh = Dsh + warp * 64;
-#pragma unroll 1
-    for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-        const int64_t n = blockIdx.x * (int64_t)kRowsPerBlock + rr * kWarpsPerBlock + warp;
-        if (n >= a.N) break;                      // no block-wide barrier below
-        float x[NG][2];
+    float *dsh = Dsh + warp * (R * 64);
+    const int64_t nb = blockIdx.x * (int64_t)kRowsPerBlock + warp * R;
+    if (nb >= a.N) return;                    // no block-wide barrier below
+    bool valid[R];
+    float x[R][NG][2];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        valid[r] = nb + r < a.N;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            const float2 v = *reinterpret_cast<const float2 *>(a.W + n * a.K + a.b0 + 64 * g + 2 * lane);
-            x[g][0] = v.x;
-            x[g][1] = v.y;
+            float2 v = make_float2(0.0f, 0.0f);
+            if (valid[r]) v = *reinterpret_cast<const float2 *>(a.W + (nb + r) * a.K + a.b0 + 64 * g + 2 * lane);
+            x[r][g][0] = v.x;
+            x[r][g][1] = v.y;
         }
+    }
+    // y[r] = sum_i dsh[r][i] M[i][2l .. 2l+1] for a 64 x 64 tile M, all rows at once
+    auto matvec = [&](const float *M, float (&y)[R][2]) {
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            const int64_t col = a.b0 + 64 * g + 2 * lane;
-            if (g > 0) *reinterpret_cast<float2 *>(a.W + n * a.K + col) = make_float2(x[g][0], x[g][1]);
-            const bool m0 = a.mask && a.mask[col], m1 = a.mask && a.mask[col + 1];
-            const float v0 = m0 ? 0.0f : x[g][0], v1 = m1 ? 0.0f : x[g][1];
+        for (int r = 0; r < R; ++r) y[r][0] = y[r][1] = 0.0f;
+        const float *mc = M + 2 * lane;
+#pragma unroll 4
+        for (int i = 0; i < 64; i += 4) {
+            float2 u[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) u[k] = *reinterpret_cast<const float2 *>(mc + (i + k) * 64);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float4 d = *reinterpret_cast<const float4 *>(dsh + r * 64 + i);
+                y[r][0] = fmaf(d.x, u[0].x, y[r][0]);
+                y[r][1] = fmaf(d.x, u[0].y, y[r][1]);
+                y[r][0] = fmaf(d.y, u[1].x, y[r][0]);
+                y[r][1] = fmaf(d.y, u[1].y, y[r][1]);
+                y[r][0] = fmaf(d.z, u[2].x, y[r][0]);
+                y[r][1] = fmaf(d.z, u[2].y, y[r][1]);
+                y[r][0] = fmaf(d.w, u[3].x, y[r][0]);
+                y[r][1] = fmaf(d.w, u[3].y, y[r][1]);
+            }
+        }
+    };
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const int64_t col = a.b0 + 64 * g + 2 * lane;
+        const bool m0 = a.mask && a.mask[col], m1 = a.mask && a.mask[col + 1];
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t n = nb + r;
+            if (g > 0 && valid[r]) *reinterpret_cast<float2 *>(a.W + n * a.K + col) = make_float2(x[r][g][0], x[r][g][1]);
+            const float v0 = m0 ? 0.0f : x[r][g][0], v1 = m1 ? 0.0f : x[r][g][1];
             // level 1: unit maximum -> scale code
             float am = fmaxf(fabsf(v0), fabsf(v1));
             float a4 = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));       // 4-element group: lanes 2k, 2k+1
@@ -567,66 +638,63 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
             const float step = ldexp_small(S, E - 2), inv = ldexp_small(__frcp_rn(S), 2 - E);
             const uint32_t q0m = enc::round_exact(fabsf(v0), inv, step), q1m = enc::round_exact(fabsf(v1), inv, step);
             const uint32_t s0 = q0m ? f_bits(v0) >> 31 : 0u, s1 = q1m ? f_bits(v1) >> 31 : 0u;
-            const float b0v = __bfloat162float(__float2bfloat16_rn(x[g][0]));
-            const float b1v = __bfloat162float(__float2bfloat16_rn(x[g][1]));
+            const float b0v = __bfloat162float(__float2bfloat16_rn(x[r][g][0]));
+            const float b1v = __bfloat162float(__float2bfloat16_rn(x[r][g][1]));
             const float q0 = m0 ? b0v : bits_f(f_bits((float)q0m * step) | (s0 << 31));
             const float q1 = m1 ? b1v : bits_f(f_bits((float)q1m * step) | (s1 << 31));
             const uint32_t nib0 = m0 ? 0u : (q0m | (s0 << 3)), nib1 = m1 ? 0u : (q1m | (s1 << 3));
-            a.codes[n * (a.K / 2) + col / 2] = (uint8_t)(nib0 | (nib1 << 4));
             const uint32_t b2 = __ballot_sync(0xffffffffu, e2 && (lane & 3) == 0);
             const uint32_t b3 = __ballot_sync(0xffffffffu, e3 && (lane & 1) == 0);
-            if (lane == 0) {
-                uint32_t mw = c;
+            if (valid[r]) {
+                a.codes[n * (a.K / 2) + col / 2] = (uint8_t)(nib0 | (nib1 << 4));
+                if (lane == 0) {
+                    uint32_t mw = c;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) mw |= ((b2 >> (4 * j)) & 1u) << (8 + j);
+                    for (int j = 0; j < 8; ++j) mw |= ((b2 >> (4 * j)) & 1u) << (8 + j);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) mw |= ((b3 >> (2 * k)) & 1u) << (16 + k);
-                a.meta[n * (a.K / 64) + col / 64] = mw;
+                    for (int k = 0; k < 16; ++k) mw |= ((b3 >> (2 * k)) & 1u) << (16 + k);
+                    a.meta[n * (a.K / 64) + col / 64] = mw;
+                }
+                if (m0) a.w_masked[n * a.n_masked + a.rank[col]] = (uint16_t)(f_bits(b0v) >> 16);
+                if (m1) a.w_masked[n * a.n_masked + a.rank[col + 1]] = (uint16_t)(f_bits(b1v) >> 16);
             }
-            if (m0) a.w_masked[n * a.n_masked + a.rank[col]] = (uint16_t)(f_bits(b0v) >> 16);
-            if (m1) a.w_masked[n * a.n_masked + a.rank[col + 1]] = (uint16_t)(f_bits(b1v) >> 16);
-            // E = D Uinv_g
+            dsh[r * 64 + 2 * lane] = x[r][g][0] - q0;
+            dsh[r * 64 + 2 * lane + 1] = x[r][g][1] - q1;
+        }
+        __syncwarp();
+        // E = D Uinv_g
+        float e[R][2];
+        matvec(Ui + g * 4096, e);
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (!valid[r]) continue;
+            // E in two TF32 parts: the lazy update's split operand
+            const uint32_t h0 = tf32_rna(e[r][0]), h1 = tf32_rna(e[r][1]);
+            const int64_t o = (nb + r) * a.ldE + a.e0 + 64 * g + 2 * lane;
+            *reinterpret_cast<float2 *>(a.Eh + o) = make_float2(__uint_as_float(h0), __uint_as_float(h1));
+            *reinterpret_cast<float2 *>(a.El + o) = make_float2(__uint_as_float(tf32_rna(e[r][0] - __uint_as_float(h0))),
+                                                              __uint_as_float(tf32_rna(e[r][1] - __uint_as_float(h1))));
+        }
+        // feedback into the later groups of the block
+        if (g + 1 < NG) {
             __syncwarp();
-            dsh[2 * lane] = x[g][0] - q0;
-            dsh[2 * lane + 1] = x[g][1] - q1;
-            __syncwarp();
-            const float *ui = Ui + g * 4096 + 2 * lane;
-            float e0 = 0.0f, e1 = 0.0f;
-            for (int i = 0; i < 64; ++i) {
-                const float d = dsh[i];
-                const float2 u = *reinterpret_cast<const float2 *>(ui + i * 64);
-                e0 = fmaf(d, u.x, e0);
-                e1 = fmaf(d, u.y, e1);
-            }
-            {
-                // E in two TF32 parts: the lazy update's split operand
-                const uint32_t h0 = tf32_rna(e0), h1 = tf32_rna(e1);
-                const int64_t o = n * a.ldE + a.e0 + 64 * g + 2 * lane;
-                *reinterpret_cast<float2 *>(a.Eh + o) = make_float2(__uint_as_float(h0), __uint_as_float(h1));
-                *reinterpret_cast<float2 *>(a.El + o) = make_float2(__uint_as_float(tf32_rna(e0 - __uint_as_float(h0))),
-                                                                  __uint_as_float(tf32_rna(e1 - __uint_as_float(h1))));
-            }
-            // feedback into the later groups of the block
-            if (g + 1 < NG) {
-                __syncwarp();
-                dsh[2 * lane] = e0;
-                dsh[2 * lane + 1] = e1;
-                __syncwarp();
 #pragma unroll
-                for (int h = g + 1; h < NG; ++h) {
-                    int p = 0;
-                    for (int gg = 0; gg < g; ++gg) p += NG - 1 - gg;
-                    p += h - g - 1;
-                    const float *uo = Uo + p * 4096 + 2 * lane;
-                    float d0 = 0.0f, d1 = 0.0f;
-                    for (int i = 0; i < 64; ++i) {
-                        const float ei = dsh[i];
-                        const float2 u = *reinterpret_cast<const float2 *>(uo + i * 64);
-                        d0 = fmaf(ei, u.x, d0);
-                        d1 = fmaf(ei, u.y, d1);
-                    }
-                    x[h][0] -= d0;
-                    x[h][1] -= d1;
+            for (int r = 0; r < R; ++r) {
+                dsh[r * 64 + 2 * lane] = e[r][0];
+                dsh[r * 64 + 2 * lane + 1] = e[r][1];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int h = g + 1; h < NG; ++h) {
+                int p = 0;
+                for (int gg = 0; gg < g; ++gg) p += NG - 1 - gg;
+                p += h - g - 1;
+                float dlt[R][2];
+                matvec(Uo + p * 4096, dlt);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    x[r][h][0] -= dlt[r][0];
+                    x[r][h][1] -= dlt[r][1];
                 }
             }
         }
@@ -908,6 +976,18 @@ struct GptqLayout {
 // columns when the block divides it (64, 128, 256), 576 for 192.
 int64_t super_cols(int64_t B) { return B * (512 / B > 1 ? 512 / B : 1); }
 
+// Largest n1 x n2 split block (doubles) at each depth of the factor's
+// recursion over n rows (the root is depth 0).
+void factor_depth_sizes(int64_t n, size_t d, std::vector<int64_t> &mx)
+{
+    if (n == TB) return;
+    const int64_t n1 = n / TB / 2 * TB, n2 = n - n1;
+    if (mx.size() <= d) mx.resize(d + 1, 0);
+    mx[d] = std::max(mx[d], n1 * n2);
+    factor_depth_sizes(n1, d + 1, mx);
+    factor_depth_sizes(n2, d + 1, mx);
+}
+
 GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
 {
     GptqLayout L{};
@@ -919,8 +999,15 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     };
     take(L.A, k * k * 8);
     take(L.Y, k * k * 8);
-    // the factor's scratch: the root split's n2 x n1 block (nested splits are smaller)
-    take(L.T, (nb - nb / 2) * (nb / 2 > 0 ? nb / 2 : 1) * TB * TB * 8);
+    // the factor's scratch: one split block per depth of the recursion (a
+    // level's block is read by its side product while deeper levels run)
+    {
+        std::vector<int64_t> mx;
+        factor_depth_sizes(K, 0, mx);
+        size_t t = 0;
+        for (int64_t v : mx) t += al256((size_t)v * 8);
+        take(L.T, t > 0 ? t : 256);
+    }
     take(L.U, k * k * 4);
     take(L.UinvG, nb * TB * TB * 4);
     take(L.UTh, k * k * 4);
@@ -946,46 +1033,93 @@ bool set_smem_once(F *kernel, size_t bytes, bool &done)
     return true;
 }
 
+// Internal streams of hif4_higptq1, per device: the call's critical chain runs
+// on `hi` (the device's greatest stream priority), forked from and joined back
+// to the caller's stream; the factor's off-path products run on `side[d]`
+// (least priority), one per depth of the recursion, so that the critical
+// chain's small kernels take SMs first as they free up.  Created on first
+// use; `mu` serializes the calls that share them.
+constexpr int kMaxDepth = 16;
+struct GptqStreams {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t hi = nullptr, side[kMaxDepth] = {};
+    cudaEvent_t in = nullptr, out = nullptr, fork[kMaxDepth] = {}, join[kMaxDepth] = {};
+};
+GptqStreams g_streams[64];
+
+hif4_status gptq_streams_ready(GptqStreams &g)
+{
+    if (g.ready) return HIF4_OK;
+    int least = 0, greatest = 0;
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&g.hi, cudaStreamNonBlocking, greatest);
+    for (int d = 0; e == cudaSuccess && d < kMaxDepth; ++d) {
+        e = cudaStreamCreateWithPriority(&g.side[d], cudaStreamNonBlocking, least);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.fork[d], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.join[d], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.in, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.out, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_failed(e);
+    g.ready = true;
+    return HIF4_OK;
+}
+
 // The factor of section "Factor": A (lower triangle of P Hd P on entry) and
-// Y = L^{-1}, both K x K; T the scratch block.
+// Y = L^{-1}, both K x K; T[d] the split block of recursion depth d.  At each
+// split, Y21 = T L11^{-1} does not depend on the lower-right block's factor,
+// so it runs on the depth's side stream while that block is factored, and is
+// joined before Y21 = -L22^{-1} Y21 (the kernels and their operands are the
+// same as in program order; only their overlap changes).
 struct Factor {
-    double *A, *Y, *T;
+    double *A, *Y;
+    double *T[kMaxDepth];
     int64_t K;
     uint32_t *status;
     cudaStream_t s;
+    GptqStreams *gs;
 
-    hif4_status gemm(bool bt, const double *a, int64_t lda, const double *b, int64_t ldb, double *c, int64_t ldc,
-                     int64_t M, int64_t N, int64_t Kd, double alpha, int beta, int tri_a, int tri_b, int lower_c)
+    hif4_status gemm(cudaStream_t st, bool bt, const double *a, int64_t lda, const double *b, int64_t ldb, double *c,
+                     int64_t ldc, int64_t M, int64_t N, int64_t Kd, double alpha, int beta, int tri_a, int tri_b,
+                     int lower_c)
     {
         Dgemm g{a, lda, b, ldb, c, ldc, (int)M, (int)N, (int)Kd, alpha, beta, tri_a, tri_b, lower_c};
         const int64_t mt = M / TB, nt = N / TB, tiles = lower_c ? mt * (mt + 1) / 2 : mt * nt;
         if (tiles < 3 * sm_count()) {             // few tiles: 32 x 32 ones, four times as many blocks
             const dim3 grid((unsigned)(N / 32), (unsigned)(M / 32));
-            return bt ? launch_pdl(k_dgemm<true, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g)
-                      : launch_pdl(k_dgemm<false, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), s, g);
+            return bt ? launch_pdl(k_dgemm<true, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), st, g)
+                      : launch_pdl(k_dgemm<false, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), st, g);
         }
         const dim3 grid((unsigned)nt, (unsigned)mt);
-        return bt ? launch_pdl(k_dgemm<true, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), s, g)
-                  : launch_pdl(k_dgemm<false, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), s, g);
+        return bt ? launch_pdl(k_dgemm<true, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), st, g)
+                  : launch_pdl(k_dgemm<false, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), st, g);
     }
 
-    // rows [o, o + n) of the factor and of its inverse
-    hif4_status run(int64_t o, int64_t n)
+    // rows [o, o + n) of the factor and of its inverse, at recursion depth d
+    hif4_status run(int64_t o, int64_t n, int d)
     {
         if (n == TB) return launch_pdl(k_leaf, dim3(1), dim3(256), kLeafSmem, s, A + o * K + o, K, Y + o * K + o, K, status);
         const int64_t n1 = n / TB / 2 * TB, n2 = n - n1, a = o, b = o + n1;
-        hif4_status st = run(a, n1);
+        hif4_status st = run(a, n1, d + 1);
         if (st != HIF4_OK) return st;
         double *A21 = A + b * K + a, *A22 = A + b * K + b, *Y11 = Y + a * K + a, *Y21 = Y + b * K + a,
-               *Y22 = Y + b * K + b;
-        if ((st = gemm(true, A21, K, Y11, K, T, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
-        if ((st = gemm(true, T, n1, T, n1, A22, K, n2, n2, n1, -1.0, 1, 0, 0, 1)) != HIF4_OK) return st;
-        if ((st = gemm(false, T, n1, Y11, K, Y21, K, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
-        if ((st = run(b, n2)) != HIF4_OK) return st;
-        if ((st = gemm(false, Y22, K, Y21, K, T, n1, n2, n1, n2, -1.0, 0, 1, 0, 0)) != HIF4_OK) return st;
+               *Y22 = Y + b * K + b, *Td = T[d];
+        if ((st = gemm(s, true, A21, K, Y11, K, Td, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
+        if ((st = gemm(s, true, Td, n1, Td, n1, A22, K, n2, n2, n1, -1.0, 1, 0, 0, 1)) != HIF4_OK) return st;
+        cudaError_t e = cudaEventRecord(gs->fork[d], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(gs->side[d], gs->fork[d], 0);
+        if (e != cudaSuccess) return cuda_failed(e);
+        if ((st = gemm(gs->side[d], false, Td, n1, Y11, K, Y21, K, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK)
+            return st;
+        if ((e = cudaEventRecord(gs->join[d], gs->side[d])) != cudaSuccess) return cuda_failed(e);
+        st = run(b, n2, d + 1);
+        if ((e = cudaStreamWaitEvent(s, gs->join[d], 0)) != cudaSuccess) return cuda_failed(e);
+        if (st != HIF4_OK) return st;
+        if ((st = gemm(s, false, Y22, K, Y21, K, Td, n1, n2, n1, n2, -1.0, 0, 1, 0, 0)) != HIF4_OK) return st;
         const int64_t pairs = n2 * n1 / 2;
         const unsigned cb = (unsigned)std::min<int64_t>((pairs + 255) / 256, 4 * (int64_t)sm_count());
-        return launch_pdl(k_copy2d, dim3(cb), dim3(256), 0, s, Y21, K, (const double *)T, n1, n2, n1);
+        return launch_pdl(k_copy2d, dim3(cb), dim3(256), 0, s, Y21, K, (const double *)Td, n1, n2, n1);
     }
 };
 
@@ -993,7 +1127,7 @@ template <int NG>
 hif4_status launch_gptq_block(const GptqArgs &a, cudaStream_t s)
 {
     constexpr int NP = NG * (NG - 1) / 2;
-    const size_t smem = sizeof(float) * ((NG + NP) * 4096 + kWarpsPerBlock * 64);
+    const size_t smem = sizeof(float) * ((NG + NP) * 4096 + kWarpsPerBlock * kRowsPerWarp * 64);
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1045,25 +1179,16 @@ extern "C" size_t hif4_higptq1_group_inputs_offset(int64_t N, int64_t K, int64_t
     return gptq_layout(N, K, blocksize == 0 ? 128 : blocksize).W;
 }
 
-extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t ldw, const float *H,
-                                    const int32_t *mask_idx, int32_t n_masked, double damp, int64_t blocksize,
-                                    uint8_t *codes, uint32_t *meta, void *w_masked, void *workspace,
-                                    size_t ws_bytes, uint32_t *status, hif4_stream_t stream)
-{
-    if (N <= 0 || K <= 0 || n_masked < 0 || !(damp >= 0.0) || !(damp < 1e30)) return HIF4_ERR_INVALID_ARG;
-    if (K % HIF4_UNIT != 0 || ldw < K) return HIF4_ERR_SHAPE;
-    const int64_t B = blocksize == 0 ? 128 : blocksize;
-    if (B <= 0 || B % HIF4_UNIT != 0 || B > 256) return HIF4_ERR_INVALID_ARG;
-    if (K > 32768 || N > ((int64_t)1 << 31) || n_masked > K) return HIF4_ERR_UNSUPPORTED;
-    if (!w || !H || !codes || !meta || (n_masked > 0 && (!mask_idx || !w_masked))) return HIF4_ERR_INVALID_ARG;
-    if (!aligned_to(w, 2) || !aligned_to(H, 4) || !aligned_to(meta, 4) ||
-        (n_masked > 0 && (!aligned_to(mask_idx, 4) || !aligned_to(w_masked, 2))))
-        return HIF4_ERR_ALIGNMENT;
-    const GptqLayout L = gptq_layout(N, K, B);
-    if (!workspace || ws_bytes < L.total) return HIF4_ERR_WORKSPACE;
-    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+namespace hif4 {
+namespace {
 
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+// Everything hif4_higptq1 enqueues, on the internal critical-chain stream s.
+hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, const float *H,
+                            const int32_t *mask_idx, int32_t n_masked, double damp, int64_t B, uint8_t *codes,
+                            uint32_t *meta, void *w_masked, void *workspace, uint32_t *status, cudaStream_t s,
+                            GptqStreams *gs)
+{
+    const GptqLayout L = gptq_layout(N, K, B);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     double *A = reinterpret_cast<double *>(ws + L.A);
     double *Y = reinterpret_cast<double *>(ws + L.Y);
@@ -1102,10 +1227,15 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     k_diag_mean<<<1, 1024, 0, s>>>(H, K, dead, mean);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     {
-        const int64_t total = N * K;
-        int64_t blocks = (total + 255) / 256;
+        const bool vec = aligned16(w) && ldw % 8 == 0;          // K is a multiple of 64
+        const int64_t work = vec ? N * K / 8 : N * K;
+        int64_t blocks = (work + 255) / 256;
         if (blocks > 8 * (int64_t)sm_count()) blocks = 8 * (int64_t)sm_count();
-        k_w_to_f32<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W, status);
+        if (vec)
+            k_w_to_f32<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W, status);
+        else
+            k_w_to_f32_any<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W,
+                                                            status);
         if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     }
     // 2. P Hd P = L' L'^T and Y = L'^{-1} (FP64, recursive), then U = P Y P
@@ -1113,8 +1243,24 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
     k_fill_reversed<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(
         H, K, dead, mean, damp, A);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    Factor F{A, Y, T, K, status, s};
-    const hif4_status fst = F.run(0, K);
+    Factor F{};
+    F.A = A;
+    F.Y = Y;
+    F.K = K;
+    F.status = status;
+    F.s = s;
+    F.gs = gs;
+    {
+        std::vector<int64_t> mx;
+        factor_depth_sizes(K, 0, mx);
+        if ((int)mx.size() > kMaxDepth) return HIF4_ERR_UNSUPPORTED;
+        uint8_t *t = reinterpret_cast<uint8_t *>(T);
+        for (size_t d = 0; d < mx.size(); ++d) {
+            F.T[d] = reinterpret_cast<double *>(t);
+            t += al256((size_t)mx[d] * 8);
+        }
+    }
+    const hif4_status fst = F.run(0, K, 0);
     if (fst != HIF4_OK) return fst;
     k_build_u<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
@@ -1181,4 +1327,44 @@ extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t
         }
     }
     return HIF4_OK;
+}
+
+} // namespace
+} // namespace hif4
+
+extern "C" hif4_status hif4_higptq1(const void *w, int64_t N, int64_t K, int64_t ldw, const float *H,
+                                    const int32_t *mask_idx, int32_t n_masked, double damp, int64_t blocksize,
+                                    uint8_t *codes, uint32_t *meta, void *w_masked, void *workspace,
+                                    size_t ws_bytes, uint32_t *status, hif4_stream_t stream)
+{
+    if (N <= 0 || K <= 0 || n_masked < 0 || !(damp >= 0.0) || !(damp < 1e30)) return HIF4_ERR_INVALID_ARG;
+    if (K % HIF4_UNIT != 0 || ldw < K) return HIF4_ERR_SHAPE;
+    const int64_t B = blocksize == 0 ? 128 : blocksize;
+    if (B <= 0 || B % HIF4_UNIT != 0 || B > 256) return HIF4_ERR_INVALID_ARG;
+    if (K > 32768 || N > ((int64_t)1 << 31) || n_masked > K) return HIF4_ERR_UNSUPPORTED;
+    if (!w || !H || !codes || !meta || (n_masked > 0 && (!mask_idx || !w_masked))) return HIF4_ERR_INVALID_ARG;
+    if (!aligned_to(w, 2) || !aligned_to(H, 4) || !aligned_to(meta, 4) ||
+        (n_masked > 0 && (!aligned_to(mask_idx, 4) || !aligned_to(w_masked, 2))))
+        return HIF4_ERR_ALIGNMENT;
+    const GptqLayout L = gptq_layout(N, K, B);
+    if (!workspace || ws_bytes < L.total) return HIF4_ERR_WORKSPACE;
+    if (!aligned_to(workspace, 256)) return HIF4_ERR_ALIGNMENT;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HIF4_ERR_CUDA;
+    GptqStreams &gs = g_streams[dev];
+    std::lock_guard<std::mutex> lk(gs.mu);
+    hif4_status st = gptq_streams_ready(gs);
+    if (st != HIF4_OK) return st;
+    // fork onto the critical-chain stream, join back whatever happens
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaEventRecord(gs.in, cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(gs.hi, gs.in, 0);
+    if (e != cudaSuccess) return cuda_failed(e);
+    st = higptq1_enqueue(w, N, K, ldw, H, mask_idx, n_masked, damp, B, codes, meta, w_masked, workspace, status,
+                         gs.hi, &gs);
+    e = cudaEventRecord(gs.out, gs.hi);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, gs.out, 0);
+    if (st == HIF4_OK && e != cudaSuccess) st = cuda_failed(e);
+    return st;
 }
