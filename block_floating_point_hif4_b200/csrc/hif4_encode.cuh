@@ -283,5 +283,48 @@ __device__ __forceinline__ void fq_unit64(const uint32_t *w, const uint32_t *mw,
     }
 }
 
+// BF16 decode of 8 elements by byte permutes (the dequantizer's and the
+// weight-decoding GEMM's).  Table word [f][which] for the scale fraction f:
+// the low (which < 2) or high bytes of the BF16 pattern of m (4 + f) 2^-35
+// for m = 0-3 (which even) or 4-7 (which odd), four per word.
+__device__ __forceinline__ uint32_t dequant_table_word(uint32_t f, uint32_t which)
+{
+    uint32_t v = 0;
+    for (uint32_t k = 0; k < 4; ++k) {
+        const uint32_t m = (which & 1u) * 4u + k;
+        const uint32_t t = m ? f_bits((float)(m * (4u + f)) * 0x1p-35f) >> 16 : 0u;
+        v |= ((which >> 1) ? (t >> 8) : (t & 0xFFu)) << (8 * k);
+    }
+    return v;
+}
+
+// BF16 output by byte-permute lookups.  Element value m S 2^(E-2) with
+// S = 2^(e6-31) (1 + f/4) equals [m (4 + f)] 2^-35 2^(e6 + E): the BF16 bits
+// of the first factor (small integers scaled by 2^-35, exact) form one
+// 8-entry table per f, split into low and high bytes; one prmt looks up 4
+// elements' bytes at once, and adding (e6 + E) << 7 to a BF16 pair word
+// scales both halves (every result is a normal number, no carry crosses the
+// halves).  m = 0 entries are masked to zero; the sign bit is the code's.
+__device__ __forceinline__ void dequant8_bf16(uint32_t cw, uint32_t e6, uint32_t Elo, uint32_t Ehi, uint4 T,
+                                              uint32_t (&out)[4])
+{
+    const uint32_t n8 = ((cw & 0x77777777u) + 0x77777777u) & 0x88888888u;   // bit 3 of nibble: m != 0
+    const uint32_t nA = n8 << 4, sA = cw << 4;                              // byte MSBs: even nibbles
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint32_t sel = (cw >> (16 * half)) & 0x7777u;
+        const uint32_t lo4 = prmt(T.x, T.y, sel), hi4 = prmt(T.z, T.w, sel);
+        const uint32_t add = imad((e6 + (half ? Ehi : Elo)) << 7, 0x10001u, 0u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int k = 2 * half + j;
+            const uint32_t v = prmt(lo4, hi4, j ? 0x7362u : 0x5140u);
+            const uint32_t msk = prmt(nA, n8, 0xCC88u + 0x1111u * k);      // 0xFFFF halves where m != 0
+            const uint32_t sg = prmt(sA, cw, 0xC888u + 0x1111u * k) & 0x80008000u;
+            out[k] = ((v + add) & msk) | sg;
+        }
+    }
+}
+
 } // namespace enc
 } // namespace hif4

@@ -101,13 +101,14 @@ __device__ __forceinline__ void epi_pack32(const uint32_t (&r)[32], const uint16
 // quarter and accumulator column base) -> output row `row` (stored only if
 // row < M), columns nb * BN ... + BN - 1: + bias, optional tanh-GELU, FP32,
 // or BF16 (round to nearest even) with optional HiF4 fake quantization of
-// the row's 64-column units.
+// the row's 64-column units (compiled in only with FQ).
+template <bool FQ>
 __device__ __forceinline__ void store_tile_rows(const Args &g, uint32_t tacc, int row, int nb, uint32_t &nonfinite)
 {
     using namespace sm100;
     const bool gelu = (g.flags & HIF4_LINEAR_GELU_TANH) != 0;
     const bool out_f32 = (g.flags & HIF4_LINEAR_OUT_F32) != 0;
-    const bool fq_out = (g.flags & HIF4_LINEAR_FAKE_QUANT_OUT) != 0;
+    const bool fq_out = FQ && (g.flags & HIF4_LINEAR_FAKE_QUANT_OUT) != 0;
     uint16_t *yrow = static_cast<uint16_t *>(g.y) + (int64_t)row * g.ldy;
     float *yrow32 = static_cast<float *>(g.y) + (int64_t)row * g.ldy;
     // HiF4 fake-quant of the output along N: a thread holds whole
@@ -355,8 +356,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
             tile_coords(t, g, mb, nb);
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, g.timeout_ns)) break;
             tc_fence_after();
-            store_tile_rows(g, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, mb * BM + q * 32 + lane, nb,
-                            nonfinite);
+            store_tile_rows<true>(g, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN, mb * BM + q * 32 + lane, nb,
+                                  nonfinite);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -372,6 +373,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
     if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
     if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
 }
+
 
 
 // ----------------------------------------------------------- host helpers

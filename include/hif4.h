@@ -142,6 +142,10 @@ hif4_status hif4_fake_quantize(const void *x, int64_t rows, int64_t cols, int64_
  *          HIF4_LINEAR_OUT_F32: store the FP32 result instead of its BF16
  *          round-to-nearest-even (the BF16 output is exactly that rounding).
  * workspace >= hif4_linear_w4a4_workspace(M, N, K) bytes, 256-byte aligned.
+ * The weight is decoded once per call into the workspace (a streaming pass
+ * at full occupancy), then read by the GEMM.  For repeated calls on a static
+ * weight, decode it once with hif4_weight_decode and call hif4_fake_quantize
+ * + hif4_gemm_bf16 per input: the same products, bit for bit.
  * Errors: SHAPE (K % 64, M/N/K <= 0), ALIGNMENT, WORKSPACE, INVALID_ARG.
  * Bad mask indices are reported through status (HIF4_FLAG_BAD_INDEX).
  */

@@ -144,3 +144,35 @@ def test_ffn_full_size(H):
     idx2 = np.nonzero(m2)[0].astype(np.int32)
     run_case(H, h, d["w2"], idx2, None, rows=rows)
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 64), (129, 256, 128), (300, 520, 640), (512, 264, 576)])
+@pytest.mark.parametrize("gelu", [False, True])
+def test_linear_equals_its_stages(H, M, N, K, gelu):
+    """hif4_linear_w4a4 is hif4_fake_quantize + hif4_weight_decode +
+    hif4_gemm_bf16, bit for bit (the staged form a caller uses to decode a
+    static weight once); protected columns at both ends of K and two
+    adjacent ones inside one 64-column unit."""
+    import torch
+    d = wl.attn_proj(M=M, K=K, N=N, seed=M + 3 * N + K)
+    idx = np.array(sorted({0, 5, 6, K // 2 + 1, K - 1}), np.int32)
+    mask = np.zeros(K, np.uint8)
+    mask[idx] = 1
+    cm = torch.from_numpy(mask).cuda()
+    wd = to_dev_bf16(d["w"])
+    wc, wm = H.quantize(wd, cm)
+    midx = torch.from_numpy(idx).cuda()
+    wmask = to_dev_bf16(np.ascontiguousarray(d["w"][:, idx]))
+    bias = to_dev_bf16(d["bias"])
+    xd = to_dev_bf16(d["x"])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = H.linear_w4a4(xd, wc, wm, N, midx, wmask, bias, gelu=gelu, status=status,
+                      out=torch.empty(M, N, dtype=torch.float32, device="cuda"))
+    xhat = H.fake_quantize(xd, cm, status=status)
+    what = torch.empty(N, K, dtype=torch.bfloat16, device="cuda")
+    H.weight_decode(wc, wm, N, K, midx, wmask, out=what, status=status)
+    ys = H.gemm_bf16(xhat, what, bias, gelu=gelu, status=status,
+                     out=torch.empty(M, N, dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    assert H.get_status(status) == 0
+    assert torch.equal(y, ys)
