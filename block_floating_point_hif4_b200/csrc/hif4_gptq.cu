@@ -573,6 +573,8 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
             for (int e = threadIdx.x; e < 4096; e += blockDim.x)
                 Uo[p * 4096 + e] = a.U[(a.b0 + 64 * g + e / 64) * a.K + a.b0 + 64 * h + e % 64];
     __syncthreads();
+    // W is written by the previous launch of the chain (U is not): wait for it here
+    pdl_enter();
     float *dsh = Dsh + warp * (R * 64);
     const int64_t nb = blockIdx.x * (int64_t)kRowsPerBlock + warp * R;
     if (nb >= a.N) return;                    // no block-wide barrier below
@@ -805,6 +807,8 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // the set-up above touches no data of the previous launch; E and W are its outputs
+    pdl_enter();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1132,8 +1136,8 @@ hif4_status launch_gptq_block(const GptqArgs &a, cudaStream_t s)
     int dev = 0;
     cudaGetDevice(&dev);
     if (!set_smem_once(k_gptq_block<NG>, smem, attr[dev & 63])) return HIF4_ERR_CUDA;
-    k_gptq_block<NG><<<(unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock), 32 * kWarpsPerBlock, smem, s>>>(a);
-    return launch_status();
+    return launch_pdl(k_gptq_block<NG>, dim3((unsigned)((a.N + kRowsPerBlock - 1) / kRowsPerBlock)),
+                      dim3(32 * kWarpsPerBlock), smem, s, a);
 }
 
 } // namespace
@@ -1289,8 +1293,7 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
         UpdArgs ua{W, K, N, c1 - c0, (int)k0, (int)c0, (int)((k1 - k0) / UBK), num_m, num_m * num_n, status,
                    (int)a0};
         const int grid = std::min(num_m * num_n, sm_count());
-        k_update_tf32<<<grid, kUThreads, kUSmem, s>>>(mAh, mAl, mBh, mBl, ua);
-        return launch_status();
+        return launch_pdl(k_update_tf32, dim3(grid), dim3(kUThreads), kUSmem, s, mAh, mAl, mBh, mBl, ua);
     };
     for (int64_t s0 = 0; s0 < K; s0 += S) {
         const int64_t s1 = s0 + S < K ? s0 + S : K;
