@@ -84,65 +84,87 @@ __global__ void k_fill_reversed(const float *H, int64_t K, const uint8_t *dead, 
 //   (L11, L11^{-1}) of A11                    recursively
 //   T   = A21 L11^{-T}                         (= L21)
 //   A22 = A22 - T T^T                          (lower tiles)
-//   Y21 = T L11^{-1}
-//   (L22, L22^{-1}) of A22                    recursively (T is reused there)
-//   Y21 = -L22^{-1} Y21                        (into T, then copied back)
+//   T2  = T L11^{-1}
+//   (L22, L22^{-1}) of A22                    recursively
+//   Y21 = -L22^{-1} T2
 // with Y holding L^{-1}: [[L11, 0], [L21, L22]]^{-1} has the off-diagonal
-// block -L22^{-1} L21 L11^{-1}.  A 64-row block is a leaf: one thread block
-// factors it and inverts its factor.  Only the diagonal tiles of L are kept
+// block -L22^{-1} L21 L11^{-1}.  The split falls on a multiple of 128 rows
+// where n allows it; a block of 128 (or 64) rows is a leaf: one thread block
+// factors it and inverts its factor.  Only the leaves' blocks of L are kept
 // (in A); every product is an FP64 GEMM that skips the tiles in which a
 // triangular operand is zero, so the whole factor costs K^3/3 + K^3/3 FLOP.
 
-constexpr int HB = TB / 2;               // half leaf: one warp's block
-constexpr int HP = HB + 1;               // padded smem row of a half block (doubles)
-constexpr size_t kLeafSmem = sizeof(double) * 7 * HB * HP;
+constexpr int HB = TB / 2;               // panel of the leaf: one warp's Cholesky block
+constexpr int HP = HB + 1;               // smem row of a diagonal (Cholesky) tile, doubles: lane = row
+constexpr int LS = HB + 4;               // smem row of a product tile, doubles: conflict-free MMA fragments
+constexpr int DT = HB * HP;              // doubles of a diagonal tile
+constexpr int LT = HB * LS;              // doubles of a product tile
+
+// d (8 x 8, two per lane: row lane / 4, columns 2 (lane % 4) + {0, 1}) +=
+// a (8 x 4, row lane / 4, column lane % 4) b (4 x 8, row lane % 4, column lane / 4)
+__device__ __forceinline__ void dmma884(double (&d)[2], double a, double b)
+{
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d[0]), "+d"(d[1])
+                 : "d"(a), "d"(b));
+}
 
 // Cholesky of the 32 x 32 lower block S (shared memory) by one warp, lane r
-// owning row r, in four panels of 8 columns: the row is held in a register
-// window whose position w is column 8 p + w, and after each panel the 8
-// finished columns go to S and the window shifts by 8.  One unrolled panel
-// body serves all four panels (the leaf runs once per 64 rows, so code size
-// - instruction fetch - matters more than the predicated work on the dead
-// window positions of the later panels).  On return S holds the factor, 0
-// above the diagonal.  Pivots that are not positive are replaced by 1 and
-// counted in bad.
+// owning row r in registers.  Column j: every lane takes the pivot d (the
+// diagonal entry as updated through column j - 1) from shared memory and
+// forms l_r = a_rj / sqrt(d) (sqrt(d) on lane j); the column goes to shared
+// memory once, lane j + 1 publishes the next pivot a_{j+1,j+1} - l^2, and
+// after one __syncwarp each lane updates its later entries a_rw -= l_r l_w
+// from 16-byte broadcast reads of the column.  The rank-one update of the
+// later columns is off the critical path, which is one shared-memory round
+// trip and one reciprocal square root per column.  On return S holds the
+// factor, 0 above the diagonal.  Pivots that are not positive are replaced
+// by 1 and counted in bad.
 __device__ __forceinline__ void warp_chol32(double (*S)[HP], int &bad)
 {
+    __shared__ __align__(16) double colb[2][HB];
+    __shared__ double piv[2];
     const int r = threadIdx.x & 31;
     double a[HB];
 #pragma unroll
     for (int c = 0; c < HB; ++c) a[c] = c <= r ? S[r][c] : 0.0;
-#pragma unroll 1
-    for (int p = 0; p < HB; p += 8) {
+    if (r == 0) piv[0] = a[0];
+    __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int J = p + j;                                     // column
-            double d = __shfl_sync(0xffffffffu, a[j], J);
-            const bool ok = d > 0.0;
-            if (!ok) d = 1.0;
-            const double rs = rsqrt(d);
-            const double l = r == J ? d * rs : a[j] * rs;           // lane J: the pivot; below it: the column
-            if (r >= J) a[j] = l;
-            bad |= (int)(!ok && r == J);
+    for (int j = 0; j < HB; ++j) {
+        double d = piv[j & 1];
+        const bool ok = d > 0.0;
+        if (!ok) d = 1.0;
+        const double rs = rsqrt(d);
+        const double l = r == j ? d * rs : (r > j ? a[j] * rs : 0.0);
+        bad |= (int)(!ok && r == j);
+        a[j] = l;
+        if (j + 1 < HB) {
+            colb[j & 1][r] = l;
+            if (r == j + 1) piv[(j + 1) & 1] = fma(-l, l, a[j + 1]);
+            __syncwarp();
+            int w = j + 1;
+            if (w & 1) {
+                a[w] = fma(-l, colb[j & 1][w], a[w]);
+                ++w;
+            }
 #pragma unroll
-            for (int w = j + 1; w < HB; ++w) {
-                const int C = p + w;                                 // column of window position w
-                const double lc = __shfl_sync(0xffffffffu, l, C & 31);
-                if (C < HB && r >= C) a[w] -= l * lc;
+            for (; w < HB; w += 2) {
+                const double2 c2 = *reinterpret_cast<const double2 *>(&colb[j & 1][w]);
+                a[w] = fma(-l, c2.x, a[w]);
+                a[w + 1] = fma(-l, c2.y, a[w + 1]);
             }
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) S[r][p + j] = p + j <= r ? a[j] : 0.0;
-#pragma unroll
-        for (int w = 0; w < HB - 8; ++w) a[w] = a[w + 8];
     }
+#pragma unroll
+    for (int c = 0; c < HB; ++c) S[r][c] = c <= r ? a[c] : 0.0;
     __syncwarp();
 }
 
-// Inverse of the 32 x 32 lower factor L (shared memory) into X (0 above the
-// diagonal), one warp: lane c computes column c by forward substitution,
-// L's rows read from shared memory as broadcasts.
-__device__ __forceinline__ void warp_inv32(const double (*L)[HP], double (*X)[HP])
+// Inverse of the 32 x 32 lower factor L (shared memory) into X (row stride
+// LS, 0 above the diagonal), one warp: lane c computes column c by forward
+// substitution, L's rows read from shared memory as broadcasts.
+__device__ __forceinline__ void warp_inv32(const double (*L)[HP], double *X)
 {
     __shared__ double rdiag[HB];
     const int c = threadIdx.x & 31;
@@ -161,124 +183,206 @@ __device__ __forceinline__ void warp_inv32(const double (*L)[HP], double (*X)[HP
         x[r] = ((r == c ? 1.0 : 0.0) - (s0 + s1)) * rdiag[r];
     }
 #pragma unroll
-    for (int r = 0; r < HB; ++r) X[r][c] = x[r];
+    for (int r = 0; r < HB; ++r) X[r * LS + c] = x[r];
     __syncwarp();
 }
 
-// One warp: the 32 x 32 lower block S (shared memory) -> its factor in S (0
-// above the diagonal) and the factor's inverse in X.  Not inlined: the leaf
-// calls it twice, so one copy of the code halves what the leaf fetches.
-__device__ __noinline__ void warp_factor_half(double (*S)[HP], double (*X)[HP], int &bad)
+// One warp: the 32 x 32 lower block S -> its factor in S (0 above the
+// diagonal) and the factor's inverse in X.  Not inlined: the leaf calls it
+// once per panel, and one copy of the code keeps what the leaf fetches small.
+__device__ __noinline__ void warp_factor_panel(double (*S)[HP], double *X, int &bad)
 {
     warp_chol32(S, bad);
     warp_inv32(S, X);
 }
 
-// One 64 x 64 diagonal block: its Cholesky factor (lower, in place in A)
-// and the factor's inverse into Y (zeros above the diagonal), as two halves:
-// warp 0 factors and inverts the 32 x 32 diagonal blocks (warp_factor_half), all
-// 8 warps form L21 = A21 L11^{-T}, A22 - L21 L21^T and
-// Y21 = -L22^{-1} L21 L11^{-1} as 32 x 32 x 32 shared-memory products.  A
-// pivot that is not positive is replaced by 1 and reported as
-// HIF4_FLAG_NOT_SPD.  256 threads.
-__global__ void __launch_bounds__(256) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
+// One warp, one 8-row strip s of a 32 x 32 product on the FP64 MMA:
+// acc[n] += A[8 s .. 8 s + 8, :] B[:, 8 n .. 8 n + 8] over the 32-deep inner
+// dimension.  A row-major (row stride LS); B row-major 32 x 32 (BT false) or
+// given as B^T row-major (BT true), row stride LS.
+template <bool BT>
+__device__ __forceinline__ void strip_mma(double (&acc)[4][2], const double *A, const double *B, int s)
 {
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    const double *ar = A + (8 * s + gid) * LS + tig;
+#pragma unroll
+    for (int k = 0; k < HB; k += 4) {
+        const double a = ar[k];
+        double b[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) b[n] = BT ? B[(8 * n + gid) * LS + k + tig] : B[(k + tig) * LS + 8 * n + gid];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) dmma884(acc[n], a, b[n]);
+    }
+}
+
+// out strip (row stride ld) = alpha acc, or (SUB) out -= acc
+template <bool SUB>
+__device__ __forceinline__ void strip_store(double *out, int ld, int s, const double (&acc)[4][2], double alpha)
+{
+    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+    double *o = out + (8 * s + gid) * ld + 2 * tig;
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            if (SUB)
+                o[8 * n + q] -= acc[n][q];
+            else
+                o[8 * n + q] = alpha * acc[n][q];
+        }
+}
+
+// Shared memory of a leaf of P panels (32 P rows): the diagonal tiles of A
+// (then L), the off-diagonal tiles of A (then L), the diagonal tiles of
+// L^{-1}, its off-diagonal tiles, and P - 1 tiles for the products
+// X_pp L_pk of the current panel.
+template <int P>
+constexpr size_t leaf_smem()
+{
+    return sizeof(double) * ((size_t)P * DT + (size_t)(P * (P - 1) + P + P - 1) * LT);
+}
+constexpr size_t kLeafSmem2 = leaf_smem<2>(), kLeafSmem4 = leaf_smem<4>();
+
+// One diagonal block of 32 P rows (P = 2 or 4): its Cholesky factor (lower,
+// in place in A) and the factor's inverse into Y (zeros above the diagonal),
+// right-looking over 32-column panels p = 0 .. P - 1 with 32 x 32 tiles in
+// shared memory.  Per panel:
+//   warp 0:    L_pp = chol(A_pp), X_pp = L_pp^{-1}
+//   all warps: L_ip = A_ip X_pp^T (i > p);  M_k = X_pp L_pk (k < p)
+//   all warps: A_ij -= L_ip L_jp^T (p < j <= i);
+//              Y_pj = -sum_{k = j}^{p - 1} M_k Y_kj (j < p, Y_jj = X_jj)
+// (the last from L Y = I: L_pp Y_pj = -sum_{k < p} L_pk Y_kj).  The
+// products run as 8 x 32 strips on the FP64 MMA, 8 warps taking strips in
+// turn.  A pivot that is not positive is replaced by 1 and reported as
+// HIF4_FLAG_NOT_SPD.  256 threads.
+template <int P>
+__global__ void __launch_bounds__(256, 1) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
+{
+    constexpr int NO = P * (P - 1) / 2;                          // off-diagonal tiles
+    constexpr int NL = HB * P;                                   // rows
     pdl_enter();
     extern __shared__ __align__(16) double smd[];
-    double(*A11)[HP] = reinterpret_cast<double(*)[HP]>(smd);    // A11, then L11
-    double(*A21)[HP] = A11 + HB;                                 // A21
-    double(*A22)[HP] = A21 + HB;                                 // A22, then L22
-    double(*L21)[HP] = A22 + HB;
-    double(*X11)[HP] = L21 + HB;                                 // L11^{-1}
-    double(*X22)[HP] = X11 + HB;                                 // L22^{-1}
-    double(*T)[HP] = X22 + HB;                                   // L21 L11^{-1}, then Y21
+    double *const Dg = smd;                                      // P diagonal tiles, row stride HP
+    double *const Og = smd + P * DT;                             // NO off-diagonal tiles of A / L
+    double *const Xg = Og + NO * LT;                             // P diagonal tiles of L^{-1}
+    double *const Yg = Xg + P * LT;                              // NO off-diagonal tiles of L^{-1}
+    double *const Mg = Yg + NO * LT;                             // P - 1 tiles X_pp L_pk
+    auto D = [&](int p) { return reinterpret_cast<double(*)[HP]>(Dg + p * DT); };
+    auto oi = [](int i, int j) { return i * (i - 1) / 2 + j; }; // i > j
+    auto O = [&](int i, int j) { return Og + oi(i, j) * LT; };
+    auto X = [&](int p) { return Xg + p * LT; };
+    auto Yo = [&](int i, int j) { return Yg + oi(i, j) * LT; };
+    auto M = [&](int k) { return Mg + k * LT; };
     __shared__ int bad_all;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-#pragma unroll 16
-    for (int e = tid; e < TB * TB; e += 256) {
-        const int r = e >> 6, c = e & 63;
-        const double v = c <= r ? A[(int64_t)r * lda + c] : 0.0;
-        if (r < HB) {
-            if (c < HB) A11[r][c] = v;
-        } else if (c < HB)
-            A21[r - HB][c] = v;
-        else
-            A22[r - HB][c - HB] = v;
+    const int tid = threadIdx.x, warp = tid >> 5;
+
+    // the lower tiles of A (zeros above the diagonal of the diagonal tiles),
+    // as 16-byte pairs: a tile row is 16 pairs
+    auto tile_of = [](int t, int &ti, int &tj) {                 // row-major over the lower tiles
+        ti = 0;
+        for (int u = t; u > ti; ++ti) u -= ti + 1;
+        tj = t - ti * (ti + 1) / 2;
+    };
+    {
+        double2 v[P + NO][2];
+#pragma unroll
+        for (int t = 0; t < P + NO; ++t) {
+            int ti, tj;
+            tile_of(t, ti, tj);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int e = tid + 256 * q, r = e >> 4, c = 2 * (e & 15);
+                v[t][q] = *reinterpret_cast<const double2 *>(A + (int64_t)(HB * ti + r) * lda + HB * tj + c);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < P + NO; ++t) {
+            int ti, tj;
+            tile_of(t, ti, tj);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int e = tid + 256 * q, r = e >> 4, c = 2 * (e & 15);
+                if (ti == tj) {
+                    D(ti)[r][c] = c <= r ? v[t][q].x : 0.0;
+                    D(ti)[r][c + 1] = c + 1 <= r ? v[t][q].y : 0.0;
+                } else {
+                    *reinterpret_cast<double2 *>(O(ti, tj) + r * LS + c) = v[t][q];
+                }
+            }
+        }
     }
     if (tid == 0) bad_all = 0;
     __syncthreads();
-    // each thread's four outputs of a 32 x 32 product: rows ro + 8 i, column lane
-    const int ro = warp;
+
     int bad = 0;
-    if (warp == 0) warp_factor_half(A11, X11, bad);
-    __syncthreads();
-    // L21 = A21 X11^T   (X11 lower: k <= c)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = ro + 8 * i;
-        double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-        for (int k = 0; k < HB; k += 2) {                       // X11[lane][k] = 0 for k > lane
-            s0 = fma(A21[r][k], X11[lane][k], s0);
-            s1 = fma(A21[r][k + 1], X11[lane][k + 1], s1);
+#pragma unroll 1
+    for (int p = 0; p < P; ++p) {
+        if (warp == 0) warp_factor_panel(D(p), X(p), bad);
+        __syncthreads();
+        // L_ip = A_ip X_pp^T (in place: a strip reads only its own rows of A_ip), M_k = X_pp L_pk
+        const int nL = 4 * (P - 1 - p), nM = 4 * p;
+        for (int t = warp; t < nL + nM; t += 8) {
+            double acc[4][2] = {};
+            const int s = t & 3;
+            if (t < nL) {
+                double *o = O(p + 1 + (t >> 2), p);
+                strip_mma<true>(acc, o, X(p), s);
+                __syncwarp();
+                strip_store<false>(o, LS, s, acc, 1.0);
+            } else {
+                const int k = (t - nL) >> 2;
+                strip_mma<false>(acc, X(p), O(p, k), s);
+                strip_store<false>(M(k), LS, s, acc, 1.0);
+            }
         }
-        L21[r][lane] = s0 + s1;
-    }
-    __syncthreads();
-    // A22 -= L21 L21^T (lower half), T = L21 X11 (X11 lower: k >= c)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = ro + 8 * i;
-        double s0 = 0.0, s1 = 0.0, t0 = 0.0, t1 = 0.0;
-#pragma unroll
-        for (int k = 0; k < HB; k += 2) {                       // X11[k][lane] = 0 for k < lane
-            s0 = fma(L21[r][k], L21[lane][k], s0);
-            s1 = fma(L21[r][k + 1], L21[lane][k + 1], s1);
-            t0 = fma(L21[r][k], X11[k][lane], t0);
-            t1 = fma(L21[r][k + 1], X11[k + 1][lane], t1);
+        __syncthreads();
+        // trailing update of the lower tiles right of panel p; row p of L^{-1}
+        const int nS = 2 * (P - 1 - p) * (P - p), nY = 4 * p;
+        for (int t = warp; t < nS + nY; t += 8) {
+            double acc[4][2] = {};
+            const int s = t & 3;
+            if (t < nS) {
+                int i = p + 1, q = t >> 2;                       // q -> (i, j), p < j <= i
+                while (q >= i - p) q -= i++ - p;
+                const int j = p + 1 + q;
+                strip_mma<true>(acc, O(i, p), O(j, p), s);
+                if (i == j)
+                    strip_store<true>(&D(j)[0][0], HP, s, acc, 0.0);
+                else
+                    strip_store<true>(O(i, j), LS, s, acc, 0.0);
+            } else {
+                const int j = (t - nS) >> 2;
+                for (int k = j; k < p; ++k) strip_mma<false>(acc, M(k), k == j ? X(j) : Yo(k, j), s);
+                strip_store<false>(Yo(p, j), LS, s, acc, -1.0);
+            }
         }
-        if (lane <= r) A22[r][lane] -= s0 + s1;
-        T[r][lane] = t0 + t1;
+        __syncthreads();
     }
-    __syncthreads();
-    if (warp == 0) {
-        warp_factor_half(A22, X22, bad);
-        if (bad) atomicOr(&bad_all, 1);
-    }
-    __syncthreads();
-    // Y21 = -X22 T   (X22 lower: k <= r); results kept in registers until all reads of T are done
-    double y21[4];
+    if (warp == 0 && bad) atomicOr(&bad_all, 1);
+
+    // L (lower tiles, zeros above the diagonal) -> A; L^{-1} (the whole
+    // block, zeros above the diagonal) -> Y; 16-byte pairs
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = ro + 8 * i;
-        double s0 = 0.0, s1 = 0.0;
+    for (int t = 0; t < P * P; ++t) {
+        const int ti = t / P, tj = t % P;
 #pragma unroll
-        for (int k = 0; k < HB; k += 2) {                       // X22[r][k] = 0 for k > r
-            s0 = fma(X22[r][k], T[k][lane], s0);
-            s1 = fma(X22[r][k + 1], T[k + 1][lane], s1);
+        for (int q = 0; q < 2; ++q) {
+            const int e = tid + 256 * q, r = e >> 4, c = 2 * (e & 15);
+            const int64_t gr = HB * ti + r, gc = HB * tj + c;
+            double2 y = make_double2(0.0, 0.0);
+            if (ti == tj) {
+                *reinterpret_cast<double2 *>(A + gr * lda + gc) = make_double2(D(ti)[r][c], D(ti)[r][c + 1]);
+                y = *reinterpret_cast<const double2 *>(X(ti) + r * LS + c);
+            } else if (ti > tj) {
+                *reinterpret_cast<double2 *>(A + gr * lda + gc) =
+                    *reinterpret_cast<const double2 *>(O(ti, tj) + r * LS + c);
+                y = *reinterpret_cast<const double2 *>(Yo(ti, tj) + r * LS + c);
+            }
+            *reinterpret_cast<double2 *>(Y + gr * ldy + gc) = y;
         }
-        y21[i] = -(s0 + s1);
     }
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 4; ++i) T[ro + 8 * i][lane] = y21[i];
-    __syncthreads();
-    for (int e = tid; e < TB * TB; e += 256) {
-        const int r = e >> 6, c = e & 63;
-        double l, y;
-        if (r < HB) {
-            l = c < HB ? A11[r][c] : 0.0;
-            y = c < HB ? X11[r][c] : 0.0;
-        } else if (c < HB) {
-            l = L21[r - HB][c];
-            y = T[r - HB][c];
-        } else {
-            l = A22[r - HB][c - HB];
-            y = X22[r - HB][c - HB];
-        }
-        if (c <= r) A[(int64_t)r * lda + c] = l;
-        Y[(int64_t)r * ldy + c] = y;
-    }
     if (tid == 0 && bad_all && status) atomicOr(status, HIF4_FLAG_NOT_SPD);
 }
 
@@ -328,15 +432,6 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_addr(smem_dst)), "l"(gmem_src)
                  : "memory");
-}
-
-// d (8 x 8, two per lane: row lane / 4, columns 2 (lane % 4) + {0, 1}) +=
-// a (8 x 4, row lane / 4, column lane % 4) b (4 x 8, row lane % 4, column lane / 4)
-__device__ __forceinline__ void dmma884(double (&d)[2], double a, double b)
-{
-    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                 : "+d"(d[0]), "+d"(d[1])
-                 : "d"(a), "d"(b));
 }
 
 template <bool BT, int T>
@@ -703,17 +798,6 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
     }
 }
 
-// dst (rows x cols, ld ldd) = src (ld lds), FP64; cols a multiple of 2.
-__global__ void k_copy2d(double *dst, int64_t ldd, const double *src, int64_t lds, int64_t rows, int64_t cols)
-{
-    pdl_enter();
-    const int64_t pairs = cols / 2, n = rows * pairs;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / pairs, c = 2 * (i - r * pairs);
-        *reinterpret_cast<double2 *>(dst + r * ldd + c) = *reinterpret_cast<const double2 *>(src + r * lds + c);
-    }
-}
-
 // The lazy update C (M x Nc, ldc) -= E B after each block, on the tcgen05
 // tensor cores, kind::tf32, as a persistent kernel: one CTA per SM walks
 // 128 x 128 tiles of C, each accumulated in
@@ -980,12 +1064,21 @@ struct GptqLayout {
 // columns when the block divides it (64, 128, 256), 576 for 192.
 int64_t super_cols(int64_t B) { return B * (512 / B > 1 ? 512 / B : 1); }
 
+// The factor's split of a diagonal block of n > 128 rows: n1 = about half,
+// a multiple of 128 rows when n is one (so that the leaves have 128 rows),
+// else of 64.
+int64_t factor_split(int64_t n)
+{
+    const int64_t u = n % (2 * TB) == 0 ? 2 * TB : TB;
+    return n / u / 2 * u;
+}
+
 // Largest n1 x n2 split block (doubles) at each depth of the factor's
 // recursion over n rows (the root is depth 0).
 void factor_depth_sizes(int64_t n, size_t d, std::vector<int64_t> &mx)
 {
-    if (n == TB) return;
-    const int64_t n1 = n / TB / 2 * TB, n2 = n - n1;
+    if (n <= 2 * TB) return;
+    const int64_t n1 = factor_split(n), n2 = n - n1;
     if (mx.size() <= d) mx.resize(d + 1, 0);
     mx[d] = std::max(mx[d], n1 * n2);
     factor_depth_sizes(n1, d + 1, mx);
@@ -1003,13 +1096,14 @@ GptqLayout gptq_layout(int64_t N, int64_t K, int64_t B)
     };
     take(L.A, k * k * 8);
     take(L.Y, k * k * 8);
-    // the factor's scratch: one split block per depth of the recursion (a
-    // level's block is read by its side product while deeper levels run)
+    // the factor's scratch: two split blocks per depth of the recursion (a
+    // level's blocks are read and written by its side product while deeper
+    // levels run)
     {
         std::vector<int64_t> mx;
         factor_depth_sizes(K, 0, mx);
         size_t t = 0;
-        for (int64_t v : mx) t += al256((size_t)v * 8);
+        for (int64_t v : mx) t += 2 * al256((size_t)v * 8);
         take(L.T, t > 0 ? t : 256);
     }
     take(L.U, k * k * 4);
@@ -1071,14 +1165,14 @@ hif4_status gptq_streams_ready(GptqStreams &g)
 }
 
 // The factor of section "Factor": A (lower triangle of P Hd P on entry) and
-// Y = L^{-1}, both K x K; T[d] the split block of recursion depth d.  At each
-// split, Y21 = T L11^{-1} does not depend on the lower-right block's factor,
-// so it runs on the depth's side stream while that block is factored, and is
-// joined before Y21 = -L22^{-1} Y21 (the kernels and their operands are the
-// same as in program order; only their overlap changes).
+// Y = L^{-1}, both K x K; T[d], T2[d] the split blocks of recursion depth d.
+// At each split, T2 = T L11^{-1} does not depend on the lower-right block's
+// factor, so it runs on the depth's side stream while that block is
+// factored, and is joined before Y21 = -L22^{-1} T2 (the kernels and their
+// operands are the same as in program order; only their overlap changes).
 struct Factor {
     double *A, *Y;
-    double *T[kMaxDepth];
+    double *T[kMaxDepth], *T2[kMaxDepth];
     int64_t K;
     uint32_t *status;
     cudaStream_t s;
@@ -1103,27 +1197,29 @@ struct Factor {
     // rows [o, o + n) of the factor and of its inverse, at recursion depth d
     hif4_status run(int64_t o, int64_t n, int d)
     {
-        if (n == TB) return launch_pdl(k_leaf, dim3(1), dim3(256), kLeafSmem, s, A + o * K + o, K, Y + o * K + o, K, status);
-        const int64_t n1 = n / TB / 2 * TB, n2 = n - n1, a = o, b = o + n1;
+        if (n == TB)
+            return launch_pdl(k_leaf<2>, dim3(1), dim3(256), kLeafSmem2, s, A + o * K + o, K, Y + o * K + o, K,
+                              status);
+        if (n == 2 * TB)
+            return launch_pdl(k_leaf<4>, dim3(1), dim3(256), kLeafSmem4, s, A + o * K + o, K, Y + o * K + o, K,
+                              status);
+        const int64_t n1 = factor_split(n), n2 = n - n1, a = o, b = o + n1;
         hif4_status st = run(a, n1, d + 1);
         if (st != HIF4_OK) return st;
         double *A21 = A + b * K + a, *A22 = A + b * K + b, *Y11 = Y + a * K + a, *Y21 = Y + b * K + a,
-               *Y22 = Y + b * K + b, *Td = T[d];
+               *Y22 = Y + b * K + b, *Td = T[d], *T2d = T2[d];
         if ((st = gemm(s, true, A21, K, Y11, K, Td, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
         if ((st = gemm(s, true, Td, n1, Td, n1, A22, K, n2, n2, n1, -1.0, 1, 0, 0, 1)) != HIF4_OK) return st;
         cudaError_t e = cudaEventRecord(gs->fork[d], s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(gs->side[d], gs->fork[d], 0);
         if (e != cudaSuccess) return cuda_failed(e);
-        if ((st = gemm(gs->side[d], false, Td, n1, Y11, K, Y21, K, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK)
+        if ((st = gemm(gs->side[d], false, Td, n1, Y11, K, T2d, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK)
             return st;
         if ((e = cudaEventRecord(gs->join[d], gs->side[d])) != cudaSuccess) return cuda_failed(e);
         st = run(b, n2, d + 1);
         if ((e = cudaStreamWaitEvent(s, gs->join[d], 0)) != cudaSuccess) return cuda_failed(e);
         if (st != HIF4_OK) return st;
-        if ((st = gemm(s, false, Y22, K, Y21, K, Td, n1, n2, n1, n2, -1.0, 0, 1, 0, 0)) != HIF4_OK) return st;
-        const int64_t pairs = n2 * n1 / 2;
-        const unsigned cb = (unsigned)std::min<int64_t>((pairs + 255) / 256, 4 * (int64_t)sm_count());
-        return launch_pdl(k_copy2d, dim3(cb), dim3(256), 0, s, Y21, K, (const double *)Td, n1, n2, n1);
+        return gemm(s, false, Y22, K, T2d, n1, Y21, K, n2, n1, n2, -1.0, 0, 1, 0, 0);
     }
 };
 
@@ -1209,13 +1305,14 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
     uint8_t *dead = ws + L.dead;
     double *mean = reinterpret_cast<double *>(ws + L.mean);
 
-    static bool attr_leaf[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false}, attr_g2[64] = {false},
+    static bool attr_leaf[64] = {false}, attr_leaf4[64] = {false}, attr_g0[64] = {false}, attr_g1[64] = {false}, attr_g2[64] = {false},
                 attr_g3[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     static bool attr_up[64] = {false};
     if (!set_smem_once(k_update_tf32, kUSmem, attr_up[dev & 63]) ||
-        !set_smem_once(k_leaf, kLeafSmem, attr_leaf[dev & 63]) ||
+        !set_smem_once(k_leaf<2>, kLeafSmem2, attr_leaf[dev & 63]) ||
+        !set_smem_once(k_leaf<4>, kLeafSmem4, attr_leaf4[dev & 63]) ||
         !set_smem_once(k_dgemm<false, 64>, gemm_smem<64>(), attr_g0[dev & 63]) ||
         !set_smem_once(k_dgemm<true, 64>, gemm_smem<64>(), attr_g1[dev & 63]) ||
         !set_smem_once(k_dgemm<false, 32>, gemm_smem<32>(), attr_g2[dev & 63]) ||
@@ -1261,6 +1358,8 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
         uint8_t *t = reinterpret_cast<uint8_t *>(T);
         for (size_t d = 0; d < mx.size(); ++d) {
             F.T[d] = reinterpret_cast<double *>(t);
+            t += al256((size_t)mx[d] * 8);
+            F.T2[d] = reinterpret_cast<double *>(t);
             t += al256((size_t)mx[d] * 8);
         }
     }

@@ -146,11 +146,12 @@ def test_small_layer_vs_oracle(H, bs):
     compare(w, Hf, idx, 0.01, bs, got)
 
 
-@pytest.mark.parametrize("K", [64, 128, 320])
+@pytest.mark.parametrize("K", [64, 128, 192, 256, 320, 448])
 def test_factor_recursion_shapes(H, K):
-    """The factor's recursion at its edges: one 64-column leaf (K = 64), one
-    split (128), and uneven splits of an odd tile count (320 = 2 + 3 tiles,
-    then 1 + 2)."""
+    """The factor's recursion at its edges: a 64-row leaf alone (K = 64), a
+    128-row leaf alone (128), the two leaf sizes side by side (192 = 64 +
+    128), one split of 128-row leaves (256), and the splits of odd 64-row
+    tile counts (320 = 128 + (64 + 128); 448 = (64 + 128) + (128 + 128))."""
     rng = np.random.default_rng(K + 7)
     N = 70
     w = _bf16(rng, (N, K), 0.02)
