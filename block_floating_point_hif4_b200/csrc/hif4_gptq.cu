@@ -260,7 +260,6 @@ template <int P>
 __global__ void __launch_bounds__(256, 1) k_leaf(double *A, int64_t lda, double *Y, int64_t ldy, uint32_t *status)
 {
     constexpr int NO = P * (P - 1) / 2;                          // off-diagonal tiles
-    constexpr int NL = HB * P;                                   // rows
     pdl_enter();
     extern __shared__ __align__(16) double smd[];
     double *const Dg = smd;                                      // P diagonal tiles, row stride HP
@@ -389,8 +388,9 @@ __global__ void __launch_bounds__(256, 1) k_leaf(double *A, int64_t lda, double 
 // FP64 GEMM on whole tiles: C = alpha op(A) op(B) (+ C if beta), on the FP64
 // tensor-core MMA (m8n8k4).  One T x T tile of C per 128-thread block (T =
 // 64, or 32 below), a T/2 x T/2 quarter per warp (T/16 x T/16 MMA tiles); the K loop
-// runs in 32-deep stages that cp.async copies double-buffer into shared
-// memory in the operands' own layouts: A row-major, B k-major (B row-major)
+// runs in 32-deep stages that cp.async copies keep NS deep in shared memory
+// (NS - 1 stages in flight ahead of the one in use: the small products'
+// whole K range at once) in the operands' own layouts: A row-major, B k-major (B row-major)
 // or n-major (BT, B^T row-major), whose fragments the MMA reads directly.  A
 // is M x K row-major; B is K x N row-major, or (BT) N x K row-major holding
 // B^T.  Triangular operands skip their zero tiles: tri_a (A lower) ends the
@@ -410,10 +410,10 @@ constexpr int stage_doubles()
 {
     return T * AS + (T * AS > KC * (T + 4) ? T * AS : KC * (T + 4));
 }
-template <int T>
+template <int T, int NS>
 constexpr size_t gemm_smem()
 {
-    return sizeof(double) * 2 * stage_doubles<T>();
+    return sizeof(double) * NS * stage_doubles<T>();
 }
 
 struct Dgemm {
@@ -434,7 +434,7 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
                  : "memory");
 }
 
-template <bool BT, int T>
+template <bool BT, int T, int NS>
 __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
 {
     pdl_enter();
@@ -474,32 +474,56 @@ __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     double acc[F][F][2] = {};
-    if (k0 < k1) {
-        issue(k0, 0);
-        int st = 0;
-        for (int k = k0; k < k1; k += KC, st ^= 1) {
-            if (k + KC < k1) {
-                issue(k + KC, st ^ 1);
-                asm volatile("cp.async.wait_group 1;" ::: "memory");
-            } else {
-                asm volatile("cp.async.wait_group 0;" ::: "memory");
+    auto compute = [&](int st) {
+        const double *As = smd + st * SD, *Bs = As + T * AS;
+#pragma unroll
+        for (int kk = 0; kk < KC; kk += 4) {
+            double a[F], b[F];
+#pragma unroll
+            for (int i = 0; i < F; ++i) a[i] = As[(wm + 8 * i + gid) * AS + kk + tig];
+#pragma unroll
+            for (int j = 0; j < F; ++j)
+                b[j] = BT ? Bs[(wn + 8 * j + gid) * AS + kk + tig] : Bs[(kk + tig) * BS + wn + 8 * j + gid];
+#pragma unroll
+            for (int i = 0; i < F; ++i)
+#pragma unroll
+                for (int j = 0; j < F; ++j) dmma884(acc[i][j], a[i], b[j]);
+        }
+    };
+    if constexpr (NS == 2) {                  // double buffer: the next stage is issued before this one is awaited
+        if (k0 < k1) {
+            issue(k0, 0);
+            int st = 0;
+            for (int k = k0; k < k1; k += KC, st ^= 1) {
+                if (k + KC < k1) {
+                    issue(k + KC, st ^ 1);
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                } else {
+                    asm volatile("cp.async.wait_group 0;" ::: "memory");
+                }
+                __syncthreads();
+                compute(st);
+                __syncthreads();              // stage st is refilled two steps on
             }
-            __syncthreads();
-            const double *As = smd + st * SD, *Bs = As + T * AS;
+        }
+    } else {
+        const int nk = k0 < k1 ? (k1 - k0) / KC : 0;
 #pragma unroll
-            for (int kk = 0; kk < KC; kk += 4) {
-                double a[F], b[F];
-#pragma unroll
-                for (int i = 0; i < F; ++i) a[i] = As[(wm + 8 * i + gid) * AS + kk + tig];
-#pragma unroll
-                for (int j = 0; j < F; ++j)
-                    b[j] = BT ? Bs[(wn + 8 * j + gid) * AS + kk + tig] : Bs[(kk + tig) * BS + wn + 8 * j + gid];
-#pragma unroll
-                for (int i = 0; i < F; ++i)
-#pragma unroll
-                    for (int j = 0; j < F; ++j) dmma884(acc[i][j], a[i], b[j]);
-            }
-            __syncthreads();                                         // stage st is refilled two steps on
+        for (int q = 0; q < NS - 1; ++q) {    // one commit group per stage, empty past the end
+            if (q < nk)
+                issue(k0 + q * KC, q);
+            else
+                asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+        for (int it = 0; it < nk; ++it) {
+            asm volatile("cp.async.wait_group %0;" ::"n"(NS - 2) : "memory");
+            __syncthreads();                  // stage it is in; stage it - 1 is consumed
+            const int nx = it + NS - 1;       // refills the slot of stage it - 1
+            if (nx < nk)
+                issue(k0 + nx * KC, nx % NS);
+            else
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            compute(it % NS);
         }
     }
 #pragma unroll
@@ -516,21 +540,6 @@ __global__ void __launch_bounds__(kGemmThreads, 3) k_dgemm(Dgemm g)
             }
             *cp = u;
         }
-}
-
-// U[i][j] = Y[K-1-i][K-1-j] for j >= i (FP32, upper), 0 below; and the
-// inverse of U's diagonal block g, Uinv_g[a][b] = L'[K-1-64g-a][K-1-64g-b]
-// for b >= a (the reversed diagonal block of the Cholesky factor).
-__global__ void k_build_u(const double *Y, const double *A, int64_t K, float *U, float *UinvG)
-{
-    const int64_t i = blockIdx.y * (int64_t)blockDim.y + threadIdx.y;
-    const int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (i >= K || j >= K) return;
-    U[i * K + j] = j >= i ? (float)Y[(K - 1 - i) * K + (K - 1 - j)] : 0.0f;
-    if (i / TB == j / TB) {
-        const int64_t g = i / TB, a = i % TB, b = j % TB;
-        UinvG[g * TB * TB + a * TB + b] = b >= a ? (float)A[(K - 1 - i) * K + (K - 1 - j)] : 0.0f;
-    }
 }
 
 // ------------------------------------------------------------ group loop
@@ -1010,14 +1019,28 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
     if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
 }
 
-// U^T split into TF32 parts (K x K, K a multiple of 32), 32 x 32 tiles through
-// shared memory so that both the reads of U and the writes of U^T coalesce.
-__global__ void k_ut_split(const float *U, int64_t K, float *UTh, float *UTl)
+// U[i][j] = Y[K-1-i][K-1-j] for j >= i (FP32, upper), 0 below; the inverse
+// of U's diagonal block g, Uinv_g[a][b] = L'[K-1-64g-a][K-1-64g-b] for b >= a
+// (the reversed diagonal block of the Cholesky factor); and U^T in TF32
+// parts, U^T = UTh + UTl (UTh = U rounded to TF32, UTl = the rest rounded to
+// TF32), the K-major B operand of the lazy update.  One 32 x 32 tile per
+// block of 32 x 8 threads, transposed through shared memory.
+__global__ void k_build_u(const double *Y, const double *A, int64_t K, float *U, float *UinvG, float *UTh,
+                          float *UTl)
 {
     __shared__ float t[32][33];
     const int64_t i0 = blockIdx.y * 32ll, j0 = blockIdx.x * 32ll;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) t[threadIdx.y + 8 * q][threadIdx.x] = U[(i0 + threadIdx.y + 8 * q) * K + j0 + threadIdx.x];
+    for (int q = 0; q < 4; ++q) {
+        const int64_t i = i0 + threadIdx.y + 8 * q, j = j0 + threadIdx.x;
+        const float u = j >= i ? (float)Y[(K - 1 - i) * K + (K - 1 - j)] : 0.0f;
+        U[i * K + j] = u;
+        t[threadIdx.y + 8 * q][threadIdx.x] = u;
+        if (i / TB == j / TB) {
+            const int64_t g = i / TB, a = i % TB, b = j % TB;
+            UinvG[g * TB * TB + a * TB + b] = b >= a ? (float)A[(K - 1 - i) * K + (K - 1 - j)] : 0.0f;
+        }
+    }
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -1135,14 +1158,18 @@ bool set_smem_once(F *kernel, size_t bytes, bool &done)
 // on `hi` (the device's greatest stream priority), forked from and joined back
 // to the caller's stream; the factor's off-path products run on `side[d]`
 // (least priority), one per depth of the recursion, so that the critical
-// chain's small kernels take SMs first as they free up.  Created on first
+// chain's small kernels take SMs first as they free up, except those of
+// blocks of at most 384 rows, which run on `side_hi[d]` (greatest priority)
+// so that they do not queue behind a large one; the FP32 working weights are
+// formed on `prep` (least priority) while the factor runs.  Created on first
 // use; `mu` serializes the calls that share them.
 constexpr int kMaxDepth = 16;
 struct GptqStreams {
     std::mutex mu;
     bool ready = false;
-    cudaStream_t hi = nullptr, side[kMaxDepth] = {};
-    cudaEvent_t in = nullptr, out = nullptr, fork[kMaxDepth] = {}, join[kMaxDepth] = {};
+    cudaStream_t hi = nullptr, prep = nullptr, side[kMaxDepth] = {}, side_hi[kMaxDepth] = {};
+    cudaEvent_t in = nullptr, out = nullptr, prep_fork = nullptr, prep_join = nullptr, fork[kMaxDepth] = {},
+                join[kMaxDepth] = {};
 };
 GptqStreams g_streams[64];
 
@@ -1152,8 +1179,12 @@ hif4_status gptq_streams_ready(GptqStreams &g)
     int least = 0, greatest = 0;
     cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&g.hi, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&g.prep, cudaStreamNonBlocking, least);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.prep_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.prep_join, cudaEventDisableTiming);
     for (int d = 0; e == cudaSuccess && d < kMaxDepth; ++d) {
         e = cudaStreamCreateWithPriority(&g.side[d], cudaStreamNonBlocking, least);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&g.side_hi[d], cudaStreamNonBlocking, greatest);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.fork[d], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&g.join[d], cudaEventDisableTiming);
     }
@@ -1186,12 +1217,12 @@ struct Factor {
         const int64_t mt = M / TB, nt = N / TB, tiles = lower_c ? mt * (mt + 1) / 2 : mt * nt;
         if (tiles < 3 * sm_count()) {             // few tiles: 32 x 32 ones, four times as many blocks
             const dim3 grid((unsigned)(N / 32), (unsigned)(M / 32));
-            return bt ? launch_pdl(k_dgemm<true, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), st, g)
-                      : launch_pdl(k_dgemm<false, 32>, grid, dim3(kGemmThreads), gemm_smem<32>(), st, g);
+            return bt ? launch_pdl(k_dgemm<true, 32, 4>, grid, dim3(kGemmThreads), gemm_smem<32, 4>(), st, g)
+                      : launch_pdl(k_dgemm<false, 32, 4>, grid, dim3(kGemmThreads), gemm_smem<32, 4>(), st, g);
         }
         const dim3 grid((unsigned)nt, (unsigned)mt);
-        return bt ? launch_pdl(k_dgemm<true, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), st, g)
-                  : launch_pdl(k_dgemm<false, 64>, grid, dim3(kGemmThreads), gemm_smem<64>(), st, g);
+        return bt ? launch_pdl(k_dgemm<true, 64, 2>, grid, dim3(kGemmThreads), gemm_smem<64, 2>(), st, g)
+                  : launch_pdl(k_dgemm<false, 64, 2>, grid, dim3(kGemmThreads), gemm_smem<64, 2>(), st, g);
     }
 
     // rows [o, o + n) of the factor and of its inverse, at recursion depth d
@@ -1210,12 +1241,12 @@ struct Factor {
                *Y22 = Y + b * K + b, *Td = T[d], *T2d = T2[d];
         if ((st = gemm(s, true, A21, K, Y11, K, Td, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
         if ((st = gemm(s, true, Td, n1, Td, n1, A22, K, n2, n2, n1, -1.0, 1, 0, 0, 1)) != HIF4_OK) return st;
+        cudaStream_t sd = n <= 384 ? gs->side_hi[d] : gs->side[d];
         cudaError_t e = cudaEventRecord(gs->fork[d], s);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(gs->side[d], gs->fork[d], 0);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sd, gs->fork[d], 0);
         if (e != cudaSuccess) return cuda_failed(e);
-        if ((st = gemm(gs->side[d], false, Td, n1, Y11, K, T2d, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK)
-            return st;
-        if ((e = cudaEventRecord(gs->join[d], gs->side[d])) != cudaSuccess) return cuda_failed(e);
+        if ((st = gemm(sd, false, Td, n1, Y11, K, T2d, n1, n2, n1, n1, 1.0, 0, 0, 1, 0)) != HIF4_OK) return st;
+        if ((e = cudaEventRecord(gs->join[d], sd)) != cudaSuccess) return cuda_failed(e);
         st = run(b, n2, d + 1);
         if ((e = cudaStreamWaitEvent(s, gs->join[d], 0)) != cudaSuccess) return cuda_failed(e);
         if (st != HIF4_OK) return st;
@@ -1313,10 +1344,10 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
     if (!set_smem_once(k_update_tf32, kUSmem, attr_up[dev & 63]) ||
         !set_smem_once(k_leaf<2>, kLeafSmem2, attr_leaf[dev & 63]) ||
         !set_smem_once(k_leaf<4>, kLeafSmem4, attr_leaf4[dev & 63]) ||
-        !set_smem_once(k_dgemm<false, 64>, gemm_smem<64>(), attr_g0[dev & 63]) ||
-        !set_smem_once(k_dgemm<true, 64>, gemm_smem<64>(), attr_g1[dev & 63]) ||
-        !set_smem_once(k_dgemm<false, 32>, gemm_smem<32>(), attr_g2[dev & 63]) ||
-        !set_smem_once(k_dgemm<true, 32>, gemm_smem<32>(), attr_g3[dev & 63]))
+        !set_smem_once(k_dgemm<false, 64, 2>, gemm_smem<64, 2>(), attr_g0[dev & 63]) ||
+        !set_smem_once(k_dgemm<true, 64, 2>, gemm_smem<64, 2>(), attr_g1[dev & 63]) ||
+        !set_smem_once(k_dgemm<false, 32, 4>, gemm_smem<32, 4>(), attr_g2[dev & 63]) ||
+        !set_smem_once(k_dgemm<true, 32, 4>, gemm_smem<32, 4>(), attr_g3[dev & 63]))
         return HIF4_ERR_CUDA;
 
     // 1. protected columns, Hessian diagonal statistics, FP32 working weights
@@ -1328,16 +1359,21 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
     k_diag_mean<<<1, 1024, 0, s>>>(H, K, dead, mean);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
     {
+        cudaError_t e = cudaEventRecord(gs->prep_fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(gs->prep, gs->prep_fork, 0);
+        if (e != cudaSuccess) return cuda_failed(e);
+        cudaStream_t ps = gs->prep;
         const bool vec = aligned16(w) && ldw % 8 == 0;          // K is a multiple of 64
         const int64_t work = vec ? N * K / 8 : N * K;
         int64_t blocks = (work + 255) / 256;
         if (blocks > 8 * (int64_t)sm_count()) blocks = 8 * (int64_t)sm_count();
         if (vec)
-            k_w_to_f32<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W, status);
+            k_w_to_f32<<<(unsigned)blocks, 256, 0, ps>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W, status);
         else
-            k_w_to_f32_any<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W,
-                                                            status);
+            k_w_to_f32_any<<<(unsigned)blocks, 256, 0, ps>>>(static_cast<const uint16_t *>(w), ldw, N, K, dead, W,
+                                                             status);
         if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+        if ((e = cudaEventRecord(gs->prep_join, ps)) != cudaSuccess) return cuda_failed(e);
     }
     // 2. P Hd P = L' L'^T and Y = L'^{-1} (FP64, recursive), then U = P Y P
     //    and the inverses of U's diagonal blocks
@@ -1365,11 +1401,12 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
     }
     const hif4_status fst = F.run(0, K, 0);
     if (fst != HIF4_OK) return fst;
-    k_build_u<<<dim3((unsigned)((K + 31) / 32), (unsigned)((K + 7) / 8)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG);
+    k_build_u<<<dim3((unsigned)(K / 32), (unsigned)(K / 32)), dim3(32, 8), 0, s>>>(Y, A, K, U, UinvG, UTh, UTl);
     if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
-    // U^T in TF32 parts: the K-major B operand of the lazy update
-    k_ut_split<<<dim3((unsigned)(K / 32), (unsigned)(K / 32)), dim3(32, 8), 0, s>>>(U, K, UTh, UTl);
-    if (launch_status() != HIF4_OK) return HIF4_ERR_CUDA;
+    {
+        const cudaError_t e = cudaStreamWaitEvent(s, gs->prep_join, 0);   // the FP32 working weights
+        if (e != cudaSuccess) return cuda_failed(e);
+    }
     CUtensorMap mBh, mBl;
     if (!make_tensor_map_f32_2d_sw128(&mBh, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN) ||
         !make_tensor_map_f32_2d_sw128(&mBl, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN))
