@@ -979,31 +979,42 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
         }
     } else {
         // ---------------------------------------------------- epilogue
+        // The TMEM read gives thread = row; each 32 x 32 chunk goes through
+        // shared memory (row stride 33: no bank conflicts either way) so that
+        // W is read and written a row at a time, lane = column (128 bytes
+        // per row).  A chunk's W values are requested before its TMEM read.
+        __shared__ float ebuf[4][32][33];
         const int q = warp & 3;                                        // TMEM lane quarter of this warp
+        float(*buf)[33] = ebuf[q];
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
             const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * UBN;
+            const int64_t r0 = (int64_t)m0 + 32 * q;                   // this warp's 32 rows
+            const int nrows = (int)(g.M - r0 < 32 ? g.M - r0 : 32);   // may be 0 or less
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kUWaitNs)) break;
             tc_fence_after();
-            const int64_t row = (int64_t)m0 + 32 * q + lane;
 #pragma unroll 1
             for (int c = 0; c < UBN / 32; ++c) {
+                const int64_t col = (int64_t)n0 + 32 * c;              // 32 columns: all inside Nc or all past it
+                const bool live = col < g.Nc;
+                float *wp = g.W + r0 * g.ldw + g.b1 + col + lane;
+                float w[32];
+                if (live) {
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr) w[rr] = rr < nrows ? wp[rr * g.ldw] : 0.0f;
+                }
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * UBN + 32 * c, r);
                 tmem_ld_wait();
-                const int64_t col = (int64_t)n0 + 32 * c;              // 32 columns: all inside Nc or all past it
-                if (row < g.M && col < g.Nc) {
-                    float4 *p = reinterpret_cast<float4 *>(g.W + row * g.ldw + g.b1 + col);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        float4 w = p[v];
-                        w.x -= __uint_as_float(r[4 * v]);
-                        w.y -= __uint_as_float(r[4 * v + 1]);
-                        w.z -= __uint_as_float(r[4 * v + 2]);
-                        w.w -= __uint_as_float(r[4 * v + 3]);
-                        p[v] = w;
-                    }
+                for (int j = 0; j < 32; ++j) buf[lane][j] = __uint_as_float(r[j]);
+                __syncwarp();
+                if (live) {
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr)
+                        if (rr < nrows) wp[rr * g.ldw] = w[rr] - buf[rr][lane];
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
