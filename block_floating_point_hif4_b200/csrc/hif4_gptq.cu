@@ -822,13 +822,21 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_gptq_block(GptqArgs a)
 // TMEM allocation and the single MMA-issuing thread; warps 2-5: epilogue,
 // thread = row.  Every wait is bounded; a time-out sets the abort flag, lets
 // the copies in flight land, and reports HIF4_FLAG_TIMEOUT.
-constexpr int UBM = 128, UBN = 128, UBK = 32, USTG = 3;
-constexpr uint32_t kUTile = UBM * UBK * 4;                // one 128 x 32 FP32 tile: 16 KB
-constexpr uint32_t kUStage = 4 * kUTile;                  // E_hi, E_lo, U^T_hi, U^T_lo
-constexpr size_t kUSmem = USTG * kUStage + 1024 + 256;
+constexpr int UBM = 128, UBK = 32;
 constexpr int kUThreads = 192;
-constexpr uint32_t kUTmemCols = 2 * UBN;
 constexpr uint64_t kUWaitNs = 2000000000ull;
+// Tiles of 128 x BN (BN = 128: a 3-stage ring of 64 KB stages; BN = 256: a
+// 2-stage ring of 96 KB stages and the whole 512-column TMEM for the two
+// accumulators).
+template <int BN>
+struct UCfg {
+    static constexpr int STG = BN == 128 ? 3 : 2;
+    static constexpr uint32_t kA = UBM * UBK * 4;           // a 128 x 32 FP32 tile of E: 16 KB
+    static constexpr uint32_t kB = BN * UBK * 4;            // a BN x 32 FP32 tile of U^T
+    static constexpr uint32_t kStage = 2 * kA + 2 * kB;     // E_hi, E_lo, U^T_hi, U^T_lo
+    static constexpr size_t kSmem = STG * kStage + 1024 + 256;
+    static constexpr uint32_t kTmemCols = 2 * BN;
+};
 
 struct UpdArgs {
     float *W;                // C = W[:, b1 : b1 + Nc], row-major, ld ldw
@@ -860,11 +868,15 @@ constexpr uint32_t idesc_tf32_f32(uint32_t M, uint32_t N)
     return (1u << 4) | (2u << 7) | (2u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kUThreads, 1)
 k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
               const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmBl, UpdArgs g)
 {
     using namespace sm100;
+    using C = UCfg<BN>;
+    constexpr int USTG = C::STG;
+    constexpr uint32_t kUStage = C::kStage;
     extern __shared__ uint8_t usm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(usm_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + USTG * kUStage);
@@ -893,7 +905,7 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
         prefetch_tensormap(&tmBl);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, kUTmemCols);
+        tmem_alloc(tmem_holder, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -909,7 +921,7 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
             uint32_t stage = 0, phase = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
-                const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * UBN;
+                const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * BN;
                 for (int kb = 0; kb < g.nkb; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kUWaitNs)) {
                         ok = false;
@@ -918,9 +930,9 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
                     uint8_t *st = sm + stage * kUStage;
                     mbar_arrive_expect_tx(&full[stage], kUStage);
                     tma_load_2d(st, &tmAh, g.a0 + kb * UBK, m0, &full[stage]);
-                    tma_load_2d(st + kUTile, &tmAl, g.a0 + kb * UBK, m0, &full[stage]);
-                    tma_load_2d(st + 2 * kUTile, &tmBh, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
-                    tma_load_2d(st + 3 * kUTile, &tmBl, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
+                    tma_load_2d(st + C::kA, &tmAl, g.a0 + kb * UBK, m0, &full[stage]);
+                    tma_load_2d(st + 2 * C::kA, &tmBh, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
+                    tma_load_2d(st + 2 * C::kA + C::kB, &tmBl, g.b0 + kb * UBK, g.b1 + n0, &full[stage]);
                     ++issued;
                     if (++stage == USTG) {
                         stage = 0;
@@ -940,21 +952,21 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------- MMA issuer
-            const uint32_t idesc = idesc_tf32_f32(UBM, UBN);
+            const uint32_t idesc = idesc_tf32_f32(UBM, BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < g.num_tiles; t += gridDim.x) {
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kUWaitNs)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + acc * UBN;
+                const uint32_t d = tmem + acc * BN;
                 for (int kb = 0; kb < g.nkb; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kUWaitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t ah = smem_addr(sm + stage * kUStage), al = ah + kUTile, bh = ah + 2 * kUTile,
-                                   bl = ah + 3 * kUTile;
+                    const uint32_t ah = smem_addr(sm + stage * kUStage), al = ah + C::kA, bh = ah + 2 * C::kA,
+                                   bl = bh + C::kB;
 #pragma unroll
                     for (int k = 0; k < UBK / 8; ++k) {                // 8 TF32 = 32 bytes per step
                         mma_tf32_tc(d, smem_desc_sw128(al + 32 * k), smem_desc_sw128(bh + 32 * k), idesc,
@@ -988,13 +1000,13 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
         float(*buf)[33] = ebuf[q];
         uint32_t acc = 0, acc_phase = 0;
         for (int t = blockIdx.x; t < g.num_tiles; t += gridDim.x) {
-            const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * UBN;
+            const int m0 = (t % g.num_m) * UBM, n0 = (t / g.num_m) * BN;
             const int64_t r0 = (int64_t)m0 + 32 * q;                   // this warp's 32 rows
             const int nrows = (int)(g.M - r0 < 32 ? g.M - r0 : 32);   // may be 0 or less
             if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kUWaitNs)) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < UBN / 32; ++c) {
+            for (int c = 0; c < BN / 32; ++c) {
                 const int64_t col = (int64_t)n0 + 32 * c;              // 32 columns: all inside Nc or all past it
                 const bool live = col < g.Nc;
                 float *wp = g.W + r0 * g.ldw + g.b1 + col + lane;
@@ -1004,7 +1016,7 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
                     for (int rr = 0; rr < 32; ++rr) w[rr] = rr < nrows ? wp[rr * g.ldw] : 0.0f;
                 }
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * UBN + 32 * c, r);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + acc * BN + 32 * c, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) buf[lane][j] = __uint_as_float(r[j]);
@@ -1026,7 +1038,7 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kUTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
     if (threadIdx.x == 0 && *abort_flag) status_or(g.status, HIF4_FLAG_TIMEOUT);
 }
 
@@ -1351,8 +1363,9 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
                 attr_g3[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    static bool attr_up[64] = {false};
-    if (!set_smem_once(k_update_tf32, kUSmem, attr_up[dev & 63]) ||
+    static bool attr_up[64] = {false}, attr_up2[64] = {false};
+    if (!set_smem_once(k_update_tf32<128>, UCfg<128>::kSmem, attr_up[dev & 63]) ||
+        !set_smem_once(k_update_tf32<256>, UCfg<256>::kSmem, attr_up2[dev & 63]) ||
         !set_smem_once(k_leaf<2>, kLeafSmem2, attr_leaf[dev & 63]) ||
         !set_smem_once(k_leaf<4>, kLeafSmem4, attr_leaf4[dev & 63]) ||
         !set_smem_once(k_dgemm<false, 64, 2>, gemm_smem<64, 2>(), attr_g0[dev & 63]) ||
@@ -1418,9 +1431,11 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
         const cudaError_t e = cudaStreamWaitEvent(s, gs->prep_join, 0);   // the FP32 working weights
         if (e != cudaSuccess) return cuda_failed(e);
     }
-    CUtensorMap mBh, mBl;
-    if (!make_tensor_map_f32_2d_sw128(&mBh, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN) ||
-        !make_tensor_map_f32_2d_sw128(&mBl, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, UBN))
+    CUtensorMap mBh, mBl, mBh2, mBl2;                  // boxes of 128 and 256 rows of U^T
+    if (!make_tensor_map_f32_2d_sw128(&mBh, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, 128) ||
+        !make_tensor_map_f32_2d_sw128(&mBl, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, 128) ||
+        !make_tensor_map_f32_2d_sw128(&mBh2, UTh, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, 256) ||
+        !make_tensor_map_f32_2d_sw128(&mBl2, UTl, (uint64_t)K, (uint64_t)K, (uint64_t)K * 4, UBK, 256))
         return HIF4_ERR_CUDA;
     // 3. the group loop, a two-level lazy update: within a super-block of
     //    S columns (whole blocks), each block's groups (with their in-block
@@ -1436,11 +1451,17 @@ hif4_status higptq1_enqueue(const void *w, int64_t N, int64_t K, int64_t ldw, co
         return HIF4_ERR_CUDA;
     auto update = [&](int64_t a0, int64_t k0, int64_t k1, int64_t c0, int64_t c1) -> hif4_status {
         // W[:, c0:c1] -= E[:, a0 : a0 + k1 - k0] U[k0:k1, c0:c1]
-        const int num_m = (int)((N + UBM - 1) / UBM), num_n = (int)((c1 - c0 + UBN - 1) / UBN);
+        // 128 x 256 tiles for the wide updates (half the E traffic per output), 128 x 128 otherwise
+        const bool wide = (c1 - c0) % 256 == 0 && c1 - c0 >= 512;
+        const int bn = wide ? 256 : 128;
+        const int num_m = (int)((N + UBM - 1) / UBM), num_n = (int)((c1 - c0 + bn - 1) / bn);
         UpdArgs ua{W, K, N, c1 - c0, (int)k0, (int)c0, (int)((k1 - k0) / UBK), num_m, num_m * num_n, status,
                    (int)a0};
         const int grid = std::min(num_m * num_n, sm_count());
-        return launch_pdl(k_update_tf32, dim3(grid), dim3(kUThreads), kUSmem, s, mAh, mAl, mBh, mBl, ua);
+        return wide ? launch_pdl(k_update_tf32<256>, dim3(grid), dim3(kUThreads), UCfg<256>::kSmem, s, mAh, mAl, mBh2,
+                                 mBl2, ua)
+                    : launch_pdl(k_update_tf32<128>, dim3(grid), dim3(kUThreads), UCfg<128>::kSmem, s, mAh, mAl, mBh,
+                                 mBl, ua);
     };
     for (int64_t s0 = 0; s0 < K; s0 += S) {
         const int64_t s1 = s0 + S < K ? s0 + S : K;
