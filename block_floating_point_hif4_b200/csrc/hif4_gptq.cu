@@ -637,7 +637,7 @@ struct GptqArgs {
                              // that group is quantized from
     int64_t N, K;
     int64_t b0;              // first column of the block
-    const float *U;          // K x K upper factor
+    const float *U;          // K x K upper factor (its blocks below the diagonal are not written)
     const float *UinvG;      // (K / 64) x 64 x 64: inverse of U's diagonal blocks
     const uint8_t *mask;     // u8 [K] or null
     const int32_t *rank;     // [K] protected rank or -1
@@ -1047,12 +1047,16 @@ k_update_tf32(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ 
 // (the reversed diagonal block of the Cholesky factor); and U^T in TF32
 // parts, U^T = UTh + UTl (UTh = U rounded to TF32, UTl = the rest rounded to
 // TF32), the K-major B operand of the lazy update.  One 32 x 32 tile per
-// block of 32 x 8 threads, transposed through shared memory.
+// block of 32 x 8 threads, transposed through shared memory.  U's (and U^T's)
+// 64 x 64 blocks below the diagonal are zero and never read (the group
+// kernel reads U's blocks right of the diagonal, the updates E U[k0:k1, c0:c1]
+// have k1 <= c0): they are left unwritten.
 __global__ void k_build_u(const double *Y, const double *A, int64_t K, float *U, float *UinvG, float *UTh,
                           float *UTl)
 {
     __shared__ float t[32][33];
     const int64_t i0 = blockIdx.y * 32ll, j0 = blockIdx.x * 32ll;
+    if (i0 / TB > j0 / TB) return;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int64_t i = i0 + threadIdx.y + 8 * q, j = j0 + threadIdx.x;
