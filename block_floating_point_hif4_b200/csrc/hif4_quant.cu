@@ -695,31 +695,41 @@ __device__ __forceinline__ void encode32(const uint32_t (&w)[16], const uint32_t
     }
     const float S = e6m2_value(c);
     const uint32_t T1 = f_bits(1.75f * S) >> 16, T2 = f_bits(3.5f * S) >> 16;
-    const uint32_t a8[4] = {A8a & 0xFFFFu, A8a >> 16, A8b & 0xFFFFu, A8b >> 16};
-    uint32_t e2[4], E[8], e2bits = 0, e3bits = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        e2[j] = a8[j] > T2;
-        const uint32_t th = e2[j] ? T2 : T1;
-        const uint32_t e3a = (A[j] & 0xFFFFu) > th, e3b = (A[j] >> 16) > th;
-        E[2 * j] = e2[j] + e3a;
-        E[2 * j + 1] = e2[j] + e3b;
-        e2bits |= e2[j] << j;
-        e3bits |= (e3a << (2 * j)) | (e3b << (2 * j + 1));
-    }
+    // Level decisions on pairs of 16-bit keys (all below 0x8000): key > T
+    // exactly when bit 15 of key + 0x7FFF - T is set, with no carry into the
+    // other half.  e2 of the 8-groups from their maxima; the 4-groups' e3
+    // against T2 where e2 is set, else T1 (selected by a byte-permute mask).
+    const uint32_t K1 = (0x7FFFu - T1) * 0x10001u, K2 = (0x7FFFu - T2) * 0x10001u;
+    const uint32_t G2a = (A8a + K2) & 0x80008000u, G2b = (A8b + K2) & 0x80008000u;
     float ih, il;
     recip_pair(c & 3u, ih, il);
     if ((c & 3u) == 0) il = bits_f(0x21800000u);             // 2^-60: keeps the exponent arithmetic valid
     const float pw0 = bits_f((160u - (c >> 2)) << 23);       // 2^(33 - E6)
     const uint32_t H0 = f_bits(ih * pw0), L0 = f_bits(il * pw0);
+    uint32_t Hk[8], Lk[8], Z = 0;                            // per 4-group: H0, L0 scaled by 2^-E
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t G = j < 2 ? G2a : G2b;
+        const uint32_t Mj = prmt(G, 0, (j & 1) ? 0xBBBBu : 0x9999u);        // all ones where e2_j
+        const uint32_t P1 = (A[j] + K1) & 0x80008000u, P2 = (A[j] + K2) & 0x80008000u;
+        const uint32_t y = ((P1 & ~Mj) | (P2 & Mj)) >> 15;                  // e3 of 4-groups 2j (bit 0), 2j+1 (bit 16)
+        const uint32_t Ep = y + (Mj & 0x10001u);                             // [E_2j, E_2j+1] in 16-bit halves
+        Hk[2 * j] = imad(Ep, 0xFF800000u, H0);                               // (the high half vanishes mod 2^32)
+        Lk[2 * j] = imad(Ep, 0xFF800000u, L0);
+        Hk[2 * j + 1] = imad(Ep & 0xFFFF0000u, 0xFFFFFF80u, H0);
+        Lk[2 * j + 1] = imad(Ep & 0xFFFF0000u, 0xFFFFFF80u, L0);
+        Z = imad(y, 1u << (2 * j), Z);
+    }
+    const uint32_t u2 = (G2a >> 15) | (G2b >> 13);           // e2 of 8-groups 0, 2 at bits 0, 2; 1, 3 at 16, 18
+    const uint32_t e2bits = (u2 & 5u) | ((u2 >> 15) & 0xAu);
+    const uint32_t e3bits = (Z & 0x55u) | ((Z >> 15) & 0xAAu);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         uint32_t tb[16];
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
             const int k = 4 * hh + (p >> 1);
-            const float H = bits_f(imad(E[k], 0xFF800000u, H0));   // exponent - E
-            const float L = bits_f(imad(E[k], 0xFF800000u, L0));
+            const float H = bits_f(Hk[k]), L = bits_f(Lk[k]);   // exponent - E
             const uint32_t m = mk[8 * hh + p];
             const u64 ax = pk(bits_f(imad(m, 65536u, 0u)), bits_f(m & 0xFFFF0000u));
             const u64 r = ffma2(ax, pk(H, H), fmul2(ax, pk(L, L)));
